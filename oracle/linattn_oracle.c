@@ -1,0 +1,230 @@
+/*
+ * linattn_oracle.c — plain fp64 CPU oracle for kernelized linear attention
+ * with the elu(x)+1 feature map.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the tests, the package's smoke check and the bench's
+ * CPU-baseline leg do.  It shares no code, header, table or helper with the
+ * CUDA library; the two meet only through the seeded input arrays.
+ *
+ * Every function walks the tokens one at a time, in the order and notation
+ * of the pages it follows, with no blocking, chunking or reordering:
+ *
+ *   phi(x)  = elu(x) + 1                       (Transformers-are-RNNs map;
+ *             "Linear Attention" knowledge-base page, section 2, "Choice of
+ *             phi"; linear-attention lesson, "What the pieces are for")
+ *   S_t     = a_t * S_{t-1} + phi(k_t) v_t^T    (running state, section 2
+ *   z_t     = a_t * z_{t-1} + phi(k_t)           "Causal recurrence"; decay
+ *                                                 a_t from the concept card's
+ *                                                 "Implementation sketch" and
+ *                                                 its SSD variant, a_t = 1 is
+ *                                                 the plain form)
+ *   o_t     = phi(q_t)^T S_t / (phi(q_t)^T z_t + eps)
+ *                                               (normalised read-out with the
+ *                                                 1e-6 of the section 3 sketch)
+ *
+ * Layouts (all row-major, C order, fp64):
+ *   q, k     [B, H, T, d_k]      v [B, H, T, d_v]      out [B, H, T, d_v]
+ *   decay    [B, H, T] (causal) or [B, H] (decode); NULL = no decay
+ *   S        [B, H, d_k, d_v]    z [B, H, d_k]
+ *
+ * Parallelism: independent (b, h) heads are spread over OpenMP threads; the
+ * arithmetic of one head is sequential and identical for any thread count.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* elu(x) + 1 with alpha = 1.  For x <= 0, elu(x) + 1 = (e^x - 1) + 1, which
+ * is e^x exactly in real arithmetic; writing e^x avoids the cancellation of
+ * the -1/+1 pair.  At x = 0 both branches give 1. */
+static double phi(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
+
+void orc_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int orc_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* One head of the causal recurrence.  fk/fq are scratch of length dk. */
+static void causal_head(const double *q, const double *k, const double *v,
+                        const double *decay, long T, int dk, int dv, double eps,
+                        double *S, double *z, double *out, double *fk, double *fq)
+{
+    for (long t = 0; t < T; ++t) {
+        const double *qt = q + t * dk, *kt = k + t * dk, *vt = v + t * dv;
+        for (int i = 0; i < dk; ++i) { fk[i] = phi(kt[i]); fq[i] = phi(qt[i]); }
+        if (decay) {
+            /* decayed form: the old state is scaled first, the new token
+             * enters undecayed */
+            const double a = decay[t];
+            for (int i = 0; i < dk; ++i) {
+                for (int j = 0; j < dv; ++j) S[i * dv + j] = a * S[i * dv + j] + fk[i] * vt[j];
+                z[i] = a * z[i] + fk[i];
+            }
+        } else {
+            /* plain form: rank-one update and vector update */
+            for (int i = 0; i < dk; ++i) {
+                for (int j = 0; j < dv; ++j) S[i * dv + j] = S[i * dv + j] + fk[i] * vt[j];
+                z[i] = z[i] + fk[i];
+            }
+        }
+        double den = 0.0;
+        for (int i = 0; i < dk; ++i) den += fq[i] * z[i];
+        double *ot = out + t * dv;
+        for (int j = 0; j < dv; ++j) {
+            double num = 0.0;
+            for (int i = 0; i < dk; ++i) num += fq[i] * S[i * dv + j];
+            ot[j] = num / (den + eps);
+        }
+    }
+}
+
+/*
+ * Causal linear attention over all heads.
+ *   S_in/z_in  : initial state, or NULL for zeros.
+ *   S_out/z_out: final state, or NULL to discard.
+ * Returns 0, or -1 on a bad argument / allocation failure.
+ */
+int orc_causal(const double *q, const double *k, const double *v, const double *decay,
+               int B, int H, long T, int dk, int dv, double eps,
+               const double *S_in, const double *z_in,
+               double *out, double *S_out, double *z_out)
+{
+    if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
+    const long BH = (long)B * H;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+        double *z = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *fk = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *fq = (double *)malloc(sizeof(double) * (size_t)dk);
+        if (!S || !z || !fk || !fq) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bh = 0; bh < BH; ++bh) {
+                if (S_in) memcpy(S, S_in + bh * dk * dv, sizeof(double) * (size_t)dk * dv);
+                else memset(S, 0, sizeof(double) * (size_t)dk * dv);
+                if (z_in) memcpy(z, z_in + bh * dk, sizeof(double) * (size_t)dk);
+                else memset(z, 0, sizeof(double) * (size_t)dk);
+                causal_head(q + bh * T * dk, k + bh * T * dk, v + bh * T * dv,
+                            decay ? decay + bh * T : NULL, T, dk, dv, eps,
+                            S, z, out + bh * T * dv, fk, fq);
+                if (S_out) memcpy(S_out + bh * dk * dv, S, sizeof(double) * (size_t)dk * dv);
+                if (z_out) memcpy(z_out + bh * dk, z, sizeof(double) * (size_t)dk);
+            }
+        }
+        free(S); free(z); free(fk); free(fq);
+    }
+    return err ? -1 : 0;
+}
+
+/*
+ * Non-causal linear attention: the prefix sums collapse to global sums over
+ * all Lk keys (knowledge-base page, section 3, first sketch):
+ *   S = S_in + sum_j phi(k_j) v_j^T,  z = z_in + sum_j phi(k_j),
+ *   o_i = phi(q_i)^T S / (phi(q_i)^T z + eps)  for each of the Lq queries.
+ * S_out/z_out receive the totals (including the state in), or NULL.
+ */
+int orc_noncausal(const double *q, const double *k, const double *v,
+                  int B, int H, long Lq, long Lk, int dk, int dv, double eps,
+                  const double *S_in, const double *z_in,
+                  double *out, double *S_out, double *z_out)
+{
+    if (B < 0 || H < 0 || Lq < 0 || Lk < 0 || dk <= 0 || dv <= 0) return -1;
+    const long BH = (long)B * H;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+        double *z = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *f = (double *)malloc(sizeof(double) * (size_t)dk);
+        if (!S || !z || !f) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bh = 0; bh < BH; ++bh) {
+                if (S_in) memcpy(S, S_in + bh * dk * dv, sizeof(double) * (size_t)dk * dv);
+                else memset(S, 0, sizeof(double) * (size_t)dk * dv);
+                if (z_in) memcpy(z, z_in + bh * dk, sizeof(double) * (size_t)dk);
+                else memset(z, 0, sizeof(double) * (size_t)dk);
+                const double *kh = k + bh * Lk * dk, *vh = v + bh * Lk * dv;
+                for (long j = 0; j < Lk; ++j) {
+                    for (int i = 0; i < dk; ++i) f[i] = phi(kh[j * dk + i]);
+                    for (int i = 0; i < dk; ++i) {
+                        for (int c = 0; c < dv; ++c) S[i * dv + c] += f[i] * vh[j * dv + c];
+                        z[i] += f[i];
+                    }
+                }
+                const double *qh = q + bh * Lq * dk;
+                double *oh = out + bh * Lq * dv;
+                for (long t = 0; t < Lq; ++t) {
+                    for (int i = 0; i < dk; ++i) f[i] = phi(qh[t * dk + i]);
+                    double den = 0.0;
+                    for (int i = 0; i < dk; ++i) den += f[i] * z[i];
+                    for (int c = 0; c < dv; ++c) {
+                        double num = 0.0;
+                        for (int i = 0; i < dk; ++i) num += f[i] * S[i * dv + c];
+                        oh[t * dv + c] = num / (den + eps);
+                    }
+                }
+                if (S_out) memcpy(S_out + bh * dk * dv, S, sizeof(double) * (size_t)dk * dv);
+                if (z_out) memcpy(z_out + bh * dk, z, sizeof(double) * (size_t)dk);
+            }
+        }
+        free(S); free(z); free(f);
+    }
+    return err ? -1 : 0;
+}
+
+/*
+ * One constant-state decode step per head: the causal loop body applied once
+ * to a carried (S, z), which are updated in place.
+ *   q, k [B, H, dk], v [B, H, dv], decay [B, H] or NULL, out [B, H, dv].
+ */
+int orc_decode_step(const double *q, const double *k, const double *v, const double *decay,
+                    int B, int H, int dk, int dv, double eps,
+                    double *S, double *z, double *out)
+{
+    if (B < 0 || H < 0 || dk <= 0 || dv <= 0 || !S || !z) return -1;
+    const long BH = (long)B * H;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *fk = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *fq = (double *)malloc(sizeof(double) * (size_t)dk);
+        if (!fk || !fq) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (long bh = 0; bh < BH; ++bh) {
+                causal_head(q + bh * dk, k + bh * dk, v + bh * dv,
+                            decay ? decay + bh : NULL, 1, dk, dv, eps,
+                            S + bh * dk * dv, z + bh * dk, out + bh * dv, fk, fq);
+            }
+        }
+        free(fk); free(fq);
+    }
+    return err ? -1 : 0;
+}

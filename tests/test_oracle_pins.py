@@ -1,0 +1,291 @@
+"""Pins for the fp64 oracle, checked against things the pages and the
+mathematics fix, never against the oracle itself:
+
+* the linear-attention lesson's worked N=8, d=4, seed-0 example and its
+  masked quadratic check (tests/golden/lesson_n8_d4_seed0.txt);
+* brute-force masked quadratic attention on tiny inputs (the lesson's
+  "same thing written as masked quadratic attention");
+* the decayed, 1-semiseparable weighted quadratic form (the lesson's "Try it
+  yourself" decay exercise; the concept card's SSD variant);
+* decay 1 being the plain causal form (concept card, SSD variant);
+* associativity of the non-causal bracketing (knowledge-base page, section 3;
+  lesson, "Two ways to bracket the same product");
+* closed forms on constructed inputs, the feature map against torch's elu,
+  invariances, state split / hand-off equivalences.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def phi_ref(x):
+    """elu(x)+1 through torch's own elu, in fp64 (library routine)."""
+    return torch.nn.functional.elu(torch.as_tensor(x, dtype=torch.float64)).numpy() + 1.0
+
+
+def quad_causal(q, k, v, eps, weights=None):
+    """Brute force masked quadratic form for one head: scores = phi(Q) phi(K)^T,
+    masked to j <= i (and weighted if given), rows normalised by their sums."""
+    fq, fk = phi_ref(q), phi_ref(k)
+    T = q.shape[0]
+    scores = fq @ fk.T
+    mask = np.tril(np.ones((T, T)))
+    scores = scores * mask
+    if weights is not None:
+        scores = scores * weights
+    return (scores @ v) / (scores.sum(-1, keepdims=True) + eps)
+
+
+def read_golden(name):
+    vals = {}
+    multi = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, val = [s.strip() for s in line.split("=", 1)]
+            if key in vals:
+                multi.setdefault(key, [vals[key]]).append(val)
+            vals[key] = val
+    return vals, multi
+
+
+def test_lesson_worked_example(orc):
+    g, multi = read_golden("lesson_n8_d4_seed0.txt")
+    N, d, eps = int(g["N"]), int(g["d"]), float(g["eps"])
+    torch.manual_seed(int(g["seed"]))
+    Q, K, V = torch.randn(N, d), torch.randn(N, d), torch.randn(N, d)
+    out, S, z = orc.causal(Q[None, None], K[None, None], V[None, None], eps=eps)
+    out = out[0, 0]
+    # the page's fp32 masked quadratic form, recomputed in fp32 with torch
+    q32, k32 = torch.nn.functional.elu(Q) + 1, torch.nn.functional.elu(K) + 1
+    sc = (q32 @ k32.T) * torch.tril(torch.ones(N, N))
+    quad32 = ((sc @ V) / (sc.sum(-1, keepdim=True) + eps)).double().numpy()
+    # the oracle agrees with the page's check at the page's tolerance, and with
+    # the fp32 result to the magnitude the page prints (4.77e-7, fp32 rounding)
+    atol = float(g["recurrent_matches_quadratic_atol"])
+    assert np.abs(out - quad32).max() <= atol
+    assert np.abs(out - quad32).max() <= 10 * float(g["max_difference_fp32"])
+    # fp64 brute force: agreement to rounding
+    np.testing.assert_allclose(out, quad_causal(Q.double().numpy(), K.double().numpy(),
+                                                V.double().numpy(), eps), rtol=1e-12, atol=1e-13)
+    # state carried: d x d numbers, independent of t
+    assert S[0, 0].size == int(g["state_numbers"]) == d * d
+    assert 2 * N * d == int(g["kv_cache_numbers_at_t8"])
+    # bracketing: (q k^T) V == q (k^T V) in the non-causal form
+    onc, _, _ = orc.noncausal(Q[None, None], K[None, None], V[None, None], eps=eps)
+    fq, fk = phi_ref(Q.double().numpy()), phi_ref(K.double().numpy())
+    left = (fq @ fk.T) @ V.double().numpy() / ((fq @ fk.T).sum(-1, keepdims=True) + eps)
+    np.testing.assert_allclose(onc[0, 0], left, rtol=1e-12, atol=1e-13)
+    assert g["scores_shape"] == f"{N}x{N}" and g["kTv_shape"] == f"{d}x{d}"
+    for row in multi["crossover"]:
+        n, a, b, r = row.split()
+        n = int(n)
+        assert n * n * d == int(a) and n * d * d == int(b) and float(r) == n * n * d / (n * d * d)
+
+
+@pytest.mark.parametrize("seed,T,dk,dv", [(1, 1, 1, 1), (2, 5, 3, 2), (3, 17, 4, 4),
+                                          (4, 64, 8, 5), (5, 33, 2, 7)])
+def test_masked_quadratic_bruteforce(orc, seed, T, dk, dv):
+    rng = np.random.default_rng(seed)
+    B, H = 2, 3
+    q = rng.standard_normal((B, H, T, dk))
+    k = rng.standard_normal((B, H, T, dk))
+    v = rng.standard_normal((B, H, T, dv))
+    out, S, z = orc.causal(q, k, v, eps=1e-6)
+    for b in range(B):
+        for h in range(H):
+            ref = quad_causal(q[b, h], k[b, h], v[b, h], 1e-6)
+            np.testing.assert_allclose(out[b, h], ref, rtol=1e-11, atol=1e-12)
+            # final state is the full prefix sum
+            fk = phi_ref(k[b, h])
+            np.testing.assert_allclose(S[b, h], fk.T @ v[b, h], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(z[b, h], fk.sum(0), rtol=1e-12)
+
+
+def _semiseparable(a):
+    """W[i, j] = prod_{l=j+1..i} a_l for j <= i, else 0 — explicit products."""
+    T = a.shape[0]
+    W = np.zeros((T, T))
+    for i in range(T):
+        for j in range(i + 1):
+            p = 1.0
+            for l in range(j + 1, i + 1):
+                p *= a[l]
+            W[i, j] = p
+    return W
+
+
+@pytest.mark.parametrize("seed,T,d", [(11, 9, 3), (12, 40, 4), (13, 64, 6)])
+def test_decayed_quadratic(orc, seed, T, d):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, 2, T, d))
+    k = rng.standard_normal((1, 2, T, d))
+    v = rng.standard_normal((1, 2, T, d))
+    a = 1.0 / (1.0 + np.exp(-(rng.standard_normal((1, 2, T)) + 2.0)))
+    out, S, z = orc.causal(q, k, v, decay=a, eps=1e-6)
+    for h in range(2):
+        W = _semiseparable(a[0, h])
+        ref = quad_causal(q[0, h], k[0, h], v[0, h], 1e-6, weights=W)
+        np.testing.assert_allclose(out[0, h], ref, rtol=1e-11, atol=1e-12)
+        # final state: sum_j (prod_{l>j} a_l) phi(k_j) v_j^T
+        fk = phi_ref(k[0, h])
+        np.testing.assert_allclose(S[0, h], (fk * W[-1][:, None]).T @ v[0, h], rtol=1e-11,
+                                   atol=1e-12)
+
+
+def test_lesson_decay_exercise(orc):
+    """S = 0.9 S + outer(k, v): no longer the unweighted quadratic form, but the
+    one weighted by 0.9^(i-j)."""
+    torch.manual_seed(0)
+    N, d = 8, 4
+    Q, K, V = (torch.randn(N, d).double().numpy() for _ in range(3))
+    a = np.full((1, 1, N), 0.9)
+    out, _, _ = orc.causal(Q[None, None], K[None, None], V[None, None], decay=a, eps=1e-6)
+    plain = quad_causal(Q, K, V, 1e-6)
+    assert np.abs(out[0, 0] - plain).max() > 1e-3
+    i, j = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
+    W = np.where(j <= i, 0.9 ** (i - j).astype(float), 0.0)
+    np.testing.assert_allclose(out[0, 0], quad_causal(Q, K, V, 1e-6, weights=W), rtol=1e-12,
+                               atol=1e-13)
+
+
+def test_decay_one_is_plain_bitwise(orc):
+    rng = np.random.default_rng(21)
+    q, k, v = (rng.standard_normal((2, 2, 50, 6)) for _ in range(3))
+    o1, S1, z1 = orc.causal(q, k, v, eps=1e-6)
+    o2, S2, z2 = orc.causal(q, k, v, decay=np.ones((2, 2, 50)), eps=1e-6)
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2) and np.array_equal(z1, z2)
+
+
+def test_feature_map_against_torch_elu(orc):
+    """Two tokens, v = (1, 0), k_1 = 0 (phi = 1): o_1 = phi(k_0) / (phi(k_0) + 1),
+    so phi(k_0) is recovered from the oracle's output and compared with torch's
+    elu(x)+1 on both branches."""
+    xs = np.array([-30.0, -3.0, -1.0, -0.25, -1e-8, 0.0, 1e-8, 0.3, 1.0, 4.0])
+    for x in xs:
+        q = np.zeros((1, 1, 2, 1))
+        k = np.array([x, 0.0]).reshape(1, 1, 2, 1)
+        v = np.array([1.0, 0.0]).reshape(1, 1, 2, 1)
+        out, _, _ = orc.causal(q, k, v, eps=0.0)
+        o = out[0, 0, 1, 0]
+        # torch forms elu(x)+1 as (expm1(x)) + 1, exact to ~1 ulp of 1.0 in
+        # absolute terms; hence the absolute floor
+        np.testing.assert_allclose(o / (1 - o), phi_ref(x), rtol=1e-12, atol=1e-15)
+
+
+def test_noncausal_associativity_and_state_in(orc):
+    rng = np.random.default_rng(31)
+    B, H, Lq, Lk, d, e = 2, 2, 23, 37, 5, 3
+    q = rng.standard_normal((B, H, Lq, d))
+    k = rng.standard_normal((B, H, Lk, d))
+    v = rng.standard_normal((B, H, Lk, e))
+    out, S, z = orc.noncausal(q, k, v, eps=1e-6)
+    for b in range(B):
+        for h in range(H):
+            fq, fk = phi_ref(q[b, h]), phi_ref(k[b, h])
+            sc = fq @ fk.T
+            ref = (sc @ v[b, h]) / (sc.sum(-1, keepdims=True) + 1e-6)
+            np.testing.assert_allclose(out[b, h], ref, rtol=1e-12, atol=1e-13)
+    # state-in equals an extra prefix of keys
+    k2 = rng.standard_normal((B, H, 11, d))
+    v2 = rng.standard_normal((B, H, 11, e))
+    o_split, S_split, z_split = orc.noncausal(q, k2, v2, eps=1e-6, S_in=S, z_in=z)
+    o_all, S_all, z_all = orc.noncausal(q, np.concatenate([k, k2], 2),
+                                        np.concatenate([v, v2], 2), eps=1e-6)
+    np.testing.assert_allclose(o_split, o_all, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S_split, S_all, rtol=1e-12, atol=1e-12)
+    # V scaled by c scales the output by c; key order does not matter
+    o_c, _, _ = orc.noncausal(q, k, 3.5 * v, eps=1e-6)
+    np.testing.assert_allclose(o_c, 3.5 * out, rtol=1e-12, atol=1e-13)
+    perm = rng.permutation(Lk)
+    o_p, _, _ = orc.noncausal(q, k[:, :, perm], v[:, :, perm], eps=1e-6)
+    np.testing.assert_allclose(o_p, out, rtol=1e-12, atol=1e-13)
+
+
+def test_causal_last_row_is_noncausal(orc):
+    rng = np.random.default_rng(41)
+    q, k, v = (rng.standard_normal((1, 3, 30, 4)) for _ in range(3))
+    oc, Sc, zc = orc.causal(q, k, v, eps=1e-6)
+    on, Sn, zn = orc.noncausal(q[:, :, -1:], k, v, eps=1e-6)
+    np.testing.assert_allclose(oc[:, :, -1:], on, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(Sc, Sn, rtol=1e-12, atol=1e-12)
+
+
+def test_closed_forms(orc):
+    rng = np.random.default_rng(51)
+    eps = 1e-6
+    # T = 1: o = v w / (w + eps), w = phi(q).phi(k)
+    q, k, v = (rng.standard_normal((1, 1, 1, 6)) for _ in range(3))
+    out, _, _ = orc.causal(q, k, v, eps=eps)
+    w = float(phi_ref(q[0, 0, 0]) @ phi_ref(k[0, 0, 0]))
+    np.testing.assert_allclose(out[0, 0, 0], v[0, 0, 0] * w / (w + eps), rtol=1e-14)
+    # constant value rows: o_t = c den_t / (den_t + eps)
+    T = 20
+    q, k = (rng.standard_normal((1, 1, T, 4)) for _ in range(2))
+    c = rng.standard_normal(3)
+    v = np.broadcast_to(c, (1, 1, T, 3)).copy()
+    out, _, _ = orc.causal(q, k, v, eps=eps)
+    fq, fk = phi_ref(q[0, 0]), phi_ref(k[0, 0])
+    den = np.array([fq[t] @ fk[: t + 1].sum(0) for t in range(T)])
+    np.testing.assert_allclose(out[0, 0], c[None] * (den / (den + eps))[:, None], rtol=1e-13)
+    # all keys equal: o_t = (sum_{j<=t} v_j) / ((t + 1) + eps / w_t)
+    kk = np.broadcast_to(rng.standard_normal(4), (1, 1, T, 4)).copy()
+    v = rng.standard_normal((1, 1, T, 3))
+    out, _, _ = orc.causal(q, kk, v, eps=eps)
+    wt = fq @ phi_ref(kk[0, 0, 0])
+    ref = np.cumsum(v[0, 0], 0) / (np.arange(1, T + 1) + eps / wt)[:, None]
+    np.testing.assert_allclose(out[0, 0], ref, rtol=1e-12)
+
+
+@pytest.mark.parametrize("with_decay", [False, True])
+def test_state_split_and_decode_handoff(orc, with_decay):
+    rng = np.random.default_rng(61 + with_decay)
+    B, H, T1, T2, d, e = 2, 2, 13, 19, 5, 4
+    q = rng.standard_normal((B, H, T1 + T2 + 1, d))
+    k = rng.standard_normal((B, H, T1 + T2 + 1, d))
+    v = rng.standard_normal((B, H, T1 + T2 + 1, e))
+    a = rng.uniform(0.5, 1.0, (B, H, T1 + T2 + 1)) if with_decay else None
+    sl = lambda x, s: None if x is None else x[:, :, s]
+    T = T1 + T2
+    o_full, S_full, z_full = orc.causal(q[:, :, :T], k[:, :, :T], v[:, :, :T], sl(a, slice(0, T)))
+    o1, S1, z1 = orc.causal(sl(q, slice(0, T1)), sl(k, slice(0, T1)), sl(v, slice(0, T1)),
+                            sl(a, slice(0, T1)))
+    o2, S2, z2 = orc.causal(sl(q, slice(T1, T)), sl(k, slice(T1, T)), sl(v, slice(T1, T)),
+                            sl(a, slice(T1, T)), S_in=S1, z_in=z1)
+    np.testing.assert_allclose(np.concatenate([o1, o2], 2), o_full, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S2, S_full, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z2, z_full, rtol=1e-12)
+    # prefill(T) then one decode step == prefill(T + 1), last row
+    od, Sd, zd = orc.decode_step(q[:, :, T], k[:, :, T], v[:, :, T], S_full, z_full,
+                                 decay=None if a is None else a[:, :, T])
+    o_next, S_next, z_next = orc.causal(q, k, v, a)
+    np.testing.assert_allclose(od, o_next[:, :, T], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(Sd, S_next, rtol=1e-12, atol=1e-12)
+
+
+def test_kb_opcount_closed_form():
+    """The knowledge-base page's op counts are T d' d_h and T^2 d_h."""
+    g, _ = read_golden("kb_opcount_d128_t100k.txt")
+    T, dp, dh = int(g["T"]), int(g["d_feature"]), int(g["d_head"])
+    tol = float(g["rel_rounding"])
+    assert abs(T * dp * dh / float(g["linear_ops_approx"]) - 1) < tol
+    assert abs(T * T * dh / float(g["softmax_ops_approx"]) - 1) < tol
+
+
+def test_oracle_thread_count_invariance(orc):
+    rng = np.random.default_rng(71)
+    q, k, v = (rng.standard_normal((3, 3, 40, 4)) for _ in range(3))
+    n = orc.max_threads()
+    orc.set_threads(1)
+    o1, _, _ = orc.causal(q, k, v)
+    orc.set_threads(max(n, 2))
+    o2, _, _ = orc.causal(q, k, v)
+    orc.set_threads(n)
+    assert np.array_equal(o1, o2)
