@@ -1,0 +1,431 @@
+"""Benchmark of the hot path on B200: causal prefill tokens/s (and % of the HBM
+roofline) on the long-context workload, followed by its decode steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one causal prefill of B=1, H=16, T=131072, d=128 (bf16 inputs,
+fp32 state, chunk 128) followed by 1024 decode steps at B=64, H=16 from fp32
+states (the decode loop is replayed from a CUDA graph).  Inputs are seeded
+and synthetic and are resident in HBM before the timed region; the prefill's
+inputs (805 MB) are larger than the 126 MB L2, so successive steps do not
+reuse cached data.  ``value`` is prefill tokens/s (B*T per prefill, summed over
+ranks); the decode rate is reported beside it.
+
+Under torchrun each rank runs the same per-GPU workload on its own GPU (heads
+are independent: no collective on the data path; weak scaling); timings are
+the max over ranks.  ``--impl reference`` times the fp64 CPU oracle on the
+host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "causal linear-attn prefill tokens/s on 1 B200 and % of roofline; decode steps/s"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ cost model
+def elem_bytes(dtype: str) -> int:
+    return {"f32": 4, "bf16": 2, "f16": 2}[dtype]
+
+
+def prefill_algorithmic_bytes(w) -> int:
+    """Minimum bytes any implementation moves: Q, K, V (and decay) read once,
+    O written once.  The fp32 state in/out is excluded (it is per head)."""
+    ht = w.B * w.H * w.T
+    per = 3 * w.d * elem_bytes(w.dtype) + w.d * elem_bytes(w.out_dtype) + (4 if w.decay else 0)
+    return ht * per
+
+
+def prefill_flops(w) -> int:
+    """Dense-tile flops of the chunked algorithm per head-token:
+    scores 2*C*d, intra P.V 2*C*d, inter phi(Q) S 2*d*d, state update 2*d*d."""
+    return w.B * w.H * w.T * (4 * w.chunk * w.d + 4 * w.d * w.d)
+
+
+def decode_bytes_per_step(w) -> int:
+    bh = w.B * w.H
+    return bh * ((w.d * w.d + w.d) * 4 * 2 + 4 * w.d * elem_bytes(w.dtype))
+
+
+def linear_vs_softmax_ops(T: int, d_feature: int, d_head: int):
+    """Op counts of the knowledge-base page's cost comparison: T d' d_h vs T^2 d_h."""
+    return T * d_feature * d_head, T * T * d_head
+
+
+# ------------------------------------------------------------------ helpers
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        smax = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[2] > 250.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, f in enumerate(r[3]) if f == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU legs
+def oracle_prefill_sample(w, q, k, v, a, tokens: int, threads: int | None = None):
+    """Time the fp64 oracle on the first ``tokens`` positions of every head."""
+    import oracle
+    oracle.build()
+    if threads:
+        oracle.set_threads(threads)
+    sl = lambda x: None if x is None else x[..., :tokens, :].contiguous() if x.dim() == 4 \
+        else x[..., :tokens].contiguous()
+    qs, ks, vs, as_ = sl(q), sl(k), sl(v), sl(a)
+    t0 = time.perf_counter()
+    oracle.causal(qs, ks, vs, as_, w.eps)
+    dt = time.perf_counter() - t0
+    return w.B * tokens / dt, dt, oracle.max_threads()
+
+
+def run_reference(args, w):
+    """--impl reference: the fp64 oracle on the host cores, bounded samples."""
+    import torch
+    from kernelized_causal_sequence_b200 import inputs
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    tokens = args.ref_tokens
+    q, k, v, a = inputs.qkv(w, T=tokens)
+    rates, times = [], []
+    for i in range(args.warmup + args.steps):
+        r, dt, cores = oracle_prefill_sample(w, q, k, v, a, tokens)
+        if i >= args.warmup:
+            rates.append(r)
+            times.append(dt)
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1)/sqrt(d) inputs of the workload's distribution)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d,
+                   "chunk": w.chunk, "decay": w.decay,
+                   "sample": f"first {tokens} tokens of all {w.B * w.H} heads per step"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{w.B * w.H} heads x {tokens} tokens, fp64 recurrence"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU leg
+def run_ours(args, w):
+    import torch
+    import kernelized_causal_sequence_b200 as la
+    from kernelized_causal_sequence_b200 import inputs
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    L = la.lib()
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- inputs resident in HBM (generated on the host once, seeded)
+    q_h, k_h, v_h, a_h = inputs.qkv(w)
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    a = None if a_h is None else a_h.to(dev)
+    out = torch.empty((w.B, w.H, w.T, w.d), dtype=w.torch_out_dtype, device=dev)
+    S = torch.zeros((w.B, w.H, w.d, w.d), dtype=torch.float32, device=dev)
+    z = torch.zeros((w.B, w.H, w.d), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, la.la_prefill_workspace_size(w.B, w.H, w.T, w.d, w.d, w.chunk)),
+                     dtype=torch.uint8, device=dev)
+
+    def prefill():
+        la.la_prefill_causal(q, k, v, decay=a, eps=w.eps, chunk=w.chunk, state_S=S, state_z=z,
+                             mode=la.LA_STATE_OUT, out=out, workspace=ws, stream=stream)
+
+    # ---- decode: states from the library's own prefill of a 512-token prompt
+    wd = inputs.WORKLOADS["decode_bf16_b64h16_d128"] if w.name.startswith("prefill") else None
+    dec = None
+    if wd is not None and args.decode_steps > 0:
+        pq, pk, pv, _ = inputs.qkv(inputs.WORKLOADS["prefill_bf16_h16_t131072_d128"], T=wd.prompt,
+                                   B=wd.B, H=wd.H, seed=wd.seed + 1)
+        dS = torch.zeros((wd.B, wd.H, wd.d, wd.d), dtype=torch.float32, device=dev)
+        dz = torch.zeros((wd.B, wd.H, wd.d), dtype=torch.float32, device=dev)
+        la.la_prefill_causal(pq.to(dev), pk.to(dev), pv.to(dev), chunk=128, state_S=dS, state_z=dz,
+                             mode=la.LA_STATE_OUT)
+        S0, z0 = dS.clone(), dz.clone()
+        n_in = min(args.decode_steps, 64)  # distinct per-step inputs, cycled
+        qs, ks, vs = [], [], []
+        for i in range(n_in):
+            qi, ki, vi, _ = inputs.decode_inputs(wd, i)
+            qs.append(qi); ks.append(ki); vs.append(vi)
+        dq = torch.stack(qs).to(dev)
+        dk = torch.stack(ks).to(dev)
+        dv = torch.stack(vs).to(dev)
+        dout = torch.empty((wd.B, wd.H, wd.d), dtype=wd.torch_out_dtype, device=dev)
+        g_stream = torch.cuda.Stream(dev)
+
+        def decode_loop(st):
+            for i in range(args.decode_steps):
+                j = i % n_in
+                la.la_decode_step(dq[j], dk[j], dv[j], dS, dz, eps=wd.eps, out=dout, stream=st)
+
+        # warm up outside capture, then capture the whole loop in one graph
+        with torch.cuda.stream(g_stream):
+            decode_loop(g_stream)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        c0 = L.la_launch_count()
+        with torch.cuda.graph(graph, stream=g_stream):
+            decode_loop(g_stream)
+        graph_launches = L.la_launch_count() - c0
+        dec = dict(graph=graph, S0=S0, z0=z0, dS=dS, dz=dz, w=wd, launches=graph_launches)
+
+    launches_before = L.la_launch_count()
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        prefill()
+        if dec:
+            dec["graph"].replay()
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches_warm = L.la_launch_count()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            prefill()
+            e1.record(stream)
+            if dec:
+                dec["graph"].replay()
+            e2.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    pre_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    dec_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    pre_avg = max_over_ranks(sum(pre_ms) / len(pre_ms), world)
+    dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), world) if dec else 0.0
+    # direct launches, plus the decode kernels each graph replay re-issues
+    launches = L.la_launch_count() - launches_warm + (args.steps * dec["launches"] if dec else 0)
+    clocks = clk.summary()
+
+    tokens_per_prefill = w.B * w.T
+    value = world * tokens_per_prefill / (pre_avg * 1e-3)
+    alg_bytes = prefill_algorithmic_bytes(w)
+    achieved = alg_bytes / (pre_avg * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": args.traffic,
+            "kernel": "la_prefill_causal (all launches of one call)",
+            "peak_source": peak_src, "algorithmic_bytes": alg_bytes,
+            "flops": prefill_flops(w),
+            "tensor_frac_of_bf16_peak": prefill_flops(w) / (pre_avg * 1e-3) / 1e12
+            / peaks["bf16_tflops"]}
+
+    # ---- end to end through the public API with host buffers (pinned)
+    e2e = None
+    if rank == 0 or world > 1:
+        qp, kp, vp = (x.pin_memory() for x in (q_h, k_h, v_h))
+        ap = None if a_h is None else a_h.pin_memory()
+        op = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp) + ((ap,) if ap is not None else ()))
+        d2h = op.numel() * op.element_size()
+        n_e2e = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            q.copy_(qp, non_blocking=True)
+            k.copy_(kp, non_blocking=True)
+            v.copy_(vp, non_blocking=True)
+            if ap is not None:
+                a.copy_(ap, non_blocking=True)
+            prefill()
+            op.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, world)
+        e2e = {"value": world * tokens_per_prefill / (e2e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(128) bf16 inputs; decode states from the "
+                "library's prefill of a seeded 512-token prompt)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "chunk": w.chunk,
+                   "decay": w.decay, "out_dtype": w.out_dtype, "parallelism": f"heads x{world} (replicas)",
+                   "l2": "prefill inputs (805 MB) larger than L2; no flush needed",
+                   "prefill_path": "tcgen05" if la.la_prefill_path(w.torch_dtype, w.d, w.d, w.chunk) == 1
+                   else "simt"},
+        "ms_per_prefill": pre_avg,
+        "roofline": roof,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if dec:
+        dbytes = decode_bytes_per_step(dec["w"])
+        per_step_ms = dec_avg / args.decode_steps
+        line["decode"] = {
+            "value": world * 1e3 / per_step_ms, "unit": "steps/s", "steps_per_bench_step": args.decode_steps,
+            "B": dec["w"].B, "H": dec["w"].H, "d": dec["w"].d, "us_per_step": per_step_ms * 1e3,
+            "roofline": {"bound": "hbm", "achieved": dbytes / (per_step_ms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": dbytes / (per_step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "note": "fp32 state (67.6 MB) stays L2-resident across the loop"},
+        }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r, dt, cores = oracle_prefill_sample(w, q_h, k_h, v_h, a_h, args.cpu_tokens)
+        line["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"first {args.cpu_tokens} tokens of all {w.B * w.H} heads, "
+                                          f"fp64 recurrence, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_bf16_h16_t131072_d128")
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--cpu-tokens", type=int, default=16384)
+    ap.add_argument("--ref-tokens", type=int, default=4096)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the dominant kernel, if measured")
+    args = ap.parse_args(argv)
+    from kernelized_causal_sequence_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    if w.kind != "causal":
+        raise SystemExit("bench workloads are causal prefills")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,137 @@
+/*
+ * linattn.h — C ABI of the B200 (sm_100a) kernelized linear-attention library
+ * (liblinattn.so).  Feature map phi(x) = elu(x) + 1, alpha = 1.
+ *
+ * The operations follow:
+ *   - "Linear Attention" knowledge-base page (lizeman.github.io/llm-arch-kb),
+ *     section 2 "Derivation" (state S = sum phi(k) v^T, normaliser
+ *     z = sum phi(k), read-out phi(q)^T S / phi(q)^T z; the causal recurrence)
+ *     and section 3 "Reference implementation" (non-causal sums, the per-token
+ *     causal loop, eps = 1e-6 added to the denominator);
+ *   - the linear-attention concept card (wikillm.com), "Implementation sketch"
+ *     (optional per-token scalar decay: state = a*state + outer(phi(k), v),
+ *     norm = a*norm + phi(k)) and its "Decaying linear attention with a scalar
+ *     state (SSD)" variant (decay 1 is the plain form; chunked algorithm with
+ *     exact products inside each chunk and a recurrence between chunks);
+ *   - the linear-attention lesson (learn.pranaymahendrakar.com), Researcher
+ *     level "Derivation" (o_i over j <= i) and "Implementation reality"
+ *     (chunks of 64 or 128, state propagated across chunks).
+ *
+ * Conventions common to every entry point
+ *   - All tensor pointers are DEVICE pointers to contiguous row-major arrays,
+ *     16-byte aligned.  The caller owns every buffer, including the workspace;
+ *     the library never allocates device memory and never synchronises.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  Every argument error detectable on
+ *     the host is reported before anything is launched, and nothing is then
+ *     written.  A failed launch returns LA_ERR_CUDA.
+ *   - Heads are independent: q, k [B, H, T, d_k], v [B, H, T, d_v],
+ *     out [B, H, T, d_v]; state S [B, H, d_k, d_v] and z [B, H, d_k], fp32.
+ *   - Supported: d_k == d_v in {32, 64, 128}; in_dtype in {F32, BF16, F16};
+ *     out_dtype == in_dtype or LA_F32.  Anything else: LA_ERR_UNSUPPORTED.
+ *   - eps must be finite and >= 0 (it is added to the denominator).
+ *   - decay values must lie in (0, 1]; this is a precondition, not checked
+ *     on the device.  decay == NULL means no decay (a = 1 everywhere).
+ *   - Results are deterministic run to run (no floating-point atomics).
+ */
+#ifndef LINATTN_H
+#define LINATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1, LA_F16 = 2 } la_dtype;
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative size, bad eps, short workspace */
+    LA_ERR_UNSUPPORTED = 2,  /* valid but not implemented: head dim, chunk, dtype combination */
+    LA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    LA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (status word set) */
+} la_status;
+
+/* State handling of the prefill / non-causal calls.
+ *   NONE : start from zeros; state_S/state_z are not read or written (may be NULL).
+ *   OUT  : start from zeros; the final state is written to state_S/state_z.
+ *   INOUT: state_S/state_z hold the initial state and receive the final one
+ *          (in place). */
+typedef enum { LA_STATE_NONE = 0, LA_STATE_OUT = 1, LA_STATE_INOUT = 2 } la_state_mode;
+
+/*
+ * Causal prefill (chunked).  For every head and every token t:
+ *   S_t = a_t S_{t-1} + phi(k_t) v_t^T,   z_t = a_t z_{t-1} + phi(k_t),
+ *   out_t = phi(q_t)^T S_t / (phi(q_t)^T z_t + eps)
+ * computed chunk by chunk: exact masked products inside each chunk of `chunk`
+ * tokens, the (S, z) state carried between chunks (segments of chunks run in
+ * parallel and are joined by a decayed prefix scan over their states).
+ *   q, k       [B, H, T, d_k] in_dtype        v [B, H, T, d_v] in_dtype
+ *   decay      [B, H, T] fp32 in (0, 1], or NULL
+ *   chunk      64 or 128
+ *   out        [B, H, T, d_v] out_dtype
+ *   workspace  device scratch of at least la_prefill_workspace_size(...)
+ *              bytes, 256-byte aligned; contents on entry are ignored.
+ * T == 0 (or B*H == 0) is valid: nothing is computed; with LA_STATE_OUT the
+ * state is set to zero, with LA_STATE_INOUT it is left unchanged.
+ */
+la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                            const float *decay, int B, int H, int T, int d_k, int d_v,
+                            float eps, int chunk, float *state_S, float *state_z,
+                            la_state_mode mode, void *out, la_dtype out_dtype,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace la_prefill_causal needs for these sizes (0 if none). */
+size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chunk);
+
+/*
+ * Non-causal form: every query attends to all Lk keys of its head.
+ *   S = S_in + sum_j phi(k_j) v_j^T,  z = z_in + sum_j phi(k_j)
+ *   out_i = phi(q_i)^T S / (phi(q_i)^T z + eps)
+ * S_in/z_in are zero unless mode == LA_STATE_INOUT.  With OUT or INOUT the
+ * totals S, z are written to state_S/state_z.
+ *   q [B, H, Lq, d_k]; k [B, H, Lk, d_k]; v [B, H, Lk, d_v]; out [B, H, Lq, d_v]
+ *   decay must be NULL (no decayed non-causal form is defined): otherwise
+ *   LA_ERR_UNSUPPORTED.
+ */
+la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                               const float *decay, int B, int H, int Lq, int Lk, int d_k,
+                               int d_v, float eps, float *state_S, float *state_z,
+                               la_state_mode mode, void *out, la_dtype out_dtype,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace la_forward_noncausal needs for these sizes. */
+size_t la_noncausal_workspace_size(int B, int H, int Lk, int d_k, int d_v);
+
+/*
+ * One constant-state decode step per head (the causal loop body once):
+ *   S <- a S + phi(k) v^T,  z <- a z + phi(k),  out = phi(q)^T S / (phi(q)^T z + eps)
+ *   q, k [B, H, d_k] in_dtype; v [B, H, d_v] in_dtype; decay [B, H] fp32 or NULL
+ *   state_S [B, H, d_k, d_v], state_z [B, H, d_k]: fp32, required, updated in place
+ *   out [B, H, d_v] out_dtype
+ */
+la_status la_decode_step(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                         const float *decay, int B, int H, int d_k, int d_v, float eps,
+                         float *state_S, float *state_z, void *out, la_dtype out_dtype,
+                         void *stream);
+
+/* Static description of a status code (never NULL). */
+const char *la_status_string(la_status s);
+
+/* Which kernel family la_prefill_causal / la_forward_noncausal would run for
+ * these arguments: 0 = fp32 CUDA-core (SIMT) kernels, 1 = tcgen05 tensor-core
+ * kernels, -1 = unsupported.  Host-only, launches nothing. */
+int la_prefill_path(la_dtype in_dtype, int d_k, int d_v, int chunk);
+
+/* Number of kernels this library has launched in this process so far, over
+ * all entry points and devices (kernels later replayed from a captured CUDA
+ * graph are counted once, at capture).  Host-only bookkeeping. */
+uint64_t la_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LINATTN_H */

@@ -1,0 +1,176 @@
+"""Python binding of liblinattn.so — B200 (sm_100a) kernelized linear attention
+with the elu(x)+1 feature map.
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  PyTorch provides device memory (outputs, state and
+workspace buffers) and the current CUDA stream.  The binding's functions carry
+the C ABI's names (``include/linattn.h``):
+
+    la_prefill_causal(q, k, v, decay=None, eps=1e-6, chunk=64, ...)
+    la_forward_noncausal(q, k, v, eps=1e-6, ...)
+    la_decode_step(q, k, v, state_S, state_z, decay=None, eps=1e-6, ...)
+
+If the shared library has not been built, importing works but every call
+raises: there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "LinAttnError", "lib", "la_prefill_causal", "la_forward_noncausal", "la_decode_step",
+    "la_prefill_workspace_size", "la_noncausal_workspace_size", "la_status_string",
+    "la_prefill_path", "la_launch_count", "LA_F32", "LA_BF16", "LA_F16", "LA_STATE_NONE", "LA_STATE_OUT",
+    "LA_STATE_INOUT", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblinattn.so")
+
+LA_F32, LA_BF16, LA_F16 = 0, 1, 2
+LA_STATE_NONE, LA_STATE_OUT, LA_STATE_INOUT = 0, 1, 2
+LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+
+_DT = {torch.float32: LA_F32, torch.bfloat16: LA_BF16, torch.float16: LA_F16}
+
+_lib = None
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+
+class LinAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {status}: {la_status_string(status)}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m kernelized_causal_sequence_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.la_prefill_causal.restype = _i
+        L.la_prefill_causal.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _i, _vp,
+                                        _vp, _i, _vp, _i, _vp, _sz, _vp]
+        L.la_prefill_workspace_size.restype = _sz
+        L.la_prefill_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
+        L.la_forward_noncausal.restype = _i
+        L.la_forward_noncausal.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _vp,
+                                           _vp, _i, _vp, _i, _vp, _sz, _vp]
+        L.la_noncausal_workspace_size.restype = _sz
+        L.la_noncausal_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+        L.la_decode_step.restype = _i
+        L.la_decode_step.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp,
+                                     _i, _vp]
+        L.la_status_string.restype = ctypes.c_char_p
+        L.la_status_string.argtypes = [_i]
+        L.la_prefill_path.restype = _i
+        L.la_prefill_path.argtypes = [_i, _i, _i, _i]
+        L.la_launch_count.restype = ctypes.c_uint64
+        L.la_launch_count.argtypes = []
+        _lib = L
+    return _lib
+
+
+def la_launch_count() -> int:
+    return int(lib().la_launch_count())
+
+
+def la_status_string(status: int) -> str:
+    return lib().la_status_string(int(status)).decode()
+
+
+def la_prefill_workspace_size(B, H, T, d_k, d_v, chunk) -> int:
+    return int(lib().la_prefill_workspace_size(B, H, T, d_k, d_v, chunk))
+
+
+def la_noncausal_workspace_size(B, H, Lk, d_k, d_v) -> int:
+    return int(lib().la_noncausal_workspace_size(B, H, Lk, d_k, d_v))
+
+
+def la_prefill_path(in_dtype, d_k, d_v, chunk) -> int:
+    if isinstance(in_dtype, torch.dtype):
+        in_dtype = _DT[in_dtype]
+    return int(lib().la_prefill_path(in_dtype, d_k, d_v, chunk))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, st):
+    if st != LA_OK:
+        raise LinAttnError(fn, st)
+
+
+def _workspace(nbytes, device):
+    # 256-byte aligned by the caching allocator
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def la_prefill_causal(q, k, v, decay=None, eps=1e-6, chunk=64, state_S=None, state_z=None,
+                      mode=None, out=None, out_dtype=None, workspace=None, stream=None):
+    """Causal chunked prefill.  q, k: [B,H,T,d_k]; v: [B,H,T,d_v] (f32/bf16/f16, CUDA,
+    contiguous); decay: [B,H,T] fp32 or None.  state_S [B,H,d_k,d_v] / state_z [B,H,d_k]
+    fp32 with ``mode`` LA_STATE_NONE/OUT/INOUT (default: OUT if given, else NONE).
+    Returns ``out`` [B,H,T,d_v]."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
+    if mode is None:
+        mode = LA_STATE_OUT if state_S is not None else LA_STATE_NONE
+    if workspace is None:
+        workspace = _workspace(la_prefill_workspace_size(B, H, T, dk, dv, chunk), q.device)
+    st = lib().la_prefill_causal(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(decay), B, H, T,
+                                 dk, dv, float(eps), int(chunk), _ptr(state_S), _ptr(state_z),
+                                 int(mode), _ptr(out), _DT[out.dtype], _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("la_prefill_causal", st)
+    return out
+
+
+def la_forward_noncausal(q, k, v, eps=1e-6, state_S=None, state_z=None, mode=None, out=None,
+                         out_dtype=None, workspace=None, stream=None, decay=None):
+    """Non-causal form.  q: [B,H,Lq,d_k]; k: [B,H,Lk,d_k]; v: [B,H,Lk,d_v]."""
+    B, H, Lq, dk = q.shape
+    Lk, dv = v.shape[2], v.shape[3]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((B, H, Lq, dv), dtype=out_dtype, device=q.device)
+    if mode is None:
+        mode = LA_STATE_OUT if state_S is not None else LA_STATE_NONE
+    if workspace is None:
+        workspace = _workspace(la_noncausal_workspace_size(B, H, Lk, dk, dv), q.device)
+    st = lib().la_forward_noncausal(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(decay), B, H,
+                                    Lq, Lk, dk, dv, float(eps), _ptr(state_S), _ptr(state_z),
+                                    int(mode), _ptr(out), _DT[out.dtype], _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("la_forward_noncausal", st)
+    return out
+
+
+def la_decode_step(q, k, v, state_S, state_z, decay=None, eps=1e-6, out=None, out_dtype=None,
+                   stream=None):
+    """One decode step; q, k: [B,H,d_k]; v: [B,H,d_v]; state updated in place."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=out_dtype, device=q.device)
+    st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(decay), B, H, dk, dv,
+                              float(eps), _ptr(state_S), _ptr(state_z), _ptr(out), _DT[out.dtype],
+                              _stream(stream))
+    _check("la_decode_step", st)
+    return out

@@ -1,0 +1,60 @@
+// common.cuh — element conversions, the feature map and small device helpers
+// shared by the library's kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace la {
+
+using bf16 = __nv_bfloat16;
+using f16 = __half;
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<bf16>(bf16 x) { return __bfloat162float(x); }
+template <> __device__ __forceinline__ float to_f32<f16>(f16 x) { return __half2float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
+template <> __device__ __forceinline__ f16 from_f32<f16>(float x) { return __float2half_rn(x); }
+
+// phi(x) = elu(x) + 1 (alpha = 1): x + 1 for x > 0, and e^x for x <= 0, which
+// equals (e^x - 1) + 1 without the cancellation.  ("Transformers are RNNs"
+// feature map, as given on the knowledge-base page, section 2, "Choice of phi".)
+__device__ __forceinline__ float phi_precise(float x) { return x > 0.f ? x + 1.f : expf(x); }
+__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+// Inclusive warp scan of the pair operator (a1, x1) o (a2, x2) = (a1 a2, a2 x1 + x2),
+// which composes the affine maps X -> a X + x of consecutive segments.
+__device__ __forceinline__ void warp_affine_scan(float &a, float &x, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        float a_up = __shfl_up_sync(0xffffffffu, a, off);
+        float x_up = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) {
+            x = fmaf(a, x_up, x);
+            a = a * a_up;
+        }
+    }
+}
+
+// Inclusive warp sum scan.
+__device__ __forceinline__ float warp_sum_scan(float x, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        float up = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += up;
+    }
+    return x;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+}  // namespace la

@@ -1,0 +1,330 @@
+// linattn_api.cu — the C ABI declared in include/linattn.h: argument checks,
+// the segment plan, workspace layout and kernel dispatch.  Every entry point
+// validates on the host first and launches nothing on error.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/linattn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "plan.h"
+#include "simt_kernels.cuh"
+#include "tc_launch.h"
+
+using namespace la;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+inline bool dtype_ok(la_dtype t) { return t == LA_F32 || t == LA_BF16 || t == LA_F16; }
+
+// Workspace layout of the segment-scan paths:
+//   [ws_state: BH * n_seg * (D*D + D) fp32][ws_A: BH * n_seg fp32][ws_total: BH * (D*D + D) fp32]
+struct WsLayout {
+    size_t state_off, A_off, total_off, bytes;
+};
+
+WsLayout ws_layout(long BH, int n_seg, int D, bool with_total) {
+    WsLayout w;
+    const size_t E = (size_t)D * D + D;
+    w.state_off = 0;
+    w.A_off = align_up(w.state_off + sizeof(float) * (size_t)BH * n_seg * E);
+    w.total_off = align_up(w.A_off + sizeof(float) * (size_t)BH * n_seg);
+    w.bytes = with_total ? align_up(w.total_off + sizeof(float) * (size_t)BH * E) : w.total_off;
+    return w;
+}
+
+// Per-(kernel, device) opt-in to large dynamic shared memory.
+template <typename K> cudaError_t allow_smem(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+la_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
+
+}  // namespace
+
+namespace la {
+std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace la
+
+namespace {
+
+// ---------------------------------------------------------------- SIMT path
+template <typename InT, typename OutT, int D>
+la_status simt_causal(SimtParams p, cudaStream_t st) {
+    const int E = D * D + D;
+    {
+        auto k1 = simt_segment_state_kernel<InT, D>;
+        const size_t sm = simt_state_smem<D>();
+        if (allow_smem(k1, sm) != cudaSuccess) return LA_ERR_CUDA;
+        k1<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p, p.T);
+    }
+    {
+        const float *sin_S = p.mode == LA_STATE_INOUT ? p.state_S : nullptr;
+        const float *sin_z = p.mode == LA_STATE_INOUT ? p.state_z : nullptr;
+        float *sout_S = p.mode != LA_STATE_NONE ? p.state_S : nullptr;
+        float *sout_z = p.mode != LA_STATE_NONE ? p.state_z : nullptr;
+        segment_scan_kernel<<<dim3((E + 31) / 32, p.BH), 256, 0, st>>>(
+            p.ws_state, p.ws_A, p.n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, nullptr);
+    }
+    {
+        auto k3 = simt_chunk_output_kernel<InT, OutT, D>;
+        const size_t sm = simt_output_smem<D>();
+        if (allow_smem(k3, sm) != cudaSuccess) return LA_ERR_CUDA;
+        k3<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p);
+    }
+    count_launches(3);
+    return cuda_status(cudaGetLastError());
+}
+
+template <typename InT, typename OutT, int D>
+la_status simt_noncausal(SimtParams p, int Lk, cudaStream_t st) {
+    const int E = D * D + D;
+    {
+        auto k1 = simt_segment_state_kernel<InT, D>;
+        const size_t sm = simt_state_smem<D>();
+        if (allow_smem(k1, sm) != cudaSuccess) return LA_ERR_CUDA;
+        k1<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p, Lk);
+    }
+    {
+        const float *sin_S = p.mode == LA_STATE_INOUT ? p.state_S : nullptr;
+        const float *sin_z = p.mode == LA_STATE_INOUT ? p.state_z : nullptr;
+        float *sout_S = p.mode != LA_STATE_NONE ? p.state_S : nullptr;
+        float *sout_z = p.mode != LA_STATE_NONE ? p.state_z : nullptr;
+        segment_scan_kernel<<<dim3((E + 31) / 32, p.BH), 256, 0, st>>>(
+            p.ws_state, p.ws_A, p.n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, p.ws_total);
+    }
+    if (p.Lq > 0) {
+        auto k3 = simt_noncausal_readout_kernel<InT, OutT, D>;
+        const size_t sm = simt_readout_smem<D>();
+        if (allow_smem(k3, sm) != cudaSuccess) return LA_ERR_CUDA;
+        k3<<<dim3((p.Lq + kReadoutQueries - 1) / kReadoutQueries, p.BH), kSimtThreads, sm, st>>>(p);
+        count_launches(1);
+    }
+    count_launches(2);
+    return cuda_status(cudaGetLastError());
+}
+
+// Dispatch over (in dtype, out dtype, head dim) for a functor template F.
+template <template <typename, typename, int> class F, typename... Args>
+la_status dispatch3(la_dtype in, la_dtype out, int D, Args... args) {
+#define LA_DISPATCH_D(IT, OT)                                       \
+    switch (D) {                                                    \
+        case 32: return F<IT, OT, 32>::run(args...);                \
+        case 64: return F<IT, OT, 64>::run(args...);                \
+        case 128: return F<IT, OT, 128>::run(args...);              \
+        default: return LA_ERR_UNSUPPORTED;                         \
+    }
+    if (in == LA_F32) { LA_DISPATCH_D(float, float) }
+    if (in == LA_BF16) {
+        if (out == LA_BF16) { LA_DISPATCH_D(bf16, bf16) }
+        LA_DISPATCH_D(bf16, float)
+    }
+    if (in == LA_F16) {
+        if (out == LA_F16) { LA_DISPATCH_D(f16, f16) }
+        LA_DISPATCH_D(f16, float)
+    }
+#undef LA_DISPATCH_D
+    return LA_ERR_UNSUPPORTED;
+}
+
+template <typename IT, typename OT, int D> struct SimtCausalF {
+    static la_status run(SimtParams p, cudaStream_t st) { return simt_causal<IT, OT, D>(p, st); }
+};
+template <typename IT, typename OT, int D> struct SimtNoncausalF {
+    static la_status run(SimtParams p, int Lk, cudaStream_t st) {
+        return simt_noncausal<IT, OT, D>(p, Lk, st);
+    }
+};
+template <typename IT, typename OT, int D> struct DecodeF {
+    static la_status run(const void *q, const void *k, const void *v, const float *decay,
+                         float eps, float *S, float *z, void *out, long BH, cudaStream_t st) {
+        decode_step_kernel<IT, OT, D><<<(unsigned)BH, kDecodeThreads, 0, st>>>(
+            (const IT *)q, (const IT *)k, (const IT *)v, decay, eps, S, z, (OT *)out);
+        count_launches(1);
+        return cuda_status(cudaGetLastError());
+    }
+};
+
+// Shared host-side checks.  Returns LA_OK when the call may proceed.
+la_status check_common(la_dtype in, la_dtype out, int d_k, int d_v, float eps) {
+    if (!dtype_ok(in) || !dtype_ok(out)) return LA_ERR_INVALID_ARG;
+    if (!(std::isfinite(eps) && eps >= 0.f)) return LA_ERR_INVALID_ARG;
+    if (d_k <= 0 || d_v <= 0) return LA_ERR_INVALID_ARG;
+    if (d_k != d_v || !dim_ok(d_k)) return LA_ERR_UNSUPPORTED;
+    if (!(out == in || out == LA_F32)) return LA_ERR_UNSUPPORTED;
+    return LA_OK;
+}
+
+la_status check_state(la_state_mode mode, const float *S, const float *z) {
+    if (mode != LA_STATE_NONE && mode != LA_STATE_OUT && mode != LA_STATE_INOUT)
+        return LA_ERR_INVALID_ARG;
+    if (mode != LA_STATE_NONE && (!S || !z || !aligned16(S) || !aligned16(z)))
+        return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+uint64_t la_launch_count(void) { return la::g_launches.load(std::memory_order_relaxed); }
+
+const char *la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "LA_OK: success";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: unsupported size, chunk or dtype";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA runtime or launch error";
+        case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT: bounded device wait expired";
+        default: return "unknown la_status";
+    }
+}
+
+int la_prefill_path(la_dtype in_dtype, int d_k, int d_v, int chunk) {
+    if (!dtype_ok(in_dtype) || d_k != d_v || !dim_ok(d_k) || (chunk != 64 && chunk != 128))
+        return -1;
+    return tc_supported(in_dtype, d_k, chunk) ? 1 : 0;
+}
+
+size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chunk) {
+    if (B <= 0 || H <= 0 || T <= 0 || d_k != d_v || !dim_ok(d_k) || (chunk != 64 && chunk != 128))
+        return 0;
+    const long BH = (long)B * H;
+    const Plan pl = make_plan(BH, T, chunk, d_k);
+    return ws_layout(BH, pl.n_seg, d_k, false).bytes;
+}
+
+size_t la_noncausal_workspace_size(int B, int H, int Lk, int d_k, int d_v) {
+    if (B <= 0 || H <= 0 || Lk < 0 || d_k != d_v || !dim_ok(d_k)) return 0;
+    const long BH = (long)B * H;
+    const Plan pl = make_plan(BH, Lk > 0 ? Lk : 1, kNoncausalChunk, d_k);
+    return ws_layout(BH, pl.n_seg, d_k, true).bytes;
+}
+
+la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                            const float *decay, int B, int H, int T, int d_k, int d_v, float eps,
+                            int chunk, float *state_S, float *state_z, la_state_mode mode,
+                            void *out, la_dtype out_dtype, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0 || T < 0) return LA_ERR_INVALID_ARG;
+    if (chunk != 64 && chunk != 128) return LA_ERR_UNSUPPORTED;
+    if ((s = check_state(mode, state_S, state_z)) != LA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    const long BH = (long)B * H;
+    if (BH == 0) return LA_OK;
+    if (T == 0) {
+        if (mode == LA_STATE_OUT) {
+            if (cudaMemsetAsync(state_S, 0, sizeof(float) * BH * d_k * d_v, st) != cudaSuccess ||
+                cudaMemsetAsync(state_z, 0, sizeof(float) * BH * d_k, st) != cudaSuccess)
+                return LA_ERR_CUDA;
+        }
+        return LA_OK;
+    }
+    if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    if (decay && !aligned16(decay)) return LA_ERR_INVALID_ARG;
+    if (BH > 65535L * 1024L || (double)BH * T * d_k > 9.0e18) return LA_ERR_UNSUPPORTED;
+    const Plan pl = make_plan(BH, T, chunk, d_k);
+    const WsLayout wl = ws_layout(BH, pl.n_seg, d_k, false);
+    if (!workspace || workspace_bytes < wl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return LA_ERR_INVALID_ARG;
+    char *ws = (char *)workspace;
+
+    if (tc_supported(in_dtype, d_k, chunk)) {
+        TcCausalArgs a;
+        a.q = q; a.k = k; a.v = v; a.decay = decay; a.out = out;
+        a.in_dtype = in_dtype; a.out_dtype = out_dtype;
+        a.ws_state = (float *)(ws + wl.state_off);
+        a.ws_A = (float *)(ws + wl.A_off);
+        a.state_S = state_S; a.state_z = state_z; a.mode = mode;
+        a.BH = BH; a.T = T; a.D = d_k; a.chunk = chunk; a.seg_len = pl.seg_len;
+        a.n_seg = pl.n_seg; a.eps = eps;
+        return tc_causal(a, st);
+    }
+    SimtParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k; p.v = v; p.decay = decay; p.out = out;
+    p.ws_state = (float *)(ws + wl.state_off);
+    p.ws_A = (float *)(ws + wl.A_off);
+    p.ws_total = nullptr;
+    p.state_S = state_S; p.state_z = state_z; p.mode = mode;
+    p.BH = (int)BH; p.T = T; p.Lq = T; p.chunk = chunk; p.seg_len = pl.seg_len; p.n_seg = pl.n_seg;
+    p.eps = eps;
+    return dispatch3<SimtCausalF>(in_dtype, out_dtype, d_k, p, st);
+}
+
+la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                               const float *decay, int B, int H, int Lq, int Lk, int d_k, int d_v,
+                               float eps, float *state_S, float *state_z, la_state_mode mode,
+                               void *out, la_dtype out_dtype, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return LA_ERR_INVALID_ARG;
+    if (decay) return LA_ERR_UNSUPPORTED;
+    if ((s = check_state(mode, state_S, state_z)) != LA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    const long BH = (long)B * H;
+    if (BH == 0) return LA_OK;
+    if (Lq > 0 && (!q || !out || !aligned16(q) || !aligned16(out))) return LA_ERR_INVALID_ARG;
+    if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return LA_ERR_INVALID_ARG;
+    if (BH > 65535L * 1024L) return LA_ERR_UNSUPPORTED;
+    const Plan pl = make_plan(BH, Lk > 0 ? Lk : 1, kNoncausalChunk, d_k);
+    const WsLayout wl = ws_layout(BH, pl.n_seg, d_k, true);
+    if (!workspace || workspace_bytes < wl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return LA_ERR_INVALID_ARG;
+    char *ws = (char *)workspace;
+
+    if (tc_noncausal_supported(in_dtype, d_k)) {
+        TcNoncausalArgs a;
+        a.q = q; a.k = k; a.v = v; a.out = out;
+        a.in_dtype = in_dtype; a.out_dtype = out_dtype;
+        a.ws_state = (float *)(ws + wl.state_off);
+        a.ws_A = (float *)(ws + wl.A_off);
+        a.ws_total = (float *)(ws + wl.total_off);
+        a.state_S = state_S; a.state_z = state_z; a.mode = mode;
+        a.BH = BH; a.Lq = Lq; a.Lk = Lk; a.D = d_k; a.seg_len = pl.seg_len; a.n_seg = pl.n_seg;
+        a.eps = eps;
+        return tc_noncausal(a, st);
+    }
+    SimtParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k; p.v = v; p.decay = nullptr; p.out = out;
+    p.ws_state = (float *)(ws + wl.state_off);
+    p.ws_A = (float *)(ws + wl.A_off);
+    p.ws_total = (float *)(ws + wl.total_off);
+    p.state_S = state_S; p.state_z = state_z; p.mode = mode;
+    p.BH = (int)BH; p.T = Lk; p.Lq = Lq; p.chunk = kNoncausalChunk; p.seg_len = pl.seg_len;
+    p.n_seg = pl.n_seg; p.eps = eps;
+    return dispatch3<SimtNoncausalF>(in_dtype, out_dtype, d_k, p, Lk, st);
+}
+
+la_status la_decode_step(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                         const float *decay, int B, int H, int d_k, int d_v, float eps,
+                         float *state_S, float *state_z, void *out, la_dtype out_dtype,
+                         void *stream) {
+    la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0) return LA_ERR_INVALID_ARG;
+    const long BH = (long)B * H;
+    if (BH == 0) return LA_OK;
+    if (!q || !k || !v || !out || !state_S || !state_z) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(state_S) || !aligned16(state_z) || (decay && !aligned16(decay)))
+        return LA_ERR_INVALID_ARG;
+    if (BH > 0x7fffffffL) return LA_ERR_UNSUPPORTED;
+    return dispatch3<DecodeF>(in_dtype, out_dtype, d_k, q, k, v, decay, eps, state_S, state_z, out,
+                              BH, (cudaStream_t)stream);
+}
+
+}  // extern "C"

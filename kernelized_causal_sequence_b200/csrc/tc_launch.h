@@ -1,0 +1,41 @@
+// tc_launch.h — host entry points of the tcgen05 (tensor-core) kernels.
+#pragma once
+#include <cuda_runtime.h>
+
+#include "../../include/linattn.h"
+
+namespace la {
+
+struct TcCausalArgs {
+    const void *q, *k, *v;
+    const float *decay;
+    void *out;
+    la_dtype in_dtype, out_dtype;
+    float *ws_state, *ws_A;
+    float *state_S, *state_z;
+    la_state_mode mode;
+    long BH;
+    int T, D, chunk, seg_len, n_seg;
+    float eps;
+};
+
+struct TcNoncausalArgs {
+    const void *q, *k, *v;
+    void *out;
+    la_dtype in_dtype, out_dtype;
+    float *ws_state, *ws_A, *ws_total;
+    float *state_S, *state_z;
+    la_state_mode mode;
+    long BH;
+    int Lq, Lk, D, seg_len, n_seg;
+    float eps;
+};
+
+void count_launches(int n);  // process-wide kernel launch counter (la_launch_count)
+
+bool tc_supported(la_dtype in_dtype, int D, int chunk);
+bool tc_noncausal_supported(la_dtype in_dtype, int D);
+la_status tc_causal(const TcCausalArgs &a, cudaStream_t st);
+la_status tc_noncausal(const TcNoncausalArgs &a, cudaStream_t st);
+
+}  // namespace la

@@ -1,0 +1,253 @@
+"""CUDA path vs the fp64 oracle, element by element, on the same seeded inputs.
+
+Bar: max over output rows of ||o_gpu - o_ref||_inf / ||o_ref||_inf below
+1e-4 for fp32 inputs and 2e-2 for bf16/fp16 inputs (fp32 state).  Full-size
+workloads run on the GPU exactly as the bench launches them; where the
+oracle would take too long, whole heads are sampled (heads are independent,
+so a sampled head's reference is exact).
+"""
+import numpy as np
+import pytest
+import torch
+
+from kernelized_causal_sequence_b200 import inputs
+from tests.conftest import row_rel_err, tol_for
+
+pytestmark = pytest.mark.gpu
+W = inputs.WORKLOADS
+DEV = "cuda"
+
+
+def gpu_prefill(la, q, k, v, decay, chunk, out_dtype, S_in=None, z_in=None, eps=1e-6):
+    B, H, T, d = q.shape
+    qd, kd, vd = (x.to(DEV) for x in (q, k, v))
+    ad = None if decay is None else decay.to(DEV)
+    S = torch.zeros((B, H, d, d), dtype=torch.float32, device=DEV)
+    z = torch.zeros((B, H, d), dtype=torch.float32, device=DEV)
+    mode = la.LA_STATE_OUT
+    if S_in is not None:
+        S.copy_(S_in)
+        z.copy_(z_in)
+        mode = la.LA_STATE_INOUT
+    out = la.la_prefill_causal(qd, kd, vd, decay=ad, eps=eps, chunk=chunk, state_S=S, state_z=z,
+                               mode=mode, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), S.cpu().numpy(), z.cpu().numpy()
+
+
+def check_prefill(la, orc, q, k, v, decay, chunk, out_dtype, tol, S_in=None, z_in=None):
+    o, S, z = gpu_prefill(la, q, k, v, decay, chunk, out_dtype, S_in, z_in)
+    ro, rS, rz = orc.causal(q, k, v, decay, 1e-6, S_in, z_in)
+    err = row_rel_err(o, ro)
+    assert err < tol, f"output rel err {err}"
+    assert row_rel_err(S.reshape(S.shape[0], S.shape[1], -1),
+                       rS.reshape(rS.shape[0], rS.shape[1], -1)) < tol
+    assert row_rel_err(z, rz) < tol
+    return err
+
+
+# --------------------------------------------------------------- small cases
+SMALL = [
+    # (dtype, d, T, chunk, decay, B, H)
+    (torch.float32, 64, 1, 64, False, 1, 1),
+    (torch.float32, 32, 65, 64, False, 2, 3),
+    (torch.float32, 128, 200, 128, True, 1, 2),
+    (torch.float32, 64, 1000, 64, True, 1, 2),
+    (torch.bfloat16, 64, 63, 64, False, 2, 2),
+    (torch.bfloat16, 64, 777, 64, True, 1, 3),
+    (torch.bfloat16, 128, 129, 128, False, 1, 2),
+    (torch.bfloat16, 128, 1500, 64, True, 2, 1),
+    (torch.bfloat16, 128, 3000, 128, False, 1, 2),
+    (torch.float16, 32, 300, 128, False, 2, 2),
+    (torch.float16, 128, 513, 64, True, 1, 2),
+]
+
+
+def _small_inputs(dtype, d, T, decay, B, H, seed):
+    rng = np.random.default_rng(seed)
+    s = 1.0 / np.sqrt(d)
+    mk = lambda: torch.from_numpy((rng.standard_normal((B, H, T, d), dtype=np.float32) * s)).to(dtype)
+    q, k, v = mk(), mk(), mk()
+    a = None
+    if decay:
+        g = rng.standard_normal((B, H, T), dtype=np.float32) + 2.0
+        a = torch.from_numpy((1.0 / (1.0 + np.exp(-g))).astype(np.float32))
+    return q, k, v, a
+
+
+@pytest.mark.parametrize("dtype,d,T,chunk,decay,B,H", SMALL)
+def test_prefill_small(la, orc, dtype, d, T, chunk, decay, B, H):
+    q, k, v, a = _small_inputs(dtype, d, T, decay, B, H, seed=T * 7 + d)
+    check_prefill(la, orc, q, k, v, a, chunk, torch.float32, tol_for(dtype))
+    if dtype != torch.float32:
+        check_prefill(la, orc, q, k, v, a, chunk, dtype, tol_for(dtype))
+
+
+def test_prefill_state_inout_and_split(la, orc):
+    dtype, d, T1, T2 = torch.bfloat16, 64, 300, 457
+    q, k, v, a = _small_inputs(dtype, d, T1 + T2, True, 2, 2, seed=5)
+    o_full, S_full, z_full = gpu_prefill(la, q, k, v, a, 64, torch.float32)
+    o1, S1, z1 = gpu_prefill(la, q[:, :, :T1], k[:, :, :T1], v[:, :, :T1], a[:, :, :T1], 64,
+                             torch.float32)
+    o2, S2, z2 = gpu_prefill(la, q[:, :, T1:], k[:, :, T1:], v[:, :, T1:], a[:, :, T1:], 64,
+                             torch.float32, S_in=torch.from_numpy(S1).to(DEV),
+                             z_in=torch.from_numpy(z1).to(DEV))
+    ro, rS, rz = orc.causal(q, k, v, a)
+    assert row_rel_err(np.concatenate([o1, o2], 2), ro) < 2e-2
+    assert row_rel_err(S2.reshape(2, 2, -1), rS.reshape(2, 2, -1)) < 2e-2
+    assert row_rel_err(o_full, ro) < 2e-2
+
+
+def test_decay_one_matches_no_decay_bitwise(la):
+    q, k, v, _ = _small_inputs(torch.bfloat16, 128, 1000, False, 1, 2, seed=9)
+    ones = torch.ones((1, 2, 1000), dtype=torch.float32)
+    o1, S1, _ = gpu_prefill(la, q, k, v, None, 64, torch.float32)
+    o2, S2, _ = gpu_prefill(la, q, k, v, ones, 64, torch.float32)
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
+
+
+def test_prefill_deterministic(la):
+    q, k, v, a = _small_inputs(torch.bfloat16, 128, 4096, True, 1, 4, seed=10)
+    o1, S1, _ = gpu_prefill(la, q, k, v, a, 64, torch.bfloat16)
+    o2, S2, _ = gpu_prefill(la, q, k, v, a, 64, torch.bfloat16)
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
+
+
+def test_chunk_64_vs_128_agree(la):
+    q, k, v, _ = _small_inputs(torch.bfloat16, 128, 2000, False, 1, 2, seed=11)
+    o1, _, _ = gpu_prefill(la, q, k, v, None, 64, torch.float32)
+    o2, _, _ = gpu_prefill(la, q, k, v, None, 128, torch.float32)
+    assert row_rel_err(o1, o2) < 2e-2
+
+
+def test_empty_and_state_only(la):
+    q = torch.empty((2, 2, 0, 64), dtype=torch.bfloat16, device=DEV)
+    S = torch.full((2, 2, 64, 64), 3.0, device=DEV)
+    z = torch.full((2, 2, 64), 3.0, device=DEV)
+    la.la_prefill_causal(q, q, q, state_S=S, state_z=z, mode=la.LA_STATE_OUT)
+    torch.cuda.synchronize()
+    assert float(S.abs().max()) == 0.0 and float(z.abs().max()) == 0.0
+    S.fill_(2.0)
+    la.la_prefill_causal(q, q, q, state_S=S, state_z=z, mode=la.LA_STATE_INOUT)
+    torch.cuda.synchronize()
+    assert float(S.min()) == 2.0
+
+
+# -------------------------------------------------------- full-size workloads
+def test_workload_causal_f32(la, orc):
+    w = W["causal_f32_t256_d64"]
+    q, k, v, a = inputs.qkv(w)
+    err = check_prefill(la, orc, q, k, v, a, w.chunk, w.torch_out_dtype, 1e-4)
+    assert err < 1e-4
+
+
+def test_workload_causal_bf16(la, orc):
+    w = W["causal_bf16_b4h8_t2048_d64"]
+    q, k, v, a = inputs.qkv(w)
+    check_prefill(la, orc, q, k, v, a, w.chunk, w.torch_out_dtype, 2e-2)
+
+
+def _sampled_heads(la, orc, w, heads):
+    q, k, v, a = inputs.qkv(w)
+    o, S, z = gpu_prefill(la, q, k, v, a, w.chunk, w.torch_out_dtype)
+    for (b, h) in heads:
+        sl = lambda x: None if x is None else x[b:b + 1, h:h + 1]
+        ro, rS, rz = orc.causal(sl(q), sl(k), sl(v), sl(a))
+        assert row_rel_err(o[b:b + 1, h:h + 1], ro) < 2e-2
+        assert row_rel_err(S[b:b + 1, h:h + 1].reshape(1, 1, -1), rS.reshape(1, 1, -1)) < 2e-2
+        assert row_rel_err(z[b:b + 1, h:h + 1], rz) < 2e-2
+
+
+def test_workload_ssd_decay(la, orc):
+    w = W["ssd_decay_bf16_b2h16_t8192_d128"]
+    _sampled_heads(la, orc, w, [(0, 0), (1, 15), (0, 7)])
+
+
+def test_workload_long_prefill(la, orc):
+    w = W["prefill_bf16_h16_t131072_d128"]
+    _sampled_heads(la, orc, w, [(0, 0), (0, 11)])
+
+
+@pytest.mark.parametrize("cross", [False, True])
+def test_workload_noncausal(la, orc, cross):
+    w = W["noncausal_f16_b8h8_l4800_d32"]
+    q, k, v, _ = inputs.qkv(w)
+    if cross:
+        k, v = inputs.cross_kv(w)
+    S = torch.zeros((w.B, w.H, w.d, w.d), device=DEV)
+    z = torch.zeros((w.B, w.H, w.d), device=DEV)
+    o = la.la_forward_noncausal(q.to(DEV), k.to(DEV), v.to(DEV), state_S=S, state_z=z,
+                                out_dtype=w.torch_out_dtype)
+    torch.cuda.synchronize()
+    ro, rS, rz = orc.noncausal(q, k, v)
+    assert row_rel_err(o.cpu().numpy(), ro) < 2e-2
+    assert row_rel_err(S.cpu().numpy().reshape(w.B, w.H, -1), rS.reshape(w.B, w.H, -1)) < 2e-2
+
+
+@pytest.mark.parametrize("dtype,d,Lq,Lk", [(torch.float32, 64, 100, 333), (torch.bfloat16, 128, 17, 1000),
+                                           (torch.float16, 32, 129, 0), (torch.bfloat16, 64, 0, 50)])
+def test_noncausal_small(la, orc, dtype, d, Lq, Lk):
+    rng = np.random.default_rng(Lq + Lk)
+    mk = lambda L: torch.from_numpy(rng.standard_normal((2, 3, L, d), dtype=np.float32)).to(dtype)
+    q, k, v = mk(Lq), mk(Lk), mk(Lk)
+    S0 = torch.from_numpy(rng.standard_normal((2, 3, d, d), dtype=np.float32))
+    z0 = torch.from_numpy(np.abs(rng.standard_normal((2, 3, d), dtype=np.float32)) + 1.0)
+    S = S0.to(DEV).clone()
+    z = z0.to(DEV).clone()
+    o = la.la_forward_noncausal(q.to(DEV), k.to(DEV), v.to(DEV), state_S=S, state_z=z,
+                                mode=la.LA_STATE_INOUT, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ro, rS, rz = orc.noncausal(q, k, v, S_in=S0, z_in=z0)
+    tol = tol_for(dtype)
+    if Lq:
+        assert row_rel_err(o.cpu().numpy(), ro) < tol
+    assert row_rel_err(S.cpu().numpy().reshape(2, 3, -1), rS.reshape(2, 3, -1)) < tol
+
+
+@pytest.mark.parametrize("dtype,d,decay", [(torch.float32, 64, False), (torch.bfloat16, 128, True),
+                                           (torch.float16, 32, True), (torch.bfloat16, 64, False)])
+def test_decode_small(la, orc, dtype, d, decay):
+    rng = np.random.default_rng(d)
+    B, H = 3, 5
+    S0 = torch.from_numpy(rng.standard_normal((B, H, d, d), dtype=np.float32))
+    z0 = torch.from_numpy(np.abs(rng.standard_normal((B, H, d), dtype=np.float32)) * 10 + 1)
+    S, z = S0.to(DEV).clone(), z0.to(DEV).clone()
+    rS, rz = S0.double().numpy(), z0.double().numpy()
+    for step in range(5):
+        mk = lambda: torch.from_numpy(rng.standard_normal((B, H, d), dtype=np.float32)).to(dtype)
+        q, k, v = mk(), mk(), mk()
+        a = torch.from_numpy(rng.uniform(0.5, 1.0, (B, H)).astype(np.float32)) if decay else None
+        o = la.la_decode_step(q.to(DEV), k.to(DEV), v.to(DEV), S, z,
+                              decay=None if a is None else a.to(DEV), out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        ro, rS, rz = orc.decode_step(q, k, v, rS, rz, decay=a)
+        tol = tol_for(dtype)
+        assert row_rel_err(o.cpu().numpy(), ro) < tol
+        assert row_rel_err(S.cpu().numpy().reshape(B, H, -1), rS.reshape(B, H, -1)) < tol
+
+
+def test_workload_decode(la, orc):
+    w = W["decode_bf16_b64h16_d128"]
+    S0, z0 = inputs.decode_state(w)
+    S, z = S0.to(DEV).clone(), z0.to(DEV).clone()
+    rS, rz = S0.double().numpy(), z0.double().numpy()
+    for step in range(6):
+        q, k, v, _ = inputs.decode_inputs(w, step)
+        o = la.la_decode_step(q.to(DEV), k.to(DEV), v.to(DEV), S, z, out_dtype=w.torch_out_dtype)
+        torch.cuda.synchronize()
+        ro, rS, rz = orc.decode_step(q, k, v, rS, rz)
+        assert row_rel_err(o.float().cpu().numpy(), ro) < 2e-2
+    assert row_rel_err(S.cpu().numpy().reshape(w.B, w.H, -1), rS.reshape(w.B, w.H, -1)) < 2e-2
+
+
+def test_prefill_then_decode_is_prefill_plus_one(la, orc):
+    q, k, v, a = _small_inputs(torch.bfloat16, 128, 513, True, 2, 2, seed=12)
+    T = 512
+    _, S, z = gpu_prefill(la, q[:, :, :T], k[:, :, :T], v[:, :, :T], a[:, :, :T], 128,
+                          torch.float32)
+    Sd, zd = torch.from_numpy(S).to(DEV), torch.from_numpy(z).to(DEV)
+    o = la.la_decode_step(q[:, :, T].to(DEV), k[:, :, T].to(DEV), v[:, :, T].to(DEV), Sd, zd,
+                          decay=a[:, :, T].to(DEV), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ro, _, _ = orc.causal(q, k, v, a)
+    assert row_rel_err(o.cpu().numpy(), ro[:, :, T]) < 2e-2
