@@ -86,6 +86,38 @@ la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtyp
 /* Bytes of workspace la_prefill_causal needs for these sizes (0 if none). */
 size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chunk);
 
+/* Size of the device scratch array behind la_prefill_causal_noalloc. */
+#define LA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * la_prefill_causal_noalloc — la_prefill_causal without a workspace argument.
+ * The pages have no counterpart: this exists for callers that cannot allocate
+ * device memory at all, such as a plugin hosted by a runtime that owns every
+ * device allocation, or a process that forbids allocation after start-up
+ * (fixed-budget serving, real-time deployments).
+ *
+ * The scratch (per-segment states) lives in a fixed array of
+ * LA_NOALLOC_SCRATCH_BYTES inside the library's device memory; every GPU that
+ * loads the library holds it until the process exits.  The caller still
+ * passes inputs, outputs and state exactly as for la_prefill_causal, and gets
+ * the same results.  The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *   - Sizes whose la_prefill_workspace_size exceeds LA_NOALLOC_SCRATCH_BYTES
+ *     return LA_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make that
+ *     first call before any stream capture.  LA_ERR_CUDA if the lookup fails.
+ *   - All calls share the one array, which keeps the last call's contents;
+ *     nothing in it needs to start at zero (every entry is written before it
+ *     is read).  Calls that overlap on the GPU (e.g. on two streams at once)
+ *     race on the array and corrupt each other's results: serialise them.
+ */
+la_status la_prefill_causal_noalloc(const void *q, const void *k, const void *v,
+                                    la_dtype in_dtype, const float *decay, int B, int H, int T,
+                                    int d_k, int d_v, float eps, int chunk, float *state_S,
+                                    float *state_z, la_state_mode mode, void *out,
+                                    la_dtype out_dtype, void *stream);
+
 /*
  * Non-causal form: every query attends to all Lk keys of its head.
  *   S = S_in + sum_j phi(k_j) v_j^T,  z = z_in + sum_j phi(k_j)
