@@ -372,7 +372,7 @@ def run_ours(args, w):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "chunk": w.chunk,
                    "decay": w.decay, "out_dtype": w.out_dtype, "parallelism": f"heads x{world} (replicas)",
                    "l2": "prefill inputs (805 MB) larger than L2; no flush needed",
-                   "prefill_path": "tcgen05" if la.la_prefill_path(w.torch_dtype, w.d, w.d, w.chunk) == 1
+                   "prefill_path": "tcgen05" if la.la_prefill_path(w.torch_dtype, w.d, w.d, w.chunk, w.decay) == 1
                    else "simt"},
         "ms_per_prefill": pre_avg,
         "roofline": roof,

@@ -28,7 +28,8 @@
  *   - Heads are independent: q, k [B, H, T, d_k], v [B, H, T, d_v],
  *     out [B, H, T, d_v]; state S [B, H, d_k, d_v] and z [B, H, d_k], fp32.
  *   - Supported: d_k == d_v in {32, 64, 128}; in_dtype in {F32, BF16, F16};
- *     out_dtype == in_dtype or LA_F32.  Anything else: LA_ERR_UNSUPPORTED.
+ *     out_dtype == in_dtype or LA_F32; B*H <= 65535.  Anything else:
+ *     LA_ERR_UNSUPPORTED.
  *   - eps must be finite and >= 0 (it is added to the denominator).
  *   - decay values must lie in (0, 1]; this is a precondition, not checked
  *     on the device.  decay == NULL means no decay (a = 1 everywhere).
@@ -152,10 +153,13 @@ la_status la_decode_step(const void *q, const void *k, const void *v, la_dtype i
 /* Static description of a status code (never NULL). */
 const char *la_status_string(la_status s);
 
-/* Which kernel family la_prefill_causal / la_forward_noncausal would run for
- * these arguments: 0 = fp32 CUDA-core (SIMT) kernels, 1 = tcgen05 tensor-core
- * kernels, -1 = unsupported.  Host-only, launches nothing. */
-int la_prefill_path(la_dtype in_dtype, int d_k, int d_v, int chunk);
+/* Which kernel family la_prefill_causal would run for these arguments
+ * (has_decay: whether a decay array is passed): 0 = fp32 CUDA-core (SIMT)
+ * kernels, 1 = tcgen05 tensor-core kernels, -1 = unsupported.  Host-only,
+ * launches nothing.  Tensor cores take 16-bit inputs with d in {64, 128};
+ * chunk 128 with decay needs more tensor memory than an SM has and runs on
+ * the CUDA-core kernels. */
+int la_prefill_path(la_dtype in_dtype, int d_k, int d_v, int chunk, int has_decay);
 
 /* Number of kernels this library has launched in this process so far, over
  * all entry points and devices (kernels later replayed from a captured CUDA

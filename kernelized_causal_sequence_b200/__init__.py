@@ -70,7 +70,7 @@ def lib() -> ctypes.CDLL:
         L.la_status_string.restype = ctypes.c_char_p
         L.la_status_string.argtypes = [_i]
         L.la_prefill_path.restype = _i
-        L.la_prefill_path.argtypes = [_i, _i, _i, _i]
+        L.la_prefill_path.argtypes = [_i, _i, _i, _i, _i]
         L.la_launch_count.restype = ctypes.c_uint64
         L.la_launch_count.argtypes = []
         _lib = L
@@ -93,10 +93,10 @@ def la_noncausal_workspace_size(B, H, Lk, d_k, d_v) -> int:
     return int(lib().la_noncausal_workspace_size(B, H, Lk, d_k, d_v))
 
 
-def la_prefill_path(in_dtype, d_k, d_v, chunk) -> int:
+def la_prefill_path(in_dtype, d_k, d_v, chunk, has_decay=False) -> int:
     if isinstance(in_dtype, torch.dtype):
         in_dtype = _DT[in_dtype]
-    return int(lib().la_prefill_path(in_dtype, d_k, d_v, chunk))
+    return int(lib().la_prefill_path(in_dtype, d_k, d_v, chunk, int(bool(has_decay))))
 
 
 def _ptr(t):

@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "plan.h"
+#include "scan.h"
 #include "simt_kernels.cuh"
 #include "tc_launch.h"
 
@@ -24,9 +25,10 @@ inline bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
 inline bool dtype_ok(la_dtype t) { return t == LA_F32 || t == LA_BF16 || t == LA_F16; }
 
 // Workspace layout of the segment-scan paths:
-//   [ws_state: BH * n_seg * (D*D + D) fp32][ws_A: BH * n_seg fp32][ws_total: BH * (D*D + D) fp32]
+//   [ws_state: BH * n_seg * (D*D + D) fp32][ws_A: BH * n_seg fp32]
+//   [ws_total: BH * (D*D + D) fp32, non-causal only][status word, 256 bytes]
 struct WsLayout {
-    size_t state_off, A_off, total_off, bytes;
+    size_t state_off, A_off, total_off, status_off, bytes;
 };
 
 WsLayout ws_layout(long BH, int n_seg, int D, bool with_total) {
@@ -35,7 +37,8 @@ WsLayout ws_layout(long BH, int n_seg, int D, bool with_total) {
     w.state_off = 0;
     w.A_off = align_up(w.state_off + sizeof(float) * (size_t)BH * n_seg * E);
     w.total_off = align_up(w.A_off + sizeof(float) * (size_t)BH * n_seg);
-    w.bytes = with_total ? align_up(w.total_off + sizeof(float) * (size_t)BH * E) : w.total_off;
+    w.status_off = with_total ? align_up(w.total_off + sizeof(float) * (size_t)BH * E) : w.total_off;
+    w.bytes = w.status_off + kAlign;
     return w;
 }
 
@@ -59,48 +62,36 @@ namespace {
 // ---------------------------------------------------------------- SIMT path
 template <typename InT, typename OutT, int D>
 la_status simt_causal(SimtParams p, cudaStream_t st) {
-    const int E = D * D + D;
     {
         auto k1 = simt_segment_state_kernel<InT, D>;
         const size_t sm = simt_state_smem<D>();
         if (allow_smem(k1, sm) != cudaSuccess) return LA_ERR_CUDA;
         k1<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p, p.T);
     }
-    {
-        const float *sin_S = p.mode == LA_STATE_INOUT ? p.state_S : nullptr;
-        const float *sin_z = p.mode == LA_STATE_INOUT ? p.state_z : nullptr;
-        float *sout_S = p.mode != LA_STATE_NONE ? p.state_S : nullptr;
-        float *sout_z = p.mode != LA_STATE_NONE ? p.state_z : nullptr;
-        segment_scan_kernel<<<dim3((E + 31) / 32, p.BH), 256, 0, st>>>(
-            p.ws_state, p.ws_A, p.n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, nullptr);
-    }
+    if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, D, p.mode, p.state_S, p.state_z,
+                            nullptr, st) != LA_OK)
+        return LA_ERR_CUDA;
     {
         auto k3 = simt_chunk_output_kernel<InT, OutT, D>;
         const size_t sm = simt_output_smem<D>();
         if (allow_smem(k3, sm) != cudaSuccess) return LA_ERR_CUDA;
         k3<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p);
     }
-    count_launches(3);
+    count_launches(2);
     return cuda_status(cudaGetLastError());
 }
 
 template <typename InT, typename OutT, int D>
 la_status simt_noncausal(SimtParams p, int Lk, cudaStream_t st) {
-    const int E = D * D + D;
     {
         auto k1 = simt_segment_state_kernel<InT, D>;
         const size_t sm = simt_state_smem<D>();
         if (allow_smem(k1, sm) != cudaSuccess) return LA_ERR_CUDA;
         k1<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p, Lk);
     }
-    {
-        const float *sin_S = p.mode == LA_STATE_INOUT ? p.state_S : nullptr;
-        const float *sin_z = p.mode == LA_STATE_INOUT ? p.state_z : nullptr;
-        float *sout_S = p.mode != LA_STATE_NONE ? p.state_S : nullptr;
-        float *sout_z = p.mode != LA_STATE_NONE ? p.state_z : nullptr;
-        segment_scan_kernel<<<dim3((E + 31) / 32, p.BH), 256, 0, st>>>(
-            p.ws_state, p.ws_A, p.n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, p.ws_total);
-    }
+    if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, D, p.mode, p.state_S, p.state_z,
+                            p.ws_total, st) != LA_OK)
+        return LA_ERR_CUDA;
     if (p.Lq > 0) {
         auto k3 = simt_noncausal_readout_kernel<InT, OutT, D>;
         const size_t sm = simt_readout_smem<D>();
@@ -108,7 +99,7 @@ la_status simt_noncausal(SimtParams p, int Lk, cudaStream_t st) {
         k3<<<dim3((p.Lq + kReadoutQueries - 1) / kReadoutQueries, p.BH), kSimtThreads, sm, st>>>(p);
         count_launches(1);
     }
-    count_launches(2);
+    count_launches(1);
     return cuda_status(cudaGetLastError());
 }
 
@@ -188,10 +179,10 @@ const char *la_status_string(la_status s) {
     }
 }
 
-int la_prefill_path(la_dtype in_dtype, int d_k, int d_v, int chunk) {
+int la_prefill_path(la_dtype in_dtype, int d_k, int d_v, int chunk, int has_decay) {
     if (!dtype_ok(in_dtype) || d_k != d_v || !dim_ok(d_k) || (chunk != 64 && chunk != 128))
         return -1;
-    return tc_supported(in_dtype, d_k, chunk) ? 1 : 0;
+    return tc_supported(in_dtype, d_k, chunk, has_decay != 0) ? 1 : 0;
 }
 
 size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chunk) {
@@ -233,19 +224,20 @@ la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtyp
     if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_INVALID_ARG;
     if (decay && !aligned16(decay)) return LA_ERR_INVALID_ARG;
-    if (BH > 65535L * 1024L || (double)BH * T * d_k > 9.0e18) return LA_ERR_UNSUPPORTED;
+    if (BH > 65535L) return LA_ERR_UNSUPPORTED;   // heads run along grid y
     const Plan pl = make_plan(BH, T, chunk, d_k);
     const WsLayout wl = ws_layout(BH, pl.n_seg, d_k, false);
     if (!workspace || workspace_bytes < wl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return LA_ERR_INVALID_ARG;
     char *ws = (char *)workspace;
 
-    if (tc_supported(in_dtype, d_k, chunk)) {
+    if (tc_supported(in_dtype, d_k, chunk, decay != nullptr)) {
         TcCausalArgs a;
         a.q = q; a.k = k; a.v = v; a.decay = decay; a.out = out;
         a.in_dtype = in_dtype; a.out_dtype = out_dtype;
         a.ws_state = (float *)(ws + wl.state_off);
         a.ws_A = (float *)(ws + wl.A_off);
+        a.status = (int *)(ws + wl.status_off);
         a.state_S = state_S; a.state_z = state_z; a.mode = mode;
         a.BH = BH; a.T = T; a.D = d_k; a.chunk = chunk; a.seg_len = pl.seg_len;
         a.n_seg = pl.n_seg; a.eps = eps;
@@ -278,7 +270,7 @@ la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_d
     if (BH == 0) return LA_OK;
     if (Lq > 0 && (!q || !out || !aligned16(q) || !aligned16(out))) return LA_ERR_INVALID_ARG;
     if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return LA_ERR_INVALID_ARG;
-    if (BH > 65535L * 1024L) return LA_ERR_UNSUPPORTED;
+    if (BH > 65535L) return LA_ERR_UNSUPPORTED;   // heads run along grid y
     const Plan pl = make_plan(BH, Lk > 0 ? Lk : 1, kNoncausalChunk, d_k);
     const WsLayout wl = ws_layout(BH, pl.n_seg, d_k, true);
     if (!workspace || workspace_bytes < wl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))

@@ -1,0 +1,95 @@
+// scan.cu — K2, the decayed exclusive prefix scan over segment states,
+// shared by the CUDA-core and tensor-core paths.
+#include "common.cuh"
+#include "scan.h"
+
+namespace la {
+
+// K2: decayed exclusive prefix scan over the segments of each head, in place.
+// Segment s maps X -> A_s X + dX_s; entering segment s the state is
+//   S_in(s) = A_{s-1} S_in(s-1) + dX_{s-1},  S_in(0) = state-in or 0,
+// and the final state is S_in(n_seg).  A block takes 32 state elements of one
+// head; a 32-segment x 32-element tile is staged through shared memory so
+// global accesses stay coalesced, and each warp scans one element across the
+// 32 segments of the tile with shuffles (lanes = segments).
+// grid (ceil((D*D + D) / 32), BH), 256 threads.
+__global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, const float *ws_A,
+                                                           int n_seg, int E, int dS,
+                                                           const float *state_in_S,
+                                                           const float *state_in_z,
+                                                           float *state_out_S, float *state_out_z,
+                                                           float *total) {
+    __shared__ float tile[32][33];
+    __shared__ float Atile[32];
+    const int bh = blockIdx.y, e0 = blockIdx.x * 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float *ws = ws_state + (size_t)bh * n_seg * E;
+    const float *Ah = ws_A + (size_t)bh * n_seg;
+
+    // carries of this warp's four elements (e0 + warp + 8 m), replicated in all lanes
+    float carry[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int e = e0 + warp + 8 * m;
+        float c = 0.f;
+        if (e < E) {
+            if (e < dS) { if (state_in_S) c = state_in_S[(size_t)bh * dS + e]; }
+            else if (state_in_z) c = state_in_z[(size_t)bh * (E - dS) + (e - dS)];
+        }
+        carry[m] = c;
+    }
+    for (int s0 = 0; s0 < n_seg; s0 += 32) {
+        __syncthreads();
+        for (int i = warp; i < 32; i += 8) {
+            const int s = s0 + i, e = e0 + lane;
+            tile[i][lane] = (s < n_seg && e < E) ? ws[(size_t)s * E + e] : 0.f;
+        }
+        if (tid < 32) Atile[tid] = (s0 + tid < n_seg) ? Ah[s0 + tid] : 1.f;
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int el = warp + 8 * m;
+            float a = Atile[lane], x = tile[lane][el];
+            warp_affine_scan(a, x, lane);
+            float pa = __shfl_up_sync(0xffffffffu, a, 1);
+            float px = __shfl_up_sync(0xffffffffu, x, 1);
+            if (lane == 0) { pa = 1.f; px = 0.f; }
+            tile[lane][el] = fmaf(pa, carry[m], px);
+            const float a31 = __shfl_sync(0xffffffffu, a, 31);
+            const float x31 = __shfl_sync(0xffffffffu, x, 31);
+            carry[m] = fmaf(a31, carry[m], x31);
+        }
+        __syncthreads();
+        for (int i = warp; i < 32; i += 8) {
+            const int s = s0 + i, e = e0 + lane;
+            if (s < n_seg && e < E) ws[(size_t)s * E + e] = tile[i][lane];
+        }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int e = e0 + warp + 8 * m;
+            if (e >= E) continue;
+            if (total) total[(size_t)bh * E + e] = carry[m];
+            if (e < dS) { if (state_out_S) state_out_S[(size_t)bh * dS + e] = carry[m]; }
+            else if (state_out_z) state_out_z[(size_t)bh * (E - dS) + (e - dS)] = carry[m];
+        }
+    }
+}
+
+
+la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n_seg, int D,
+                              int mode, float *state_S, float *state_z, float *total,
+                              cudaStream_t st) {
+    const int E = D * D + D;
+    const float *sin_S = mode == LA_STATE_INOUT ? state_S : nullptr;
+    const float *sin_z = mode == LA_STATE_INOUT ? state_z : nullptr;
+    float *sout_S = mode != LA_STATE_NONE ? state_S : nullptr;
+    float *sout_z = mode != LA_STATE_NONE ? state_z : nullptr;
+    segment_scan_kernel<<<dim3((E + 31) / 32, (unsigned)BH), 256, 0, st>>>(
+        ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, total);
+    count_launches(1);
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+}  // namespace la

@@ -136,78 +136,6 @@ __global__ void __launch_bounds__(kSimtThreads) simt_segment_state_kernel(SimtPa
     if (tid == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = Aseg;
 }
 
-// K2: decayed exclusive prefix scan over the segments of each head, in place.
-// Segment s maps X -> A_s X + dX_s; entering segment s the state is
-//   S_in(s) = A_{s-1} S_in(s-1) + dX_{s-1},  S_in(0) = state-in or 0,
-// and the final state is S_in(n_seg).  A block takes 32 state elements of one
-// head; a 32-segment x 32-element tile is staged through shared memory so
-// global accesses stay coalesced, and each warp scans one element across the
-// 32 segments of the tile with shuffles (lanes = segments).
-// grid (ceil((D*D + D) / 32), BH), 256 threads.
-__global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, const float *ws_A,
-                                                           int n_seg, int E, int dS,
-                                                           const float *state_in_S,
-                                                           const float *state_in_z,
-                                                           float *state_out_S, float *state_out_z,
-                                                           float *total) {
-    __shared__ float tile[32][33];
-    __shared__ float Atile[32];
-    const int bh = blockIdx.y, e0 = blockIdx.x * 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    float *ws = ws_state + (size_t)bh * n_seg * E;
-    const float *Ah = ws_A + (size_t)bh * n_seg;
-
-    // carries of this warp's four elements (e0 + warp + 8 m), replicated in all lanes
-    float carry[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const int e = e0 + warp + 8 * m;
-        float c = 0.f;
-        if (e < E) {
-            if (e < dS) { if (state_in_S) c = state_in_S[(size_t)bh * dS + e]; }
-            else if (state_in_z) c = state_in_z[(size_t)bh * (E - dS) + (e - dS)];
-        }
-        carry[m] = c;
-    }
-    for (int s0 = 0; s0 < n_seg; s0 += 32) {
-        __syncthreads();
-        for (int i = warp; i < 32; i += 8) {
-            const int s = s0 + i, e = e0 + lane;
-            tile[i][lane] = (s < n_seg && e < E) ? ws[(size_t)s * E + e] : 0.f;
-        }
-        if (tid < 32) Atile[tid] = (s0 + tid < n_seg) ? Ah[s0 + tid] : 1.f;
-        __syncthreads();
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int el = warp + 8 * m;
-            float a = Atile[lane], x = tile[lane][el];
-            warp_affine_scan(a, x, lane);
-            float pa = __shfl_up_sync(0xffffffffu, a, 1);
-            float px = __shfl_up_sync(0xffffffffu, x, 1);
-            if (lane == 0) { pa = 1.f; px = 0.f; }
-            tile[lane][el] = fmaf(pa, carry[m], px);
-            const float a31 = __shfl_sync(0xffffffffu, a, 31);
-            const float x31 = __shfl_sync(0xffffffffu, x, 31);
-            carry[m] = fmaf(a31, carry[m], x31);
-        }
-        __syncthreads();
-        for (int i = warp; i < 32; i += 8) {
-            const int s = s0 + i, e = e0 + lane;
-            if (s < n_seg && e < E) ws[(size_t)s * E + e] = tile[i][lane];
-        }
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int e = e0 + warp + 8 * m;
-            if (e >= E) continue;
-            if (total) total[(size_t)bh * E + e] = carry[m];
-            if (e < dS) { if (state_out_S) state_out_S[(size_t)bh * dS + e] = carry[m]; }
-            else if (state_out_z) state_out_z[(size_t)bh * (E - dS) + (e - dS)] = carry[m];
-        }
-    }
-}
-
 template <int D> __host__ __device__ constexpr size_t simt_output_smem() {
     return sizeof(float) * (D * D + D + 3 * kSub * D + kSub * (kSub + 1) + 128);
 }

@@ -1,11 +1,128 @@
-// tc_kernels.cu — tcgen05 tensor-core kernels (bf16/fp16 inputs, fp32 state).
+// tc_kernels.cu — host side of the tcgen05 prefill: tensor maps, launch
+// configuration and the K1 (state build) -> K2 (scan) -> K3 (chunk output)
+// sequence on the caller's stream.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <type_traits>
+
+#include "scan.h"
 #include "tc_launch.h"
+#include "tc_prefill.cuh"
 
 namespace la {
 
-bool tc_supported(la_dtype, int, int) { return false; }
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D map over a [BH][T][D] 16-bit tensor; box = 64 columns x C rows x 1 head,
+// 128-byte swizzle, zero fill beyond T.
+bool make_map(CUtensorMap *m, const void *base, la_dtype dt, long BH, int T, int D, int C) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)C, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapDataType t =
+        dt == LA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = enc(m, t, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int C, int D, bool DECAY, int MODE, typename InT, typename OutT>
+la_status launch_tc(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                    const tc::TcParams &p, long BH, cudaStream_t st) {
+    using G = tc::Cfg<C, D, DECAY, MODE>;
+    auto kern = tc::tc_prefill_kernel<C, D, DECAY, MODE, InT, OutT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES) !=
+        cudaSuccess)
+        return LA_ERR_CUDA;
+    kern<<<dim3(p.n_seg, (unsigned)BH), tc::kThreads, G::SMEM_BYTES, st>>>(mq, mk, mv, p);
+    count_launches(1);
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+template <int C, int D, bool DECAY, typename InT, typename OutT>
+la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, a.q, a.in_dtype, a.BH, a.T, D, C) || !make_map(&mk, a.k, a.in_dtype, a.BH, a.T, D, C) ||
+        !make_map(&mv, a.v, a.in_dtype, a.BH, a.T, D, C))
+        return LA_ERR_CUDA;
+    tc::TcParams p;
+    p.decay = a.decay;
+    p.out = a.out;
+    p.ws_state = a.ws_state;
+    p.ws_A = a.ws_A;
+    p.status = a.status;
+    p.T = a.T;
+    p.seg_len = a.seg_len;
+    p.n_seg = a.n_seg;
+    p.eps = a.eps;
+    if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return LA_ERR_CUDA;
+    // K1: per-segment state contributions
+    la_status s = launch_tc<C, D, DECAY, tc::kStateOnly, InT, float>(mq, mk, mv, p, a.BH, st);
+    if (s != LA_OK) return s;
+    // K2: decayed exclusive scan over segments (+ state in/out)
+    s = launch_segment_scan(a.ws_state, a.ws_A, a.BH, a.n_seg, D, a.mode, a.state_S, a.state_z,
+                            nullptr, st);
+    if (s != LA_OK) return s;
+    // K3: chunked output from the segment-entry states
+    return launch_tc<C, D, DECAY, tc::kOutput, InT, OutT>(mq, mk, mv, p, a.BH, st);
+}
+
+template <typename InT, typename OutT>
+la_status dispatch_cd(const TcCausalArgs &a, cudaStream_t st) {
+    const bool dec = a.decay != nullptr;
+    if (a.D == 128) {
+        if (a.chunk == 128) return dec ? LA_ERR_UNSUPPORTED : run_causal<128, 128, false, InT, OutT>(a, st);
+        return dec ? run_causal<64, 128, true, InT, OutT>(a, st) : run_causal<64, 128, false, InT, OutT>(a, st);
+    }
+    if (a.D == 64) {
+        if (a.chunk == 128) return dec ? LA_ERR_UNSUPPORTED : run_causal<128, 64, false, InT, OutT>(a, st);
+        return dec ? run_causal<64, 64, true, InT, OutT>(a, st) : run_causal<64, 64, false, InT, OutT>(a, st);
+    }
+    return LA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+bool tc_supported(la_dtype in_dtype, int D, int chunk, bool has_decay) {
+    if (in_dtype != LA_BF16 && in_dtype != LA_F16) return false;
+    if (D != 64 && D != 128) return false;
+    if (chunk != 64 && chunk != 128) return false;
+    if (chunk == 128 && has_decay) return false;   // TMEM budget: see Cfg
+    return true;
+}
+
 bool tc_noncausal_supported(la_dtype, int) { return false; }
-la_status tc_causal(const TcCausalArgs &, cudaStream_t) { return LA_ERR_UNSUPPORTED; }
+
+la_status tc_causal(const TcCausalArgs &a, cudaStream_t st) {
+    if (a.in_dtype == LA_BF16) {
+        if (a.out_dtype == LA_BF16) return dispatch_cd<bf16, bf16>(a, st);
+        return dispatch_cd<bf16, float>(a, st);
+    }
+    if (a.in_dtype == LA_F16) {
+        if (a.out_dtype == LA_F16) return dispatch_cd<f16, f16>(a, st);
+        return dispatch_cd<f16, float>(a, st);
+    }
+    return LA_ERR_UNSUPPORTED;
+}
+
 la_status tc_noncausal(const TcNoncausalArgs &, cudaStream_t) { return LA_ERR_UNSUPPORTED; }
 
 }  // namespace la

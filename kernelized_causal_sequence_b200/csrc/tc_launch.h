@@ -12,6 +12,7 @@ struct TcCausalArgs {
     void *out;
     la_dtype in_dtype, out_dtype;
     float *ws_state, *ws_A;
+    int *status;
     float *state_S, *state_z;
     la_state_mode mode;
     long BH;
@@ -33,7 +34,7 @@ struct TcNoncausalArgs {
 
 void count_launches(int n);  // process-wide kernel launch counter (la_launch_count)
 
-bool tc_supported(la_dtype in_dtype, int D, int chunk);
+bool tc_supported(la_dtype in_dtype, int D, int chunk, bool has_decay);
 bool tc_noncausal_supported(la_dtype in_dtype, int D);
 la_status tc_causal(const TcCausalArgs &a, cudaStream_t st);
 la_status tc_noncausal(const TcNoncausalArgs &a, cudaStream_t st);

@@ -59,7 +59,11 @@ def test_prefill_path_selection(L):
     assert la.la_prefill_path(la.LA_F32, 64, 64, 64) == 0
     assert la.la_prefill_path(la.LA_BF16, 64, 64, 96) == -1
     assert la.la_prefill_path(la.LA_BF16, 48, 48, 64) == -1
-    assert la.la_prefill_path(la.LA_BF16, 128, 128, 128) in (0, 1)
+    # 16-bit inputs with d in {64, 128} run on tensor cores, except chunk 128 with decay
+    assert la.la_prefill_path(la.LA_BF16, 128, 128, 128) == 1
+    assert la.la_prefill_path(la.LA_F16, 64, 64, 64, has_decay=True) == 1
+    assert la.la_prefill_path(la.LA_BF16, 128, 128, 128, has_decay=True) == 0
+    assert la.la_prefill_path(la.LA_BF16, 32, 32, 64) == 0
 
 
 def _prefill(L, q=P, k=P, v=P, dt=la.LA_BF16, decay=None, B=1, H=2, T=128, dk=64, dv=64,
