@@ -244,7 +244,7 @@ def run_ours(args, w):
     # ---- decode: states from the library's own prefill of a 512-token prompt
     wd = inputs.WORKLOADS["decode_bf16_b64h16_d128"] if w.name.startswith("prefill") else None
     dec = None
-    if wd is not None and args.decode_steps > 0:
+    if wd is not None and args.decode_steps > 0 and w.decay is False:
         pq, pk, pv, _ = inputs.qkv(inputs.WORKLOADS["prefill_bf16_h16_t131072_d128"], T=wd.prompt,
                                    B=wd.B, H=wd.H, seed=wd.seed + 1)
         dS = torch.zeros((wd.B, wd.H, wd.d, wd.d), dtype=torch.float32, device=dev)
@@ -332,7 +332,7 @@ def run_ours(args, w):
 
     # ---- end to end through the public API with host buffers (pinned)
     e2e = None
-    if rank == 0 or world > 1:
+    if not args.no_e2e:
         qp, kp, vp = (x.pin_memory() for x in (q_h, k_h, v_h))
         ap = None if a_h is None else a_h.pin_memory()
         op = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -392,10 +392,11 @@ def run_ours(args, w):
                          "note": "fp32 state (67.6 MB) stays L2-resident across the loop"},
         }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r, dt, cores = oracle_prefill_sample(w, q_h, k_h, v_h, a_h, args.cpu_tokens)
+        tok = args.cpu_tokens or w.T
+        r, dt, cores = oracle_prefill_sample(w, q_h, k_h, v_h, a_h, tok)
         line["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"first {args.cpu_tokens} tokens of all {w.B * w.H} heads, "
-                                          f"fp64 recurrence, {dt:.1f} s"}
+                                "sample": f"first {tok} of {w.T} tokens of all {w.B * w.H} heads "
+                                          f"(the whole prefill when equal), fp64 recurrence, {dt:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -412,7 +413,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_bf16_h16_t131072_d128")
     ap.add_argument("--decode-steps", type=int, default=1024)
-    ap.add_argument("--cpu-tokens", type=int, default=16384)
+    ap.add_argument("--cpu-tokens", type=int, default=0,
+                    help="tokens per head for the CPU oracle sample (0 = the whole workload)")
+    ap.add_argument("--T", type=int, default=0, help="override the workload's sequence length")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=4096)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
@@ -420,6 +424,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     from kernelized_causal_sequence_b200 import inputs
     w = inputs.WORKLOADS[args.workload]
+    if args.T:
+        import dataclasses
+        w = dataclasses.replace(w, T=args.T, name=f"{w.name}@T{args.T}")
     if w.kind != "causal":
         raise SystemExit("bench workloads are causal prefills")
     if args.impl == "reference":

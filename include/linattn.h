@@ -153,6 +153,11 @@ la_status la_decode_step(const void *q, const void *k, const void *v, la_dtype i
 /* Static description of a status code (never NULL). */
 const char *la_status_string(la_status s);
 
+/* Text of the last failure that made an entry point return LA_ERR_CUDA on
+ * the calling thread ("<step>: <CUDA error>"), or "" if none.  The pointer
+ * stays valid until the thread's next failing call. */
+const char *la_last_error_string(void);
+
 /* Which kernel family la_prefill_causal would run for these arguments
  * (has_decay: whether a decay array is passed): 0 = fp32 CUDA-core (SIMT)
  * kernels, 1 = tcgen05 tensor-core kernels, -1 = unsupported.  Host-only,

@@ -41,7 +41,10 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 
 class LinAttnError(RuntimeError):
     def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn} returned {status}: {la_status_string(status)}")
+        msg = f"{fn} returned {status}: {la_status_string(status)}"
+        if status == LA_ERR_CUDA:
+            msg += f" ({lib().la_last_error_string().decode()})"
+        super().__init__(msg)
         self.status = status
 
 
@@ -73,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.la_prefill_path.argtypes = [_i, _i, _i, _i, _i]
         L.la_launch_count.restype = ctypes.c_uint64
         L.la_launch_count.argtypes = []
+        L.la_last_error_string.restype = ctypes.c_char_p
+        L.la_last_error_string.argtypes = []
         _lib = L
     return _lib
 

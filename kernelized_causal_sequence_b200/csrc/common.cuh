@@ -21,11 +21,30 @@ template <> __device__ __forceinline__ float from_f32<float>(float x) { return x
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
 template <> __device__ __forceinline__ f16 from_f32<f16>(float x) { return __float2half_rn(x); }
 
+// 2^x with the hardware approximation instruction (relative error ~2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// log2(x) with the hardware approximation instruction.
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
 // phi(x) = elu(x) + 1 (alpha = 1): x + 1 for x > 0, and e^x for x <= 0, which
 // equals (e^x - 1) + 1 without the cancellation.  ("Transformers are RNNs"
 // feature map, as given on the knowledge-base page, section 2, "Choice of phi".)
+// The fp32-input path uses the library expf; the 16-bit paths, whose operands
+// are rounded to bf16 anyway, take e^x = 2^(x log2 e) on the ex2 unit.
 __device__ __forceinline__ float phi_precise(float x) { return x > 0.f ? x + 1.f : expf(x); }
-__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+__device__ __forceinline__ float phi_fast(float x) {
+    const float e = ex2_approx(x * kLog2e);
+    return x > 0.f ? x + 1.f : e;
+}
 
 // Inclusive warp scan of the pair operator (a1, x1) o (a2, x2) = (a1 a2, a2 x1 + x2),
 // which composes the affine maps X -> a X + x of consecutive segments.

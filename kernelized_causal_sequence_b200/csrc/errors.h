@@ -1,0 +1,19 @@
+// errors.h — per-thread record of the last CUDA failure behind LA_ERR_CUDA,
+// readable through la_last_error_string().
+#pragma once
+#include <cuda_runtime.h>
+
+#include "linattn.h"
+
+namespace la {
+
+// Records "where: <CUDA error text>" and returns LA_ERR_CUDA.
+la_status cuda_fail(const char *where, cudaError_t e);
+// Records a message (for non-runtime failures) and returns LA_ERR_CUDA.
+la_status cuda_fail_msg(const char *where, const char *msg);
+// LA_OK if e is cudaSuccess, else cuda_fail(where, e).
+inline la_status cuda_check(const char *where, cudaError_t e) {
+    return e == cudaSuccess ? LA_OK : cuda_fail(where, e);
+}
+
+}  // namespace la

@@ -4,11 +4,13 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 
-#include "../../include/linattn.h"
+#include "linattn.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "errors.h"
 #include "plan.h"
 #include "scan.h"
 #include "simt_kernels.cuh"
@@ -48,13 +50,21 @@ template <typename K> cudaError_t allow_smem(K kernel, size_t bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-la_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
 
 }  // namespace
 
 namespace la {
 std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+thread_local char g_last_error[256] = "";
+la_status cuda_fail_msg(const char *where, const char *msg) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, msg);
+    return LA_ERR_CUDA;
+}
+la_status cuda_fail(const char *where, cudaError_t e) {
+    return cuda_fail_msg(where, cudaGetErrorString(e));
+}
 }  // namespace la
 
 namespace {
@@ -65,7 +75,8 @@ la_status simt_causal(SimtParams p, cudaStream_t st) {
     {
         auto k1 = simt_segment_state_kernel<InT, D>;
         const size_t sm = simt_state_smem<D>();
-        if (allow_smem(k1, sm) != cudaSuccess) return LA_ERR_CUDA;
+        la_status e = cuda_check("segment_state smem attribute", allow_smem(k1, sm));
+        if (e != LA_OK) return e;
         k1<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p, p.T);
     }
     if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, D, p.mode, p.state_S, p.state_z,
@@ -74,11 +85,12 @@ la_status simt_causal(SimtParams p, cudaStream_t st) {
     {
         auto k3 = simt_chunk_output_kernel<InT, OutT, D>;
         const size_t sm = simt_output_smem<D>();
-        if (allow_smem(k3, sm) != cudaSuccess) return LA_ERR_CUDA;
+        la_status e = cuda_check("chunk_output smem attribute", allow_smem(k3, sm));
+        if (e != LA_OK) return e;
         k3<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p);
     }
     count_launches(2);
-    return cuda_status(cudaGetLastError());
+    return cuda_check("causal kernel launch", cudaGetLastError());
 }
 
 template <typename InT, typename OutT, int D>
@@ -86,7 +98,8 @@ la_status simt_noncausal(SimtParams p, int Lk, cudaStream_t st) {
     {
         auto k1 = simt_segment_state_kernel<InT, D>;
         const size_t sm = simt_state_smem<D>();
-        if (allow_smem(k1, sm) != cudaSuccess) return LA_ERR_CUDA;
+        la_status e = cuda_check("segment_state smem attribute", allow_smem(k1, sm));
+        if (e != LA_OK) return e;
         k1<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p, Lk);
     }
     if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, D, p.mode, p.state_S, p.state_z,
@@ -95,12 +108,13 @@ la_status simt_noncausal(SimtParams p, int Lk, cudaStream_t st) {
     if (p.Lq > 0) {
         auto k3 = simt_noncausal_readout_kernel<InT, OutT, D>;
         const size_t sm = simt_readout_smem<D>();
-        if (allow_smem(k3, sm) != cudaSuccess) return LA_ERR_CUDA;
+        la_status e = cuda_check("readout smem attribute", allow_smem(k3, sm));
+        if (e != LA_OK) return e;
         k3<<<dim3((p.Lq + kReadoutQueries - 1) / kReadoutQueries, p.BH), kSimtThreads, sm, st>>>(p);
         count_launches(1);
     }
     count_launches(1);
-    return cuda_status(cudaGetLastError());
+    return cuda_check("non-causal kernel launch", cudaGetLastError());
 }
 
 // Dispatch over (in dtype, out dtype, head dim) for a functor template F.
@@ -140,7 +154,7 @@ template <typename IT, typename OT, int D> struct DecodeF {
         decode_step_kernel<IT, OT, D><<<(unsigned)BH, kDecodeThreads, 0, st>>>(
             (const IT *)q, (const IT *)k, (const IT *)v, decay, eps, S, z, (OT *)out);
         count_launches(1);
-        return cuda_status(cudaGetLastError());
+        return cuda_check("decode_step launch", cudaGetLastError());
     }
 };
 
@@ -167,6 +181,8 @@ la_status check_state(la_state_mode mode, const float *S, const float *z) {
 extern "C" {
 
 uint64_t la_launch_count(void) { return la::g_launches.load(std::memory_order_relaxed); }
+
+const char *la_last_error_string(void) { return la::g_last_error; }
 
 const char *la_status_string(la_status s) {
     switch (s) {
@@ -215,9 +231,9 @@ la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtyp
     if (BH == 0) return LA_OK;
     if (T == 0) {
         if (mode == LA_STATE_OUT) {
-            if (cudaMemsetAsync(state_S, 0, sizeof(float) * BH * d_k * d_v, st) != cudaSuccess ||
-                cudaMemsetAsync(state_z, 0, sizeof(float) * BH * d_k, st) != cudaSuccess)
-                return LA_ERR_CUDA;
+            la_status e = cuda_check("state memset", cudaMemsetAsync(state_S, 0, sizeof(float) * BH * d_k * d_v, st));
+            if (e == LA_OK) e = cuda_check("state memset", cudaMemsetAsync(state_z, 0, sizeof(float) * BH * d_k, st));
+            if (e != LA_OK) return e;
         }
         return LA_OK;
     }

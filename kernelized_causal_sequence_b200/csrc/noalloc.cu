@@ -15,7 +15,7 @@
 // with cudaGetSymbolAddress and cached.
 #include <mutex>
 
-#include "../../include/linattn.h"
+#include "linattn.h"
 #include <cuda_runtime.h>
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
@@ -52,7 +52,7 @@ extern "C" la_status la_prefill_causal_noalloc(const void *q, const void *k, con
         la_prefill_workspace_size(B, H, T, d_k, d_v, chunk) > (size_t)LA_NOALLOC_SCRATCH_BYTES)
         return LA_ERR_UNSUPPORTED;
     void *scratch = scratch_for_current_device();
-    if (!scratch) return LA_ERR_CUDA;
+    if (!scratch) return LA_ERR_CUDA;   // device address lookup failed
     return la_prefill_causal(q, k, v, in_dtype, decay, B, H, T, d_k, d_v, eps, chunk, state_S,
                              state_z, mode, out, out_dtype, scratch,
                              (size_t)LA_NOALLOC_SCRATCH_BYTES, stream);

@@ -17,24 +17,30 @@ struct Plan {
     int n_seg;    // segments per head
 };
 
-// Segments per head: enough CTAs for two per SM across all heads, but no
-// segment shorter than `min_tokens` unless the head itself is shorter.
+// Segments per head.  Each segment is one CTA (one per SM), so the critical
+// path is (waves of CTAs) x (chunks per segment): choose the segment count
+// that minimises it, preferring fewer segments (less scan traffic) on ties.
+// Segments are kept at least `min_chunks` long so the per-segment state
+// (D*D + D fp32 written, scanned, read back) stays a small fraction of the
+// segment's own input bytes.
 inline Plan make_plan(long BH, long T, int chunk, int D) {
     Plan p;
     p.chunk = chunk;
     const long n_chunks = (T + chunk - 1) / chunk;
-    const long want_ctas = 2L * kNumSMs;
-    long segs = (want_ctas + BH - 1) / BH;
-    // keep the scan traffic (4 passes over D*D fp32 per segment) below ~1/8
-    // of the segment's own q/k/v/o bytes (~8*D bytes per token at 16 bits)
-    long min_tokens = (long)D * 16;
-    if (min_tokens < chunk) min_tokens = chunk;
-    long min_chunks = (min_tokens + chunk - 1) / chunk;
+    long min_chunks = ((long)D * 4 + chunk - 1) / chunk;   // >= 4*D tokens per segment
+    if (min_chunks < 1) min_chunks = 1;
     long max_segs = n_chunks / min_chunks;
     if (max_segs < 1) max_segs = 1;
-    if (segs > max_segs) segs = max_segs;
-    if (segs < 1) segs = 1;
-    long G = (n_chunks + segs - 1) / segs;
+    if (max_segs > 4096) max_segs = 4096;
+    long best_segs = 1, best_cost = -1;
+    for (long segs = 1; segs <= max_segs; ++segs) {
+        const long G = (n_chunks + segs - 1) / segs;
+        const long real = (n_chunks + G - 1) / G;
+        const long waves = (BH * real + kNumSMs - 1) / kNumSMs;
+        const long cost = waves * (G + 2);   // ~2 chunks of per-CTA fill, set-up and drain
+        if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_segs = segs; }
+    }
+    const long G = (n_chunks + best_segs - 1) / best_segs;
     p.seg_len = (int)(G * chunk);
     p.n_seg = (int)((n_chunks + G - 1) / G);
     return p;

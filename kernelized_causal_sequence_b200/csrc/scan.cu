@@ -1,6 +1,7 @@
 // scan.cu — K2, the decayed exclusive prefix scan over segment states,
 // shared by the CUDA-core and tensor-core paths.
 #include "common.cuh"
+#include "errors.h"
 #include "scan.h"
 
 namespace la {
@@ -89,7 +90,7 @@ la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n
     segment_scan_kernel<<<dim3((E + 31) / 32, (unsigned)BH), 256, 0, st>>>(
         ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, total);
     count_launches(1);
-    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    return cuda_check("segment_scan launch", cudaGetLastError());
 }
 
 }  // namespace la

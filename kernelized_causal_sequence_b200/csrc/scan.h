@@ -2,7 +2,7 @@
 #pragma once
 #include <cuda_runtime.h>
 
-#include "../../include/linattn.h"
+#include "linattn.h"
 
 namespace la {
 

@@ -6,6 +6,7 @@
 #include <mutex>
 #include <type_traits>
 
+#include "errors.h"
 #include "scan.h"
 #include "tc_launch.h"
 #include "tc_prefill.cuh"
@@ -27,17 +28,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3-D map over a [BH][T][D] 16-bit tensor; box = 64 columns x C rows x 1 head,
-// 128-byte swizzle, zero fill beyond T.
+// 3-D map over a [BH][T][D] tensor; box = 128 bytes of columns x C rows x 1
+// head, 128-byte swizzle, zero fill (loads) / clipping (stores) beyond T.
 bool make_map(CUtensorMap *m, const void *base, la_dtype dt, long BH, int T, int D, int C) {
     auto enc = encode_fn();
     if (!enc) return false;
+    const int es = dt == LA_F32 ? 4 : 2;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)C, 1};
+    cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)T * D * es};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / es), (cuuint32_t)C, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    const CUtensorMapDataType t =
-        dt == LA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapDataType t = dt == LA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                  : dt == LA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     CUresult r = enc(m, t, 3, const_cast<void *>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -46,23 +49,24 @@ bool make_map(CUtensorMap *m, const void *base, la_dtype dt, long BH, int T, int
 
 template <int C, int D, bool DECAY, int MODE, typename InT, typename OutT>
 la_status launch_tc(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                    const tc::TcParams &p, long BH, cudaStream_t st) {
+                    const CUtensorMap &mo, const tc::TcParams &p, long BH, cudaStream_t st) {
     using G = tc::Cfg<C, D, DECAY, MODE>;
     auto kern = tc::tc_prefill_kernel<C, D, DECAY, MODE, InT, OutT>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES) !=
-        cudaSuccess)
-        return LA_ERR_CUDA;
-    kern<<<dim3(p.n_seg, (unsigned)BH), tc::kThreads, G::SMEM_BYTES, st>>>(mq, mk, mv, p);
+    la_status e = cuda_check("tensor-core kernel smem attribute",
+                             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES));
+    if (e != LA_OK) return e;
+    kern<<<dim3(p.n_seg, (unsigned)BH), tc::kThreads, G::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
     count_launches(1);
-    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    return cuda_check("tensor-core kernel launch", cudaGetLastError());
 }
 
 template <int C, int D, bool DECAY, typename InT, typename OutT>
 la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, a.q, a.in_dtype, a.BH, a.T, D, C) || !make_map(&mk, a.k, a.in_dtype, a.BH, a.T, D, C) ||
-        !make_map(&mv, a.v, a.in_dtype, a.BH, a.T, D, C))
-        return LA_ERR_CUDA;
+        !make_map(&mv, a.v, a.in_dtype, a.BH, a.T, D, C) ||
+        !make_map(&mo, a.out, a.out_dtype, a.BH, a.T, D, C == 128 ? 32 : 16))   // per-warp row blocks
+        return cuda_fail_msg("cuTensorMapEncodeTiled", "tensor map encoding failed");
     tc::TcParams p;
     p.decay = a.decay;
     p.out = a.out;
@@ -73,16 +77,17 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
     p.seg_len = a.seg_len;
     p.n_seg = a.n_seg;
     p.eps = a.eps;
-    if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return LA_ERR_CUDA;
+    la_status e0 = cuda_check("status memset", cudaMemsetAsync(a.status, 0, sizeof(int), st));
+    if (e0 != LA_OK) return e0;
     // K1: per-segment state contributions
-    la_status s = launch_tc<C, D, DECAY, tc::kStateOnly, InT, float>(mq, mk, mv, p, a.BH, st);
+    la_status s = launch_tc<C, D, DECAY, tc::kStateOnly, InT, float>(mq, mk, mv, mo, p, a.BH, st);
     if (s != LA_OK) return s;
     // K2: decayed exclusive scan over segments (+ state in/out)
     s = launch_segment_scan(a.ws_state, a.ws_A, a.BH, a.n_seg, D, a.mode, a.state_S, a.state_z,
                             nullptr, st);
     if (s != LA_OK) return s;
     // K3: chunked output from the segment-entry states
-    return launch_tc<C, D, DECAY, tc::kOutput, InT, OutT>(mq, mk, mv, p, a.BH, st);
+    return launch_tc<C, D, DECAY, tc::kOutput, InT, OutT>(mq, mk, mv, mo, p, a.BH, st);
 }
 
 template <typename InT, typename OutT>

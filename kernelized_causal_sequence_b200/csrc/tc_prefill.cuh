@@ -16,8 +16,8 @@
 // the linear-attention lesson's "Implementation reality": quadratic inside a
 // chunk, the state carried across chunks; the concept card's SSD variant for
 // the scalar decay.)  With decay, w_j = prod_{l>j in chunk} a_l, the mask is
-// exp(L_i - L_j) for j <= i (L = chunk-local inclusive cumsum of log a), the
-// inter term of row i is scaled by exp(L_i), and the state is rescaled by the
+// 2^(L_i - L_j) for j <= i (L = chunk-local inclusive cumsum of log2 a), the
+// inter term of row i is scaled by 2^(L_i), and the state is rescaled by the
 // chunk's total decay before each update.
 //
 // Warp roles (320 threads):
@@ -58,9 +58,18 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr bool QT = OUT && C == 128;    // phi(Q) held in TMEM
     static constexpr bool PT = OUT && C == 128;    // P held in TMEM
     static constexpr bool SPLIT = OUT && DECAY;    // separate inter / intra accumulators
-    static constexpr int NKV = 2;                  // K/V stages
+    // K/V stages: two in output mode (shared memory is full); the state-only
+    // pass has room for more, which hides the load latency of its short chunks
+    static constexpr int KV_BYTES = (2 + (DECAY ? 1 : 0)) * C * D * 2;
+    static constexpr int NKV = OUT ? 2 : (KV_BYTES <= 48 * 1024 ? 4 : 3);
     static constexpr int NQ = OUT ? (QT ? 1 : 2) : 0;
     static constexpr int ROWS_PER_WARP = (C == 128) ? 32 : 16;   // M=64 uses lanes 0-15
+    // Work split of the feature map between the two warpgroups: the phi
+    // warpgroup forms the first KSPLIT quarters of the key rows, the epilogue
+    // warpgroup the rest; with phi(Q) in TMEM and two column boxes, the
+    // epilogue warpgroup also forms the second box of phi(Q).
+    static constexpr bool QSPLIT = QT && KB == 2;
+    static constexpr int KSPLIT = QSPLIT ? 3 : 2;
 
     // ---- shared memory (offsets from a 1024-byte aligned base)
     static constexpr int KV_STAGE = 2 * TILE + (DECAY ? TILE : 0);  // K, V, (w o phi(K))
@@ -72,12 +81,16 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int PB = (OUT && !PT) ? C * C * 2 : 0;
     static constexpr int OFF_ZB = OFF_P + PB;                        // z as MMA operand [16][D]
     static constexpr int ZB = OUT ? 16 * D * 2 : 0;
-    static constexpr int OFF_ONES = OFF_ZB + ZB;                     // ones operand [16][C]
-    static constexpr int ONES = 16 * C * 2;
-    static constexpr int OFF_F = OFF_ONES + ONES;                    // fp32 scratch
-    static constexpr int F_L = 0;                                    // [NKV][C] log-decay cumsum
+    static constexpr int OFF_STG = OFF_ZB + ZB;                      // output staging, 4 warps x [R][128 B]
+    static constexpr int STG = OUT ? 4 * ROWS_PER_WARP * 128 : 0;
+    static constexpr int OFF_F = OFF_STG + STG;                      // fp32 scratch
+    static constexpr int F_L = 0;                                    // [NKV][C] log2-decay cumsum
     static constexpr int F_G = F_L + (DECAY ? NKV * C : 0);          // [NKV] chunk decay
-    static constexpr int F_END = F_G + NKV;
+    // per-warp column sums of w o phi(K) (8 warps: 4 phi + 4 epilogue), one
+    // buffer per K/V stage in output mode, one running set in state-only mode
+    static constexpr int NRED = OUT ? 3 : 1;   // 3: the slot of chunk c is reused by chunk c+3 only
+    static constexpr int F_RED = (F_G + NKV + 3) / 4 * 4;            // [NRED][8][D], 16-byte aligned
+    static constexpr int F_END = F_RED + NRED * 8 * D;
     static constexpr int OFF_BAR = (OFF_F + F_END * 4 + 7) / 8 * 8;
     // barrier indices
     static constexpr int B_KV_FULL = 0, B_KV_EMPTY = B_KV_FULL + NKV, B_PHI = B_KV_EMPTY + NKV;
@@ -86,7 +99,8 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int B_P_READY = B_SC_FULL + 1, B_MMA4 = B_P_READY + 1;
     static constexpr int B_O_FULL = B_MMA4 + 1, B_O_EMPTY = B_O_FULL + 1;
     static constexpr int B_DS_FULL = B_O_EMPTY + 1, B_S_READY = B_DS_FULL + 1;
-    static constexpr int B_DRAIN = B_S_READY + 1, NBAR = B_DRAIN + 1;
+    static constexpr int B_DRAIN = B_S_READY + 1, B_L_READY = B_DRAIN + 1;
+    static constexpr int NBAR = B_L_READY + NKV;
     static constexpr int OFF_TMEMADDR = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEMADDR + 4;
     static constexpr int OFF_END = OFF_ABORT + 4;
@@ -97,8 +111,7 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int T_O = OUT ? C : 0;
     static constexpr int T_O2 = T_O + (OUT ? D : 0);
     static constexpr int T_S = T_O2 + (SPLIT ? D : 0);
-    static constexpr int T_Z = T_S + D;
-    static constexpr int T_DEN = T_Z + 16;
+    static constexpr int T_DEN = T_S + D;                     // phi(Q) z of the carried state
     static constexpr int T_Q = T_DEN + (OUT ? 16 : 0);
     static constexpr int T_USED = T_Q + (QT ? D / 2 : 0);
     static constexpr int TMEM_COLS = tmem_alloc_cols(T_USED);
@@ -108,6 +121,9 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static_assert(!(C == 128 && DECAY && OUT), "chunk 128 with decay exceeds TMEM");
     static_assert(T_USED <= 512, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(OFF_F % 16 == 0 && (F_RED * 4) % 16 == 0, "float4 column-sum stores need 16-byte alignment");
+    static_assert(OFF_STG % 1024 == 0 && OFF_SBF % 1024 == 0 && OFF_P % 1024 == 0 && OFF_ZB % 16 == 0 &&
+                  OFF_Q % 1024 == 0 && KV_STAGE % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 };
 
 struct TcParams {
@@ -163,16 +179,337 @@ template <> __device__ __forceinline__ void unpack8<f16>(const uint4 &u, float (
     }
 }
 
+// phi on a packed pair of bf16 values: phi(x) = max(x, 0) + e^(min(x, 0))
+// (x + 1 for x > 0, e^x for x <= 0).  min/max/add run on the pair; e^m is
+// taken as 2^(m log2 e) on the fp32 ex2 unit (measured faster here than the
+// packed bf16x2 ex2) and rounded once to bf16.  For x > 0 the result is
+// x + 1 rounded once to bf16.
+__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x2) {
+    uint32_t m, pz, r;
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(x2), "r"(0u));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(pz) : "r"(x2), "r"(0u));
+    const float e0 = ex2_approx(__uint_as_float(m << 16) * kLog2e);
+    const float e1 = ex2_approx(__uint_as_float(m & 0xFFFF0000u) * kLog2e);
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(pz), "r"(pack_bf16x2(e0, e1)));
+    return r;
+}
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint4 phi_bf16x8(const uint4 &u) {
+    return make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w));
+}
+
 __device__ __forceinline__ uint4 pack8_bf16(const float (&x)[8]) {
     return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                       pack_bf16x2(x[6], x[7]));
+}
+
+
+// S row `a` (32 fp32 values from column col0) -> the bf16 MN-major operand
+// [D/64 column blocks][D rows][128 bytes], 128-byte swizzled.
+template <int D>
+__device__ __forceinline__ void write_state_row(uint8_t *sbf, int a, int col0, const float (&vals)[32]) {
+    uint8_t *blk = sbf + (col0 / 64) * (D * 128);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = vals[8 * m + e];
+        *reinterpret_cast<uint4 *>(blk + sw128_off(a, ((col0 % 64) / 8) + m)) = pack8_bf16(x);
+    }
+}
+
+// phi applied in place to a staged [C][D] tile (KB boxes of [C][128 B]),
+// rows >= n zeroed.  With DECAY, w_j phi(k_j) is also written to `kw`
+// (w_j = exp(L_end - L_j)); with FP16 inputs the V tile is converted to bf16.
+// Thread tw (0..127) owns one 16-byte column chunk of one box on every PH-th
+// row; with PH a multiple of 8 its swizzled chunk position is the same on
+// all its rows, and all loads of a batch are issued before any arithmetic.
+// The tile's rows are split into NPART equal parts; this call does part PART
+// (the two warpgroups each take one part of the key tile).
+// When ZSUM, zp[e] accumulates this thread's column sums of the operand the
+// state update uses (w o phi(K) with decay, phi(K) without), for its 8 columns.
+template <typename InT, int C, int D, bool DECAY, bool CONVERT_V, int PB = 0, int PE = 1, int NPART = 1,
+          bool ZSUM = false>
+__device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *kw, uint8_t *vt, int tw, int n,
+                                         const float *L, float Lend, float (&zp)[8]) {
+    constexpr int KB = D / 64, BOXB = C * 128;
+    constexpr int PH = 128 / (8 * KB);
+    constexpr int NIT = C / PH;
+    constexpr int IPART = NIT / NPART;
+    constexpr int BATCH = IPART < 8 ? IPART : 8;
+    static_assert(NIT % NPART == 0 && IPART % BATCH == 0, "row split");
+    const int lc = tw & 7, b = (tw >> 3) % KB, ph = tw / (8 * KB);
+    const uint32_t base = b * BOXB + ph * 128 + ((lc ^ (ph & 7)) << 4);
+#pragma unroll 1
+    for (int i0 = PB * IPART; i0 < PE * IPART; i0 += BATCH) {
+        uint4 raw[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) raw[i] = *reinterpret_cast<const uint4 *>(tile + base + (i0 + i) * PH * 128);
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            const int r = ph + (i0 + i) * PH;
+            const uint32_t off = base + (i0 + i) * PH * 128;
+            const bool valid = r < n;
+            uint4 used;   // the bf16 operand of the state update for these 8 columns
+            if constexpr (std::is_same<InT, bf16>::value) {
+                uint4 f = phi_bf16x8(raw[i]);
+                if (!valid) f = make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(tile + off) = f;
+                used = f;
+                if constexpr (DECAY) {
+                    const float w = valid ? ex2_approx(Lend - L[r]) : 0.f;
+                    const uint32_t w2 = pack_bf16x2(w, w);
+                    used = make_uint4(mul_bf16x2(f.x, w2), mul_bf16x2(f.y, w2), mul_bf16x2(f.z, w2),
+                                      mul_bf16x2(f.w, w2));
+                    *reinterpret_cast<uint4 *>(kw + off) = used;
+                }
+            } else {
+                float x[8];
+                unpack8<InT>(raw[i], x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = valid ? phi_fast(x[e]) : 0.f;
+                used = pack8_bf16(x);
+                *reinterpret_cast<uint4 *>(tile + off) = used;
+                if constexpr (DECAY) {
+                    const float w = valid ? ex2_approx(Lend - L[r]) : 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] *= w;
+                    used = pack8_bf16(x);
+                    *reinterpret_cast<uint4 *>(kw + off) = used;
+                }
+            }
+            if constexpr (ZSUM) {
+                const uint32_t uw[4] = {used.x, used.y, used.z, used.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    zp[2 * e] += bf16lo(uw[e]);
+                    zp[2 * e + 1] += bf16hi(uw[e]);
+                }
+            }
+        }
+        if constexpr (CONVERT_V) {
+            uint4 rv[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) rv[i] = *reinterpret_cast<const uint4 *>(vt + base + (i0 + i) * PH * 128);
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                float y[8];
+                unpack8<InT>(rv[i], y);
+                *reinterpret_cast<uint4 *>(vt + base + (i0 + i) * PH * 128) = pack8_bf16(y);
+            }
+        }
+    }
+}
+
+// Column sums of one key part: combine the row phases held by lanes of this
+// warp, then lanes owning a (column-chunk, box) write their 8 sums to
+// red[wslot][col].  Warp-collective.
+template <int D>
+__device__ __forceinline__ void publish_zsum(float (&zp)[8], float *red, int wslot, int tw) {
+    constexpr int KB = D / 64;
+    const int lane = tw & 31;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        zp[e] += __shfl_xor_sync(0xffffffffu, zp[e], 16);
+        if constexpr (KB == 1) zp[e] += __shfl_xor_sync(0xffffffffu, zp[e], 8);
+    }
+    const int owners = 8 * KB;   // lanes 0 .. owners-1 hold distinct column chunks
+    if (lane < owners) {
+        const int lc = lane & 7, b = lane >> 3;
+        float4 *dst = reinterpret_cast<float4 *>(red + wslot * D + b * 64 + lc * 8);
+        dst[0] = make_float4(zp[0], zp[1], zp[2], zp[3]);
+        dst[1] = make_float4(zp[4], zp[5], zp[6], zp[7]);
+    }
+}
+
+// Output mode: publish this chunk's column sums to red[stage].  State-only
+// mode: keep a decayed running sum per thread (zrun <- gamma_c zrun + zp) and
+// publish it after the segment's last chunk.
+template <typename G>
+__device__ __forceinline__ void zsum_update(float (&zp)[8], float (&zrun)[8], float *Fsm, int s,
+                                            int c, int nch, int wslot, int tw) {
+    if constexpr (G::OUT) {
+        publish_zsum<G::D>(zp, Fsm + G::F_RED + (c % G::NRED) * 8 * G::D, wslot, tw);
+    } else {
+        const float g = G::DECAY ? Fsm[G::F_G + s] : 1.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) zrun[e] = fmaf(g, zrun[e], zp[e]);
+        if (c == nch - 1) publish_zsum<G::D>(zrun, Fsm + G::F_RED, wslot, tw);
+    }
+}
+
+// phi of chunk c: decay cumsum (DECAY), K (and w o phi(K)), Q (output mode:
+// into TMEM for C = 128, in place otherwise); then arrives on phi_done.
+// Returns false if the CTA is aborting.
+template <int C, int D, bool DECAY, int MODE, typename InT>
+__device__ __forceinline__ bool phi_stage(uint8_t *smem, uint64_t *bar, float *Fsm, const AbortCtx ab,
+                                       const TcParams &p, uint32_t tmem, long t_begin, long t_end,
+                                       int bh, int c, int nch, int tw, float &Aseg, float (&zrun)[8]) {
+    using G = Cfg<C, D, DECAY, MODE>;
+    const int lane = tw & 31, q = (kPhiWarp0 + (tw >> 5)) & 3;
+    const int s = c % G::NKV;
+    const long t0 = t_begin + (long)c * C;
+    const int n = (int)min((long)C, t_end - t0);
+    if (!mbar_wait(&bar[G::B_KV_FULL + s], (c / G::NKV) & 1, ab, 8)) return false;
+    float *L = Fsm + G::F_L + s * C;
+    if constexpr (DECAY) {
+        if (tw < 32) {
+            const float *a = p.decay + (size_t)bh * p.T + t0;
+            float carry = 0.f;
+#pragma unroll
+            for (int j0 = 0; j0 < C; j0 += 32) {
+                const int j = j0 + lane;
+                float x = (j < n) ? lg2_approx(a[j]) : 0.f;   // log2 units
+                x = warp_sum_scan(x, lane) + carry;
+                L[j] = x;   // rows >= n repeat the chunk total (never used)
+                carry = __shfl_sync(0xffffffffu, x, 31);
+            }
+            if (lane == 0) {
+                const float g = ex2_approx(carry);
+                Fsm[G::F_G + s] = g;
+                Aseg *= g;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[G::B_L_READY + s]);   // for the other warpgroup
+        }
+        named_bar_sync(1, 128);
+    }
+    uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
+    constexpr bool CONV = !std::is_same<InT, bf16>::value;
+    // the first parts of the key rows; the epilogue warpgroup takes the rest
+    float zp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    phi_tile<InT, C, D, DECAY, CONV, 0, G::KSPLIT, 4, true>(kt, kt + 2 * G::TILE, kt + G::TILE, tw, n, L,
+                                                           DECAY ? L[n - 1] : 0.f, zp);
+    zsum_update<G>(zp, zrun, Fsm, s, c, nch, tw >> 5, tw);
+    if constexpr (G::OUT) {
+        const int sq = G::QT ? 0 : (c & 1);
+        const int use = G::QT ? c : (c >> 1);
+        if (!mbar_wait(&bar[G::B_Q_FULL + sq], use & 1, ab, 9)) return false;
+        uint8_t *qs = smem + G::OFF_Q + sq * G::TILE;
+        if constexpr (G::QT) {
+            // row r = 32q + lane: phi(q_r) as bf16 pairs -> TMEM (A operand),
+            // one 64-column box (32 TMEM columns) at a time
+            const int r = q * 32 + lane;
+            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+            constexpr int NBQ = G::QSPLIT ? 1 : G::KB;   // boxes formed here
+#pragma unroll 1
+            for (int b = 0; b < NBQ; ++b) {
+                uint4 raw[8];
+#pragma unroll
+                for (int lc = 0; lc < 8; ++lc)
+                    raw[lc] = *reinterpret_cast<const uint4 *>(qs + b * G::BOXB + sw128_off(r, lc));
+                uint32_t packed[32];
+#pragma unroll
+                for (int lc = 0; lc < 8; ++lc) {
+                    if constexpr (std::is_same<InT, bf16>::value) {
+                        const uint4 f = phi_bf16x8(raw[lc]);
+                        packed[lc * 4 + 0] = f.x;
+                        packed[lc * 4 + 1] = f.y;
+                        packed[lc * 4 + 2] = f.z;
+                        packed[lc * 4 + 3] = f.w;
+                    } else {
+                        float x[8];
+                        unpack8<InT>(raw[lc], x);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            packed[lc * 4 + e] = pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
+                    }
+                }
+                if (b == NBQ - 1) {
+                    // this warpgroup's reads of the raw Q slot are done
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar[G::B_Q_EMPTY]);
+                }
+                if (b == 0) {
+                    if (c > 0 && !mbar_wait(&bar[G::B_QT_EMPTY], (c - 1) & 1, ab, 10)) return false;
+                    tc_fence_after();
+                }
+                tmem_st32(tmem + lane_base + G::T_Q + b * 32, packed);
+            }
+            tmem_st_wait();
+        } else {
+            float unused[8];
+            phi_tile<InT, C, D, false, false>(qs, nullptr, nullptr, tw, C, nullptr, 0.f, unused);
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
+    return true;
+}
+
+// Second half of the key rows of chunk c, done by the epilogue warpgroup
+// (thread index et = 0..127); arrives on phi_done.  False if aborting.
+template <int C, int D, bool DECAY, int MODE, typename InT>
+__device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *bar, float *Fsm,
+                                                     const AbortCtx ab, uint32_t tmem, long t_begin,
+                                                     long t_end, int c, int nch, int et,
+                                                     float (&zrun)[8]) {
+    using G = Cfg<C, D, DECAY, MODE>;
+    const int s = c % G::NKV;
+    const long t0 = t_begin + (long)c * C;
+    const int n = (int)min((long)C, t_end - t0);
+    if (!mbar_wait(&bar[G::B_KV_FULL + s], (c / G::NKV) & 1, ab, 15)) return false;
+    const float *L = Fsm + G::F_L + s * C;
+    if constexpr (DECAY)
+        if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 16)) return false;
+    uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
+    constexpr bool CONV = !std::is_same<InT, bf16>::value;
+    float zp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    phi_tile<InT, C, D, DECAY, CONV, G::KSPLIT, 4, 4, true>(kt, kt + 2 * G::TILE, kt + G::TILE, et, n, L,
+                                                           DECAY ? L[n - 1] : 0.f, zp);
+    zsum_update<G>(zp, zrun, Fsm, s, c, nch, 4 + (et >> 5), et);
+    if constexpr (G::QSPLIT) {
+        // second column box of phi(Q) for rows 32q + lane -> TMEM
+        const int lane = et & 31, q = et >> 5;
+        if (!mbar_wait(&bar[G::B_Q_FULL], c & 1, ab, 18)) return false;
+        const uint8_t *qs = smem + G::OFF_Q + G::BOXB;
+        const int r = q * 32 + lane;
+        uint4 raw[8];
+#pragma unroll
+        for (int lc = 0; lc < 8; ++lc) raw[lc] = *reinterpret_cast<const uint4 *>(qs + sw128_off(r, lc));
+        uint32_t packed[32];
+#pragma unroll
+        for (int lc = 0; lc < 8; ++lc) {
+            if constexpr (std::is_same<InT, bf16>::value) {
+                const uint4 f = phi_bf16x8(raw[lc]);
+                packed[lc * 4 + 0] = f.x;
+                packed[lc * 4 + 1] = f.y;
+                packed[lc * 4 + 2] = f.z;
+                packed[lc * 4 + 3] = f.w;
+            } else {
+                float x[8];
+                unpack8<InT>(raw[lc], x);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    packed[lc * 4 + e] = pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[G::B_Q_EMPTY]);
+        if (c > 0 && !mbar_wait(&bar[G::B_QT_EMPTY], (c - 1) & 1, ab, 19)) return false;
+        tc_fence_after();
+        tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + G::T_Q + 32, packed);
+        tmem_st_wait();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if ((et & 31) == 0) mbar_arrive(&bar[G::B_PHI + s]);
+    return true;
 }
 
 // ---------------------------------------------------------------------------
 template <int C, int D, bool DECAY, int MODE, typename InT, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, TcParams p) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  TcParams p) {
     using G = Cfg<C, D, DECAY, MODE>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -194,11 +531,12 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int s = 0; s < G::NKV; ++s) {
             mbar_init(&bar[G::B_KV_FULL + s], 1);
             mbar_init(&bar[G::B_KV_EMPTY + s], 1);
-            mbar_init(&bar[G::B_PHI + s], 4);
+            mbar_init(&bar[G::B_PHI + s], 8);   // 4 phi warps + 4 epilogue warps
+            mbar_init(&bar[G::B_L_READY + s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar[G::B_Q_FULL + s], 1);
-            mbar_init(&bar[G::B_Q_EMPTY + s], G::QT ? 4 : 1);
+            mbar_init(&bar[G::B_Q_EMPTY + s], G::QT ? (G::QSPLIT ? 8 : 4) : 1);
         }
         mbar_init(&bar[G::B_QT_EMPTY], 1);
         mbar_init(&bar[G::B_SC_FULL], 1);
@@ -211,10 +549,8 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(&bar[G::B_DRAIN], 1);
         fence_mbar_init();
     }
-    // constant operands: all-ones [16][C] and (OUT) a zeroed z operand [16][D]
+    // (output mode) the z operand [16][D] starts zeroed: only its row 0 is used
     {
-        uint32_t *ones = reinterpret_cast<uint32_t *>(smem + G::OFF_ONES);
-        for (int i = threadIdx.x; i < G::ONES / 4; i += kThreads) ones[i] = 0x3F803F80u;
         if constexpr (G::OUT) {
             uint32_t *zb = reinterpret_cast<uint32_t *>(smem + G::OFF_ZB);
             for (int i = threadIdx.x; i < G::ZB / 4; i += kThreads) zb[i] = 0u;
@@ -223,7 +559,10 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_addr_smem, G::TMEM_COLS);
     if (warp == kTmaWarp && lane == 0) {
-        if constexpr (G::OUT) prefetch_tmap(&tm_q);
+        if constexpr (G::OUT) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_o);
+        }
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
     }
@@ -281,50 +620,53 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             constexpr uint32_t ID_INT = idesc_bf16(C, D, false, true);
             constexpr uint32_t ID_DEN = idesc_bf16(C, 16, false, false);
             constexpr uint32_t ID_DS = idesc_bf16(D, D, true, true);
-            constexpr uint32_t ID_DZ = idesc_bf16(D, 16, true, false);
             constexpr uint32_t ID_PV = idesc_bf16(C, D, false, true);
             const uint32_t sb = smem_u32(smem);
+            // Base descriptors; a K-step advances the start address field
+            // (address >> 4 in the low 14 bits, which never carries here:
+            // shared memory is < 256 KB), so descriptor + (offset >> 4).
+            auto nosw = [](uint32_t addr, uint32_t sbo) -> uint64_t {   // no-swizzle K-major
+                return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) |
+                       ((uint64_t)(sbo >> 4) << 32) | (1ull << 46);
+            };
+            const uint64_t dS0 = sdesc_sw128(sb + G::OFF_SBF, D * 128, 1024);   // S (MN-major)
+            const uint64_t dZ0 = nosw(sb + G::OFF_ZB, (D / 8) * 128);           // z [16][D]
+            const uint64_t dP0 = sdesc_sw128(sb + G::OFF_P, 16, 1024);          // P (K-major, smem)
             for (int c = 0; c < nch; ++c) {
                 const int s = c % G::NKV;
                 const uint32_t kt = sb + G::OFF_KV + s * G::KV_STAGE;   // phi(K)
-                const uint32_t vt = kt + G::TILE;                        // V
-                const uint32_t at = DECAY ? kt + 2 * G::TILE : kt;       // state-update A operand
+                const uint64_t dKk = sdesc_sw128(kt, 16, 1024);                        // phi(K), K-major
+                const uint64_t dKm = sdesc_sw128(DECAY ? kt + 2 * G::TILE : kt, G::BOXB, 1024);  // MN-major
+                const uint64_t dVm = sdesc_sw128(kt + G::TILE, G::BOXB, 1024);         // V, MN-major
                 if (!mbar_wait(&bar[G::B_PHI + s], (c / G::NKV) & 1, ab, 3)) break;
                 tc_fence_after();
                 if constexpr (G::OUT) {
-                    const uint32_t qt = sb + G::OFF_Q + (G::QT ? 0 : (c & 1)) * G::TILE;  // phi(Q) (smem)
+                    const uint64_t dQk = sdesc_sw128(sb + G::OFF_Q + (G::QT ? 0 : (c & 1)) * G::TILE, 16, 1024);
                     // MMA1: scores = phi(Q) phi(K)^T (scores buffer free once MMA4 of c-1 is done)
                     if (c > 0 && !mbar_wait(&bar[G::B_MMA4], (c - 1) & 1, ab, 4)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t koff = (kk >> 2) * G::BOXB + (kk & 3) * 32;
-                        const uint64_t bdesc = sdesc_sw128(kt + koff, 16, 1024);
+                        const uint32_t koff = ((kk >> 2) * G::BOXB + (kk & 3) * 32) >> 4;
                         if constexpr (G::QT)
-                            mma_ts(tmem + G::T_SC, tmem + G::T_Q + kk * 8, bdesc, ID_SC, kk > 0);
+                            mma_ts(tmem + G::T_SC, tmem + G::T_Q + kk * 8, dKk + koff, ID_SC, kk > 0);
                         else
-                            mma_ss(tmem + G::T_SC, sdesc_sw128(qt + koff, 16, 1024), bdesc, ID_SC, kk > 0);
+                            mma_ss(tmem + G::T_SC, dQk + koff, dKk + koff, ID_SC, kk > 0);
                     }
                     mma_commit(&bar[G::B_SC_FULL]);
                     // MMA2 + MMAd: inter term and its denominator with the state entering c
                     if (!mbar_wait(&bar[G::B_S_READY], c & 1, ab, 5)) break;
                     if (c > 0 && !mbar_wait(&bar[G::B_O_EMPTY], (c - 1) & 1, ab, 6)) break;
                     tc_fence_after();
-                    const uint32_t sbf = sb + G::OFF_SBF, zb = sb + G::OFF_ZB;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t bS = sdesc_sw128(sbf + kk * 2048, D * 128, 1024);
-                        const uint64_t bZ = [&] {
-                            const uint32_t a = zb + kk * 256;
-                            return (uint64_t)((a >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) |
-                                   ((uint64_t)(((D / 8) * 128) >> 4) << 32) | (1ull << 46);
-                        }();
+                        const uint64_t bS = dS0 + (uint64_t)((kk * 2048) >> 4);
+                        const uint64_t bZ = dZ0 + (uint64_t)((kk * 256) >> 4);
                         if constexpr (G::QT) {
                             mma_ts(tmem + G::T_O, tmem + G::T_Q + kk * 8, bS, ID_INT, kk > 0);
                             mma_ts(tmem + G::T_DEN, tmem + G::T_Q + kk * 8, bZ, ID_DEN, kk > 0);
                         } else {
-                            const uint32_t koff = (kk >> 2) * G::BOXB + (kk & 3) * 32;
-                            const uint64_t aQ = sdesc_sw128(qt + koff, 16, 1024);
+                            const uint64_t aQ = dQk + (uint64_t)(((kk >> 2) * G::BOXB + (kk & 3) * 32) >> 4);
                             mma_ss(tmem + G::T_O, aQ, bS, ID_INT, kk > 0);
                             mma_ss(tmem + G::T_DEN, aQ, bZ, ID_DEN, kk > 0);
                         }
@@ -335,31 +677,27 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if ((c == 0 || DECAY) && !mbar_wait(&bar[G::B_S_READY], c & 1, ab, 5)) break;
                     tc_fence_after();
                 }
-                // MMA3 + MMAz: state update with this chunk's keys and values
+                // MMA3: state update with this chunk's keys and values (z is summed
+                // on the CUDA cores while phi(K) is formed)
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk) {
-                    const uint64_t aK = sdesc_sw128(at + kk * 2048, G::BOXB, 1024);
-                    const uint64_t bV = sdesc_sw128(vt + kk * 2048, G::BOXB, 1024);
-                    const uint32_t oa = sb + G::OFF_ONES + kk * 256;
-                    const uint64_t b1 = (uint64_t)((oa >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) |
-                                        ((uint64_t)(((C / 8) * 128) >> 4) << 32) | (1ull << 46);
-                    mma_ss(tmem + G::T_S, aK, bV, ID_DS, 1);
-                    mma_ss(tmem + G::T_Z, aK, b1, ID_DZ, 1);
-                }
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_ss(tmem + G::T_S, dKm + (uint64_t)((kk * 2048) >> 4),
+                           dVm + (uint64_t)((kk * 2048) >> 4), ID_DS, 1);
                 if (G::OUT || DECAY || c == nch - 1) mma_commit(&bar[G::B_DS_FULL]);
                 if constexpr (G::OUT) {
                     // MMA4: exact intra-chunk product with the masked, decayed scores
                     if (!mbar_wait(&bar[G::B_P_READY], c & 1, ab, 7)) break;
                     tc_fence_after();
+                    // O (+)= P V
                     const uint32_t dst = tmem + (G::SPLIT ? G::T_O2 : G::T_O);
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk) {
-                        const uint64_t bV = sdesc_sw128(vt + kk * 2048, G::BOXB, 1024);
+                        const uint64_t bV = dVm + (uint64_t)((kk * 2048) >> 4);
+                        const uint32_t acc = G::SPLIT ? (kk > 0) : 1;
                         if constexpr (G::PT)
-                            mma_ts(dst, tmem + G::T_SC + kk * 8, bV, ID_PV, G::SPLIT ? (kk > 0) : 1);
+                            mma_ts(dst, tmem + G::T_SC + kk * 8, bV, ID_PV, acc);
                         else
-                            mma_ss(dst, sdesc_sw128(sb + G::OFF_P + kk * 32, 16, 1024), bV, ID_PV,
-                                   G::SPLIT ? (kk > 0) : 1);
+                            mma_ss(dst, dP0 + (uint64_t)((kk * 32) >> 4), bV, ID_PV, acc);
                     }
                     mma_commit(&bar[G::B_MMA4]);
                     mma_commit(&bar[G::B_O_FULL]);
@@ -378,117 +716,8 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int q = warp & 3;                              // TMEM lane quarter
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         float Aseg = 1.f;  // product of chunk decays (state-only mode)
+        float zrun[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // running column sums (state-only)
         bool ok = true;
-
-        // phi on one staged chunk; returns false on abort
-        auto phi_chunk = [&](int c) -> bool {
-            const int s = c % G::NKV;
-            const long t0 = t_begin + (long)c * C;
-            const int n = (int)min((long)C, t_end - t0);
-            if (!mbar_wait(&bar[G::B_KV_FULL + s], (c / G::NKV) & 1, ab, 8)) return false;
-            float *L = Fsm + G::F_L + s * C;
-            if constexpr (DECAY) {
-                if (tw < 32) {
-                    const float *a = p.decay + (size_t)bh * p.T + t0;
-                    float carry = 0.f;
-                    for (int j0 = 0; j0 < C; j0 += 32) {
-                        const int j = j0 + lane;
-                        float x = (j < n) ? logf(a[j]) : 0.f;
-                        x = warp_sum_scan(x, lane) + carry;
-                        L[j] = x;   // rows >= n repeat the chunk total (never used)
-                        carry = __shfl_sync(0xffffffffu, x, 31);
-                    }
-                    if (lane == 0) {
-                        const float g = expf(carry);
-                        Fsm[G::F_G + s] = g;
-                        Aseg *= g;
-                    }
-                }
-                named_bar_sync(1, 128);
-            }
-            uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
-            // K: phi in place (rows >= n zeroed); with decay also w o phi(K)
-            {
-                const int lc = tw & 7;
-                constexpr int PH = 128 / (8 * G::KB);
-                const int b = (tw >> 3) % G::KB, ph = tw / (8 * G::KB);
-                const float Lend = DECAY ? L[n - 1] : 0.f;
-                for (int r = ph; r < C; r += PH) {
-                    const uint32_t off = b * G::BOXB + sw128_off(r, lc);
-                    uint4 *src = reinterpret_cast<uint4 *>(kt + off);
-                    float x[8];
-                    unpack8<InT>(*src, x);
-                    const bool valid = r < n;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = valid ? phi_fast(x[e]) : 0.f;
-                    *src = pack8_bf16(x);
-                    if constexpr (DECAY) {
-                        const float w = valid ? __expf(Lend - L[r]) : 0.f;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] *= w;
-                        *reinterpret_cast<uint4 *>(kt + 2 * G::TILE + off) = pack8_bf16(x);
-                    }
-                    if constexpr (sizeof(InT) == 2 && !std::is_same<InT, bf16>::value) {
-                        // fp16 values -> bf16 operands
-                        uint4 *vs = reinterpret_cast<uint4 *>(kt + G::TILE + off);
-                        float y[8];
-                        unpack8<InT>(*vs, y);
-                        *vs = pack8_bf16(y);
-                    }
-                }
-            }
-            if constexpr (G::OUT) {
-                const int sq = G::QT ? 0 : (c & 1);
-                const int use = G::QT ? c : (c >> 1);
-                if (!mbar_wait(&bar[G::B_Q_FULL + sq], use & 1, ab, 9)) return false;
-                uint8_t *qs = smem + G::OFF_Q + sq * G::TILE;
-                if constexpr (G::QT) {
-                    // row i = 32q + lane: phi(q_i) -> TMEM (A operand, bf16 pairs)
-                    if (c > 0 && !mbar_wait(&bar[G::B_QT_EMPTY], (c - 1) & 1, ab, 10)) return false;
-                    tc_fence_after();
-                    const int r = q * 32 + lane;
-                    uint32_t packed[D / 2];
-#pragma unroll
-                    for (int b = 0; b < G::KB; ++b)
-#pragma unroll
-                        for (int lc = 0; lc < 8; ++lc) {
-                            float x[8];
-                            unpack8<InT>(*reinterpret_cast<const uint4 *>(qs + b * G::BOXB + sw128_off(r, lc)), x);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                packed[b * 32 + lc * 4 + e] = pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
-                        }
-                    // raw Q slot may be refilled
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar[G::B_Q_EMPTY]);
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h) {
-                        uint32_t chunk32[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) chunk32[i] = packed[h * 32 + i];
-                        tmem_st32(tmem + lane_base + G::T_Q + h * 32, chunk32);
-                    }
-                    tmem_st_wait();
-                } else {
-                    const int lc = tw & 7;
-                    constexpr int PH = 128 / (8 * G::KB);
-                    const int b = (tw >> 3) % G::KB, ph = tw / (8 * G::KB);
-                    for (int r = ph; r < C; r += PH) {
-                        uint4 *src = reinterpret_cast<uint4 *>(qs + b * G::BOXB + sw128_off(r, lc));
-                        float x[8];
-                        unpack8<InT>(*src, x);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = phi_fast(x[e]);
-                        *src = pack8_bf16(x);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
-            return true;
-        };
 
         // state rows owned by this thread: TMEM lane quarter q, rows of the
         // M = D accumulator (D = 64: lanes 0-15 of each quarter)
@@ -496,28 +725,17 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const bool srow_ok = lane < SROWS;
         const int a_row = q * SROWS + lane;   // state row (feature index)
 
-        auto write_state_operands = [&](const float *srow, int col0, float zval) {
-            // S row a (32 values from column col0) -> bf16 MN-major operand
-            uint8_t *sbf = smem + G::OFF_SBF + (col0 / 64) * (D * 128);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = srow[8 * m + e];
-                const int lcol = ((col0 % 64) / 8) + m;
-                *reinterpret_cast<uint4 *>(sbf + sw128_off(a_row, lcol)) = pack8_bf16(x);
-            }
-            (void)zval;
-        };
-
-        if (nch > 0) ok = phi_chunk(0);
+        if (nch > 0)
+            ok = phi_stage<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, p, tmem, t_begin, t_end, bh, 0, nch,
+                                                   tw, Aseg, zrun);
+        float zreg = 0.f;   // z of this thread's state row (output mode)
         // ---- segment start: state entering the segment -> TMEM (and operands)
         if (ok) {
             tc_fence_after();
             const float g0 = DECAY ? Fsm[G::F_G + 0] : 1.f;
             const float *st = p.ws_state + ((size_t)bh * p.n_seg + seg) * (D * D + D);
             {
-#pragma unroll
+#pragma unroll 1
                 for (int cb = 0; cb < D / 32; ++cb) {
                     float vals[32];
                     uint32_t u[32];
@@ -527,17 +745,10 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         u[i] = __float_as_uint(vals[i] * g0);
                     }
                     tmem_st32(tmem + lane_base + G::T_S + cb * 32, u);
-                    if constexpr (G::OUT) if (srow_ok) write_state_operands(vals, cb * 32, 0.f);
+                    if constexpr (G::OUT) if (srow_ok) write_state_row<D>(smem + G::OFF_SBF, a_row, cb * 32, vals);
                 }
                 const float zin = (G::OUT && srow_ok) ? st[(size_t)D * D + a_row] : 0.f;
-                uint32_t uz[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) uz[i] = __float_as_uint(zin * g0);
-                asm volatile(
-                    "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-                    ::"r"(tmem + lane_base + G::T_Z), "r"(uz[0]), "r"(uz[1]), "r"(uz[2]), "r"(uz[3]), "r"(uz[4]),
-                      "r"(uz[5]), "r"(uz[6]), "r"(uz[7]), "r"(uz[8]), "r"(uz[9]), "r"(uz[10]), "r"(uz[11]),
-                      "r"(uz[12]), "r"(uz[13]), "r"(uz[14]), "r"(uz[15]) : "memory");
+                zreg = zin;
                 if constexpr (G::OUT) {
                     if (srow_ok) {
                         // z operand: row n = 0 of the [16][D] K-major no-swizzle layout
@@ -554,17 +765,23 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
 
         for (int c = 0; ok && c < nch; ++c) {
-            if (c + 1 < nch) { if (!(ok = phi_chunk(c + 1))) break; }
+            if (c + 1 < nch) {
+                ok = phi_stage<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, p, tmem, t_begin, t_end, bh, c + 1,
+                                                       nch, tw, Aseg, zrun);
+                if (!ok) break;
+            }
             const bool need = G::OUT || DECAY || c == nch - 1;
             if (!need) continue;
             if (!mbar_wait(&bar[G::B_DS_FULL], (G::OUT || DECAY) ? (c & 1) : 0, ab, 11)) { ok = false; break; }
+            // the column sums of chunk c are published before phi_done(c)
+            if (!mbar_wait(&bar[G::B_PHI + (c % G::NKV)], (c / G::NKV) & 1, ab, 17)) { ok = false; break; }
             tc_fence_after();
             const bool last = c == nch - 1;
             const float gnext = (DECAY && !last) ? Fsm[G::F_G + ((c + 1) % G::NKV)] : 1.f;
             if (last && !G::OUT) {
                 // state-only mode: write the segment's (dS, dz, A) to the workspace
                 float *dst = p.ws_state + ((size_t)bh * p.n_seg + seg) * (D * D + D);
-#pragma unroll
+#pragma unroll 1
                 for (int cb = 0; cb < D / 32; ++cb) {
                     uint32_t u[32];
                     tmem_ld32(tmem + lane_base + G::T_S + cb * 32, u);
@@ -577,16 +794,19 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                                 __uint_as_float(u[4 * i + 2]), __uint_as_float(u[4 * i + 3]));
                     }
                 }
-                uint32_t u[32];
-                tmem_ld32(tmem + lane_base + G::T_Z, u);
-                tmem_ld_wait();
-                if (srow_ok) dst[(size_t)D * D + a_row] = __uint_as_float(u[0]);
+                if (srow_ok) {
+                    const float *red = Fsm + G::F_RED;
+                    float zs = 0.f;
+#pragma unroll
+                    for (int w8 = 0; w8 < 8; ++w8) zs += red[w8 * D + a_row];
+                    dst[(size_t)D * D + a_row] = zs;
+                }
                 if (tw == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = Aseg;
                 break;
             }
             if (last && G::OUT) break;   // the final state of a segment is produced by the scan
             // state entering chunk c+1: bf16 operands, and (decay) rescale in TMEM
-#pragma unroll
+#pragma unroll 1
             for (int cb = 0; cb < D / 32; ++cb) {
                 uint32_t u[32];
                 tmem_ld32(tmem + lane_base + G::T_S + cb * 32, u);
@@ -594,33 +814,23 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 float vals[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) vals[i] = __uint_as_float(u[i]);
-                if constexpr (G::OUT) if (srow_ok) write_state_operands(vals, cb * 32, 0.f);
+                if constexpr (G::OUT) if (srow_ok) write_state_row<D>(smem + G::OFF_SBF, a_row, cb * 32, vals);
                 if constexpr (DECAY) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(vals[i] * gnext);
                     tmem_st32(tmem + lane_base + G::T_S + cb * 32, u);
                 }
             }
-            {
-                uint32_t u[32];
-                tmem_ld32(tmem + lane_base + G::T_Z, u);
-                tmem_ld_wait();
-                const float zc = __uint_as_float(u[0]);
-                if constexpr (G::OUT) {
-                    if (srow_ok) {
-                        bf16 *zb = reinterpret_cast<bf16 *>(smem + G::OFF_ZB);
-                        zb[(a_row / 8) * 64 + (a_row % 8)] = __float2bfloat16_rn(zc);
-                    }
-                }
-                if constexpr (DECAY) {
-                    uint32_t uz[16];
+            if constexpr (G::OUT) {
+                // z after chunk c: z <- gamma_c z + (column sums of w o phi(K) over the chunk)
+                if (srow_ok) {
+                    const float *red = Fsm + G::F_RED + (c % G::NRED) * 8 * D;
+                    float dz = 0.f;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) uz[i] = __float_as_uint(zc * gnext);
-                    asm volatile(
-                        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-                        ::"r"(tmem + lane_base + G::T_Z), "r"(uz[0]), "r"(uz[1]), "r"(uz[2]), "r"(uz[3]), "r"(uz[4]),
-                          "r"(uz[5]), "r"(uz[6]), "r"(uz[7]), "r"(uz[8]), "r"(uz[9]), "r"(uz[10]), "r"(uz[11]),
-                          "r"(uz[12]), "r"(uz[13]), "r"(uz[14]), "r"(uz[15]) : "memory");
+                    for (int w8 = 0; w8 < 8; ++w8) dz += red[w8 * D + a_row];
+                    zreg = fmaf(DECAY ? Fsm[G::F_G + (c % G::NKV)] : 1.f, zreg, dz);
+                    bf16 *zb = reinterpret_cast<bf16 *>(smem + G::OFF_ZB);
+                    zb[(a_row / 8) * 64 + (a_row % 8)] = __float2bfloat16_rn(zreg);
                 }
             }
             if constexpr (DECAY) tmem_st_wait();
@@ -629,14 +839,23 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_S_READY]);
         }
-    } else if constexpr (G::OUT) {
+    } else if constexpr (!G::OUT) {
+        // ================= warps 0-3 in state-only mode: second half of phi(K)
+        float zrun[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < nch; ++c)
+            if (!phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, tmem, t_begin, t_end, c, nch,
+                                                              threadIdx.x, zrun))
+                break;
+    } else {
         // ================= epilogue (warps 0-3)
         const int q = warp;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const bool rvalid_lane = lane < G::ROWS_PER_WARP;
         const int i = q * G::ROWS_PER_WARP + lane;   // row of the chunk held by this thread
-        OutT *O = reinterpret_cast<OutT *>(p.out) + (size_t)bh * p.T * D;
-        for (int c = 0; c < nch; ++c) {
+        float zrun[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // unused in output mode
+        bool eok = nch == 0 || phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, tmem, t_begin,
+                                                                             t_end, 0, nch, threadIdx.x, zrun);
+        for (int c = 0; eok && c < nch; ++c) {
             const int s = c % G::NKV;
             const long t0 = t_begin + (long)c * C;
             const int n = (int)min((long)C, t_end - t0);
@@ -645,34 +864,51 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_after();
             const float *L = Fsm + G::F_L + s * C;
             const float Li = (DECAY && rvalid_lane) ? L[min(i, C - 1)] : 0.f;
+            // scores -> P, two 32-column blocks per TMEM round trip.  For this
+            // warp's rows [r0, r0 + R) a block lies fully below the diagonal
+            // (no mask), fully above it (P = 0, scores not read) or on it.
+            // The row sums of P are formed by an MMA (P times ones).
+            const int r0 = q * G::ROWS_PER_WARP, r1 = r0 + G::ROWS_PER_WARP - 1;
             float rowsum = 0.f;
+#pragma unroll 1
+            for (int cb0 = 0; cb0 < C / 32; cb0 += 2) {
+                uint32_t u[2][32];
+                bool live[2];
 #pragma unroll
-            for (int cb = 0; cb < C / 32; ++cb) {
-                uint32_t u[32];
-                tmem_ld32(tmem + lane_base + G::T_SC + cb * 32, u);
-                tmem_ld_wait();
-                float pv[32];
-#pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int j = cb * 32 + k;
-                    float v = (j <= i) ? __uint_as_float(u[k]) : 0.f;
-                    if constexpr (DECAY) v = (j <= i) ? v * __expf(Li - L[j]) : 0.f;
-                    pv[k] = v;
-                    rowsum += v;
+                for (int h = 0; h < 2; ++h) {
+                    live[h] = (cb0 + h) * 32 <= r1;
+                    if (live[h]) tmem_ld32(tmem + lane_base + G::T_SC + (cb0 + h) * 32, u[h]);
                 }
-                if constexpr (G::PT) {
+                tmem_ld_wait();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int cb = cb0 + h;
                     uint32_t pk[16];
+                    if (!live[h]) {
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(pv[2 * k], pv[2 * k + 1]);
-                    tmem_st16(tmem + lane_base + G::T_SC + cb * 16, pk);
-                } else if (rvalid_lane) {
-                    uint8_t *pr = smem + G::OFF_P;
+                        for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                    } else {
+                        const bool full = cb * 32 + 31 < r0;   // every j < every row of the warp
+                        float pv[32];
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        float x[8];
+                        for (int k = 0; k < 32; ++k) {
+                            const int j = cb * 32 + k;
+                            float v = __uint_as_float(u[h][k]);
+                            if constexpr (DECAY) v *= ex2_approx(Li - L[j]);
+                            pv[k] = (full || j <= i) ? v : 0.f;
+                            rowsum += pv[k];
+                        }
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = pv[8 * m + e];
-                        *reinterpret_cast<uint4 *>(pr + sw128_off(i, cb * 4 + m)) = pack8_bf16(x);
+                        for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(pv[2 * k], pv[2 * k + 1]);
+                    }
+                    if constexpr (G::PT) {
+                        tmem_st16(tmem + lane_base + G::T_SC + cb * 16, pk);
+                    } else if (rvalid_lane) {
+                        uint8_t *pr = smem + G::OFF_P;
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            *reinterpret_cast<uint4 *>(pr + sw128_off(i, cb * 4 + m)) =
+                                make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
                     }
                 }
             }
@@ -681,37 +917,79 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_P_READY]);
-            const float gi = DECAY ? __expf(Li) : 1.f;
+            const float gi = DECAY ? ex2_approx(Li) : 1.f;
+            // while MMA4 runs: the second half of the next chunk's keys
+            if (c + 1 < nch &&
+                !phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, tmem, t_begin, t_end, c + 1,
+                                                              nch, threadIdx.x, zrun))
+                break;
 
             if (!mbar_wait(&bar[G::B_O_FULL], c & 1, ab, 14)) break;
             tc_fence_after();
-            float den;
-            {
-                uint32_t u[32];
-                tmem_ld32(tmem + lane_base + G::T_DEN, u);   // columns beyond 16 unused
-                tmem_ld_wait();
-                den = gi * __uint_as_float(u[0]) + rowsum + p.eps;
-            }
-            const float inv = 1.f / den;
-            const bool store = rvalid_lane && i < n;
+            // output: one 128-byte-wide column box at a time is scaled, converted,
+            // written swizzled to this warp's staging rows and stored by TMA
+            // (each warp stores its own rows; rows beyond T are clipped)
+            constexpr int CPB = 128 / (int)sizeof(OutT);     // columns per box
+            constexpr int NBOX = D / CPB;
+            uint8_t *stg = smem + G::OFF_STG + q * (G::ROWS_PER_WARP * 128);   // this warp's rows
+            float inv = 0.f;
+#pragma unroll 1
+            for (int bx = 0; bx < NBOX; ++bx) {
+                float o[CPB];
+                {
+                    uint32_t u[CPB], u2[CPB], ud[16];
+                    if (bx == 0) tmem_ld16(tmem + lane_base + G::T_DEN, ud);
 #pragma unroll
-            for (int cb = 0; cb < D / 32; ++cb) {
-                uint32_t u[32];
-                tmem_ld32(tmem + lane_base + G::T_O + cb * 32, u);
-                tmem_ld_wait();
-                float o[32];
-                if constexpr (G::SPLIT) {
-                    uint32_t u2[32];
-                    tmem_ld32(tmem + lane_base + G::T_O2 + cb * 32, u2);
+                    for (int h = 0; h < CPB / 32; ++h) {
+                        tmem_ld32(tmem + lane_base + G::T_O + bx * CPB + h * 32,
+                                  *reinterpret_cast<uint32_t(*)[32]>(&u[h * 32]));
+                        if constexpr (G::SPLIT)
+                            tmem_ld32(tmem + lane_base + G::T_O2 + bx * CPB + h * 32,
+                                      *reinterpret_cast<uint32_t(*)[32]>(&u2[h * 32]));
+                    }
                     tmem_ld_wait();
+                    if (bx == 0) {
+                        // denominator: (decayed) phi(q).z of the carried state + row sum of P + eps
+                        inv = 1.f / (gi * __uint_as_float(ud[0]) + rowsum + p.eps);
+                    }
 #pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        o[k] = (gi * __uint_as_float(u[k]) + __uint_as_float(u2[k])) * inv;
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(u[k]) * inv;
+                    for (int k = 0; k < CPB; ++k) {
+                        if constexpr (G::SPLIT)
+                            o[k] = (gi * __uint_as_float(u[k]) + __uint_as_float(u2[k])) * inv;
+                        else
+                            o[k] = __uint_as_float(u[k]) * inv;
+                    }
                 }
-                if (store) store_row32<OutT>(O + (size_t)(t0 + i) * D + cb * 32, o);
+                // this warp's previous store must have read its staging rows
+                if (lane == 0) bulk_wait_read0();
+                __syncwarp();
+                if (rvalid_lane) {
+                    if constexpr (sizeof(OutT) == 4) {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m)
+                            *reinterpret_cast<float4 *>(stg + sw128_off(lane, m)) =
+                                make_float4(o[4 * m], o[4 * m + 1], o[4 * m + 2], o[4 * m + 3]);
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            float x[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] = o[8 * m + e];
+                            uint4 w;
+                            if constexpr (std::is_same<OutT, bf16>::value) w = pack8_bf16(x);
+                            else
+                                w = make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]),
+                                               pack_f16x2(x[4], x[5]), pack_f16x2(x[6], x[7]));
+                            *reinterpret_cast<uint4 *>(stg + sw128_off(lane, m)) = w;
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&tm_o, stg, bx * CPB, (int)t0 + q * G::ROWS_PER_WARP, bh);
+                    bulk_commit();
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -720,6 +998,9 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
 
     // ---------------- teardown
+    if constexpr (G::OUT) {
+        if (warp < 4 && lane == 0) bulk_wait0();   // output stores complete
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == kMmaWarp) {

@@ -98,12 +98,22 @@ def test_prefill_state_inout_and_split(la, orc):
     assert row_rel_err(o_full, ro) < 2e-2
 
 
-def test_decay_one_matches_no_decay_bitwise(la):
+def test_decay_one_matches_no_decay(la):
+    """Decay 1 is the plain causal form.  On the fp32 CUDA-core path every
+    decay factor is exactly 1 (2^0), so the results are bitwise equal; the
+    tensor-core path keeps separate inter/intra accumulators when a decay is
+    given, so only the fp32 summation order differs."""
+    q, k, v, _ = _small_inputs(torch.float32, 64, 700, False, 1, 2, seed=9)
+    ones = torch.ones((1, 2, 700), dtype=torch.float32)
+    o1, S1, _ = gpu_prefill(la, q, k, v, None, 64, torch.float32)
+    o2, S2, _ = gpu_prefill(la, q, k, v, ones, 64, torch.float32)
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
     q, k, v, _ = _small_inputs(torch.bfloat16, 128, 1000, False, 1, 2, seed=9)
     ones = torch.ones((1, 2, 1000), dtype=torch.float32)
     o1, S1, _ = gpu_prefill(la, q, k, v, None, 64, torch.float32)
     o2, S2, _ = gpu_prefill(la, q, k, v, ones, 64, torch.float32)
-    assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
+    assert row_rel_err(o2, o1) < 1e-4
+    assert row_rel_err(S2.reshape(1, 2, -1), S1.reshape(1, 2, -1)) < 1e-5
 
 
 def test_prefill_deterministic(la):
