@@ -215,6 +215,71 @@ def run_reference(args, w):
     return 0
 
 
+# ------------------------------------------------------------------ per-workload timings
+def time_calls(fn, iters, flush=None):
+    """Mean device time (ms) of fn() over iters calls, CUDA events on the
+    current stream; `flush` (untimed) runs before every call."""
+    import torch
+    st = torch.cuda.current_stream()
+    tot = 0.0
+    for _ in range(iters):
+        if flush is not None:
+            flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        fn()
+        e1.record(st)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    return tot / iters
+
+
+def measure_workloads(dev, peaks, iters=10):
+    """Time every other workload of the hot path once (the per-row numbers
+    beside the headline).  L2 is flushed (a 512 MB write) before each call."""
+    import torch
+    import kernelized_causal_sequence_b200 as la
+    from kernelized_causal_sequence_b200 import inputs
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = lambda: flush_buf.zero_()
+    res = {}
+    for name in ("causal_f32_t256_d64", "causal_bf16_b4h8_t2048_d64", "ssd_decay_bf16_b2h16_t8192_d128"):
+        w = inputs.WORKLOADS[name]
+        q, k, v, a = (None if x is None else x.to(dev) for x in inputs.qkv(w))
+        out = torch.empty((w.B, w.H, w.T, w.d), dtype=w.torch_out_dtype, device=dev)
+        S = torch.zeros((w.B, w.H, w.d, w.d), device=dev)
+        z = torch.zeros((w.B, w.H, w.d), device=dev)
+        ws = torch.empty(max(1, la.la_prefill_workspace_size(w.B, w.H, w.T, w.d, w.d, w.chunk)),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: la.la_prefill_causal(q, k, v, decay=a, eps=w.eps, chunk=w.chunk, state_S=S,
+                                          state_z=z, out=out, workspace=ws)
+        fn()
+        ms = time_calls(fn, iters, flush)
+        b = prefill_algorithmic_bytes(w)
+        res[name] = {"ms": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3), "algorithmic_bytes": b,
+                     "hbm_frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "path": "tcgen05" if la.la_prefill_path(w.torch_dtype, w.d, w.d, w.chunk, w.decay) == 1
+                     else "simt"}
+    w = inputs.WORKLOADS["noncausal_f16_b8h8_l4800_d32"]
+    for cross in (False, True):
+        q, k, v, _ = inputs.qkv(w)
+        if cross:
+            k, v = inputs.cross_kv(w)
+        q, k, v = q.to(dev), k.to(dev), v.to(dev)
+        out = torch.empty((w.B, w.H, w.T, w.d), dtype=w.torch_out_dtype, device=dev)
+        ws = torch.empty(max(1, la.la_noncausal_workspace_size(w.B, w.H, w.Lk, w.d, w.d)),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: la.la_forward_noncausal(q, k, v, eps=w.eps, out=out, workspace=ws)
+        fn()
+        ms = time_calls(fn, iters, flush)
+        b = w.B * w.H * (w.T * w.d * 2 + w.Lk * 2 * w.d * 2 + w.T * w.d * 4)
+        res[w.name + ("_cross" if cross else "_self")] = {
+            "ms": ms, "query_tokens_per_s": w.B * w.T / (ms * 1e-3), "algorithmic_bytes": b,
+            "hbm_frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del flush_buf
+    return res
+
+
 # ------------------------------------------------------------------ GPU leg
 def run_ours(args, w):
     import torch
@@ -391,6 +456,8 @@ def run_ours(args, w):
                          "frac": dbytes / (per_step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                          "note": "fp32 state (67.6 MB) stays L2-resident across the loop"},
         }
+    if rank == 0 and not args.no_workloads:
+        line["workloads"] = measure_workloads(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tok = args.cpu_tokens or w.T
         r, dt, cores = oracle_prefill_sample(w, q_h, k_h, v_h, a_h, tok)
@@ -417,6 +484,8 @@ def main(argv=None):
                     help="tokens per head for the CPU oracle sample (0 = the whole workload)")
     ap.add_argument("--T", type=int, default=0, help="override the workload's sequence length")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-row timings of the other workloads")
     ap.add_argument("--ref-tokens", type=int, default=4096)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,

@@ -10,6 +10,7 @@
 #include "linattn.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "nc32_kernels.cuh"
 #include "errors.h"
 #include "plan.h"
 #include "scan.h"
@@ -143,9 +144,31 @@ la_status dispatch3(la_dtype in, la_dtype out, int D, Args... args) {
 template <typename IT, typename OT, int D> struct SimtCausalF {
     static la_status run(SimtParams p, cudaStream_t st) { return simt_causal<IT, OT, D>(p, st); }
 };
+// Head dim 32: column-per-lane state and read-out kernels (nc32_kernels.cuh).
+template <typename InT, typename OutT>
+la_status nc32_noncausal(SimtParams p, int Lk, cudaStream_t st) {
+    nc32_state_kernel<InT><<<dim3(p.n_seg, p.BH), kNc32Warps * 32, 0, st>>>(
+        (const InT *)p.k, (const InT *)p.v, Lk, p.seg_len, p.n_seg, p.ws_state, p.ws_A);
+    count_launches(1);
+    la_status e = cuda_check("nc32 state launch", cudaGetLastError());
+    if (e != LA_OK) return e;
+    e = launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, 32, p.mode, p.state_S, p.state_z,
+                            p.ws_total, st);
+    if (e != LA_OK) return e;
+    if (p.Lq > 0) {
+        nc32_readout_kernel<InT, OutT>
+            <<<dim3((p.Lq + kNc32Queries - 1) / kNc32Queries, p.BH), kNc32Warps * 32, 0, st>>>(
+                (const InT *)p.q, p.Lq, p.ws_total, p.eps, (OutT *)p.out);
+        count_launches(1);
+        e = cuda_check("nc32 read-out launch", cudaGetLastError());
+    }
+    return e;
+}
+
 template <typename IT, typename OT, int D> struct SimtNoncausalF {
     static la_status run(SimtParams p, int Lk, cudaStream_t st) {
-        return simt_noncausal<IT, OT, D>(p, Lk, st);
+        if constexpr (D == 32) return nc32_noncausal<IT, OT>(p, Lk, st);
+        else return simt_noncausal<IT, OT, D>(p, Lk, st);
     }
 };
 template <typename IT, typename OT, int D> struct DecodeF {
@@ -212,7 +235,7 @@ size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chun
 size_t la_noncausal_workspace_size(int B, int H, int Lk, int d_k, int d_v) {
     if (B <= 0 || H <= 0 || Lk < 0 || d_k != d_v || !dim_ok(d_k)) return 0;
     const long BH = (long)B * H;
-    const Plan pl = make_plan(BH, Lk > 0 ? Lk : 1, kNoncausalChunk, d_k);
+    const Plan pl = make_nc_plan(BH, Lk, d_k);
     return ws_layout(BH, pl.n_seg, d_k, true).bytes;
 }
 
@@ -287,7 +310,7 @@ la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_d
     if (Lq > 0 && (!q || !out || !aligned16(q) || !aligned16(out))) return LA_ERR_INVALID_ARG;
     if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return LA_ERR_INVALID_ARG;
     if (BH > 65535L) return LA_ERR_UNSUPPORTED;   // heads run along grid y
-    const Plan pl = make_plan(BH, Lk > 0 ? Lk : 1, kNoncausalChunk, d_k);
+    const Plan pl = make_nc_plan(BH, Lk, d_k);
     const WsLayout wl = ws_layout(BH, pl.n_seg, d_k, true);
     if (!workspace || workspace_bytes < wl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return LA_ERR_INVALID_ARG;
@@ -312,7 +335,7 @@ la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_d
     p.ws_A = (float *)(ws + wl.A_off);
     p.ws_total = (float *)(ws + wl.total_off);
     p.state_S = state_S; p.state_z = state_z; p.mode = mode;
-    p.BH = (int)BH; p.T = Lk; p.Lq = Lq; p.chunk = kNoncausalChunk; p.seg_len = pl.seg_len;
+    p.BH = (int)BH; p.T = Lk; p.Lq = Lq; p.chunk = pl.chunk; p.seg_len = pl.seg_len;
     p.n_seg = pl.n_seg; p.eps = eps;
     return dispatch3<SimtNoncausalF>(in_dtype, out_dtype, d_k, p, Lk, st);
 }

@@ -27,7 +27,10 @@ inline Plan make_plan(long BH, long T, int chunk, int D) {
     Plan p;
     p.chunk = chunk;
     const long n_chunks = (T + chunk - 1) / chunk;
-    long min_chunks = ((long)D * 4 + chunk - 1) / chunk;   // >= 4*D tokens per segment
+    // >= 4*D tokens per segment, unless the whole problem has fewer chunks than
+    // two waves of SMs (then latency, not scan traffic, is what matters)
+    long min_chunks = ((long)D * 4 + chunk - 1) / chunk;
+    if (BH * n_chunks < 2L * kNumSMs) min_chunks = 1;
     if (min_chunks < 1) min_chunks = 1;
     long max_segs = n_chunks / min_chunks;
     if (max_segs < 1) max_segs = 1;
@@ -43,6 +46,25 @@ inline Plan make_plan(long BH, long T, int chunk, int D) {
     const long G = (n_chunks + best_segs - 1) / best_segs;
     p.seg_len = (int)(G * chunk);
     p.n_seg = (int)((n_chunks + G - 1) / G);
+    return p;
+}
+
+// Key segments of the non-causal form.  At head dim 32 the CUDA-core state
+// kernel runs several CTAs per SM, so aim for ~4 CTAs per SM over all heads,
+// with segments of at least 64 keys; other head dims use the chunk plan.
+inline Plan make_nc_plan(long BH, long Lk, int D) {
+    if (D != 32) return make_plan(BH, Lk > 0 ? Lk : 1, kNoncausalChunk, D);
+    Plan p;
+    p.chunk = 64;
+    const long L = Lk > 0 ? Lk : 1;
+    long segs = (4L * kNumSMs + BH - 1) / BH;
+    const long max_segs = (L + 63) / 64;
+    if (segs > max_segs) segs = max_segs;
+    if (segs < 1) segs = 1;
+    long seg_len = (L + segs - 1) / segs;
+    seg_len = (seg_len + 63) / 64 * 64;
+    p.seg_len = (int)seg_len;
+    p.n_seg = (int)((L + seg_len - 1) / seg_len);
     return p;
 }
 
