@@ -234,9 +234,10 @@ def time_calls(fn, iters, flush=None):
     return tot / iters
 
 
-def measure_workloads(dev, peaks, iters=10):
+def measure_workloads(dev, peaks, iters=10, only=None):
     """Time every other workload of the hot path once (the per-row numbers
-    beside the headline).  L2 is flushed (a 512 MB write) before each call."""
+    beside the headline).  L2 is flushed (a 512 MB write) before each call.
+    ``only`` restricts the run to one workload name (profiling runs)."""
     import torch
     import kernelized_causal_sequence_b200 as la
     from kernelized_causal_sequence_b200 import inputs
@@ -244,6 +245,8 @@ def measure_workloads(dev, peaks, iters=10):
     flush = lambda: flush_buf.zero_()
     res = {}
     for name in ("causal_f32_t256_d64", "causal_bf16_b4h8_t2048_d64", "ssd_decay_bf16_b2h16_t8192_d128"):
+        if only is not None and name != only:
+            continue
         w = inputs.WORKLOADS[name]
         q, k, v, a = (None if x is None else x.to(dev) for x in inputs.qkv(w))
         out = torch.empty((w.B, w.H, w.T, w.d), dtype=w.torch_out_dtype, device=dev)
@@ -262,6 +265,8 @@ def measure_workloads(dev, peaks, iters=10):
                      else "simt"}
     w = inputs.WORKLOADS["noncausal_f16_b8h8_l4800_d32"]
     for cross in (False, True):
+        if only is not None and only != w.name:
+            continue
         q, k, v, _ = inputs.qkv(w)
         if cross:
             k, v = inputs.cross_kv(w)
@@ -472,6 +477,18 @@ def run_ours(args, w):
     return 0
 
 
+def run_case(args):
+    """One per-row workload alone (no headline, no decode, no CPU leg)."""
+    import torch
+    peaks, _ = load_peaks()
+    dev = torch.device("cuda", 0)
+    res = measure_workloads(dev, peaks, iters=max(1, args.steps), only=args.case)
+    if not res:
+        raise SystemExit(f"unknown case {args.case!r}")
+    print(json.dumps({"case": args.case, **res}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -490,8 +507,13 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the dominant kernel, if measured")
+    ap.add_argument("--case", default=None,
+                    help="time only this workload (one of the per-row workloads) with --steps "
+                         "calls and print its figures; used for focused profiling runs")
     args = ap.parse_args(argv)
     from kernelized_causal_sequence_b200 import inputs
+    if args.case is not None:
+        return run_case(args)
     w = inputs.WORKLOADS[args.workload]
     if args.T:
         import dataclasses

@@ -6,7 +6,8 @@
 
 namespace la {
 
-// K2: decayed exclusive prefix scan over the segments of each head, in place.
+// K2: decayed exclusive prefix scan over the segments of each head, in place
+// (this form: many segments per head).
 // Segment s maps X -> A_s X + dX_s; entering segment s the state is
 //   S_in(s) = A_{s-1} S_in(s-1) + dX_{s-1},  S_in(0) = state-in or 0,
 // and the final state is S_in(n_seg).  A block takes 32 state elements of one
@@ -79,6 +80,48 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, cons
 }
 
 
+// K2 for few segments per head (the common case): one thread per state
+// element walks the head's segments in order, with the loads of eight
+// segments in flight at a time, so each block streams whole coalesced rows of
+// the workspace.  The segment factors A_s of the head are staged in shared
+// memory.  grid (ceil((D*D + D) / 256), BH), 256 threads.
+constexpr int kSeqScanMaxSeg = 64;
+constexpr int kSeqScanBatch = 8;
+__global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, const float *ws_A,
+                                                               int n_seg, int E, int dS,
+                                                               const float *state_in_S,
+                                                               const float *state_in_z,
+                                                               float *state_out_S, float *state_out_z,
+                                                               float *total) {
+    __shared__ float Ash[kSeqScanMaxSeg];
+    const int bh = blockIdx.y;
+    const int e = blockIdx.x * 256 + threadIdx.x;
+    if (threadIdx.x < n_seg) Ash[threadIdx.x] = ws_A[(size_t)bh * n_seg + threadIdx.x];
+    __syncthreads();
+    if (e >= E) return;
+    float *ws = ws_state + (size_t)bh * n_seg * E + e;
+    float carry = 0.f;
+    if (e < dS) { if (state_in_S) carry = state_in_S[(size_t)bh * dS + e]; }
+    else if (state_in_z) carry = state_in_z[(size_t)bh * (E - dS) + (e - dS)];
+#pragma unroll 1
+    for (int s0 = 0; s0 < n_seg; s0 += kSeqScanBatch) {
+        float x[kSeqScanBatch];
+#pragma unroll
+        for (int i = 0; i < kSeqScanBatch; ++i)
+            x[i] = (s0 + i < n_seg) ? ws[(size_t)(s0 + i) * E] : 0.f;
+#pragma unroll
+        for (int i = 0; i < kSeqScanBatch; ++i) {
+            if (s0 + i < n_seg) {
+                ws[(size_t)(s0 + i) * E] = carry;   // state entering segment s0 + i
+                carry = fmaf(Ash[s0 + i], carry, x[i]);
+            }
+        }
+    }
+    if (total) total[(size_t)bh * E + e] = carry;
+    if (e < dS) { if (state_out_S) state_out_S[(size_t)bh * dS + e] = carry; }
+    else if (state_out_z) state_out_z[(size_t)bh * (E - dS) + (e - dS)] = carry;
+}
+
 la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n_seg, int D,
                               int mode, float *state_S, float *state_z, float *total,
                               cudaStream_t st) {
@@ -87,8 +130,13 @@ la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n
     const float *sin_z = mode == LA_STATE_INOUT ? state_z : nullptr;
     float *sout_S = mode != LA_STATE_NONE ? state_S : nullptr;
     float *sout_z = mode != LA_STATE_NONE ? state_z : nullptr;
-    segment_scan_kernel<<<dim3((E + 31) / 32, (unsigned)BH), 256, 0, st>>>(
-        ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, total);
+    if (n_seg <= kSeqScanMaxSeg) {
+        segment_scan_seq_kernel<<<dim3((E + 255) / 256, (unsigned)BH), 256, 0, st>>>(
+            ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, total);
+    } else {
+        segment_scan_kernel<<<dim3((E + 31) / 32, (unsigned)BH), 256, 0, st>>>(
+            ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, total);
+    }
     count_launches(1);
     return cuda_check("segment_scan launch", cudaGetLastError());
 }

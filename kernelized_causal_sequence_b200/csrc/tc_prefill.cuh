@@ -8,7 +8,7 @@
 //   MMA2  O      = phi(Q) S                            (C x D,  K = D)   inter-chunk term
 //   MMAd  den    = phi(Q) z                            (C x 16, K = D)
 //   MMA3  S     += (w o phi(K))^T V                    (D x D,  K = C)   state update
-//   MMAz  z     += (w o phi(K))^T 1                    (D x 16, K = C)
+//   MMAz  z     += (w o phi(K))^T 1                    (D x 16, K = C)   ones operand
 //   MMA4  O     += P V,  P = scores o mask o decay     (C x D,  K = C)   exact intra-chunk part
 //   out   = O / (den_inter + rowsum(P) + eps)
 //
@@ -81,16 +81,15 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int PB = (OUT && !PT) ? C * C * 2 : 0;
     static constexpr int OFF_ZB = OFF_P + PB;                        // z as MMA operand [16][D]
     static constexpr int ZB = OUT ? 16 * D * 2 : 0;
-    static constexpr int OFF_STG = OFF_ZB + ZB;                      // output staging, 4 warps x [R][128 B]
+    static constexpr int OFF_ONES = OFF_ZB + ZB;                     // ones operand [16][C] of MMAz
+    static constexpr int ONES = 16 * C * 2;
+    static constexpr int OFF_STG = (OFF_ONES + ONES + 1023) / 1024 * 1024;   // output staging, 4 warps x [R][128 B]
     static constexpr int STG = OUT ? 4 * ROWS_PER_WARP * 128 : 0;
     static constexpr int OFF_F = OFF_STG + STG;                      // fp32 scratch
     static constexpr int F_L = 0;                                    // [NKV][C] log2-decay cumsum
     static constexpr int F_G = F_L + (DECAY ? NKV * C : 0);          // [NKV] chunk decay
-    // per-warp column sums of w o phi(K) (8 warps: 4 phi + 4 epilogue), one
-    // buffer per K/V stage in output mode, one running set in state-only mode
-    static constexpr int NRED = OUT ? 3 : 1;   // 3: the slot of chunk c is reused by chunk c+3 only
-    static constexpr int F_RED = (F_G + NKV + 3) / 4 * 4;            // [NRED][8][D], 16-byte aligned
-    static constexpr int F_END = F_RED + NRED * 8 * D;
+    static constexpr int F_LE = F_G + NKV;                           // [NKV] log2 weight origin
+    static constexpr int F_END = F_LE + NKV;
     static constexpr int OFF_BAR = (OFF_F + F_END * 4 + 7) / 8 * 8;
     // barrier indices
     static constexpr int B_KV_FULL = 0, B_KV_EMPTY = B_KV_FULL + NKV, B_PHI = B_KV_EMPTY + NKV;
@@ -111,7 +110,8 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int T_O = OUT ? C : 0;
     static constexpr int T_O2 = T_O + (OUT ? D : 0);
     static constexpr int T_S = T_O2 + (SPLIT ? D : 0);
-    static constexpr int T_DEN = T_S + D;                     // phi(Q) z of the carried state
+    static constexpr int T_Z = T_S + D;                       // z (column 0; MMAz accumulator)
+    static constexpr int T_DEN = T_Z + 16;                    // phi(Q) z of the carried state
     static constexpr int T_Q = T_DEN + (OUT ? 16 : 0);
     static constexpr int T_USED = T_Q + (QT ? D / 2 : 0);
     static constexpr int TMEM_COLS = tmem_alloc_cols(T_USED);
@@ -121,7 +121,7 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static_assert(!(C == 128 && DECAY && OUT), "chunk 128 with decay exceeds TMEM");
     static_assert(T_USED <= 512, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static_assert(OFF_F % 16 == 0 && (F_RED * 4) % 16 == 0, "float4 column-sum stores need 16-byte alignment");
+    static_assert(OFF_ONES % 16 == 0, "no-swizzle operand alignment");
     static_assert(OFF_STG % 1024 == 0 && OFF_SBF % 1024 == 0 && OFF_P % 1024 == 0 && OFF_ZB % 16 == 0 &&
                   OFF_Q % 1024 == 0 && KV_STAGE % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 };
@@ -230,12 +230,9 @@ __device__ __forceinline__ void write_state_row(uint8_t *sbf, int a, int col0, c
 // all its rows, and all loads of a batch are issued before any arithmetic.
 // The tile's rows are split into NPART equal parts; this call does part PART
 // (the two warpgroups each take one part of the key tile).
-// When ZSUM, zp[e] accumulates this thread's column sums of the operand the
-// state update uses (w o phi(K) with decay, phi(K) without), for its 8 columns.
-template <typename InT, int C, int D, bool DECAY, bool CONVERT_V, int PB = 0, int PE = 1, int NPART = 1,
-          bool ZSUM = false>
+template <typename InT, int C, int D, bool DECAY, bool CONVERT_V, int PB = 0, int PE = 1, int NPART = 1>
 __device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *kw, uint8_t *vt, int tw, int n,
-                                         const float *L, float Lend, float (&zp)[8]) {
+                                         const float *L, float Lend) {
     constexpr int KB = D / 64, BOXB = C * 128;
     constexpr int PH = 128 / (8 * KB);
     constexpr int NIT = C / PH;
@@ -254,40 +251,28 @@ __device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *kw, uint8_t *vt
             const int r = ph + (i0 + i) * PH;
             const uint32_t off = base + (i0 + i) * PH * 128;
             const bool valid = r < n;
-            uint4 used;   // the bf16 operand of the state update for these 8 columns
             if constexpr (std::is_same<InT, bf16>::value) {
                 uint4 f = phi_bf16x8(raw[i]);
                 if (!valid) f = make_uint4(0u, 0u, 0u, 0u);
                 *reinterpret_cast<uint4 *>(tile + off) = f;
-                used = f;
                 if constexpr (DECAY) {
                     const float w = valid ? ex2_approx(Lend - L[r]) : 0.f;
                     const uint32_t w2 = pack_bf16x2(w, w);
-                    used = make_uint4(mul_bf16x2(f.x, w2), mul_bf16x2(f.y, w2), mul_bf16x2(f.z, w2),
-                                      mul_bf16x2(f.w, w2));
-                    *reinterpret_cast<uint4 *>(kw + off) = used;
+                    *reinterpret_cast<uint4 *>(kw + off) =
+                        make_uint4(mul_bf16x2(f.x, w2), mul_bf16x2(f.y, w2), mul_bf16x2(f.z, w2),
+                                   mul_bf16x2(f.w, w2));
                 }
             } else {
                 float x[8];
                 unpack8<InT>(raw[i], x);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = valid ? phi_fast(x[e]) : 0.f;
-                used = pack8_bf16(x);
-                *reinterpret_cast<uint4 *>(tile + off) = used;
+                *reinterpret_cast<uint4 *>(tile + off) = pack8_bf16(x);
                 if constexpr (DECAY) {
                     const float w = valid ? ex2_approx(Lend - L[r]) : 0.f;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) x[e] *= w;
-                    used = pack8_bf16(x);
-                    *reinterpret_cast<uint4 *>(kw + off) = used;
-                }
-            }
-            if constexpr (ZSUM) {
-                const uint32_t uw[4] = {used.x, used.y, used.z, used.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    zp[2 * e] += bf16lo(uw[e]);
-                    zp[2 * e + 1] += bf16hi(uw[e]);
+                    *reinterpret_cast<uint4 *>(kw + off) = pack8_bf16(x);
                 }
             }
         }
@@ -305,42 +290,10 @@ __device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *kw, uint8_t *vt
     }
 }
 
-// Column sums of one key part: combine the row phases held by lanes of this
-// warp, then lanes owning a (column-chunk, box) write their 8 sums to
-// red[wslot][col].  Warp-collective.
-template <int D>
-__device__ __forceinline__ void publish_zsum(float (&zp)[8], float *red, int wslot, int tw) {
-    constexpr int KB = D / 64;
-    const int lane = tw & 31;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        zp[e] += __shfl_xor_sync(0xffffffffu, zp[e], 16);
-        if constexpr (KB == 1) zp[e] += __shfl_xor_sync(0xffffffffu, zp[e], 8);
-    }
-    const int owners = 8 * KB;   // lanes 0 .. owners-1 hold distinct column chunks
-    if (lane < owners) {
-        const int lc = lane & 7, b = lane >> 3;
-        float4 *dst = reinterpret_cast<float4 *>(red + wslot * D + b * 64 + lc * 8);
-        dst[0] = make_float4(zp[0], zp[1], zp[2], zp[3]);
-        dst[1] = make_float4(zp[4], zp[5], zp[6], zp[7]);
-    }
-}
-
-// Output mode: publish this chunk's column sums to red[stage].  State-only
-// mode: keep a decayed running sum per thread (zrun <- gamma_c zrun + zp) and
-// publish it after the segment's last chunk.
-template <typename G>
-__device__ __forceinline__ void zsum_update(float (&zp)[8], float (&zrun)[8], float *Fsm, int s,
-                                            int c, int nch, int wslot, int tw) {
-    if constexpr (G::OUT) {
-        publish_zsum<G::D>(zp, Fsm + G::F_RED + (c % G::NRED) * 8 * G::D, wslot, tw);
-    } else {
-        const float g = G::DECAY ? Fsm[G::F_G + s] : 1.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) zrun[e] = fmaf(g, zrun[e], zp[e]);
-        if (c == nch - 1) publish_zsum<G::D>(zrun, Fsm + G::F_RED, wslot, tw);
-    }
-}
+// The chunk handled at step c: output mode walks the segment forwards (the
+// state is carried), the state-only pass walks it backwards so that the
+// decay from each key to the segment's end is known when its chunk is read.
+template <bool OUT> __device__ __forceinline__ int chunk_at(int c, int nch) { return OUT ? c : nch - 1 - c; }
 
 // phi of chunk c: decay cumsum (DECAY), K (and w o phi(K)), Q (output mode:
 // into TMEM for C = 128, in place otherwise); then arrives on phi_done.
@@ -348,22 +301,41 @@ __device__ __forceinline__ void zsum_update(float (&zp)[8], float (&zrun)[8], fl
 template <int C, int D, bool DECAY, int MODE, typename InT>
 __device__ __forceinline__ bool phi_stage(uint8_t *smem, uint64_t *bar, float *Fsm, const AbortCtx ab,
                                        const TcParams &p, uint32_t tmem, long t_begin, long t_end,
-                                       int bh, int c, int nch, int tw, float &Aseg, float (&zrun)[8]) {
+                                       int bh, int c, int nch, int tw, float &Aseg,
+                                       float (&apre)[C / 32], float &lam) {
     using G = Cfg<C, D, DECAY, MODE>;
     const int lane = tw & 31, q = (kPhiWarp0 + (tw >> 5)) & 3;
     const int s = c % G::NKV;
-    const long t0 = t_begin + (long)c * C;
+    const long t0 = t_begin + (long)chunk_at<G::OUT>(c, nch) * C;
     const int n = (int)min((long)C, t_end - t0);
     if (!mbar_wait(&bar[G::B_KV_FULL + s], (c / G::NKV) & 1, ab, 8)) return false;
     float *L = Fsm + G::F_L + s * C;
     if constexpr (DECAY) {
         if (tw < 32) {
+            // the decays of chunk c were loaded into registers during chunk c-1;
+            // start the loads of chunk c+1 now so their latency is hidden
             const float *a = p.decay + (size_t)bh * p.T + t0;
+            float cur[C / 32];
+#pragma unroll
+            for (int h = 0; h < C / 32; ++h) {
+                const int j = h * 32 + lane;
+                cur[h] = (c == 0) ? ((j < n) ? a[j] : 1.f) : apre[h];
+            }
+            if (c + 1 < nch) {
+                const long t1 = t_begin + (long)chunk_at<G::OUT>(c + 1, nch) * C;
+                const int n1 = (int)min((long)C, t_end - t1);
+                const float *a1 = p.decay + (size_t)bh * p.T + t1;
+#pragma unroll
+                for (int h = 0; h < C / 32; ++h) {
+                    const int j = h * 32 + lane;
+                    apre[h] = (j < n1) ? a1[j] : 1.f;
+                }
+            }
             float carry = 0.f;
 #pragma unroll
-            for (int j0 = 0; j0 < C; j0 += 32) {
-                const int j = j0 + lane;
-                float x = (j < n) ? lg2_approx(a[j]) : 0.f;   // log2 units
+            for (int h = 0; h < C / 32; ++h) {
+                const int j = h * 32 + lane;
+                float x = (j < n) ? lg2_approx(cur[h]) : 0.f;   // log2 units
                 x = warp_sum_scan(x, lane) + carry;
                 L[j] = x;   // rows >= n repeat the chunk total (never used)
                 carry = __shfl_sync(0xffffffffu, x, 31);
@@ -372,6 +344,11 @@ __device__ __forceinline__ bool phi_stage(uint8_t *smem, uint64_t *bar, float *F
                 const float g = ex2_approx(carry);
                 Fsm[G::F_G + s] = g;
                 Aseg *= g;
+                // weights w_j = 2^(origin - L_j): the chunk's end in output mode;
+                // in state-only mode the segment's end (lam = log2 decay of the
+                // chunks after this one, all processed already)
+                Fsm[G::F_LE + s] = G::OUT ? carry : carry + lam;
+                lam += carry;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_L_READY + s]);   // for the other warpgroup
@@ -381,10 +358,8 @@ __device__ __forceinline__ bool phi_stage(uint8_t *smem, uint64_t *bar, float *F
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
     constexpr bool CONV = !std::is_same<InT, bf16>::value;
     // the first parts of the key rows; the epilogue warpgroup takes the rest
-    float zp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    phi_tile<InT, C, D, DECAY, CONV, 0, G::KSPLIT, 4, true>(kt, kt + 2 * G::TILE, kt + G::TILE, tw, n, L,
-                                                           DECAY ? L[n - 1] : 0.f, zp);
-    zsum_update<G>(zp, zrun, Fsm, s, c, nch, tw >> 5, tw);
+    phi_tile<InT, C, D, DECAY, CONV, 0, G::KSPLIT, 4>(kt, kt + 2 * G::TILE, kt + G::TILE, tw, n, L,
+                                                     DECAY ? Fsm[G::F_LE + s] : 0.f);
     if constexpr (G::OUT) {
         const int sq = G::QT ? 0 : (c & 1);
         const int use = G::QT ? c : (c >> 1);
@@ -432,8 +407,7 @@ __device__ __forceinline__ bool phi_stage(uint8_t *smem, uint64_t *bar, float *F
             }
             tmem_st_wait();
         } else {
-            float unused[8];
-            phi_tile<InT, C, D, false, false>(qs, nullptr, nullptr, tw, C, nullptr, 0.f, unused);
+            phi_tile<InT, C, D, false, false>(qs, nullptr, nullptr, tw, C, nullptr, 0.f);
         }
     }
     fence_proxy_async_smem();
@@ -448,11 +422,10 @@ __device__ __forceinline__ bool phi_stage(uint8_t *smem, uint64_t *bar, float *F
 template <int C, int D, bool DECAY, int MODE, typename InT>
 __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *bar, float *Fsm,
                                                      const AbortCtx ab, uint32_t tmem, long t_begin,
-                                                     long t_end, int c, int nch, int et,
-                                                     float (&zrun)[8]) {
+                                                     long t_end, int c, int nch, int et) {
     using G = Cfg<C, D, DECAY, MODE>;
     const int s = c % G::NKV;
-    const long t0 = t_begin + (long)c * C;
+    const long t0 = t_begin + (long)chunk_at<G::OUT>(c, nch) * C;
     const int n = (int)min((long)C, t_end - t0);
     if (!mbar_wait(&bar[G::B_KV_FULL + s], (c / G::NKV) & 1, ab, 15)) return false;
     const float *L = Fsm + G::F_L + s * C;
@@ -460,10 +433,8 @@ __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *ba
         if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 16)) return false;
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
     constexpr bool CONV = !std::is_same<InT, bf16>::value;
-    float zp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    phi_tile<InT, C, D, DECAY, CONV, G::KSPLIT, 4, 4, true>(kt, kt + 2 * G::TILE, kt + G::TILE, et, n, L,
-                                                           DECAY ? L[n - 1] : 0.f, zp);
-    zsum_update<G>(zp, zrun, Fsm, s, c, nch, 4 + (et >> 5), et);
+    phi_tile<InT, C, D, DECAY, CONV, G::KSPLIT, 4, 4>(kt, kt + 2 * G::TILE, kt + G::TILE, et, n, L,
+                                                     DECAY ? Fsm[G::F_LE + s] : 0.f);
     if constexpr (G::QSPLIT) {
         // second column box of phi(Q) for rows 32q + lane -> TMEM
         const int lane = et & 31, q = et >> 5;
@@ -549,12 +520,15 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(&bar[G::B_DRAIN], 1);
         fence_mbar_init();
     }
-    // (output mode) the z operand [16][D] starts zeroed: only its row 0 is used
+    // (output mode) the z operand [16][D] starts zeroed: only its row 0 is used;
+    // the ones operand of MMAz is all ones (every column of its result is z)
     {
         if constexpr (G::OUT) {
             uint32_t *zb = reinterpret_cast<uint32_t *>(smem + G::OFF_ZB);
             for (int i = threadIdx.x; i < G::ZB / 4; i += kThreads) zb[i] = 0u;
         }
+        uint32_t *ones = reinterpret_cast<uint32_t *>(smem + G::OFF_ONES);
+        for (int i = threadIdx.x; i < G::ONES / 4; i += kThreads) ones[i] = 0x3F803F80u;   // bf16 1.0 pairs
         fence_proxy_async_smem();
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_addr_smem, G::TMEM_COLS);
@@ -578,7 +552,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             int issued_kv[G::NKV] = {}, issued_q[2] = {};
             for (int c = 0; c < nch; ++c) {
                 const int s = c % G::NKV;
-                const int y = (int)(t_begin + (long)c * C);
+                const int y = (int)(t_begin + (long)chunk_at<G::OUT>(c, nch) * C);
                 if constexpr (G::OUT) {
                     const int sq = G::QT ? 0 : (c & 1);
                     const int use = G::QT ? c : (c >> 1);
@@ -621,6 +595,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             constexpr uint32_t ID_DEN = idesc_bf16(C, 16, false, false);
             constexpr uint32_t ID_DS = idesc_bf16(D, D, true, true);
             constexpr uint32_t ID_PV = idesc_bf16(C, D, false, true);
+            constexpr uint32_t ID_Z = idesc_bf16(D, 16, true, false);
             const uint32_t sb = smem_u32(smem);
             // Base descriptors; a K-step advances the start address field
             // (address >> 4 in the low 14 bits, which never carries here:
@@ -632,6 +607,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint64_t dS0 = sdesc_sw128(sb + G::OFF_SBF, D * 128, 1024);   // S (MN-major)
             const uint64_t dZ0 = nosw(sb + G::OFF_ZB, (D / 8) * 128);           // z [16][D]
             const uint64_t dP0 = sdesc_sw128(sb + G::OFF_P, 16, 1024);          // P (K-major, smem)
+            const uint64_t dOnes = nosw(sb + G::OFF_ONES, (C / 8) * 128);       // ones [16][C]
             for (int c = 0; c < nch; ++c) {
                 const int s = c % G::NKV;
                 const uint32_t kt = sb + G::OFF_KV + s * G::KV_STAGE;   // phi(K)
@@ -674,16 +650,19 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if constexpr (G::QT) mma_commit(&bar[G::B_QT_EMPTY]);
                     else mma_commit(&bar[G::B_Q_EMPTY + (c & 1)]);
                 } else {
-                    if ((c == 0 || DECAY) && !mbar_wait(&bar[G::B_S_READY], c & 1, ab, 5)) break;
+                    if (c == 0 && !mbar_wait(&bar[G::B_S_READY], 0, ab, 5)) break;
                     tc_fence_after();
                 }
-                // MMA3: state update with this chunk's keys and values (z is summed
-                // on the CUDA cores while phi(K) is formed)
+                // MMA3 + MMAz: state update with this chunk's keys and values
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_ss(tmem + G::T_S, dKm + (uint64_t)((kk * 2048) >> 4),
                            dVm + (uint64_t)((kk * 2048) >> 4), ID_DS, 1);
-                if (G::OUT || DECAY || c == nch - 1) mma_commit(&bar[G::B_DS_FULL]);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_ss(tmem + G::T_Z, dKm + (uint64_t)((kk * 2048) >> 4),
+                           dOnes + (uint64_t)((kk * 256) >> 4), ID_Z, 1);
+                if (G::OUT || c == nch - 1) mma_commit(&bar[G::B_DS_FULL]);
                 if constexpr (G::OUT) {
                     // MMA4: exact intra-chunk product with the masked, decayed scores
                     if (!mbar_wait(&bar[G::B_P_READY], c & 1, ab, 7)) break;
@@ -716,7 +695,10 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int q = warp & 3;                              // TMEM lane quarter
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         float Aseg = 1.f;  // product of chunk decays (state-only mode)
-        float zrun[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // running column sums (state-only)
+        float apre[C / 32];   // decays of the next chunk (warp kPhiWarp0)
+#pragma unroll
+        for (int h = 0; h < C / 32; ++h) apre[h] = 1.f;
+        float lam = 0.f;      // log2 decay of the chunks already processed (state-only mode)
         bool ok = true;
 
         // state rows owned by this thread: TMEM lane quarter q, rows of the
@@ -727,8 +709,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
         if (nch > 0)
             ok = phi_stage<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, p, tmem, t_begin, t_end, bh, 0, nch,
-                                                   tw, Aseg, zrun);
-        float zreg = 0.f;   // z of this thread's state row (output mode)
+                                                   tw, Aseg, apre, lam);
         // ---- segment start: state entering the segment -> TMEM (and operands)
         if (ok) {
             tc_fence_after();
@@ -748,7 +729,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if constexpr (G::OUT) if (srow_ok) write_state_row<D>(smem + G::OFF_SBF, a_row, cb * 32, vals);
                 }
                 const float zin = (G::OUT && srow_ok) ? st[(size_t)D * D + a_row] : 0.f;
-                zreg = zin;
+                tmem_st1(tmem + lane_base + G::T_Z, __float_as_uint(zin * g0));
                 if constexpr (G::OUT) {
                     if (srow_ok) {
                         // z operand: row n = 0 of the [16][D] K-major no-swizzle layout
@@ -767,15 +748,15 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int c = 0; ok && c < nch; ++c) {
             if (c + 1 < nch) {
                 ok = phi_stage<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, p, tmem, t_begin, t_end, bh, c + 1,
-                                                       nch, tw, Aseg, zrun);
+                                                       nch, tw, Aseg, apre, lam);
                 if (!ok) break;
             }
-            const bool need = G::OUT || DECAY || c == nch - 1;
+            const bool need = G::OUT || c == nch - 1;
             if (!need) continue;
-            if (!mbar_wait(&bar[G::B_DS_FULL], (G::OUT || DECAY) ? (c & 1) : 0, ab, 11)) { ok = false; break; }
-            // the column sums of chunk c are published before phi_done(c)
-            if (!mbar_wait(&bar[G::B_PHI + (c % G::NKV)], (c / G::NKV) & 1, ab, 17)) { ok = false; break; }
+            if (!mbar_wait(&bar[G::B_DS_FULL], G::OUT ? (c & 1) : 0, ab, 11)) { ok = false; break; }
             tc_fence_after();
+            uint32_t zbits;   // z of this thread's state row after chunk c
+            tmem_ld1(tmem + lane_base + G::T_Z, zbits);
             const bool last = c == nch - 1;
             const float gnext = (DECAY && !last) ? Fsm[G::F_G + ((c + 1) % G::NKV)] : 1.f;
             if (last && !G::OUT) {
@@ -794,13 +775,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                                 __uint_as_float(u[4 * i + 2]), __uint_as_float(u[4 * i + 3]));
                     }
                 }
-                if (srow_ok) {
-                    const float *red = Fsm + G::F_RED;
-                    float zs = 0.f;
-#pragma unroll
-                    for (int w8 = 0; w8 < 8; ++w8) zs += red[w8 * D + a_row];
-                    dst[(size_t)D * D + a_row] = zs;
-                }
+                if (srow_ok) dst[(size_t)D * D + a_row] = __uint_as_float(zbits);
                 if (tw == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = Aseg;
                 break;
             }
@@ -822,17 +797,13 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             }
             if constexpr (G::OUT) {
-                // z after chunk c: z <- gamma_c z + (column sums of w o phi(K) over the chunk)
+                // z entering chunk c+1 (MMAz has added this chunk's w o phi(K) column sums)
                 if (srow_ok) {
-                    const float *red = Fsm + G::F_RED + (c % G::NRED) * 8 * D;
-                    float dz = 0.f;
-#pragma unroll
-                    for (int w8 = 0; w8 < 8; ++w8) dz += red[w8 * D + a_row];
-                    zreg = fmaf(DECAY ? Fsm[G::F_G + (c % G::NKV)] : 1.f, zreg, dz);
                     bf16 *zb = reinterpret_cast<bf16 *>(smem + G::OFF_ZB);
-                    zb[(a_row / 8) * 64 + (a_row % 8)] = __float2bfloat16_rn(zreg);
+                    zb[(a_row / 8) * 64 + (a_row % 8)] = __float2bfloat16_rn(__uint_as_float(zbits));
                 }
             }
+            if constexpr (DECAY) tmem_st1(tmem + lane_base + G::T_Z, __float_as_uint(__uint_as_float(zbits) * gnext));
             if constexpr (DECAY) tmem_st_wait();
             fence_proxy_async_smem();
             tc_fence_before();
@@ -841,10 +812,9 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
     } else if constexpr (!G::OUT) {
         // ================= warps 0-3 in state-only mode: second half of phi(K)
-        float zrun[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int c = 0; c < nch; ++c)
             if (!phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, tmem, t_begin, t_end, c, nch,
-                                                              threadIdx.x, zrun))
+                                                              threadIdx.x))
                 break;
     } else {
         // ================= epilogue (warps 0-3)
@@ -852,9 +822,8 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const bool rvalid_lane = lane < G::ROWS_PER_WARP;
         const int i = q * G::ROWS_PER_WARP + lane;   // row of the chunk held by this thread
-        float zrun[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // unused in output mode
         bool eok = nch == 0 || phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, tmem, t_begin,
-                                                                             t_end, 0, nch, threadIdx.x, zrun);
+                                                                             t_end, 0, nch, threadIdx.x);
         for (int c = 0; eok && c < nch; ++c) {
             const int s = c % G::NKV;
             const long t0 = t_begin + (long)c * C;
@@ -921,7 +890,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // while MMA4 runs: the second half of the next chunk's keys
             if (c + 1 < nch &&
                 !phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, tmem, t_begin, t_end, c + 1,
-                                                              nch, threadIdx.x, zrun))
+                                                              nch, threadIdx.x))
                 break;
 
             if (!mbar_wait(&bar[G::B_O_FULL], c & 1, ab, 14)) break;

@@ -60,6 +60,9 @@ SMALL = [
     (torch.bfloat16, 128, 3000, 128, False, 1, 2),
     (torch.float16, 32, 300, 128, False, 2, 2),
     (torch.float16, 128, 513, 64, True, 1, 2),
+    # more than 64 segments per head (the scan's shuffle form)
+    (torch.bfloat16, 128, 5000, 64, True, 1, 1),
+    (torch.float32, 64, 10000, 64, False, 1, 1),
 ]
 
 
