@@ -20,13 +20,16 @@
 // inter term of row i is scaled by 2^(L_i), and the state is rescaled by the
 // chunk's total decay before each update.
 //
-// Warp roles (320 threads):
-//   warps 0-3  epilogue: scores -> P (mask, decay, row sums), output division
-//              and store.  Warp w reads TMEM lanes 32w..32w+31.
-//   warp  4    TMA producer (one elected thread).
-//   warp  5    TMEM allocator and MMA issuer (one elected thread).
-//   warps 6-9  feature map phi on the staged tiles, decay cumsum, and the
-//              state epilogue (TMEM S -> bf16 operand, decay rescale).
+// Warp roles (448 threads; at most four warps share a scheduler, which caps
+// registers at 128 per thread):
+//   warps 0-3    epilogue: scores -> P (mask, decay, row sums), output division
+//                and store.  Warp w reads TMEM lanes 32w..32w+31.  In the
+//                state-only pass: the second half of phi(K).
+//   warp  4      TMA producer (one elected thread).
+//   warp  5      TMEM allocator and MMA issuer (one elected thread).
+//   warps 6-9    phi(Q) (into TMEM for chunk 128) and the state epilogue
+//                (TMEM S -> bf16 operand, decay rescale).
+//   warps 10-13  decay cumsum and phi(K) (w o phi(K) with decay).
 //
 // Every wait is bounded (see tc_ptx.cuh); on expiry the CTA raises its abort
 // flag and the status word, drains its copies and MMAs, frees TMEM, returns.
@@ -41,8 +44,8 @@ namespace tc {
 
 enum Mode { kStateOnly = 0, kOutput = 1 };
 
-constexpr int kThreads = 320;
-constexpr int kEpiWarp0 = 0, kTmaWarp = 4, kMmaWarp = 5, kPhiWarp0 = 6;
+constexpr int kThreads = 448;
+constexpr int kEpiWarp0 = 0, kTmaWarp = 4, kMmaWarp = 5, kPhiWarp0 = 6, kKWarp0 = 10;
 
 constexpr int tmem_alloc_cols(int used) {
     return used <= 32 ? 32 : used <= 64 ? 64 : used <= 128 ? 128 : used <= 256 ? 256 : 512;
@@ -64,12 +67,6 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int NKV = OUT ? 2 : (KV_BYTES <= 48 * 1024 ? 4 : 3);
     static constexpr int NQ = OUT ? (QT ? 1 : 2) : 0;
     static constexpr int ROWS_PER_WARP = (C == 128) ? 32 : 16;   // M=64 uses lanes 0-15
-    // Work split of the feature map between the two warpgroups: the phi
-    // warpgroup forms the first KSPLIT quarters of the key rows, the epilogue
-    // warpgroup the rest; with phi(Q) in TMEM and two column boxes, the
-    // epilogue warpgroup also forms the second box of phi(Q).
-    static constexpr bool QSPLIT = QT && KB == 2;
-    static constexpr int KSPLIT = QSPLIT ? 3 : 2;
 
     // ---- shared memory (offsets from a 1024-byte aligned base)
     static constexpr int KV_STAGE = 2 * TILE + (DECAY ? TILE : 0);  // K, V, (w o phi(K))
@@ -295,25 +292,25 @@ __device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *kw, uint8_t *vt
 // decay from each key to the segment's end is known when its chunk is read.
 template <bool OUT> __device__ __forceinline__ int chunk_at(int c, int nch) { return OUT ? c : nch - 1 - c; }
 
-// phi of chunk c: decay cumsum (DECAY), K (and w o phi(K)), Q (output mode:
-// into TMEM for C = 128, in place otherwise); then arrives on phi_done.
-// Returns false if the CTA is aborting.
+// Keys of chunk c (K warpgroup, thread index tk = 0..127): the decay cumsum
+// (warp 0; DECAY), then phi(K) (and w o phi(K)) in place; in output mode all
+// key rows, in state-only mode the first half (warps 0-3 take the rest).
+// Arrives on phi_done.  Returns false if the CTA is aborting.
 template <int C, int D, bool DECAY, int MODE, typename InT>
-__device__ __forceinline__ bool phi_stage(uint8_t *smem, uint64_t *bar, float *Fsm, const AbortCtx ab,
-                                       const TcParams &p, uint32_t tmem, long t_begin, long t_end,
-                                       int bh, int c, int nch, int tw, float &Aseg,
-                                       float (&apre)[C / 32], float &lam) {
+__device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm, const AbortCtx ab,
+                                        const TcParams &p, long t_begin, long t_end, int bh, int c,
+                                        int nch, int tk, float &Aseg, float (&apre)[C / 32], float &lam) {
     using G = Cfg<C, D, DECAY, MODE>;
-    const int lane = tw & 31, q = (kPhiWarp0 + (tw >> 5)) & 3;
+    const int lane = tk & 31;
     const int s = c % G::NKV;
     const long t0 = t_begin + (long)chunk_at<G::OUT>(c, nch) * C;
     const int n = (int)min((long)C, t_end - t0);
     if (!mbar_wait(&bar[G::B_KV_FULL + s], (c / G::NKV) & 1, ab, 8)) return false;
     float *L = Fsm + G::F_L + s * C;
     if constexpr (DECAY) {
-        if (tw < 32) {
+        if (tk < 32) {
             // the decays of chunk c were loaded into registers during chunk c-1;
-            // start the loads of chunk c+1 now so their latency is hidden
+            // start the loads of the next chunk now so their latency is hidden
             const float *a = p.decay + (size_t)bh * p.T + t0;
             float cur[C / 32];
 #pragma unroll
@@ -351,78 +348,90 @@ __device__ __forceinline__ bool phi_stage(uint8_t *smem, uint64_t *bar, float *F
                 lam += carry;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[G::B_L_READY + s]);   // for the other warpgroup
+            if (lane == 0) mbar_arrive(&bar[G::B_L_READY + s]);   // for the other warpgroups
         }
         named_bar_sync(1, 128);
     }
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
     constexpr bool CONV = !std::is_same<InT, bf16>::value;
-    // the first parts of the key rows; the epilogue warpgroup takes the rest
-    phi_tile<InT, C, D, DECAY, CONV, 0, G::KSPLIT, 4>(kt, kt + 2 * G::TILE, kt + G::TILE, tw, n, L,
-                                                     DECAY ? Fsm[G::F_LE + s] : 0.f);
-    if constexpr (G::OUT) {
-        const int sq = G::QT ? 0 : (c & 1);
-        const int use = G::QT ? c : (c >> 1);
-        if (!mbar_wait(&bar[G::B_Q_FULL + sq], use & 1, ab, 9)) return false;
-        uint8_t *qs = smem + G::OFF_Q + sq * G::TILE;
-        if constexpr (G::QT) {
-            // row r = 32q + lane: phi(q_r) as bf16 pairs -> TMEM (A operand),
-            // one 64-column box (32 TMEM columns) at a time
-            const int r = q * 32 + lane;
-            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-            constexpr int NBQ = G::QSPLIT ? 1 : G::KB;   // boxes formed here
-#pragma unroll 1
-            for (int b = 0; b < NBQ; ++b) {
-                uint4 raw[8];
-#pragma unroll
-                for (int lc = 0; lc < 8; ++lc)
-                    raw[lc] = *reinterpret_cast<const uint4 *>(qs + b * G::BOXB + sw128_off(r, lc));
-                uint32_t packed[32];
-#pragma unroll
-                for (int lc = 0; lc < 8; ++lc) {
-                    if constexpr (std::is_same<InT, bf16>::value) {
-                        const uint4 f = phi_bf16x8(raw[lc]);
-                        packed[lc * 4 + 0] = f.x;
-                        packed[lc * 4 + 1] = f.y;
-                        packed[lc * 4 + 2] = f.z;
-                        packed[lc * 4 + 3] = f.w;
-                    } else {
-                        float x[8];
-                        unpack8<InT>(raw[lc], x);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            packed[lc * 4 + e] = pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
-                    }
-                }
-                if (b == NBQ - 1) {
-                    // this warpgroup's reads of the raw Q slot are done
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar[G::B_Q_EMPTY]);
-                }
-                if (b == 0) {
-                    if (c > 0 && !mbar_wait(&bar[G::B_QT_EMPTY], (c - 1) & 1, ab, 10)) return false;
-                    tc_fence_after();
-                }
-                tmem_st32(tmem + lane_base + G::T_Q + b * 32, packed);
-            }
-            tmem_st_wait();
-        } else {
-            phi_tile<InT, C, D, false, false>(qs, nullptr, nullptr, tw, C, nullptr, 0.f);
-        }
-    }
+    const float Lend = DECAY ? Fsm[G::F_LE + s] : 0.f;
+    if constexpr (G::OUT)
+        phi_tile<InT, C, D, DECAY, CONV, 0, 1, 1>(kt, kt + 2 * G::TILE, kt + G::TILE, tk, n, L, Lend);
+    else
+        phi_tile<InT, C, D, DECAY, CONV, 0, 2, 4>(kt, kt + 2 * G::TILE, kt + G::TILE, tk, n, L, Lend);
     fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
+    return true;
+}
+
+// Queries of chunk c (phi warpgroup, output mode, tw = 0..127): phi(Q) into
+// TMEM as the A operand (chunk 128: row r = 32q + lane, the thread's TMEM lane)
+// or in place in shared memory (chunk 64).  Arrives on phi_done.
+template <int C, int D, bool DECAY, int MODE, typename InT>
+__device__ __forceinline__ bool q_stage(uint8_t *smem, uint64_t *bar, const AbortCtx ab, uint32_t tmem,
+                                        int c, int tw) {
+    using G = Cfg<C, D, DECAY, MODE>;
+    const int lane = tw & 31, q = (kPhiWarp0 + (tw >> 5)) & 3;
+    const int s = c % G::NKV;
+    const int sq = G::QT ? 0 : (c & 1);
+    const int use = G::QT ? c : (c >> 1);
+    if (!mbar_wait(&bar[G::B_Q_FULL + sq], use & 1, ab, 9)) return false;
+    uint8_t *qs = smem + G::OFF_Q + sq * G::TILE;
+    if constexpr (G::QT) {
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+#pragma unroll 1
+        for (int b = 0; b < G::KB; ++b) {
+            uint4 raw[8];
+#pragma unroll
+            for (int lc = 0; lc < 8; ++lc)
+                raw[lc] = *reinterpret_cast<const uint4 *>(qs + b * G::BOXB + sw128_off(r, lc));
+            uint32_t packed[32];
+#pragma unroll
+            for (int lc = 0; lc < 8; ++lc) {
+                if constexpr (std::is_same<InT, bf16>::value) {
+                    const uint4 f = phi_bf16x8(raw[lc]);
+                    packed[lc * 4 + 0] = f.x;
+                    packed[lc * 4 + 1] = f.y;
+                    packed[lc * 4 + 2] = f.z;
+                    packed[lc * 4 + 3] = f.w;
+                } else {
+                    float x[8];
+                    unpack8<InT>(raw[lc], x);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        packed[lc * 4 + e] = pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
+                }
+            }
+            if (b == G::KB - 1) {
+                // this warp's reads of the raw Q slot are done
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[G::B_Q_EMPTY]);
+            }
+            if (b == 0) {
+                if (c > 0 && !mbar_wait(&bar[G::B_QT_EMPTY], (c - 1) & 1, ab, 10)) return false;
+                tc_fence_after();
+            }
+            tmem_st32(tmem + lane_base + G::T_Q + b * 32, packed);
+        }
+        tmem_st_wait();
+    } else {
+        phi_tile<InT, C, D, false, false>(qs, nullptr, nullptr, tw, C, nullptr, 0.f);
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
     return true;
 }
 
-// Second half of the key rows of chunk c, done by the epilogue warpgroup
-// (thread index et = 0..127); arrives on phi_done.  False if aborting.
+// State-only mode: second half of the key rows of chunk c, done by warps
+// 0-3 (thread index et = 0..127); arrives on phi_done.  False if aborting.
 template <int C, int D, bool DECAY, int MODE, typename InT>
 __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *bar, float *Fsm,
-                                                     const AbortCtx ab, uint32_t tmem, long t_begin,
-                                                     long t_end, int c, int nch, int et) {
+                                                     const AbortCtx ab, long t_begin, long t_end, int c,
+                                                     int nch, int et) {
     using G = Cfg<C, D, DECAY, MODE>;
     const int s = c % G::NKV;
     const long t0 = t_begin + (long)chunk_at<G::OUT>(c, nch) * C;
@@ -433,43 +442,9 @@ __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *ba
         if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 16)) return false;
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
     constexpr bool CONV = !std::is_same<InT, bf16>::value;
-    phi_tile<InT, C, D, DECAY, CONV, G::KSPLIT, 4, 4>(kt, kt + 2 * G::TILE, kt + G::TILE, et, n, L,
-                                                     DECAY ? Fsm[G::F_LE + s] : 0.f);
-    if constexpr (G::QSPLIT) {
-        // second column box of phi(Q) for rows 32q + lane -> TMEM
-        const int lane = et & 31, q = et >> 5;
-        if (!mbar_wait(&bar[G::B_Q_FULL], c & 1, ab, 18)) return false;
-        const uint8_t *qs = smem + G::OFF_Q + G::BOXB;
-        const int r = q * 32 + lane;
-        uint4 raw[8];
-#pragma unroll
-        for (int lc = 0; lc < 8; ++lc) raw[lc] = *reinterpret_cast<const uint4 *>(qs + sw128_off(r, lc));
-        uint32_t packed[32];
-#pragma unroll
-        for (int lc = 0; lc < 8; ++lc) {
-            if constexpr (std::is_same<InT, bf16>::value) {
-                const uint4 f = phi_bf16x8(raw[lc]);
-                packed[lc * 4 + 0] = f.x;
-                packed[lc * 4 + 1] = f.y;
-                packed[lc * 4 + 2] = f.z;
-                packed[lc * 4 + 3] = f.w;
-            } else {
-                float x[8];
-                unpack8<InT>(raw[lc], x);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    packed[lc * 4 + e] = pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[G::B_Q_EMPTY]);
-        if (c > 0 && !mbar_wait(&bar[G::B_QT_EMPTY], (c - 1) & 1, ab, 19)) return false;
-        tc_fence_after();
-        tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + G::T_Q + 32, packed);
-        tmem_st_wait();
-    }
+    phi_tile<InT, C, D, DECAY, CONV, 2, 4, 4>(kt, kt + 2 * G::TILE, kt + G::TILE, et, n, L,
+                                             DECAY ? Fsm[G::F_LE + s] : 0.f);
     fence_proxy_async_smem();
-    tc_fence_before();
     __syncwarp();
     if ((et & 31) == 0) mbar_arrive(&bar[G::B_PHI + s]);
     return true;
@@ -502,12 +477,12 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int s = 0; s < G::NKV; ++s) {
             mbar_init(&bar[G::B_KV_FULL + s], 1);
             mbar_init(&bar[G::B_KV_EMPTY + s], 1);
-            mbar_init(&bar[G::B_PHI + s], 8);   // 4 phi warps + 4 epilogue warps
+            mbar_init(&bar[G::B_PHI + s], 8);   // key warps + (query warps | warps 0-3)
             mbar_init(&bar[G::B_L_READY + s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar[G::B_Q_FULL + s], 1);
-            mbar_init(&bar[G::B_Q_EMPTY + s], G::QT ? (G::QSPLIT ? 8 : 4) : 1);
+            mbar_init(&bar[G::B_Q_EMPTY + s], G::QT ? 4 : 1);
         }
         mbar_init(&bar[G::B_QT_EMPTY], 1);
         mbar_init(&bar[G::B_SC_FULL], 1);
@@ -689,16 +664,25 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mma_commit(&bar[G::B_DRAIN]);
             mbar_wait(&bar[G::B_DRAIN], 0, timed, 0);
         }
+    } else if (warp >= kKWarp0) {
+        // ================= keys: decay cumsum and phi(K) (warps 10-13)
+        const int tk = threadIdx.x - kKWarp0 * 32;   // 0..127
+        float Aseg = 1.f;                            // product of chunk decays (state-only mode)
+        float apre[C / 32];                          // decays of the next chunk (warp kKWarp0)
+#pragma unroll
+        for (int h = 0; h < C / 32; ++h) apre[h] = 1.f;
+        float lam = 0.f;   // log2 decay of the chunks already processed (state-only mode)
+        bool ok = true;
+        for (int c = 0; ok && c < nch; ++c)
+            ok = k_stage<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, p, t_begin, t_end, bh, c, nch, tk, Aseg,
+                                                 apre, lam);
+        if constexpr (!G::OUT)
+            if (ok && tk == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = Aseg;
     } else if (warp >= kPhiWarp0) {
-        // ================= feature map, decay, state epilogue (warps 6-9)
+        // ================= phi(Q) and the state epilogue (warps 6-9)
         const int tw = threadIdx.x - kPhiWarp0 * 32;        // 0..127
         const int q = warp & 3;                              // TMEM lane quarter
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        float Aseg = 1.f;  // product of chunk decays (state-only mode)
-        float apre[C / 32];   // decays of the next chunk (warp kPhiWarp0)
-#pragma unroll
-        for (int h = 0; h < C / 32; ++h) apre[h] = 1.f;
-        float lam = 0.f;      // log2 decay of the chunks already processed (state-only mode)
         bool ok = true;
 
         // state rows owned by this thread: TMEM lane quarter q, rows of the
@@ -707,15 +691,18 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const bool srow_ok = lane < SROWS;
         const int a_row = q * SROWS + lane;   // state row (feature index)
 
-        if (nch > 0)
-            ok = phi_stage<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, p, tmem, t_begin, t_end, bh, 0, nch,
-                                                   tw, Aseg, apre, lam);
+        if constexpr (G::OUT)
+            if (nch > 0) ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, 0, tw);
         // ---- segment start: state entering the segment -> TMEM (and operands)
-        if (ok) {
+        if (ok && nch > 0) {
+            float g0 = 1.f;   // decay of chunk 0 (the state is rescaled before its update)
+            if constexpr (DECAY && G::OUT) {
+                ok = mbar_wait(&bar[G::B_L_READY + 0], 0, ab, 17);
+                g0 = Fsm[G::F_G + 0];
+            }
             tc_fence_after();
-            const float g0 = DECAY ? Fsm[G::F_G + 0] : 1.f;
             const float *st = p.ws_state + ((size_t)bh * p.n_seg + seg) * (D * D + D);
-            {
+            if (ok) {
 #pragma unroll 1
                 for (int cb = 0; cb < D / 32; ++cb) {
                     float vals[32];
@@ -738,30 +725,21 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                 }
                 tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[G::B_S_READY]);
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[G::B_S_READY]);
         }
 
-        for (int c = 0; ok && c < nch; ++c) {
-            if (c + 1 < nch) {
-                ok = phi_stage<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, p, tmem, t_begin, t_end, bh, c + 1,
-                                                       nch, tw, Aseg, apre, lam);
-                if (!ok) break;
-            }
-            const bool need = G::OUT || c == nch - 1;
-            if (!need) continue;
-            if (!mbar_wait(&bar[G::B_DS_FULL], G::OUT ? (c & 1) : 0, ab, 11)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t zbits;   // z of this thread's state row after chunk c
-            tmem_ld1(tmem + lane_base + G::T_Z, zbits);
-            const bool last = c == nch - 1;
-            const float gnext = (DECAY && !last) ? Fsm[G::F_G + ((c + 1) % G::NKV)] : 1.f;
-            if (last && !G::OUT) {
-                // state-only mode: write the segment's (dS, dz, A) to the workspace
+        if constexpr (!G::OUT) {
+            // state-only mode: write the segment's (dS, dz) to the workspace
+            // (A is written by the key warps)
+            if (ok && nch > 0 && mbar_wait(&bar[G::B_DS_FULL], 0, ab, 11)) {
+                tc_fence_after();
                 float *dst = p.ws_state + ((size_t)bh * p.n_seg + seg) * (D * D + D);
+                uint32_t zbits;
+                tmem_ld1(tmem + lane_base + G::T_Z, zbits);
 #pragma unroll 1
                 for (int cb = 0; cb < D / 32; ++cb) {
                     uint32_t u[32];
@@ -776,58 +754,69 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                 }
                 if (srow_ok) dst[(size_t)D * D + a_row] = __uint_as_float(zbits);
-                if (tw == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = Aseg;
-                break;
             }
-            if (last && G::OUT) break;   // the final state of a segment is produced by the scan
-            // state entering chunk c+1: bf16 operands, and (decay) rescale in TMEM
-#pragma unroll 1
-            for (int cb = 0; cb < D / 32; ++cb) {
-                uint32_t u[32];
-                tmem_ld32(tmem + lane_base + G::T_S + cb * 32, u);
-                tmem_ld_wait();
-                float vals[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) vals[i] = __uint_as_float(u[i]);
-                if constexpr (G::OUT) if (srow_ok) write_state_row<D>(smem + G::OFF_SBF, a_row, cb * 32, vals);
-                if constexpr (DECAY) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(vals[i] * gnext);
-                    tmem_st32(tmem + lane_base + G::T_S + cb * 32, u);
+        } else {
+            for (int c = 0; ok && c < nch; ++c) {
+                if (c + 1 < nch) {
+                    ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, c + 1, tw);
+                    if (!ok) break;
                 }
-            }
-            if constexpr (G::OUT) {
-                // z entering chunk c+1 (MMAz has added this chunk's w o phi(K) column sums)
+                if (c == nch - 1) break;   // the final state of a segment is produced by the scan
+                if (!mbar_wait(&bar[G::B_DS_FULL], c & 1, ab, 11)) { ok = false; break; }
+                float gnext = 1.f;   // decay of chunk c+1
+                if constexpr (DECAY) {
+                    const int s1 = (c + 1) % G::NKV;
+                    if (!mbar_wait(&bar[G::B_L_READY + s1], ((c + 1) / G::NKV) & 1, ab, 18)) { ok = false; break; }
+                    gnext = Fsm[G::F_G + s1];
+                }
+                tc_fence_after();
+                uint32_t zbits;   // z of this thread's state row entering chunk c+1
+                tmem_ld1(tmem + lane_base + G::T_Z, zbits);
+                // state entering chunk c+1: bf16 operands, and (decay) rescale in TMEM
+#pragma unroll 1
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    uint32_t u[32];
+                    tmem_ld32(tmem + lane_base + G::T_S + cb * 32, u);
+                    tmem_ld_wait();
+                    float vals[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) vals[i] = __uint_as_float(u[i]);
+                    if (srow_ok) write_state_row<D>(smem + G::OFF_SBF, a_row, cb * 32, vals);
+                    if constexpr (DECAY) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(vals[i] * gnext);
+                        tmem_st32(tmem + lane_base + G::T_S + cb * 32, u);
+                    }
+                }
                 if (srow_ok) {
                     bf16 *zb = reinterpret_cast<bf16 *>(smem + G::OFF_ZB);
                     zb[(a_row / 8) * 64 + (a_row % 8)] = __float2bfloat16_rn(__uint_as_float(zbits));
                 }
+                if constexpr (DECAY) {
+                    tmem_st1(tmem + lane_base + G::T_Z, __float_as_uint(__uint_as_float(zbits) * gnext));
+                    tmem_st_wait();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[G::B_S_READY]);
             }
-            if constexpr (DECAY) tmem_st1(tmem + lane_base + G::T_Z, __float_as_uint(__uint_as_float(zbits) * gnext));
-            if constexpr (DECAY) tmem_st_wait();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[G::B_S_READY]);
         }
     } else if constexpr (!G::OUT) {
         // ================= warps 0-3 in state-only mode: second half of phi(K)
         for (int c = 0; c < nch; ++c)
-            if (!phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, tmem, t_begin, t_end, c, nch,
+            if (!phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, t_begin, t_end, c, nch,
                                                               threadIdx.x))
                 break;
     } else {
-        // ================= epilogue (warps 0-3)
+        // ================= epilogue (warps 0-3): scores -> P, output division and store
         const int q = warp;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const bool rvalid_lane = lane < G::ROWS_PER_WARP;
         const int i = q * G::ROWS_PER_WARP + lane;   // row of the chunk held by this thread
-        bool eok = nch == 0 || phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, tmem, t_begin,
-                                                                             t_end, 0, nch, threadIdx.x);
-        for (int c = 0; eok && c < nch; ++c) {
+        for (int c = 0; c < nch; ++c) {
             const int s = c % G::NKV;
             const long t0 = t_begin + (long)c * C;
-            const int n = (int)min((long)C, t_end - t0);
             if (!mbar_wait(&bar[G::B_PHI + s], (c / G::NKV) & 1, ab, 12)) break;
             if (!mbar_wait(&bar[G::B_SC_FULL], c & 1, ab, 13)) break;
             tc_fence_after();
@@ -836,7 +825,6 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // scores -> P, two 32-column blocks per TMEM round trip.  For this
             // warp's rows [r0, r0 + R) a block lies fully below the diagonal
             // (no mask), fully above it (P = 0, scores not read) or on it.
-            // The row sums of P are formed by an MMA (P times ones).
             const int r0 = q * G::ROWS_PER_WARP, r1 = r0 + G::ROWS_PER_WARP - 1;
             float rowsum = 0.f;
 #pragma unroll 1
@@ -858,17 +846,19 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         for (int k = 0; k < 16; ++k) pk[k] = 0u;
                     } else {
                         const bool full = cb * 32 + 31 < r0;   // every j < every row of the warp
-                        float pv[32];
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) {
-                            const int j = cb * 32 + k;
-                            float v = __uint_as_float(u[h][k]);
-                            if constexpr (DECAY) v *= ex2_approx(Li - L[j]);
-                            pv[k] = (full || j <= i) ? v : 0.f;
-                            rowsum += pv[k];
+                        for (int k = 0; k < 16; ++k) {
+                            const int j = cb * 32 + 2 * k;
+                            float v0 = __uint_as_float(u[h][2 * k]), v1 = __uint_as_float(u[h][2 * k + 1]);
+                            if constexpr (DECAY) {
+                                v0 *= ex2_approx(Li - L[j]);
+                                v1 *= ex2_approx(Li - L[j + 1]);
+                            }
+                            v0 = (full || j <= i) ? v0 : 0.f;
+                            v1 = (full || j + 1 <= i) ? v1 : 0.f;
+                            rowsum += v0 + v1;
+                            pk[k] = pack_bf16x2(v0, v1);
                         }
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(pv[2 * k], pv[2 * k + 1]);
                     }
                     if constexpr (G::PT) {
                         tmem_st16(tmem + lane_base + G::T_SC + cb * 16, pk);
@@ -887,51 +877,42 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_P_READY]);
             const float gi = DECAY ? ex2_approx(Li) : 1.f;
-            // while MMA4 runs: the second half of the next chunk's keys
-            if (c + 1 < nch &&
-                !phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, tmem, t_begin, t_end, c + 1,
-                                                              nch, threadIdx.x))
-                break;
 
             if (!mbar_wait(&bar[G::B_O_FULL], c & 1, ab, 14)) break;
             tc_fence_after();
-            // output: one 128-byte-wide column box at a time is scaled, converted,
-            // written swizzled to this warp's staging rows and stored by TMA
-            // (each warp stores its own rows; rows beyond T are clipped)
+            // output: 32 columns per TMEM round trip, scaled, converted and
+            // written swizzled to this warp's staging rows; each completed
+            // 128-byte-wide column box is stored by TMA (each warp stores its
+            // own rows; rows beyond T are clipped)
             constexpr int CPB = 128 / (int)sizeof(OutT);     // columns per box
-            constexpr int NBOX = D / CPB;
+            constexpr int GPB = CPB / 32;                    // 32-column groups per box
             uint8_t *stg = smem + G::OFF_STG + q * (G::ROWS_PER_WARP * 128);   // this warp's rows
             float inv = 0.f;
 #pragma unroll 1
-            for (int bx = 0; bx < NBOX; ++bx) {
-                float o[CPB];
+            for (int g = 0; g < D / 32; ++g) {
+                const int bx = g / GPB, gb = g % GPB;
+                float o[32];
                 {
-                    uint32_t u[CPB], u2[CPB], ud[16];
-                    if (bx == 0) tmem_ld16(tmem + lane_base + G::T_DEN, ud);
-#pragma unroll
-                    for (int h = 0; h < CPB / 32; ++h) {
-                        tmem_ld32(tmem + lane_base + G::T_O + bx * CPB + h * 32,
-                                  *reinterpret_cast<uint32_t(*)[32]>(&u[h * 32]));
-                        if constexpr (G::SPLIT)
-                            tmem_ld32(tmem + lane_base + G::T_O2 + bx * CPB + h * 32,
-                                      *reinterpret_cast<uint32_t(*)[32]>(&u2[h * 32]));
-                    }
+                    uint32_t u[32], u2[32], ud = 0u;
+                    if (g == 0) tmem_ld1(tmem + lane_base + G::T_DEN, ud);
+                    tmem_ld32(tmem + lane_base + G::T_O + g * 32, u);
+                    if constexpr (G::SPLIT) tmem_ld32(tmem + lane_base + G::T_O2 + g * 32, u2);
                     tmem_ld_wait();
-                    if (bx == 0) {
-                        // denominator: (decayed) phi(q).z of the carried state + row sum of P + eps
-                        inv = 1.f / (gi * __uint_as_float(ud[0]) + rowsum + p.eps);
-                    }
+                    // denominator: (decayed) phi(q).z of the carried state + row sum of P + eps
+                    if (g == 0) inv = 1.f / (gi * __uint_as_float(ud) + rowsum + p.eps);
 #pragma unroll
-                    for (int k = 0; k < CPB; ++k) {
+                    for (int k = 0; k < 32; ++k) {
                         if constexpr (G::SPLIT)
                             o[k] = (gi * __uint_as_float(u[k]) + __uint_as_float(u2[k])) * inv;
                         else
                             o[k] = __uint_as_float(u[k]) * inv;
                     }
                 }
-                // this warp's previous store must have read its staging rows
-                if (lane == 0) bulk_wait_read0();
-                __syncwarp();
+                if (gb == 0) {
+                    // this warp's previous store must have read its staging rows
+                    if (lane == 0) bulk_wait_read0();
+                    __syncwarp();
+                }
                 if (rvalid_lane) {
                     if constexpr (sizeof(OutT) == 4) {
 #pragma unroll
@@ -940,7 +921,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 make_float4(o[4 * m], o[4 * m + 1], o[4 * m + 2], o[4 * m + 3]);
                     } else {
 #pragma unroll
-                        for (int m = 0; m < 8; ++m) {
+                        for (int m = 0; m < 4; ++m) {
                             float x[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) x[e] = o[8 * m + e];
@@ -949,15 +930,17 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             else
                                 w = make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]),
                                                pack_f16x2(x[4], x[5]), pack_f16x2(x[6], x[7]));
-                            *reinterpret_cast<uint4 *>(stg + sw128_off(lane, m)) = w;
+                            *reinterpret_cast<uint4 *>(stg + sw128_off(lane, gb * 4 + m)) = w;
                         }
                     }
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_3d(&tm_o, stg, bx * CPB, (int)t0 + q * G::ROWS_PER_WARP, bh);
-                    bulk_commit();
+                if (gb == GPB - 1) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tm_o, stg, bx * CPB, (int)t0 + q * G::ROWS_PER_WARP, bh);
+                        bulk_commit();
+                    }
                 }
             }
             tc_fence_before();
