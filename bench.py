@@ -155,6 +155,12 @@ def barrier(world):
         dist.barrier()
 
 
+def job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: every rank processes ``units_per_rank`` units
+    (weak scaling), and the job takes the slowest rank's ``ms``."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
@@ -389,7 +395,7 @@ def run_ours(args, w):
     clocks = clk.summary()
 
     tokens_per_prefill = w.B * w.T
-    value = world * tokens_per_prefill / (pre_avg * 1e-3)
+    value = job_rate(world, tokens_per_prefill, pre_avg)
     alg_bytes = prefill_algorithmic_bytes(w)
     achieved = alg_bytes / (pre_avg * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -430,7 +436,7 @@ def run_ours(args, w):
         s1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, world)
-        e2e = {"value": world * tokens_per_prefill / (e2e_ms * 1e-3), "unit": UNIT,
+        e2e = {"value": job_rate(world, tokens_per_prefill, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     line = {
@@ -454,7 +460,7 @@ def run_ours(args, w):
         dbytes = decode_bytes_per_step(dec["w"])
         per_step_ms = dec_avg / args.decode_steps
         line["decode"] = {
-            "value": world * 1e3 / per_step_ms, "unit": "steps/s", "steps_per_bench_step": args.decode_steps,
+            "value": job_rate(world, 1, per_step_ms), "unit": "steps/s", "steps_per_bench_step": args.decode_steps,
             "B": dec["w"].B, "H": dec["w"].H, "d": dec["w"].d, "us_per_step": per_step_ms * 1e3,
             "roofline": {"bound": "hbm", "achieved": dbytes / (per_step_ms * 1e-3) / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
