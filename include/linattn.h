@@ -84,6 +84,24 @@ la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtyp
                             la_state_mode mode, void *out, la_dtype out_dtype,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * la_prefill_causal_ev — la_prefill_causal that also records caller-owned
+ * CUDA events on `stream` at the boundaries of the kernels it launches, so a
+ * caller can time each pass on the device without synchronising:
+ *   events[0] before the state pass (K1), events[1] before the segment scan,
+ *   events[2] before the output pass, events[3] after it.
+ * `events` is NULL (then this is la_prefill_causal) or an array of 4
+ * cudaEvent_t created by the caller (a NULL entry is skipped); the library
+ * records them and never creates, waits on or destroys them.  A failed record
+ * returns LA_ERR_CUDA.  On the T == 0 / B*H == 0 paths nothing is recorded.
+ */
+la_status la_prefill_causal_ev(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                               const float *decay, int B, int H, int T, int d_k, int d_v,
+                               float eps, int chunk, float *state_S, float *state_z,
+                               la_state_mode mode, void *out, la_dtype out_dtype,
+                               void *workspace, size_t workspace_bytes, void *stream,
+                               void *const *events);
+
 /* Bytes of workspace la_prefill_causal needs for these sizes (0 if none). */
 size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chunk);
 
@@ -165,6 +183,13 @@ const char *la_last_error_string(void);
  * chunk 128 with decay needs more tensor memory than an SM has and runs on
  * the CUDA-core kernels. */
 int la_prefill_path(la_dtype in_dtype, int d_k, int d_v, int chunk, int has_decay);
+
+/* The segment plan la_prefill_causal uses for these sizes: each head's T
+ * tokens are cut into *n_seg segments of *seg_len tokens (the last may be
+ * shorter), one CTA per segment.  Host-only, launches nothing.  Returns
+ * LA_ERR_INVALID_ARG for negative sizes, null outputs or chunk not in
+ * {64, 128}. */
+la_status la_prefill_plan(int B, int H, int T, int d_k, int chunk, int *n_seg, int *seg_len);
 
 /* Number of kernels this library has launched in this process so far, over
  * all entry points and devices (kernels later replayed from a captured CUDA

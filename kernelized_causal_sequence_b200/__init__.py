@@ -60,6 +60,9 @@ def lib() -> ctypes.CDLL:
         L.la_prefill_causal.restype = _i
         L.la_prefill_causal.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _i, _vp,
                                         _vp, _i, _vp, _i, _vp, _sz, _vp]
+        L.la_prefill_causal_ev.restype = _i
+        L.la_prefill_causal_ev.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _i, _vp,
+                                           _vp, _i, _vp, _i, _vp, _sz, _vp, _vp]
         L.la_prefill_workspace_size.restype = _sz
         L.la_prefill_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
         L.la_forward_noncausal.restype = _i
@@ -72,6 +75,8 @@ def lib() -> ctypes.CDLL:
                                      _i, _vp]
         L.la_status_string.restype = ctypes.c_char_p
         L.la_status_string.argtypes = [_i]
+        L.la_prefill_plan.restype = _i
+        L.la_prefill_plan.argtypes = [_i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)]
         L.la_prefill_path.restype = _i
         L.la_prefill_path.argtypes = [_i, _i, _i, _i, _i]
         L.la_launch_count.restype = ctypes.c_uint64
@@ -92,6 +97,13 @@ def la_status_string(status: int) -> str:
 
 def la_prefill_workspace_size(B, H, T, d_k, d_v, chunk) -> int:
     return int(lib().la_prefill_workspace_size(B, H, T, d_k, d_v, chunk))
+
+
+def la_prefill_plan(B, H, T, d_k, chunk):
+    """(segments per head, tokens per segment) of la_prefill_causal's plan."""
+    n, sl = ctypes.c_int(0), ctypes.c_int(0)
+    _check("la_prefill_plan", lib().la_prefill_plan(B, H, T, d_k, chunk, ctypes.byref(n), ctypes.byref(sl)))
+    return n.value, sl.value
 
 
 def la_noncausal_workspace_size(B, H, Lk, d_k, d_v) -> int:
@@ -124,11 +136,14 @@ def _workspace(nbytes, device):
 
 
 def la_prefill_causal(q, k, v, decay=None, eps=1e-6, chunk=64, state_S=None, state_z=None,
-                      mode=None, out=None, out_dtype=None, workspace=None, stream=None):
+                      mode=None, out=None, out_dtype=None, workspace=None, stream=None,
+                      events=None):
     """Causal chunked prefill.  q, k: [B,H,T,d_k]; v: [B,H,T,d_v] (f32/bf16/f16, CUDA,
     contiguous); decay: [B,H,T] fp32 or None.  state_S [B,H,d_k,d_v] / state_z [B,H,d_k]
     fp32 with ``mode`` LA_STATE_NONE/OUT/INOUT (default: OUT if given, else NONE).
-    Returns ``out`` [B,H,T,d_v]."""
+    ``events``: None, or 4 recorded-once ``torch.cuda.Event(enable_timing=True)``
+    objects that la_prefill_causal_ev records around the state pass, the scan and
+    the output pass.  Returns ``out`` [B,H,T,d_v]."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     out_dtype = q.dtype if out_dtype is None else out_dtype
@@ -138,11 +153,21 @@ def la_prefill_causal(q, k, v, decay=None, eps=1e-6, chunk=64, state_S=None, sta
         mode = LA_STATE_OUT if state_S is not None else LA_STATE_NONE
     if workspace is None:
         workspace = _workspace(la_prefill_workspace_size(B, H, T, dk, dv, chunk), q.device)
-    st = lib().la_prefill_causal(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(decay), B, H, T,
-                                 dk, dv, float(eps), int(chunk), _ptr(state_S), _ptr(state_z),
-                                 int(mode), _ptr(out), _DT[out.dtype], _ptr(workspace),
-                                 workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("la_prefill_causal", st)
+    args = (_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(decay), B, H, T, dk, dv, float(eps),
+            int(chunk), _ptr(state_S), _ptr(state_z), int(mode), _ptr(out), _DT[out.dtype],
+            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if events is None:
+        st = lib().la_prefill_causal(*args)
+        _check("la_prefill_causal", st)
+    else:
+        if len(events) != 4:
+            raise ValueError("events: 4 CUDA events")
+        for e in events:   # torch creates the CUDA event at its first record
+            if int(e.cuda_event) == 0:
+                e.record()
+        arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(int(e.cuda_event)) for e in events])
+        st = lib().la_prefill_causal_ev(*args, arr)
+        _check("la_prefill_causal_ev", st)
     return out
 
 

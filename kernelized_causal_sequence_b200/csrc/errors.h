@@ -16,4 +16,10 @@ inline la_status cuda_check(const char *where, cudaError_t e) {
     return e == cudaSuccess ? LA_OK : cuda_fail(where, e);
 }
 
+// Records caller event i of `events` (an array of cudaEvent_t, or null) on st.
+inline la_status record_event(void *const *events, int i, cudaStream_t st) {
+    if (events == nullptr || events[i] == nullptr) return LA_OK;
+    return cuda_check("event record", cudaEventRecord((cudaEvent_t)events[i], st));
+}
+
 }  // namespace la

@@ -73,6 +73,7 @@ namespace {
 // ---------------------------------------------------------------- SIMT path
 template <typename InT, typename OutT, int D>
 la_status simt_causal(SimtParams p, cudaStream_t st) {
+    if (record_event(p.events, 0, st) != LA_OK) return LA_ERR_CUDA;
     {
         auto k1 = simt_segment_state_kernel<InT, D>;
         const size_t sm = simt_state_smem<D>();
@@ -80,9 +81,11 @@ la_status simt_causal(SimtParams p, cudaStream_t st) {
         if (e != LA_OK) return e;
         k1<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p, p.T);
     }
+    if (record_event(p.events, 1, st) != LA_OK) return LA_ERR_CUDA;
     if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, D, p.mode, p.state_S, p.state_z,
                             nullptr, st) != LA_OK)
         return LA_ERR_CUDA;
+    if (record_event(p.events, 2, st) != LA_OK) return LA_ERR_CUDA;
     {
         auto k3 = simt_chunk_output_kernel<InT, OutT, D>;
         const size_t sm = simt_output_smem<D>();
@@ -91,7 +94,9 @@ la_status simt_causal(SimtParams p, cudaStream_t st) {
         k3<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p);
     }
     count_launches(2);
-    return cuda_check("causal kernel launch", cudaGetLastError());
+    la_status e = cuda_check("causal kernel launch", cudaGetLastError());
+    if (e != LA_OK) return e;
+    return record_event(p.events, 3, st);
 }
 
 template <typename InT, typename OutT, int D>
@@ -218,6 +223,15 @@ const char *la_status_string(la_status s) {
     }
 }
 
+la_status la_prefill_plan(int B, int H, int T, int d_k, int chunk, int *n_seg, int *seg_len) {
+    if (B < 0 || H < 0 || T < 0 || d_k <= 0 || !n_seg || !seg_len || (chunk != 64 && chunk != 128))
+        return LA_ERR_INVALID_ARG;
+    const Plan pl = make_plan((long)B * H, T > 0 ? T : 1, chunk, d_k);
+    *n_seg = pl.n_seg;
+    *seg_len = pl.seg_len;
+    return LA_OK;
+}
+
 int la_prefill_path(la_dtype in_dtype, int d_k, int d_v, int chunk, int has_decay) {
     if (!dtype_ok(in_dtype) || d_k != d_v || !dim_ok(d_k) || (chunk != 64 && chunk != 128))
         return -1;
@@ -244,6 +258,16 @@ la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtyp
                             int chunk, float *state_S, float *state_z, la_state_mode mode,
                             void *out, la_dtype out_dtype, void *workspace,
                             size_t workspace_bytes, void *stream) {
+    return la_prefill_causal_ev(q, k, v, in_dtype, decay, B, H, T, d_k, d_v, eps, chunk, state_S,
+                                state_z, mode, out, out_dtype, workspace, workspace_bytes, stream,
+                                nullptr);
+}
+
+la_status la_prefill_causal_ev(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                               const float *decay, int B, int H, int T, int d_k, int d_v, float eps,
+                               int chunk, float *state_S, float *state_z, la_state_mode mode,
+                               void *out, la_dtype out_dtype, void *workspace,
+                               size_t workspace_bytes, void *stream, void *const *events) {
     la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
     if (s != LA_OK) return s;
     if (B < 0 || H < 0 || T < 0) return LA_ERR_INVALID_ARG;
@@ -280,6 +304,7 @@ la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtyp
         a.state_S = state_S; a.state_z = state_z; a.mode = mode;
         a.BH = BH; a.T = T; a.D = d_k; a.chunk = chunk; a.seg_len = pl.seg_len;
         a.n_seg = pl.n_seg; a.eps = eps;
+        a.events = events;
         return tc_causal(a, st);
     }
     SimtParams p;
@@ -291,6 +316,7 @@ la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtyp
     p.state_S = state_S; p.state_z = state_z; p.mode = mode;
     p.BH = (int)BH; p.T = T; p.Lq = T; p.chunk = chunk; p.seg_len = pl.seg_len; p.n_seg = pl.n_seg;
     p.eps = eps;
+    p.events = events;
     return dispatch3<SimtCausalF>(in_dtype, out_dtype, d_k, p, st);
 }
 

@@ -34,6 +34,7 @@ struct SimtParams {
     int mode;               // la_state_mode
     int BH, T, Lq, chunk, seg_len, n_seg;
     float eps;
+    void *const *events;    // host only: 4 cudaEvent_t recorded around K1, K2, K3, or null
 };
 
 constexpr int kSimtThreads = 256;

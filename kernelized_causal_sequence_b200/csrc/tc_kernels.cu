@@ -49,13 +49,13 @@ bool make_map(CUtensorMap *m, const void *base, la_dtype dt, long BH, int T, int
 
 template <int C, int D, bool DECAY, int MODE, typename InT, typename OutT>
 la_status launch_tc(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                    const CUtensorMap &mo, const tc::TcParams &p, long BH, cudaStream_t st) {
+                    const CUtensorMap &mo, const tc::TcParams &p, long BH, int n_ctas_x, cudaStream_t st) {
     using G = tc::Cfg<C, D, DECAY, MODE>;
     auto kern = tc::tc_prefill_kernel<C, D, DECAY, MODE, InT, OutT>;
     la_status e = cuda_check("tensor-core kernel smem attribute",
                              cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES));
     if (e != LA_OK) return e;
-    kern<<<dim3(p.n_seg, (unsigned)BH), tc::kThreads, G::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    kern<<<dim3(n_ctas_x, (unsigned)BH), tc::kThreads, G::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
     count_launches(1);
     return cuda_check("tensor-core kernel launch", cudaGetLastError());
 }
@@ -79,15 +79,21 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
     p.eps = a.eps;
     la_status e0 = cuda_check("status memset", cudaMemsetAsync(a.status, 0, sizeof(int), st));
     if (e0 != LA_OK) return e0;
-    // K1: per-segment state contributions
-    la_status s = launch_tc<C, D, DECAY, tc::kStateOnly, InT, float>(mq, mk, mv, mo, p, a.BH, st);
+    la_status s = record_event(a.events, 0, st);
     if (s != LA_OK) return s;
+    // K1: per-segment state contributions
+    s = launch_tc<C, D, DECAY, tc::kStateOnly, InT, float>(mq, mk, mv, mo, p, a.BH, a.n_seg, st);
+    if (s != LA_OK) return s;
+    if ((s = record_event(a.events, 1, st)) != LA_OK) return s;
     // K2: decayed exclusive scan over segments (+ state in/out)
     s = launch_segment_scan(a.ws_state, a.ws_A, a.BH, a.n_seg, D, a.mode, a.state_S, a.state_z,
                             nullptr, st);
     if (s != LA_OK) return s;
+    if ((s = record_event(a.events, 2, st)) != LA_OK) return s;
     // K3: chunked output from the segment-entry states
-    return launch_tc<C, D, DECAY, tc::kOutput, InT, OutT>(mq, mk, mv, mo, p, a.BH, st);
+    s = launch_tc<C, D, DECAY, tc::kOutput, InT, OutT>(mq, mk, mv, mo, p, a.BH, a.n_seg, st);
+    if (s != LA_OK) return s;
+    return record_event(a.events, 3, st);
 }
 
 template <typename InT, typename OutT>

@@ -18,6 +18,7 @@ struct TcCausalArgs {
     long BH;
     int T, D, chunk, seg_len, n_seg;
     float eps;
+    void *const *events;   // 4 cudaEvent_t recorded around K1, K2, K3, or null
 };
 
 struct TcNoncausalArgs {

@@ -119,3 +119,14 @@ def test_header_documents_each_entry_point():
     for name in ("la_prefill_causal", "la_forward_noncausal", "la_decode_step"):
         i = src.index(name + "(")
         assert "/*" in src[max(0, i - 1500):i], f"{name} lacks a comment block"
+
+
+def test_prefill_plan(L):
+    # long-context workload: 16 heads x 1024 chunks of 128 -> 9 segments (144 CTAs)
+    assert la.la_prefill_plan(1, 16, 131072, 128, 128) == (9, 14592)
+    # SSD workload: 32 heads x 128 chunks of 64 -> 4 segments (128 CTAs)
+    assert la.la_prefill_plan(2, 16, 8192, 128, 64) == (4, 2048)
+    n, sl = la.la_prefill_plan(1, 1, 5000, 128, 64)
+    assert n * sl >= 5000 and (n - 1) * sl < 5000 and sl % 64 == 0
+    with pytest.raises(la.LinAttnError):
+        la.la_prefill_plan(1, 1, 100, 64, 96)
