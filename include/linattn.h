@@ -179,9 +179,9 @@ const char *la_last_error_string(void);
 /* Which kernel family la_prefill_causal would run for these arguments
  * (has_decay: whether a decay array is passed): 0 = fp32 CUDA-core (SIMT)
  * kernels, 1 = tcgen05 tensor-core kernels, -1 = unsupported.  Host-only,
- * launches nothing.  Tensor cores take 16-bit inputs with d in {64, 128};
- * chunk 128 with decay needs more tensor memory than an SM has and runs on
- * the CUDA-core kernels. */
+ * launches nothing.  Tensor cores take 16-bit inputs with d in {64, 128}
+ * (either chunk, with or without decay); fp32 inputs and d = 32 run on the
+ * CUDA cores. */
 int la_prefill_path(la_dtype in_dtype, int d_k, int d_v, int chunk, int has_decay);
 
 /* The segment plan la_prefill_causal uses for these sizes: each head's T

@@ -149,10 +149,10 @@ la_status dispatch3(la_dtype in, la_dtype out, int D, Args... args) {
 template <typename IT, typename OT, int D> struct SimtCausalF {
     static la_status run(SimtParams p, cudaStream_t st) { return simt_causal<IT, OT, D>(p, st); }
 };
-// Head dim 32: column-per-lane state and read-out kernels (nc32_kernels.cuh).
+// Head dim 32: register-blocked CUDA-core state and read-out kernels (nc32_kernels.cuh).
 template <typename InT, typename OutT>
 la_status nc32_noncausal(SimtParams p, int Lk, cudaStream_t st) {
-    nc32_state_kernel<InT><<<dim3(p.n_seg, p.BH), kNc32Warps * 32, 0, st>>>(
+    nc32_state_kernel<InT><<<dim3(p.n_seg, p.BH), kNc32Threads, 0, st>>>(
         (const InT *)p.k, (const InT *)p.v, Lk, p.seg_len, p.n_seg, p.ws_state, p.ws_A);
     count_launches(1);
     la_status e = cuda_check("nc32 state launch", cudaGetLastError());
@@ -162,7 +162,7 @@ la_status nc32_noncausal(SimtParams p, int Lk, cudaStream_t st) {
     if (e != LA_OK) return e;
     if (p.Lq > 0) {
         nc32_readout_kernel<InT, OutT>
-            <<<dim3((p.Lq + kNc32Queries - 1) / kNc32Queries, p.BH), kNc32Warps * 32, 0, st>>>(
+            <<<dim3((p.Lq + kNc32Queries - 1) / kNc32Queries, p.BH), kNc32Threads, 0, st>>>(
                 (const InT *)p.q, p.Lq, p.ws_total, p.eps, (OutT *)p.out);
         count_launches(1);
         e = cuda_check("nc32 read-out launch", cudaGetLastError());

@@ -3,123 +3,226 @@
 // S = phi(K)^T V, z = sum_j phi(k_j), out_i = phi(q_i)^T S / (phi(q_i)^T z + eps)).
 //
 // At d = 32 the per-token contraction is 32 x 32, too narrow for the
-// tensor-core shapes (M >= 64) and small enough that the work is bound by
-// memory traffic.  Both kernels give each lane of a warp one column of the
-// 32 x 32 state, so that a whole row of phi(k) or phi(q) is one broadcast
-// read of shared memory and 32 fused multiply-adds per lane.
+// tensor-core shapes (M >= 64), and the work is bound by memory traffic and
+// FMA issue.  Both kernels stage tiles of 128 rows through shared memory with
+// 16-byte coalesced loads (the next tile's loads are in flight while the
+// current one is used) and give every thread a 4 x 4 block of outputs, so each
+// pair of shared-memory loads feeds 16 fused multiply-adds.
 #pragma once
 #include "common.cuh"
 
 namespace la {
 
-constexpr int kNc32Warps = 8;
-constexpr int kNc32Batch = 8;   // keys staged per warp per step
+constexpr int kNc32Threads = 256;
+constexpr int kNc32Tile = 128;   // rows (keys or queries) per shared-memory tile
+
+// 16-byte chunks of one [kNc32Tile][32] tile that each thread loads.
+template <typename InT> struct Nc32Io {
+    static constexpr int ELEMS = 16 / (int)sizeof(InT);            // elements per chunk
+    static constexpr int CPR = 32 / ELEMS;                          // chunks per row
+    static constexpr int NLD = kNc32Tile * CPR / kNc32Threads;      // chunks per thread
+};
+
+template <typename InT>
+__device__ __forceinline__ void nc32_unpack(const uint4 &u, float (&x)[Nc32Io<InT>::ELEMS]);
+template <> __device__ __forceinline__ void nc32_unpack<float>(const uint4 &u, float (&x)[4]) {
+    x[0] = __uint_as_float(u.x); x[1] = __uint_as_float(u.y);
+    x[2] = __uint_as_float(u.z); x[3] = __uint_as_float(u.w);
+}
+template <> __device__ __forceinline__ void nc32_unpack<bf16>(const uint4 &u, float (&x)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+template <> __device__ __forceinline__ void nc32_unpack<f16>(const uint4 &u, float (&x)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+
+// Loads this thread's chunks of rows [r0, r0 + kNc32Tile) of a [*, 32] matrix
+// (rows >= r1 read as zero).
+template <typename InT>
+__device__ __forceinline__ void nc32_load_tile(const InT *__restrict__ base, long r0, long r1,
+                                               uint4 (&raw)[Nc32Io<InT>::NLD]) {
+    using I = Nc32Io<InT>;
+#pragma unroll
+    for (int i = 0; i < I::NLD; ++i) {
+        const int u = threadIdx.x + kNc32Threads * i;
+        const long r = r0 + u / I::CPR;
+        raw[i] = (r < r1) ? *reinterpret_cast<const uint4 *>(base + r * 32 + (u % I::CPR) * I::ELEMS)
+                          : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
 
 // Per-segment partial state over keys [s*seg_len, min(Lk, (s+1)*seg_len)).
+// Thread t owns rows a0..a0+3 and columns b0..b0+3 of S (a0 = 4*((t%64)/8),
+// b0 = 4*(t%8)) for the keys of one quarter of each tile (t/64); the four
+// quarters are added at the end in a fixed order (deterministic).
 // grid (n_seg, BH), 256 threads; writes ws_state[bh][seg] = (S, z) and
 // ws_A[bh][seg] = 1 (no decay), the layout the segment scan consumes.
 template <typename InT>
-__global__ void __launch_bounds__(kNc32Warps * 32)
+__global__ void __launch_bounds__(kNc32Threads)
 nc32_state_kernel(const InT *__restrict__ k, const InT *__restrict__ v, int Lk, int seg_len,
                   int n_seg, float *__restrict__ ws_state, float *__restrict__ ws_A) {
-    __shared__ float fk[kNc32Warps][kNc32Batch][32];
-    __shared__ float red[kNc32Warps][33][32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    using I = Nc32Io<InT>;
+    // phi(k) rows, v rows; after the last tile the same memory holds the
+    // per-quarter partial (S, z) for the final sum
+    __shared__ __align__(16) float sm[2 * kNc32Tile * 32];
+    float(*fk)[32] = reinterpret_cast<float(*)[32]>(sm);
+    float(*vv)[32] = reinterpret_cast<float(*)[32]>(sm + kNc32Tile * 32);
+    float(*red)[33][32] = reinterpret_cast<float(*)[33][32]>(sm);
+    static_assert(4 * 33 * 32 <= 2 * kNc32Tile * 32, "reduction fits the tile buffers");
+    const int t = threadIdx.x, kg = t >> 6, a0 = ((t & 63) >> 3) * 4, b0 = (t & 7) * 4;
     const int seg = blockIdx.x, bh = blockIdx.y;
     const long j0 = (long)seg * seg_len, j1 = min((long)Lk, j0 + seg_len);
     const InT *K = k + (size_t)bh * Lk * 32;
     const InT *V = v + (size_t)bh * Lk * 32;
-    float S[32];   // column `lane` of this warp's partial state
+    float acc[4][4] = {}, zacc[4] = {};
+    uint4 rk[I::NLD], rv[I::NLD];
+    nc32_load_tile<InT>(K, j0, j1, rk);
+    nc32_load_tile<InT>(V, j0, j1, rv);
+#pragma unroll 1
+    for (long jt = j0; jt < j1; jt += kNc32Tile) {
+        __syncthreads();   // the previous tile has been used
 #pragma unroll
-    for (int a = 0; a < 32; ++a) S[a] = 0.f;
-    float z = 0.f;  // z[lane]
-    for (long jb = j0 + (long)warp * kNc32Batch; jb < j1; jb += (long)kNc32Warps * kNc32Batch) {
-        float vb[kNc32Batch];
+        for (int i = 0; i < I::NLD; ++i) {
+            const int u = t + kNc32Threads * i, row = u / I::CPR, col = (u % I::CPR) * I::ELEMS;
+            const bool valid = jt + row < j1;
+            float x[I::ELEMS], y[I::ELEMS];
+            nc32_unpack<InT>(rk[i], x);
+            nc32_unpack<InT>(rv[i], y);
 #pragma unroll
-        for (int t = 0; t < kNc32Batch; ++t) {
-            const long j = jb + t;
-            float kf = 0.f, vf = 0.f;
-            if (j < j1) {
-                kf = phi_precise(to_f32(K[(size_t)j * 32 + lane]));
-                vf = to_f32(V[(size_t)j * 32 + lane]);
-            }
-            fk[warp][t][lane] = kf;
-            vb[t] = vf;
-            z += kf;
-        }
-        __syncwarp();
-#pragma unroll
-        for (int t = 0; t < kNc32Batch; ++t) {
-            const float4 *row = reinterpret_cast<const float4 *>(fk[warp][t]);
-#pragma unroll
-            for (int a4 = 0; a4 < 8; ++a4) {
-                const float4 f = row[a4];
-                S[4 * a4 + 0] = fmaf(f.x, vb[t], S[4 * a4 + 0]);
-                S[4 * a4 + 1] = fmaf(f.y, vb[t], S[4 * a4 + 1]);
-                S[4 * a4 + 2] = fmaf(f.z, vb[t], S[4 * a4 + 2]);
-                S[4 * a4 + 3] = fmaf(f.w, vb[t], S[4 * a4 + 3]);
+            for (int e = 0; e < I::ELEMS; e += 4) {
+                *reinterpret_cast<float4 *>(&fk[row][col + e]) =
+                    valid ? make_float4(phi_precise(x[e]), phi_precise(x[e + 1]), phi_precise(x[e + 2]),
+                                        phi_precise(x[e + 3]))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(&vv[row][col + e]) = make_float4(y[e], y[e + 1], y[e + 2], y[e + 3]);
             }
         }
-        __syncwarp();
+        __syncthreads();
+        if (jt + kNc32Tile < j1) {   // next tile in flight while this one is used
+            nc32_load_tile<InT>(K, jt + kNc32Tile, j1, rk);
+            nc32_load_tile<InT>(V, jt + kNc32Tile, j1, rv);
+        }
+#pragma unroll 4
+        for (int jj = 0; jj < kNc32Tile / 4; ++jj) {
+            const int j = kg * (kNc32Tile / 4) + jj;
+            const float4 f = *reinterpret_cast<const float4 *>(&fk[j][a0]);
+            const float4 w = *reinterpret_cast<const float4 *>(&vv[j][b0]);
+            const float fa[4] = {f.x, f.y, f.z, f.w}, wb[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(fa[r], wb[c], acc[r][c]);
+                zacc[r] += fa[r];
+            }
+        }
     }
-    // reduce the warps' partials (fixed order: deterministic)
+    // add the four key quarters (fixed order)
+    __syncthreads();   // the tile buffers are reused
 #pragma unroll
-    for (int a = 0; a < 32; ++a) red[warp][a][lane] = S[a];
-    red[warp][32][lane] = z;
+    for (int r = 0; r < 4; ++r) {
+        *reinterpret_cast<float4 *>(&red[kg][a0 + r][b0]) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+        if (b0 == 0) red[kg][32][a0 + r] = zacc[r];
+    }
     __syncthreads();
     float *dst = ws_state + ((size_t)bh * n_seg + seg) * (32 * 32 + 32);
-    for (int e = threadIdx.x; e < 33 * 32; e += kNc32Warps * 32) {
+    for (int e = t; e < 33 * 32; e += kNc32Threads) {
         const int a = e / 32, b = e % 32;
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kNc32Warps; ++w) acc += red[w][a][b];
-        dst[e] = acc;   // rows 0..31 are S[a][b]; row 32 is z[b]
+        dst[e] = ((red[0][a][b] + red[1][a][b]) + red[2][a][b]) + red[3][a][b];   // row 32: z
     }
-    if (threadIdx.x == 0) ws_A[(size_t)bh * n_seg + seg] = 1.f;
+    if (t == 0) ws_A[(size_t)bh * n_seg + seg] = 1.f;
 }
 
-constexpr int kNc32Queries = 32 * kNc32Warps;   // queries per CTA (one 32-query block per warp)
+constexpr int kNc32Queries = 4 * kNc32Tile;   // queries per CTA (four tiles)
+
+template <typename OutT> __device__ __forceinline__ void nc32_store4(OutT *dst, float o0, float o1, float o2, float o3);
+template <> __device__ __forceinline__ void nc32_store4<float>(float *dst, float o0, float o1, float o2, float o3) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(o0, o1, o2, o3);
+}
+template <> __device__ __forceinline__ void nc32_store4<bf16>(bf16 *dst, float o0, float o1, float o2, float o3) {
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(o0, o1), p1 = __floats2bfloat162_rn(o2, o3);
+    *reinterpret_cast<uint2 *>(dst) =
+        make_uint2(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1));
+}
+template <> __device__ __forceinline__ void nc32_store4<f16>(f16 *dst, float o0, float o1, float o2, float o3) {
+    const __half2 p0 = __floats2half2_rn(o0, o1), p1 = __floats2half2_rn(o2, o3);
+    *reinterpret_cast<uint2 *>(dst) =
+        make_uint2(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1));
+}
 
 // out_i = phi(q_i)^T S / (phi(q_i)^T z + eps) with the head's total (S, z).
-// grid (ceil(Lq / 256), BH), 256 threads.
+// phi(q) of a 128-query tile is staged transposed, [feature][query], with the
+// query index XOR-swizzled by 8 x (the feature's 8-column block) so the
+// transposing stores of a warp hit 32 different banks; thread t owns queries
+// i0..i0+3 (i0 = 4*(t/8)) and columns b0..b0+3 (b0 = 4*(t%8)) of each tile.
+// grid (ceil(Lq / 512), BH), 256 threads.
 template <typename InT, typename OutT>
-__global__ void __launch_bounds__(kNc32Warps * 32)
+__global__ void __launch_bounds__(kNc32Threads)
 nc32_readout_kernel(const InT *__restrict__ q, int Lq, const float *__restrict__ total, float eps,
                     OutT *__restrict__ out) {
-    __shared__ float fq[kNc32Warps][32][33];
-    __shared__ float dens[kNc32Warps][32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    using I = Nc32Io<InT>;
+    __shared__ __align__(16) float Ssm[32][32];
+    __shared__ float zsm[32];
+    __shared__ __align__(16) float fq[32][kNc32Tile];
+    const int t = threadIdx.x, i0 = (t >> 3) * 4, b0 = (t & 7) * 4;
     const int bh = blockIdx.y;
     const float *tot = total + (size_t)bh * (32 * 32 + 32);
-    float Sc[32], zr[32];
-#pragma unroll
-    for (int a = 0; a < 32; ++a) {
-        Sc[a] = tot[a * 32 + lane];   // column `lane` of S
-        zr[a] = tot[32 * 32 + a];     // z (every lane)
-    }
-    const long i0 = (long)blockIdx.x * kNc32Queries + (long)warp * 32;
-    if (i0 >= Lq) return;
+    for (int e = t; e < 32 * 32; e += kNc32Threads) Ssm[e / 32][e % 32] = tot[e];
+    if (t < 32) zsm[t] = tot[32 * 32 + t];
+    const long q0 = (long)blockIdx.x * kNc32Queries, q1 = min((long)Lq, q0 + kNc32Queries);
     const InT *Q = q + (size_t)bh * Lq * 32;
     OutT *O = out + (size_t)bh * Lq * 32;
-    const int nq = (int)min(32L, (long)Lq - i0);
-    // stage phi(q) of the block's 32 queries (row i in fq[warp][i][.])
-    for (int i = 0; i < 32; ++i)
-        fq[warp][i][lane] = (i < nq) ? phi_precise(to_f32(Q[(size_t)(i0 + i) * 32 + lane])) : 0.f;
-    __syncwarp();
-    // lane i: denominator of query i
-    {
-        float d = 0.f;
+    uint4 rq[I::NLD];
+    if (q0 < q1) nc32_load_tile<InT>(Q, q0, q1, rq);
+#pragma unroll 1
+    for (long it = q0; it < q1; it += kNc32Tile) {
+        __syncthreads();   // S staged; the previous tile has been used
 #pragma unroll
-        for (int a = 0; a < 32; ++a) d = fmaf(fq[warp][lane][a], zr[a], d);
-        dens[warp][lane] = d + eps;
-    }
-    __syncwarp();
-    // lane b: numerators of column b for the 32 queries
-    for (int i = 0; i < nq; ++i) {
-        float num = 0.f;
+        for (int i = 0; i < I::NLD; ++i) {
+            const int u = t + kNc32Threads * i, row = u / I::CPR, col = (u % I::CPR) * I::ELEMS;
+            float x[I::ELEMS];
+            nc32_unpack<InT>(rq[i], x);
 #pragma unroll
-        for (int a = 0; a < 32; ++a) num = fmaf(fq[warp][i][a], Sc[a], num);
-        O[(size_t)(i0 + i) * 32 + lane] = from_f32<OutT>(num / dens[warp][i]);
+            for (int e = 0; e < I::ELEMS; ++e) {
+                const int c = col + e;
+                fq[c][row ^ ((c >> 3) << 3)] = phi_precise(x[e]);
+            }
+        }
+        __syncthreads();
+        if (it + kNc32Tile < q1) nc32_load_tile<InT>(Q, it + kNc32Tile, q1, rq);
+        float acc[4][4] = {}, den[4] = {};
+#pragma unroll 8
+        for (int a = 0; a < 32; ++a) {
+            const float4 f = *reinterpret_cast<const float4 *>(&fq[a][i0 ^ ((a >> 3) << 3)]);
+            const float4 s = *reinterpret_cast<const float4 *>(&Ssm[a][b0]);
+            const float za = zsm[a];
+            const float fr[4] = {f.x, f.y, f.z, f.w}, sc[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(fr[r], sc[c], acc[r][c]);
+                den[r] = fmaf(fr[r], za, den[r]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const long i = it + i0 + r;
+            if (i < q1) {
+                const float inv = 1.f / (den[r] + eps);
+                nc32_store4<OutT>(O + i * 32 + b0, acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv,
+                                  acc[r][3] * inv);
+            }
+        }
     }
 }
 

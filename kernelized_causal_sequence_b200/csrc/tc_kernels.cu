@@ -100,11 +100,13 @@ template <typename InT, typename OutT>
 la_status dispatch_cd(const TcCausalArgs &a, cudaStream_t st) {
     const bool dec = a.decay != nullptr;
     if (a.D == 128) {
-        if (a.chunk == 128) return dec ? LA_ERR_UNSUPPORTED : run_causal<128, 128, false, InT, OutT>(a, st);
+        if (a.chunk == 128)
+            return dec ? run_causal<128, 128, true, InT, OutT>(a, st) : run_causal<128, 128, false, InT, OutT>(a, st);
         return dec ? run_causal<64, 128, true, InT, OutT>(a, st) : run_causal<64, 128, false, InT, OutT>(a, st);
     }
     if (a.D == 64) {
-        if (a.chunk == 128) return dec ? LA_ERR_UNSUPPORTED : run_causal<128, 64, false, InT, OutT>(a, st);
+        if (a.chunk == 128)
+            return dec ? run_causal<128, 64, true, InT, OutT>(a, st) : run_causal<128, 64, false, InT, OutT>(a, st);
         return dec ? run_causal<64, 64, true, InT, OutT>(a, st) : run_causal<64, 64, false, InT, OutT>(a, st);
     }
     return LA_ERR_UNSUPPORTED;
@@ -116,7 +118,7 @@ bool tc_supported(la_dtype in_dtype, int D, int chunk, bool has_decay) {
     if (in_dtype != LA_BF16 && in_dtype != LA_F16) return false;
     if (D != 64 && D != 128) return false;
     if (chunk != 64 && chunk != 128) return false;
-    if (chunk == 128 && has_decay) return false;   // TMEM budget: see Cfg
+    (void)has_decay;
     return true;
 }
 

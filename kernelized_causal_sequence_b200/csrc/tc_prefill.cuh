@@ -18,7 +18,10 @@
 // the scalar decay.)  With decay, w_j = prod_{l>j in chunk} a_l, the mask is
 // 2^(L_i - L_j) for j <= i (L = chunk-local inclusive cumsum of log2 a), the
 // inter term of row i is scaled by 2^(L_i), and the state is rescaled by the
-// chunk's total decay before each update.
+// chunk's total decay before each update.  MMA1 reads the plain phi(Q) and
+// phi(K); once it has, the two tiles are rescaled in place (rows of phi(Q) by
+// 2^(L_i) for MMA2/MMAd, rows of phi(K) by w_j for MMA3/MMAz), so a single
+// accumulator holds the inter and intra terms and no second K tile is needed.
 //
 // Warp roles (448 threads; at most four warps share a scheduler, which caps
 // registers at 128 per thread):
@@ -29,7 +32,7 @@
 //   warp  5      TMEM allocator and MMA issuer (one elected thread).
 //   warps 6-9    phi(Q) (into TMEM for chunk 128) and the state epilogue
 //                (TMEM S -> bf16 operand, decay rescale).
-//   warps 10-13  decay cumsum and phi(K) (w o phi(K) with decay).
+//   warps 10-13  decay cumsum and phi(K) (then w o phi(K) in place).
 //
 // Every wait is bounded (see tc_ptx.cuh); on expiry the CTA raises its abort
 // flag and the status word, drains its copies and MMAs, frees TMEM, returns.
@@ -60,16 +63,19 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int TILE = C * D * 2;         // bytes of one [C][D] bf16 tile
     static constexpr bool QT = OUT && C == 128;    // phi(Q) held in TMEM
     static constexpr bool PT = OUT && C == 128;    // P held in TMEM
-    static constexpr bool SPLIT = OUT && DECAY;    // separate inter / intra accumulators
+    // With decay the inter term of row i is scaled by 2^(L_i): phi(Q) rows are
+    // rescaled in place once MMA1 has read them, so one accumulator holds
+    // inter + intra; likewise phi(K) becomes w o phi(K) in place for MMA3.
+    static constexpr bool QS = OUT && DECAY;
     // K/V stages: two in output mode (shared memory is full); the state-only
     // pass has room for more, which hides the load latency of its short chunks
-    static constexpr int KV_BYTES = (2 + (DECAY ? 1 : 0)) * C * D * 2;
+    static constexpr int KV_BYTES = 2 * C * D * 2;
     static constexpr int NKV = OUT ? 2 : (KV_BYTES <= 48 * 1024 ? 4 : 3);
     static constexpr int NQ = OUT ? (QT ? 1 : 2) : 0;
     static constexpr int ROWS_PER_WARP = (C == 128) ? 32 : 16;   // M=64 uses lanes 0-15
 
     // ---- shared memory (offsets from a 1024-byte aligned base)
-    static constexpr int KV_STAGE = 2 * TILE + (DECAY ? TILE : 0);  // K, V, (w o phi(K))
+    static constexpr int KV_STAGE = 2 * TILE;                        // K (phi(K) in place), V
     static constexpr int OFF_KV = 0;
     static constexpr int OFF_Q = OFF_KV + NKV * KV_STAGE;
     static constexpr int OFF_SBF = OFF_Q + NQ * TILE;                // S as bf16 MMA operand
@@ -95,7 +101,8 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int B_P_READY = B_SC_FULL + 1, B_MMA4 = B_P_READY + 1;
     static constexpr int B_O_FULL = B_MMA4 + 1, B_O_EMPTY = B_O_FULL + 1;
     static constexpr int B_DS_FULL = B_O_EMPTY + 1, B_S_READY = B_DS_FULL + 1;
-    static constexpr int B_DRAIN = B_S_READY + 1, B_L_READY = B_DRAIN + 1;
+    static constexpr int B_DRAIN = B_S_READY + 1, B_KW_READY = B_DRAIN + 1, B_QS_READY = B_KW_READY + 1;
+    static constexpr int B_L_READY = B_QS_READY + 1;
     static constexpr int NBAR = B_L_READY + NKV;
     static constexpr int OFF_TMEMADDR = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEMADDR + 4;
@@ -105,8 +112,7 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     // ---- TMEM columns
     static constexpr int T_SC = 0;
     static constexpr int T_O = OUT ? C : 0;
-    static constexpr int T_O2 = T_O + (OUT ? D : 0);
-    static constexpr int T_S = T_O2 + (SPLIT ? D : 0);
+    static constexpr int T_S = T_O + (OUT ? D : 0);
     static constexpr int T_Z = T_S + D;                       // z (column 0; MMAz accumulator)
     static constexpr int T_DEN = T_Z + 16;                    // phi(Q) z of the carried state
     static constexpr int T_Q = T_DEN + (OUT ? 16 : 0);
@@ -115,7 +121,7 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
 
     static_assert(D == 64 || D == 128, "tensor-core path: D in {64, 128}");
     static_assert(C == 64 || C == 128, "tensor-core path: chunk in {64, 128}");
-    static_assert(!(C == 128 && DECAY && OUT), "chunk 128 with decay exceeds TMEM");
+
     static_assert(T_USED <= 512, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(OFF_ONES % 16 == 0, "no-swizzle operand alignment");
@@ -220,16 +226,16 @@ __device__ __forceinline__ void write_state_row(uint8_t *sbf, int a, int col0, c
 }
 
 // phi applied in place to a staged [C][D] tile (KB boxes of [C][128 B]),
-// rows >= n zeroed.  With DECAY, w_j phi(k_j) is also written to `kw`
-// (w_j = exp(L_end - L_j)); with FP16 inputs the V tile is converted to bf16.
+// rows >= n zeroed.  With WEIGHT each row is also multiplied by
+// w_r = 2^(Lend - L_r) (the state-only pass: the key's decay to the segment
+// end); with FP16 inputs the V tile is converted to bf16.
 // Thread tw (0..127) owns one 16-byte column chunk of one box on every PH-th
 // row; with PH a multiple of 8 its swizzled chunk position is the same on
 // all its rows, and all loads of a batch are issued before any arithmetic.
-// The tile's rows are split into NPART equal parts; this call does part PART
-// (the two warpgroups each take one part of the key tile).
-template <typename InT, int C, int D, bool DECAY, bool CONVERT_V, int PB = 0, int PE = 1, int NPART = 1>
-__device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *kw, uint8_t *vt, int tw, int n,
-                                         const float *L, float Lend) {
+// The tile's rows are split into NPART equal parts; this call does parts
+// [PB, PE) (the two warpgroups of the state-only pass each take half).
+template <typename InT, int C, int D, bool WEIGHT, bool CONVERT_V, int PB = 0, int PE = 1, int NPART = 1>
+__device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *vt, int tw, int n, const float *L, float Lend) {
     constexpr int KB = D / 64, BOXB = C * 128;
     constexpr int PH = 128 / (8 * KB);
     constexpr int NIT = C / PH;
@@ -251,26 +257,20 @@ __device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *kw, uint8_t *vt
             if constexpr (std::is_same<InT, bf16>::value) {
                 uint4 f = phi_bf16x8(raw[i]);
                 if (!valid) f = make_uint4(0u, 0u, 0u, 0u);
-                *reinterpret_cast<uint4 *>(tile + off) = f;
-                if constexpr (DECAY) {
+                if constexpr (WEIGHT) {
                     const float w = valid ? ex2_approx(Lend - L[r]) : 0.f;
                     const uint32_t w2 = pack_bf16x2(w, w);
-                    *reinterpret_cast<uint4 *>(kw + off) =
-                        make_uint4(mul_bf16x2(f.x, w2), mul_bf16x2(f.y, w2), mul_bf16x2(f.z, w2),
+                    f = make_uint4(mul_bf16x2(f.x, w2), mul_bf16x2(f.y, w2), mul_bf16x2(f.z, w2),
                                    mul_bf16x2(f.w, w2));
                 }
+                *reinterpret_cast<uint4 *>(tile + off) = f;
             } else {
                 float x[8];
                 unpack8<InT>(raw[i], x);
+                const float w = WEIGHT ? (valid ? ex2_approx(Lend - L[r]) : 0.f) : 1.f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = valid ? phi_fast(x[e]) : 0.f;
+                for (int e = 0; e < 8; ++e) x[e] = valid ? phi_fast(x[e]) * w : 0.f;
                 *reinterpret_cast<uint4 *>(tile + off) = pack8_bf16(x);
-                if constexpr (DECAY) {
-                    const float w = valid ? ex2_approx(Lend - L[r]) : 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] *= w;
-                    *reinterpret_cast<uint4 *>(kw + off) = pack8_bf16(x);
-                }
             }
         }
         if constexpr (CONVERT_V) {
@@ -283,6 +283,35 @@ __device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *kw, uint8_t *vt
                 unpack8<InT>(rv[i], y);
                 *reinterpret_cast<uint4 *>(vt + base + (i0 + i) * PH * 128) = pack8_bf16(y);
             }
+        }
+    }
+}
+
+// Multiplies the rows of a staged bf16 [C][D] tile in place: row r by
+// 2^(Lend - L_r) (KEYS: w o phi(K) for the state update, chunk-relative) or by
+// 2^(L_r) (queries: the decay of the carried state at query r).  Same thread
+// mapping as phi_tile, all rows, thread tw = 0..127.
+template <int C, int D, bool KEYS>
+__device__ __forceinline__ void scale_rows(uint8_t *tile, int tw, const float *L, float Lend) {
+    constexpr int KB = D / 64, BOXB = C * 128;
+    constexpr int PH = 128 / (8 * KB);
+    constexpr int NIT = C / PH;
+    constexpr int BATCH = NIT < 8 ? NIT : 8;
+    const int lc = tw & 7, b = (tw >> 3) % KB, ph = tw / (8 * KB);
+    const uint32_t base = b * BOXB + ph * 128 + ((lc ^ (ph & 7)) << 4);
+#pragma unroll 1
+    for (int i0 = 0; i0 < NIT; i0 += BATCH) {
+        uint4 raw[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) raw[i] = *reinterpret_cast<const uint4 *>(tile + base + (i0 + i) * PH * 128);
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            const int r = ph + (i0 + i) * PH;
+            const float w = ex2_approx(KEYS ? Lend - L[r] : L[r]);
+            const uint32_t w2 = pack_bf16x2(w, w);
+            const uint4 f = raw[i];
+            *reinterpret_cast<uint4 *>(tile + base + (i0 + i) * PH * 128) =
+                make_uint4(mul_bf16x2(f.x, w2), mul_bf16x2(f.y, w2), mul_bf16x2(f.z, w2), mul_bf16x2(f.w, w2));
         }
     }
 }
@@ -355,10 +384,12 @@ __device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
     constexpr bool CONV = !std::is_same<InT, bf16>::value;
     const float Lend = DECAY ? Fsm[G::F_LE + s] : 0.f;
+    // output mode: plain phi(K) (MMA1 needs it; the decay weights are applied
+    // in place after MMA1, see k_weight); state-only: w o phi(K) directly
     if constexpr (G::OUT)
-        phi_tile<InT, C, D, DECAY, CONV, 0, 1, 1>(kt, kt + 2 * G::TILE, kt + G::TILE, tk, n, L, Lend);
+        phi_tile<InT, C, D, false, CONV, 0, 1, 1>(kt, kt + G::TILE, tk, n, L, Lend);
     else
-        phi_tile<InT, C, D, DECAY, CONV, 0, 2, 4>(kt, kt + 2 * G::TILE, kt + G::TILE, tk, n, L, Lend);
+        phi_tile<InT, C, D, DECAY, CONV, 0, 2, 4>(kt, kt + G::TILE, tk, n, L, Lend);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
@@ -417,12 +448,67 @@ __device__ __forceinline__ bool q_stage(uint8_t *smem, uint64_t *bar, const Abor
         }
         tmem_st_wait();
     } else {
-        phi_tile<InT, C, D, false, false>(qs, nullptr, nullptr, tw, C, nullptr, 0.f);
+        phi_tile<InT, C, D, false, false>(qs, nullptr, tw, C, nullptr, 0.f);
         fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
+    return true;
+}
+
+// Output mode with decay, keys of chunk c once MMA1 has read phi(K): the tile
+// becomes w o phi(K) in place (w_j = 2^(L_end - L_j)) for MMA3; arrives on
+// kw_ready.  False if aborting.
+template <int C, int D, bool DECAY, int MODE>
+__device__ __forceinline__ bool k_weight(uint8_t *smem, uint64_t *bar, float *Fsm, const AbortCtx ab, int c,
+                                         int tk) {
+    using G = Cfg<C, D, DECAY, MODE>;
+    const int s = c % G::NKV;
+    if (!mbar_wait(&bar[G::B_SC_FULL], c & 1, ab, 21)) return false;
+    scale_rows<C, D, true>(smem + G::OFF_KV + s * G::KV_STAGE, tk, Fsm + G::F_L + s * C, Fsm[G::F_LE + s]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if ((tk & 31) == 0) mbar_arrive(&bar[G::B_KW_READY]);
+    return true;
+}
+
+// Output mode with decay, queries of chunk c once MMA1 has read phi(Q): row i
+// is scaled by 2^(L_i) (the decay of the carried state at query i) for MMA2
+// and MMAd — in TMEM (chunk 128: this thread's row) or in shared memory
+// (chunk 64).  Arrives on qs_ready.  False if aborting.
+template <int C, int D, bool DECAY, int MODE>
+__device__ __forceinline__ bool q_weight(uint8_t *smem, uint64_t *bar, float *Fsm, const AbortCtx ab,
+                                         uint32_t tmem, int c, int tw) {
+    using G = Cfg<C, D, DECAY, MODE>;
+    const int lane = tw & 31, q = (kPhiWarp0 + (tw >> 5)) & 3;
+    const int s = c % G::NKV;
+    if (!mbar_wait(&bar[G::B_SC_FULL], c & 1, ab, 22)) return false;
+    if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 23)) return false;
+    const float *L = Fsm + G::F_L + s * C;
+    tc_fence_after();
+    if constexpr (G::QT) {
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const float w = ex2_approx(L[r]);
+        const uint32_t w2 = pack_bf16x2(w, w);
+#pragma unroll 1
+        for (int b = 0; b < G::KB; ++b) {
+            uint32_t u[32];
+            tmem_ld32(tmem + lane_base + G::T_Q + b * 32, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) u[k] = mul_bf16x2(u[k], w2);
+            tmem_st32(tmem + lane_base + G::T_Q + b * 32, u);
+        }
+        tmem_st_wait();
+    } else {
+        scale_rows<C, D, false>(smem + G::OFF_Q + (c & 1) * G::TILE, tw, L, 0.f);
+        fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar[G::B_QS_READY]);
     return true;
 }
 
@@ -442,8 +528,7 @@ __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *ba
         if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 16)) return false;
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
     constexpr bool CONV = !std::is_same<InT, bf16>::value;
-    phi_tile<InT, C, D, DECAY, CONV, 2, 4, 4>(kt, kt + 2 * G::TILE, kt + G::TILE, et, n, L,
-                                             DECAY ? Fsm[G::F_LE + s] : 0.f);
+    phi_tile<InT, C, D, DECAY, CONV, 2, 4, 4>(kt, kt + G::TILE, et, n, L, DECAY ? Fsm[G::F_LE + s] : 0.f);
     fence_proxy_async_smem();
     __syncwarp();
     if ((et & 31) == 0) mbar_arrive(&bar[G::B_PHI + s]);
@@ -493,6 +578,8 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(&bar[G::B_DS_FULL], 1);
         mbar_init(&bar[G::B_S_READY], 4);
         mbar_init(&bar[G::B_DRAIN], 1);
+        mbar_init(&bar[G::B_KW_READY], 4);   // key warps
+        mbar_init(&bar[G::B_QS_READY], 4);   // query warps
         fence_mbar_init();
     }
     // (output mode) the z operand [16][D] starts zeroed: only its row 0 is used;
@@ -587,7 +674,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int s = c % G::NKV;
                 const uint32_t kt = sb + G::OFF_KV + s * G::KV_STAGE;   // phi(K)
                 const uint64_t dKk = sdesc_sw128(kt, 16, 1024);                        // phi(K), K-major
-                const uint64_t dKm = sdesc_sw128(DECAY ? kt + 2 * G::TILE : kt, G::BOXB, 1024);  // MN-major
+                const uint64_t dKm = sdesc_sw128(kt, G::BOXB, 1024);                   // (w o) phi(K), MN-major
                 const uint64_t dVm = sdesc_sw128(kt + G::TILE, G::BOXB, 1024);         // V, MN-major
                 if (!mbar_wait(&bar[G::B_PHI + s], (c / G::NKV) & 1, ab, 3)) break;
                 tc_fence_after();
@@ -606,8 +693,10 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                     mma_commit(&bar[G::B_SC_FULL]);
                     // MMA2 + MMAd: inter term and its denominator with the state entering c
+                    // (with decay: from the 2^(L_i)-scaled phi(Q))
                     if (!mbar_wait(&bar[G::B_S_READY], c & 1, ab, 5)) break;
                     if (c > 0 && !mbar_wait(&bar[G::B_O_EMPTY], (c - 1) & 1, ab, 6)) break;
+                    if (G::QS && !mbar_wait(&bar[G::B_QS_READY], c & 1, ab, 24)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
@@ -629,6 +718,10 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     tc_fence_after();
                 }
                 // MMA3 + MMAz: state update with this chunk's keys and values
+                if (G::QS) {
+                    if (!mbar_wait(&bar[G::B_KW_READY], c & 1, ab, 25)) break;
+                    tc_fence_after();
+                }
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_ss(tmem + G::T_S, dKm + (uint64_t)((kk * 2048) >> 4),
@@ -643,11 +736,11 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if (!mbar_wait(&bar[G::B_P_READY], c & 1, ab, 7)) break;
                     tc_fence_after();
                     // O (+)= P V
-                    const uint32_t dst = tmem + (G::SPLIT ? G::T_O2 : G::T_O);
+                    const uint32_t dst = tmem + G::T_O;
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk) {
                         const uint64_t bV = dVm + (uint64_t)((kk * 2048) >> 4);
-                        const uint32_t acc = G::SPLIT ? (kk > 0) : 1;
+                        const uint32_t acc = 1;
                         if constexpr (G::PT)
                             mma_ts(dst, tmem + G::T_SC + kk * 8, bV, ID_PV, acc);
                         else
@@ -673,9 +766,11 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int h = 0; h < C / 32; ++h) apre[h] = 1.f;
         float lam = 0.f;   // log2 decay of the chunks already processed (state-only mode)
         bool ok = true;
-        for (int c = 0; ok && c < nch; ++c)
+        for (int c = 0; ok && c < nch; ++c) {
             ok = k_stage<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, p, t_begin, t_end, bh, c, nch, tk, Aseg,
                                                  apre, lam);
+            if constexpr (G::QS) if (ok) ok = k_weight<C, D, DECAY, MODE>(smem, bar, Fsm, ab, c, tk);
+        }
         if constexpr (!G::OUT)
             if (ok && tk == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = Aseg;
     } else if (warp >= kPhiWarp0) {
@@ -757,6 +852,10 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         } else {
             for (int c = 0; ok && c < nch; ++c) {
+                if constexpr (G::QS) {
+                    ok = q_weight<C, D, DECAY, MODE>(smem, bar, Fsm, ab, tmem, c, tw);
+                    if (!ok) break;
+                }
                 if (c + 1 < nch) {
                     ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, c + 1, tw);
                     if (!ok) break;
@@ -876,7 +975,6 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_P_READY]);
-            const float gi = DECAY ? ex2_approx(Li) : 1.f;
 
             if (!mbar_wait(&bar[G::B_O_FULL], c & 1, ab, 14)) break;
             tc_fence_after();
@@ -893,20 +991,14 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int bx = g / GPB, gb = g % GPB;
                 float o[32];
                 {
-                    uint32_t u[32], u2[32], ud = 0u;
+                    uint32_t u[32], ud = 0u;
                     if (g == 0) tmem_ld1(tmem + lane_base + G::T_DEN, ud);
                     tmem_ld32(tmem + lane_base + G::T_O + g * 32, u);
-                    if constexpr (G::SPLIT) tmem_ld32(tmem + lane_base + G::T_O2 + g * 32, u2);
                     tmem_ld_wait();
                     // denominator: (decayed) phi(q).z of the carried state + row sum of P + eps
-                    if (g == 0) inv = 1.f / (gi * __uint_as_float(ud) + rowsum + p.eps);
+                    if (g == 0) inv = 1.f / (__uint_as_float(ud) + rowsum + p.eps);
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        if constexpr (G::SPLIT)
-                            o[k] = (gi * __uint_as_float(u[k]) + __uint_as_float(u2[k])) * inv;
-                        else
-                            o[k] = __uint_as_float(u[k]) * inv;
-                    }
+                    for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(u[k]) * inv;
                 }
                 if (gb == 0) {
                     // this warp's previous store must have read its staging rows

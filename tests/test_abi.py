@@ -62,7 +62,7 @@ def test_prefill_path_selection(L):
     # 16-bit inputs with d in {64, 128} run on tensor cores, except chunk 128 with decay
     assert la.la_prefill_path(la.LA_BF16, 128, 128, 128) == 1
     assert la.la_prefill_path(la.LA_F16, 64, 64, 64, has_decay=True) == 1
-    assert la.la_prefill_path(la.LA_BF16, 128, 128, 128, has_decay=True) == 0
+    assert la.la_prefill_path(la.LA_BF16, 128, 128, 128, has_decay=True) == 1
     assert la.la_prefill_path(la.LA_BF16, 32, 32, 64) == 0
 
 

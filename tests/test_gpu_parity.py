@@ -60,6 +60,10 @@ SMALL = [
     (torch.bfloat16, 128, 3000, 128, False, 1, 2),
     (torch.float16, 32, 300, 128, False, 2, 2),
     (torch.float16, 128, 513, 64, True, 1, 2),
+    # chunk 128 with decay on the tensor cores (in-place decay weights)
+    (torch.bfloat16, 128, 1000, 128, True, 1, 2),
+    (torch.bfloat16, 64, 777, 128, True, 2, 1),
+    (torch.float16, 128, 2500, 128, True, 1, 1),
     # more than 64 segments per head (the scan's shuffle form)
     (torch.bfloat16, 128, 5000, 64, True, 1, 1),
     (torch.float32, 64, 10000, 64, False, 1, 1),
@@ -126,11 +130,27 @@ def test_prefill_deterministic(la):
     assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
 
 
-def test_chunk_64_vs_128_agree(la):
-    q, k, v, _ = _small_inputs(torch.bfloat16, 128, 2000, False, 1, 2, seed=11)
-    o1, _, _ = gpu_prefill(la, q, k, v, None, 64, torch.float32)
-    o2, _, _ = gpu_prefill(la, q, k, v, None, 128, torch.float32)
+@pytest.mark.parametrize("decay", [False, True])
+def test_chunk_64_vs_128_agree(la, decay):
+    q, k, v, a = _small_inputs(torch.bfloat16, 128, 2000, decay, 1, 2, seed=11)
+    o1, S1, _ = gpu_prefill(la, q, k, v, a, 64, torch.float32)
+    o2, S2, _ = gpu_prefill(la, q, k, v, a, 128, torch.float32)
     assert row_rel_err(o1, o2) < 2e-2
+    assert row_rel_err(S1.reshape(1, 2, -1), S2.reshape(1, 2, -1)) < 2e-2
+
+
+def test_workload_ssd_decay_chunk128(la, orc):
+    """The SSD-decay workload's inputs processed with 128-token chunks (the
+    result equals the per-token recurrence up to rounding for any chunk)."""
+    w = W["ssd_decay_bf16_b2h16_t8192_d128"]
+    q, k, v, a = inputs.qkv(w)
+    o = la.la_prefill_causal(q.to(DEV), k.to(DEV), v.to(DEV), decay=a.to(DEV), chunk=128)
+    torch.cuda.synchronize()
+    o = o.float().cpu().numpy()
+    for b, h in ((0, 0), (1, 15)):
+        ro, _, _ = orc.causal(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1],
+                              a[b:b + 1, h:h + 1])
+        assert row_rel_err(o[b:b + 1, h:h + 1], ro) < 2e-2
 
 
 def test_empty_and_state_only(la):
@@ -198,7 +218,9 @@ def test_workload_noncausal(la, orc, cross):
 
 
 @pytest.mark.parametrize("dtype,d,Lq,Lk", [(torch.float32, 64, 100, 333), (torch.bfloat16, 128, 17, 1000),
-                                           (torch.float16, 32, 129, 0), (torch.bfloat16, 64, 0, 50)])
+                                           (torch.float16, 32, 129, 0), (torch.bfloat16, 64, 0, 50),
+                                           (torch.float32, 32, 300, 700), (torch.bfloat16, 32, 1000, 517),
+                                           (torch.float16, 32, 513, 5000)])
 def test_noncausal_small(la, orc, dtype, d, Lq, Lk):
     rng = np.random.default_rng(Lq + Lk)
     mk = lambda L: torch.from_numpy(rng.standard_normal((2, 3, L, d), dtype=np.float32)).to(dtype)
@@ -264,3 +286,16 @@ def test_prefill_then_decode_is_prefill_plus_one(la, orc):
     torch.cuda.synchronize()
     ro, _, _ = orc.causal(q, k, v, a)
     assert row_rel_err(o.cpu().numpy(), ro[:, :, T]) < 2e-2
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_noncausal_d32_native_out(la, orc, dtype):
+    """d = 32 read-out writing the input dtype (ragged query and key tiles)."""
+    rng = np.random.default_rng(32)
+    mk = lambda L: torch.from_numpy(rng.standard_normal((1, 4, L, 32), dtype=np.float32) * 0.5).to(dtype)
+    q, k, v = mk(333), mk(1100), mk(1100)
+    o = la.la_forward_noncausal(q.to(DEV), k.to(DEV), v.to(DEV), out_dtype=dtype)
+    torch.cuda.synchronize()
+    ro, _, _ = orc.noncausal(q, k, v)
+    assert o.dtype == dtype
+    assert row_rel_err(o.float().cpu().numpy(), ro) < 2e-2
