@@ -250,10 +250,18 @@ def measure_workloads(dev, peaks, iters=10, only=None):
     flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     flush = lambda: flush_buf.zero_()
     res = {}
-    for name in ("causal_f32_t256_d64", "causal_bf16_b4h8_t2048_d64", "ssd_decay_bf16_b2h16_t8192_d128"):
+    import dataclasses
+    rows = [("causal_f32_t256_d64", None), ("causal_bf16_b4h8_t2048_d64", None),
+            ("ssd_decay_bf16_b2h16_t8192_d128", None),
+            # the same SSD inputs with 128-token chunks (equal results up to rounding)
+            ("ssd_decay_bf16_b2h16_t8192_d128", 128)]
+    for name, chunk in rows:
         if only is not None and name != only:
             continue
         w = inputs.WORKLOADS[name]
+        if chunk is not None:
+            w = dataclasses.replace(w, chunk=chunk)
+        key = name if chunk is None else f"{name}@chunk{chunk}"
         q, k, v, a = (None if x is None else x.to(dev) for x in inputs.qkv(w))
         out = torch.empty((w.B, w.H, w.T, w.d), dtype=w.torch_out_dtype, device=dev)
         S = torch.zeros((w.B, w.H, w.d, w.d), device=dev)
@@ -265,10 +273,10 @@ def measure_workloads(dev, peaks, iters=10, only=None):
         fn()
         ms = time_calls(fn, iters, flush)
         b = prefill_algorithmic_bytes(w)
-        res[name] = {"ms": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3), "algorithmic_bytes": b,
-                     "hbm_frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                     "path": "tcgen05" if la.la_prefill_path(w.torch_dtype, w.d, w.d, w.chunk, w.decay) == 1
-                     else "simt"}
+        res[key] = {"ms": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3), "algorithmic_bytes": b,
+                    "hbm_frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "chunk": w.chunk,
+                    "path": "tcgen05" if la.la_prefill_path(w.torch_dtype, w.d, w.d, w.chunk, w.decay) == 1
+                    else "simt"}
     w = inputs.WORKLOADS["noncausal_f16_b8h8_l4800_d32"]
     for cross in (False, True):
         if only is not None and only != w.name:

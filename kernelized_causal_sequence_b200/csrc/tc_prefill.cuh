@@ -240,7 +240,9 @@ __device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *vt, int tw, int
     constexpr int PH = 128 / (8 * KB);
     constexpr int NIT = C / PH;
     constexpr int IPART = NIT / NPART;
-    constexpr int BATCH = IPART < 8 ? IPART : 8;
+    // two rows per batch: the loop body stays small (this kernel's warp roles
+    // compete for the instruction cache; measured faster than 4 or 8)
+    constexpr int BATCH = IPART < 2 ? IPART : 2;
     static_assert(NIT % NPART == 0 && IPART % BATCH == 0, "row split");
     const int lc = tw & 7, b = (tw >> 3) % KB, ph = tw / (8 * KB);
     const uint32_t base = b * BOXB + ph * 128 + ((lc ^ (ph & 7)) << 4);
@@ -921,23 +923,24 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_after();
             const float *L = Fsm + G::F_L + s * C;
             const float Li = (DECAY && rvalid_lane) ? L[min(i, C - 1)] : 0.f;
-            // scores -> P, two 32-column blocks per TMEM round trip.  For this
-            // warp's rows [r0, r0 + R) a block lies fully below the diagonal
-            // (no mask), fully above it (P = 0, scores not read) or on it.
+            // scores -> P, one 32-column block per TMEM round trip (small code;
+            // measured faster than two).  For this warp's rows [r0, r0 + R) a
+            // block lies fully below the diagonal (no mask), fully above it
+            // (P = 0, scores not read) or on it.
             const int r0 = q * G::ROWS_PER_WARP, r1 = r0 + G::ROWS_PER_WARP - 1;
             float rowsum = 0.f;
 #pragma unroll 1
-            for (int cb0 = 0; cb0 < C / 32; cb0 += 2) {
-                uint32_t u[2][32];
-                bool live[2];
+            for (int cb0 = 0; cb0 < C / 32; cb0 += 1) {
+                uint32_t u[1][32];
+                bool live[1];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < 1; ++h) {
                     live[h] = (cb0 + h) * 32 <= r1;
                     if (live[h]) tmem_ld32(tmem + lane_base + G::T_SC + (cb0 + h) * 32, u[h]);
                 }
                 tmem_ld_wait();
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < 1; ++h) {
                     const int cb = cb0 + h;
                     uint32_t pk[16];
                     if (!live[h]) {

@@ -67,9 +67,16 @@ __device__ __forceinline__ void raise_abort(const AbortCtx &ab, int code) {
 
 // Bounded wait on a phase parity.  Returns false if the CTA is aborting or
 // the limit expired (then the abort is raised).
+// The polling loop is out of line: it is reached only when the phase is not
+// complete at the first try, and keeping ~25 copies of it inline costs
+// instruction-cache space the working loops need.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, const AbortCtx ab, int code);
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const AbortCtx &ab,
                                           int code) {
     if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, ab, code);
+}
+__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, const AbortCtx ab, int code) {
     const uint64_t t0 = globaltimer_ns();
     uint32_t n = 0;
     while (true) {
