@@ -161,9 +161,11 @@ la_status nc32_noncausal(SimtParams p, int Lk, cudaStream_t st) {
                             p.ws_total, st);
     if (e != LA_OK) return e;
     if (p.Lq > 0) {
+        const int tpc = nc32_tiles_per_cta(p.BH, p.Lq);
+        const long span = (long)tpc * kNc32Tile;
         nc32_readout_kernel<InT, OutT>
-            <<<dim3((p.Lq + kNc32Queries - 1) / kNc32Queries, p.BH), kNc32Threads, 0, st>>>(
-                (const InT *)p.q, p.Lq, p.ws_total, p.eps, (OutT *)p.out);
+            <<<dim3((unsigned)((p.Lq + span - 1) / span), p.BH), kNc32Threads, 0, st>>>(
+                (const InT *)p.q, p.Lq, tpc, p.ws_total, p.eps, (OutT *)p.out);
         count_launches(1);
         e = cuda_check("nc32 read-out launch", cudaGetLastError());
     }

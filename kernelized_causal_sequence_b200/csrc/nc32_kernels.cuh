@@ -64,12 +64,13 @@ __device__ __forceinline__ void nc32_load_tile(const InT *__restrict__ base, lon
 
 // Per-segment partial state over keys [s*seg_len, min(Lk, (s+1)*seg_len)).
 // Thread t owns rows a0..a0+3 and columns b0..b0+3 of S (a0 = 4*((t%64)/8),
-// b0 = 4*(t%8)) for the keys of one quarter of each tile (t/64); the four
-// quarters are added at the end in a fixed order (deterministic).
+// b0 = 4*(t%8)) for the keys of one quarter of each tile (t/64); z is summed
+// per tile by each warp over 16 rows (lane = feature).  The partials are
+// added at the end in a fixed order (deterministic).
 // grid (n_seg, BH), 256 threads; writes ws_state[bh][seg] = (S, z) and
 // ws_A[bh][seg] = 1 (no decay), the layout the segment scan consumes.
 template <typename InT>
-__global__ void __launch_bounds__(kNc32Threads)
+__global__ void __launch_bounds__(kNc32Threads, 4)
 nc32_state_kernel(const InT *__restrict__ k, const InT *__restrict__ v, int Lk, int seg_len,
                   int n_seg, float *__restrict__ ws_state, float *__restrict__ ws_A) {
     using I = Nc32Io<InT>;
@@ -78,14 +79,16 @@ nc32_state_kernel(const InT *__restrict__ k, const InT *__restrict__ v, int Lk, 
     __shared__ __align__(16) float sm[2 * kNc32Tile * 32];
     float(*fk)[32] = reinterpret_cast<float(*)[32]>(sm);
     float(*vv)[32] = reinterpret_cast<float(*)[32]>(sm + kNc32Tile * 32);
-    float(*red)[33][32] = reinterpret_cast<float(*)[33][32]>(sm);
-    static_assert(4 * 33 * 32 <= 2 * kNc32Tile * 32, "reduction fits the tile buffers");
+    float(*red)[32][32] = reinterpret_cast<float(*)[32][32]>(sm);
+    float(*redz)[32] = reinterpret_cast<float(*)[32]>(sm + 4 * 32 * 32);
+    static_assert(4 * 32 * 32 + 8 * 32 <= 2 * kNc32Tile * 32, "reduction fits the tile buffers");
     const int t = threadIdx.x, kg = t >> 6, a0 = ((t & 63) >> 3) * 4, b0 = (t & 7) * 4;
+    const int warp = t >> 5, lane = t & 31;
     const int seg = blockIdx.x, bh = blockIdx.y;
     const long j0 = (long)seg * seg_len, j1 = min((long)Lk, j0 + seg_len);
     const InT *K = k + (size_t)bh * Lk * 32;
     const InT *V = v + (size_t)bh * Lk * 32;
-    float acc[4][4] = {}, zacc[4] = {};
+    float acc[4][4] = {}, zpart = 0.f;   // zpart: z[lane] over this warp's rows of each tile
     uint4 rk[I::NLD], rv[I::NLD];
     nc32_load_tile<InT>(K, j0, j1, rk);
     nc32_load_tile<InT>(V, j0, j1, rv);
@@ -120,30 +123,34 @@ nc32_state_kernel(const InT *__restrict__ k, const InT *__restrict__ v, int Lk, 
             const float4 w = *reinterpret_cast<const float4 *>(&vv[j][b0]);
             const float fa[4] = {f.x, f.y, f.z, f.w}, wb[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(fa[r], wb[c], acc[r][c]);
-                zacc[r] += fa[r];
-            }
         }
+#pragma unroll 4
+        for (int jj = 0; jj < kNc32Tile / 8; ++jj) zpart += fk[warp * (kNc32Tile / 8) + jj][lane];
     }
     // add the four key quarters (fixed order)
     __syncthreads();   // the tile buffers are reused
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < 4; ++r)
         *reinterpret_cast<float4 *>(&red[kg][a0 + r][b0]) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-        if (b0 == 0) red[kg][32][a0 + r] = zacc[r];
-    }
+    redz[warp][lane] = zpart;
     __syncthreads();
     float *dst = ws_state + ((size_t)bh * n_seg + seg) * (32 * 32 + 32);
-    for (int e = t; e < 33 * 32; e += kNc32Threads) {
+    for (int e = t; e < 32 * 32; e += kNc32Threads) {
         const int a = e / 32, b = e % 32;
-        dst[e] = ((red[0][a][b] + red[1][a][b]) + red[2][a][b]) + red[3][a][b];   // row 32: z
+        dst[e] = ((red[0][a][b] + red[1][a][b]) + red[2][a][b]) + red[3][a][b];
+    }
+    if (t < 32) {
+        float zs = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) zs += redz[w][t];
+        dst[32 * 32 + t] = zs;
     }
     if (t == 0) ws_A[(size_t)bh * n_seg + seg] = 1.f;
 }
 
-constexpr int kNc32Queries = 4 * kNc32Tile;   // queries per CTA (four tiles)
 
 template <typename OutT> __device__ __forceinline__ void nc32_store4(OutT *dst, float o0, float o1, float o2, float o3);
 template <> __device__ __forceinline__ void nc32_store4<float>(float *dst, float o0, float o1, float o2, float o3) {
@@ -165,21 +172,25 @@ template <> __device__ __forceinline__ void nc32_store4<f16>(f16 *dst, float o0,
 // query index XOR-swizzled by 8 x (the feature's 8-column block) so the
 // transposing stores of a warp hit 32 different banks; thread t owns queries
 // i0..i0+3 (i0 = 4*(t/8)) and columns b0..b0+3 (b0 = 4*(t%8)) of each tile.
-// grid (ceil(Lq / 512), BH), 256 threads.
+// The denominators of a tile are formed once per query (threads 0..127)
+// before the product loop.  grid (ceil(Lq / (128 * tiles_per_cta)), BH),
+// 256 threads.
 template <typename InT, typename OutT>
-__global__ void __launch_bounds__(kNc32Threads)
-nc32_readout_kernel(const InT *__restrict__ q, int Lq, const float *__restrict__ total, float eps,
-                    OutT *__restrict__ out) {
+__global__ void __launch_bounds__(kNc32Threads, 4)
+nc32_readout_kernel(const InT *__restrict__ q, int Lq, int tiles_per_cta, const float *__restrict__ total,
+                    float eps, OutT *__restrict__ out) {
     using I = Nc32Io<InT>;
     __shared__ __align__(16) float Ssm[32][32];
     __shared__ float zsm[32];
     __shared__ __align__(16) float fq[32][kNc32Tile];
+    __shared__ float inv_den[kNc32Tile];
     const int t = threadIdx.x, i0 = (t >> 3) * 4, b0 = (t & 7) * 4;
     const int bh = blockIdx.y;
     const float *tot = total + (size_t)bh * (32 * 32 + 32);
     for (int e = t; e < 32 * 32; e += kNc32Threads) Ssm[e / 32][e % 32] = tot[e];
     if (t < 32) zsm[t] = tot[32 * 32 + t];
-    const long q0 = (long)blockIdx.x * kNc32Queries, q1 = min((long)Lq, q0 + kNc32Queries);
+    const long span = (long)tiles_per_cta * kNc32Tile;
+    const long q0 = (long)blockIdx.x * span, q1 = min((long)Lq, q0 + span);
     const InT *Q = q + (size_t)bh * Lq * 32;
     OutT *O = out + (size_t)bh * Lq * 32;
     uint4 rq[I::NLD];
@@ -200,25 +211,29 @@ nc32_readout_kernel(const InT *__restrict__ q, int Lq, const float *__restrict__
         }
         __syncthreads();
         if (it + kNc32Tile < q1) nc32_load_tile<InT>(Q, it + kNc32Tile, q1, rq);
-        float acc[4][4] = {}, den[4] = {};
+        if (t < kNc32Tile) {   // denominator of query t of the tile
+            float d = 0.f;
+#pragma unroll 8
+            for (int a = 0; a < 32; ++a) d = fmaf(fq[a][t ^ ((a >> 3) << 3)], zsm[a], d);
+            inv_den[t] = 1.f / (d + eps);
+        }
+        float acc[4][4] = {};
 #pragma unroll 8
         for (int a = 0; a < 32; ++a) {
             const float4 f = *reinterpret_cast<const float4 *>(&fq[a][i0 ^ ((a >> 3) << 3)]);
             const float4 s = *reinterpret_cast<const float4 *>(&Ssm[a][b0]);
-            const float za = zsm[a];
             const float fr[4] = {f.x, f.y, f.z, f.w}, sc[4] = {s.x, s.y, s.z, s.w};
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(fr[r], sc[c], acc[r][c]);
-                den[r] = fmaf(fr[r], za, den[r]);
-            }
         }
+        __syncthreads();   // inv_den of this tile
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const long i = it + i0 + r;
             if (i < q1) {
-                const float inv = 1.f / (den[r] + eps);
+                const float inv = inv_den[i0 + r];
                 nc32_store4<OutT>(O + i * 32 + b0, acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv,
                                   acc[r][3] * inv);
             }

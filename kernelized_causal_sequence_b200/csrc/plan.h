@@ -49,23 +49,33 @@ inline Plan make_plan(long BH, long T, int chunk, int D) {
     return p;
 }
 
-// Key segments of the non-causal form.  At head dim 32 the CUDA-core state
-// kernel runs several CTAs per SM, so aim for ~4 CTAs per SM over all heads,
-// with segments of at least 64 keys; other head dims use the chunk plan.
+// Key segments of the non-causal form.  At head dimension 32 the CUDA-core
+// state kernel fits four 256-thread CTAs per SM, so the plan fills one wave
+// of 4 x 148 CTAs over all heads, with segments of whole 128-key tiles;
+// other head dims use the chunk plan.
+constexpr int kNc32CtasPerSm = 4;
+constexpr int kNc32TileRows = 128;
 inline Plan make_nc_plan(long BH, long Lk, int D) {
     if (D != 32) return make_plan(BH, Lk > 0 ? Lk : 1, kNoncausalChunk, D);
     Plan p;
-    p.chunk = 64;
+    p.chunk = kNc32TileRows;
     const long L = Lk > 0 ? Lk : 1;
-    long segs = (4L * kNumSMs + BH - 1) / BH;
-    const long max_segs = (L + 63) / 64;
-    if (segs > max_segs) segs = max_segs;
+    long segs = (long)kNc32CtasPerSm * kNumSMs / (BH > 0 ? BH : 1);
     if (segs < 1) segs = 1;
     long seg_len = (L + segs - 1) / segs;
-    seg_len = (seg_len + 63) / 64 * 64;
+    seg_len = (seg_len + kNc32TileRows - 1) / kNc32TileRows * kNc32TileRows;
     p.seg_len = (int)seg_len;
     p.n_seg = (int)((L + seg_len - 1) / seg_len);
     return p;
+}
+
+// Query tiles per read-out CTA at head dimension 32: one wave of
+// 4 x 148 CTAs over all heads.
+inline int nc32_tiles_per_cta(long BH, long Lq) {
+    const long tiles = (Lq + kNc32TileRows - 1) / kNc32TileRows;
+    const long slots = (long)kNc32CtasPerSm * kNumSMs;
+    long t = (tiles * BH + slots - 1) / slots;
+    return (int)(t < 1 ? 1 : t);
 }
 
 }  // namespace la
