@@ -279,9 +279,18 @@ def measure_workloads(dev, peaks, iters=10, only=None):
                                           state_z=z, out=out, workspace=ws)
         fn()
         ms = time_calls(fn, iters, flush)
+        # per-pass split of one more (flushed) call, from the library's events
+        kev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush()
+        la.la_prefill_causal(q, k, v, decay=a, eps=w.eps, chunk=w.chunk, state_S=S, state_z=z,
+                             out=out, workspace=ws, events=kev)
+        torch.cuda.synchronize(dev)
+        split = {nm: kev[j].elapsed_time(kev[j + 1]) for j, nm in enumerate(("K1_ms", "K2_ms", "K3_ms"))}
         b = prefill_algorithmic_bytes(w)
         res[key] = {"ms": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3), "algorithmic_bytes": b,
                     "hbm_frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "chunk": w.chunk,
+                    "passes_ms": split,
+                    "segments_per_head": la.la_prefill_plan(w.B, w.H, w.T, w.d, w.chunk)[0],
                     "path": "tcgen05" if la.la_prefill_path(w.torch_dtype, w.d, w.d, w.chunk, w.decay) == 1
                     else "simt"}
     w = inputs.WORKLOADS["noncausal_f16_b8h8_l4800_d32"]
