@@ -40,6 +40,20 @@ struct SimtParams {
 constexpr int kSimtThreads = 256;
 constexpr int kSub = 32;
 
+// This thread's elements of rows [r0, r0 + kSub) of a [*, D] matrix (rows at
+// or beyond r0 + rn read as 0), converted to fp32.  The loads are all issued
+// before any is used, so a tile costs one memory round trip.
+constexpr int simt_per_thread(int D) { return kSub * D / kSimtThreads; }
+template <typename InT, int D>
+__device__ __forceinline__ void simt_load_rows(const InT *base, long r0, int rn,
+                                               float (&x)[simt_per_thread(D)]) {
+#pragma unroll
+    for (int u = 0; u < simt_per_thread(D); ++u) {
+        const int idx = threadIdx.x + u * kSimtThreads, j = idx / D, a = idx % D;
+        x[u] = (j < rn) ? to_f32(base[(size_t)(r0 + j) * D + a]) : 0.f;
+    }
+}
+
 // Chunk-local inclusive cumulative sum of log a (warp 0 only).
 __device__ __forceinline__ void chunk_log_cumsum(const float *a, int n, float *Lc) {
     const int lane = threadIdx.x & 31;
@@ -99,17 +113,21 @@ __global__ void __launch_bounds__(kSimtThreads) simt_segment_state_kernel(SimtPa
             Aseg *= g;
         }
         for (int j0 = 0; j0 < n; j0 += kSub) {
-            for (int idx = tid; idx < kSub * D; idx += kSimtThreads) {
-                const int j = idx / D, a = idx % D;
-                float f = 0.f, x = 0.f;
-                if (j0 + j < n) {
-                    const size_t off = (size_t)(c0 + j0 + j) * D + a;
-                    f = phi_precise(to_f32(K[off]));
-                    if (A) f *= expf(Lend - Lc[j0 + j]);
-                    x = to_f32(V[off]);
+            {
+                float kx[simt_per_thread(D)], vx[simt_per_thread(D)];
+                simt_load_rows<InT, D>(K, c0 + j0, n - j0, kx);
+                simt_load_rows<InT, D>(V, c0 + j0, n - j0, vx);
+#pragma unroll
+                for (int u = 0; u < simt_per_thread(D); ++u) {
+                    const int idx = tid + u * kSimtThreads, j = idx / D;
+                    float f = 0.f;
+                    if (j0 + j < n) {
+                        f = phi_precise(kx[u]);
+                        if (A) f *= expf(Lend - Lc[j0 + j]);
+                    }
+                    fk[idx] = f;
+                    vv[idx] = vx[u];
                 }
-                fk[idx] = f;
-                vv[idx] = x;
             }
             __syncthreads();
             for (int j = 0; j < kSub; ++j) {
@@ -138,7 +156,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_segment_state_kernel(SimtPa
 }
 
 template <int D> __host__ __device__ constexpr size_t simt_output_smem() {
-    return sizeof(float) * (D * D + D + 3 * kSub * D + kSub * (kSub + 1) + 128);
+    return sizeof(float) * (D * D + D + 2 * kSub * (D + 1) + kSub * D + kSub * (kSub + 1) + 128);
 }
 
 // K3: chunked causal output.  grid (n_seg, BH), 256 threads.
@@ -146,12 +164,16 @@ template <typename InT, typename OutT, int D>
 __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtParams p) {
     constexpr int TR = D / 16;
     constexpr int CPT = D / 8;  // output columns per thread (32 rows x 8 column groups)
+    // phi(q) and phi(k) rows are padded to D + 1 floats: the scores loop reads
+    // 32 different key rows at the same column in one warp, and the inter-term
+    // loop 4 different query rows, which would otherwise share a bank
+    constexpr int RS = D + 1;
     extern __shared__ float smem[];
     float *S = smem;                    // [D][D]
     float *z = S + D * D;               // [D]
-    float *fq = z + D;                  // [kSub][D]
-    float *fk = fq + kSub * D;          // [kSub][D]
-    float *vv = fk + kSub * D;          // [kSub][D]
+    float *fq = z + D;                  // [kSub][D + 1]
+    float *fk = fq + kSub * RS;         // [kSub][D + 1]
+    float *vv = fk + kSub * RS;         // [kSub][D]
     float *P = vv + kSub * D;           // [kSub][kSub + 1]
     float *Lc = P + kSub * (kSub + 1);  // [128]
     const int seg = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
@@ -174,9 +196,14 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
         if (A) chunk_log_cumsum(A + c0, n, Lc);
         __syncthreads();
         for (int q0 = 0; q0 < n; q0 += kSub) {
-            for (int idx = tid; idx < kSub * D; idx += kSimtThreads) {
-                const int j = idx / D, a = idx % D;
-                fq[idx] = (q0 + j < n) ? phi_precise(to_f32(Q[(size_t)(c0 + q0 + j) * D + a])) : 0.f;
+            {
+                float qx[simt_per_thread(D)];
+                simt_load_rows<InT, D>(Q, c0 + q0, n - q0, qx);
+#pragma unroll
+                for (int u = 0; u < simt_per_thread(D); ++u) {
+                    const int idx = tid + u * kSimtThreads, j = idx / D, a = idx % D;
+                    fq[j * RS + a] = (q0 + j < n) ? phi_precise(qx[u]) : 0.f;
+                }
             }
             __syncthreads();
             const int il = q0 + row;
@@ -190,7 +217,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
                 for (int c = 0; c < CPT; ++c) s[c] = 0.f;
                 float dz = 0.f;
                 for (int a = 0; a < D; ++a) {
-                    const float f = fq[row * D + a];
+                    const float f = fq[row * RS + a];
                     dz = fmaf(f, z[a], dz);
 #pragma unroll
                     for (int c = 0; c < CPT; ++c) s[c] = fmaf(f, S[a * D + cg * CPT + c], s[c]);
@@ -200,16 +227,16 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
                 den = g * dz;
             }
             for (int k0 = 0; k0 <= q0; k0 += kSub) {
-                for (int idx = tid; idx < kSub * D; idx += kSimtThreads) {
-                    const int j = idx / D, a = idx % D;
-                    float f = 0.f, x = 0.f;
-                    if (k0 + j < n) {
-                        const size_t off = (size_t)(c0 + k0 + j) * D + a;
-                        f = phi_precise(to_f32(K[off]));
-                        x = to_f32(V[off]);
+                {
+                    float kx[simt_per_thread(D)], vx[simt_per_thread(D)];
+                    simt_load_rows<InT, D>(K, c0 + k0, n - k0, kx);
+                    simt_load_rows<InT, D>(V, c0 + k0, n - k0, vx);
+#pragma unroll
+                    for (int u = 0; u < simt_per_thread(D); ++u) {
+                        const int idx = tid + u * kSimtThreads, j = idx / D, a = idx % D;
+                        fk[j * RS + a] = (k0 + j < n) ? phi_precise(kx[u]) : 0.f;
+                        vv[idx] = vx[u];
                     }
-                    fk[idx] = f;
-                    vv[idx] = x;
                 }
                 __syncthreads();
                 for (int e = tid; e < kSub * kSub; e += kSimtThreads) {
@@ -217,7 +244,15 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
                     const int gi = q0 + i, gj = k0 + j;
                     float sc = 0.f;
                     if (gj <= gi && gi < n) {
-                        for (int a = 0; a < D; ++a) sc = fmaf(fq[i * D + a], fk[j * D + a], sc);
+                        // four independent partial sums (a dependent chain of D FMAs
+                        // would serialise on their latency)
+                        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                        for (int a = 0; a < D; a += 4) {
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) s4[u] = fmaf(fq[i * RS + a + u], fk[j * RS + a + u], s4[u]);
+                        }
+                        sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
                         if (A) sc *= expf(Lc[gi] - Lc[gj]);
                     }
                     P[i * (kSub + 1) + j] = sc;
@@ -252,23 +287,27 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
         if (tid < D) zreg = (A ? expf(Lend) : 1.f) * z[tid];
         for (int k0 = 0; k0 < n; k0 += kSub) {
             __syncthreads();
-            for (int idx = tid; idx < kSub * D; idx += kSimtThreads) {
-                const int j = idx / D, a = idx % D;
-                float f = 0.f, x = 0.f;
-                if (k0 + j < n) {
-                    const size_t off = (size_t)(c0 + k0 + j) * D + a;
-                    f = phi_precise(to_f32(K[off]));
-                    if (A) f *= expf(Lend - Lc[k0 + j]);
-                    x = to_f32(V[off]);
+            {
+                float kx[simt_per_thread(D)], vx[simt_per_thread(D)];
+                simt_load_rows<InT, D>(K, c0 + k0, n - k0, kx);
+                simt_load_rows<InT, D>(V, c0 + k0, n - k0, vx);
+#pragma unroll
+                for (int u = 0; u < simt_per_thread(D); ++u) {
+                    const int idx = tid + u * kSimtThreads, j = idx / D, a = idx % D;
+                    float f = 0.f;
+                    if (k0 + j < n) {
+                        f = phi_precise(kx[u]);
+                        if (A) f *= expf(Lend - Lc[k0 + j]);
+                    }
+                    fk[j * RS + a] = f;
+                    vv[idx] = vx[u];
                 }
-                fk[idx] = f;
-                vv[idx] = x;
             }
             __syncthreads();
             for (int j = 0; j < kSub; ++j) {
                 float ar[TR], bc[TR];
 #pragma unroll
-                for (int r = 0; r < TR; ++r) ar[r] = fk[j * D + ty * TR + r];
+                for (int r = 0; r < TR; ++r) ar[r] = fk[j * RS + ty * TR + r];
 #pragma unroll
                 for (int c = 0; c < TR; ++c) bc[c] = vv[j * D + tx * TR + c];
 #pragma unroll
@@ -277,7 +316,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
                     for (int c = 0; c < TR; ++c) sreg[r][c] = fmaf(ar[r], bc[c], sreg[r][c]);
             }
             if (tid < D)
-                for (int j = 0; j < kSub; ++j) zreg += fk[j * D + tid];
+                for (int j = 0; j < kSub; ++j) zreg += fk[j * RS + tid];
         }
         __syncthreads();
 #pragma unroll
@@ -290,7 +329,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
 }
 
 template <int D> __host__ __device__ constexpr size_t simt_readout_smem() {
-    return sizeof(float) * (D * D + D + kSub * D);
+    return sizeof(float) * (D * D + D + kSub * (D + 1));
 }
 
 constexpr int kReadoutQueries = 128;
@@ -303,7 +342,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_noncausal_readout_kernel(Si
     extern __shared__ float smem[];
     float *S = smem;          // [D][D]
     float *z = S + D * D;     // [D]
-    float *fq = z + D;        // [kSub][D]
+    float *fq = z + D;        // [kSub][D + 1] (padded: 4 query rows per warp)
+    constexpr int RS = D + 1;
     const int bh = blockIdx.y, tid = threadIdx.x;
     const int row = tid / 8, cg = tid % 8;
     const float *tot = p.ws_total + (size_t)bh * (D * D + D);
@@ -314,9 +354,14 @@ __global__ void __launch_bounds__(kSimtThreads) simt_noncausal_readout_kernel(Si
     const int qe = min(p.Lq, qb + kReadoutQueries);
     for (int q0 = qb; q0 < qe; q0 += kSub) {
         __syncthreads();
-        for (int idx = tid; idx < kSub * D; idx += kSimtThreads) {
-            const int j = idx / D, a = idx % D;
-            fq[idx] = (q0 + j < qe) ? phi_precise(to_f32(Q[(size_t)(q0 + j) * D + a])) : 0.f;
+        {
+            float qx[simt_per_thread(D)];
+            simt_load_rows<InT, D>(Q, q0, qe - q0, qx);
+#pragma unroll
+            for (int u = 0; u < simt_per_thread(D); ++u) {
+                const int idx = tid + u * kSimtThreads, j = idx / D, a = idx % D;
+                fq[j * RS + a] = (q0 + j < qe) ? phi_precise(qx[u]) : 0.f;
+            }
         }
         __syncthreads();
         float s[CPT];
@@ -324,7 +369,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_noncausal_readout_kernel(Si
         for (int c = 0; c < CPT; ++c) s[c] = 0.f;
         float dz = 0.f;
         for (int a = 0; a < D; ++a) {
-            const float f = fq[row * D + a];
+            const float f = fq[row * RS + a];
             dz = fmaf(f, z[a], dz);
 #pragma unroll
             for (int c = 0; c < CPT; ++c) s[c] = fmaf(f, S[a * D + cg * CPT + c], s[c]);
