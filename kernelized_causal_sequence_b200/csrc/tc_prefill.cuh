@@ -323,9 +323,64 @@ __device__ __forceinline__ void scale_rows(uint8_t *tile, int tw, const float *L
 // decay from each key to the segment's end is known when its chunk is read.
 template <bool OUT> __device__ __forceinline__ int chunk_at(int c, int nch) { return OUT ? c : nch - 1 - c; }
 
-// Keys of chunk c (K warpgroup, thread index tk = 0..127): the decay cumsum
-// (warp 0; DECAY), then phi(K) (and w o phi(K)) in place; in output mode all
-// key rows, in state-only mode the first half (warps 0-3 take the rest).
+// Decay cumsum of chunk c by one warp: L_j (chunk-local inclusive cumsum of
+// log2 a) to shared memory, the chunk decay g = 2^(L_end) and the weight
+// origin; arrives on l_ready.  The decays of chunk c were loaded into
+// registers during chunk c-1; the loads of the next chunk start here so their
+// latency is hidden.  The caller has waited until the stage's L slot is free.
+template <int C, int D, bool DECAY, int MODE>
+__device__ __forceinline__ void decay_cumsum(uint64_t *bar, float *Fsm, const TcParams &p, long t_begin,
+                                             long t_end, int bh, int c, int nch, int lane, float &Aseg,
+                                             float (&apre)[C / 32], float &lam) {
+    using G = Cfg<C, D, DECAY, MODE>;
+    const int s = c % G::NKV;
+    const long t0 = t_begin + (long)chunk_at<G::OUT>(c, nch) * C;
+    const int n = (int)min((long)C, t_end - t0);
+    float *L = Fsm + G::F_L + s * C;
+    const float *a = p.decay + (size_t)bh * p.T + t0;
+    float cur[C / 32];
+#pragma unroll
+    for (int h = 0; h < C / 32; ++h) {
+        const int j = h * 32 + lane;
+        cur[h] = (c == 0) ? ((j < n) ? a[j] : 1.f) : apre[h];
+    }
+    if (c + 1 < nch) {
+        const long t1 = t_begin + (long)chunk_at<G::OUT>(c + 1, nch) * C;
+        const int n1 = (int)min((long)C, t_end - t1);
+        const float *a1 = p.decay + (size_t)bh * p.T + t1;
+#pragma unroll
+        for (int h = 0; h < C / 32; ++h) {
+            const int j = h * 32 + lane;
+            apre[h] = (j < n1) ? a1[j] : 1.f;
+        }
+    }
+    float carry = 0.f;
+#pragma unroll
+    for (int h = 0; h < C / 32; ++h) {
+        const int j = h * 32 + lane;
+        float x = (j < n) ? lg2_approx(cur[h]) : 0.f;   // log2 units
+        x = warp_sum_scan(x, lane) + carry;
+        L[j] = x;   // rows >= n repeat the chunk total (never used)
+        carry = __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) {
+        const float g = ex2_approx(carry);
+        Fsm[G::F_G + s] = g;
+        Aseg *= g;
+        // weights w_j = 2^(origin - L_j): the chunk's end in output mode; in
+        // state-only mode the segment's end (lam = log2 decay of the chunks
+        // after this one, all processed already)
+        Fsm[G::F_LE + s] = G::OUT ? carry : carry + lam;
+        lam += carry;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar[G::B_L_READY + s]);
+}
+
+// Keys of chunk c (K warpgroup, thread index tk = 0..127): phi(K) in place (in
+// output mode all key rows, in state-only mode the first half, weighted by
+// the decay to the segment end; warps 0-3 take the rest); in output mode
+// with decay, warp 0 then forms the chunk's decay cumsum.
 // Arrives on phi_done.  Returns false if the CTA is aborting.
 template <int C, int D, bool DECAY, int MODE, typename InT>
 __device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm, const AbortCtx ab,
@@ -338,51 +393,10 @@ __device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm
     const int n = (int)min((long)C, t_end - t0);
     if (!mbar_wait(&bar[G::B_KV_FULL + s], (c / G::NKV) & 1, ab, 8)) return false;
     float *L = Fsm + G::F_L + s * C;
-    if constexpr (DECAY) {
-        if (tk < 32) {
-            // the decays of chunk c were loaded into registers during chunk c-1;
-            // start the loads of the next chunk now so their latency is hidden
-            const float *a = p.decay + (size_t)bh * p.T + t0;
-            float cur[C / 32];
-#pragma unroll
-            for (int h = 0; h < C / 32; ++h) {
-                const int j = h * 32 + lane;
-                cur[h] = (c == 0) ? ((j < n) ? a[j] : 1.f) : apre[h];
-            }
-            if (c + 1 < nch) {
-                const long t1 = t_begin + (long)chunk_at<G::OUT>(c + 1, nch) * C;
-                const int n1 = (int)min((long)C, t_end - t1);
-                const float *a1 = p.decay + (size_t)bh * p.T + t1;
-#pragma unroll
-                for (int h = 0; h < C / 32; ++h) {
-                    const int j = h * 32 + lane;
-                    apre[h] = (j < n1) ? a1[j] : 1.f;
-                }
-            }
-            float carry = 0.f;
-#pragma unroll
-            for (int h = 0; h < C / 32; ++h) {
-                const int j = h * 32 + lane;
-                float x = (j < n) ? lg2_approx(cur[h]) : 0.f;   // log2 units
-                x = warp_sum_scan(x, lane) + carry;
-                L[j] = x;   // rows >= n repeat the chunk total (never used)
-                carry = __shfl_sync(0xffffffffu, x, 31);
-            }
-            if (lane == 0) {
-                const float g = ex2_approx(carry);
-                Fsm[G::F_G + s] = g;
-                Aseg *= g;
-                // weights w_j = 2^(origin - L_j): the chunk's end in output mode;
-                // in state-only mode the segment's end (lam = log2 decay of the
-                // chunks after this one, all processed already)
-                Fsm[G::F_LE + s] = G::OUT ? carry : carry + lam;
-                lam += carry;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[G::B_L_READY + s]);   // for the other warpgroups
-        }
-        named_bar_sync(1, 128);
-    }
+    // state-only mode: the weights need the decay cumsum, which the idle phi(Q)
+    // warps compute ahead of the key warps
+    if constexpr (DECAY && !G::OUT)
+        if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 29)) return false;
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
     constexpr bool CONV = !std::is_same<InT, bf16>::value;
     const float Lend = DECAY ? Fsm[G::F_LE + s] : 0.f;
@@ -395,6 +409,9 @@ __device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
+    // output mode: phi(K) did not need the decays; the cumsum follows it (warp 0)
+    if constexpr (DECAY && G::OUT)
+        if (tk < 32) decay_cumsum<C, D, DECAY, MODE>(bar, Fsm, p, t_begin, t_end, bh, c, nch, lane, Aseg, apre, lam);
     return true;
 }
 
@@ -468,6 +485,7 @@ __device__ __forceinline__ bool k_weight(uint8_t *smem, uint64_t *bar, float *Fs
     using G = Cfg<C, D, DECAY, MODE>;
     const int s = c % G::NKV;
     if (!mbar_wait(&bar[G::B_SC_FULL], c & 1, ab, 21)) return false;
+    if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 30)) return false;
     scale_rows<C, D, true>(smem + G::OFF_KV + s * G::KV_STAGE, tk, Fsm + G::F_L + s * C, Fsm[G::F_LE + s]);
     fence_proxy_async_smem();
     __syncwarp();
@@ -773,8 +791,6 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                                  apre, lam);
             if constexpr (G::QS) if (ok) ok = k_weight<C, D, DECAY, MODE>(smem, bar, Fsm, ab, c, tk);
         }
-        if constexpr (!G::OUT)
-            if (ok && tk == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = Aseg;
     } else if (warp >= kPhiWarp0) {
         // ================= phi(Q) and the state epilogue (warps 6-9)
         const int tw = threadIdx.x - kPhiWarp0 * 32;        // 0..127
@@ -830,8 +846,23 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
 
         if constexpr (!G::OUT) {
+            // state-only mode with decay: warp 0 forms every chunk's decay cumsum
+            // ahead of the key warps (each once its stage's L slot is free)
+            float Aseg = 1.f;   // product of the chunk decays (the segment's A)
+            if constexpr (DECAY) {
+                if (tw < 32) {
+                    float apre[C / 32];
+#pragma unroll
+                    for (int h = 0; h < C / 32; ++h) apre[h] = 1.f;
+                    float lam = 0.f;
+                    for (int c = 0; ok && c < nch; ++c) {
+                        if (!mbar_wait(&bar[G::B_KV_FULL + c % G::NKV], (c / G::NKV) & 1, ab, 31)) { ok = false; break; }
+                        decay_cumsum<C, D, DECAY, MODE>(bar, Fsm, p, t_begin, t_end, bh, c, nch, lane, Aseg, apre, lam);
+                    }
+                }
+            }
+            if (tw == 0 && ok && nch > 0) p.ws_A[(size_t)bh * p.n_seg + seg] = Aseg;
             // state-only mode: write the segment's (dS, dz) to the workspace
-            // (A is written by the key warps)
             if (ok && nch > 0 && mbar_wait(&bar[G::B_DS_FULL], 0, ab, 11)) {
                 tc_fence_after();
                 float *dst = p.ws_state + ((size_t)bh * p.n_seg + seg) * (D * D + D);
@@ -920,6 +951,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const long t0 = t_begin + (long)c * C;
             if (!mbar_wait(&bar[G::B_PHI + s], (c / G::NKV) & 1, ab, 12)) break;
             if (!mbar_wait(&bar[G::B_SC_FULL], c & 1, ab, 13)) break;
+            if (DECAY && !mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 28)) break;
             tc_fence_after();
             const float *L = Fsm + G::F_L + s * C;
             const float Li = (DECAY && rvalid_lane) ? L[min(i, C - 1)] : 0.f;
