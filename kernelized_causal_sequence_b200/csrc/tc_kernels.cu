@@ -81,8 +81,18 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
     if (e0 != LA_OK) return e0;
     la_status s = record_event(a.events, 0, st);
     if (s != LA_OK) return s;
-    // K1: per-segment state contributions
-    s = launch_tc<C, D, DECAY, tc::kStateOnly, InT, float>(mq, mk, mv, mo, p, a.BH, a.n_seg, st);
+    // K1: per-segment state contributions.  A segment's contribution does not
+    // depend on the chunk, so K1 always walks it in 128-token tiles (fewer,
+    // longer pipeline steps); segments are whole 64-token chunks and the last
+    // tile of a segment may be a half tile.
+    if constexpr (C == 64) {
+        CUtensorMap mk1, mv1;
+        if (!make_map(&mk1, a.k, a.in_dtype, a.BH, a.T, D, 128) || !make_map(&mv1, a.v, a.in_dtype, a.BH, a.T, D, 128))
+            return cuda_fail_msg("cuTensorMapEncodeTiled", "tensor map encoding failed");
+        s = launch_tc<128, D, DECAY, tc::kStateOnly, InT, float>(mq, mk1, mv1, mo, p, a.BH, a.n_seg, st);
+    } else {
+        s = launch_tc<C, D, DECAY, tc::kStateOnly, InT, float>(mq, mk, mv, mo, p, a.BH, a.n_seg, st);
+    }
     if (s != LA_OK) return s;
     if ((s = record_event(a.events, 1, st)) != LA_OK) return s;
     // K2: decayed exclusive scan over segments (+ state in/out)
