@@ -847,7 +847,9 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
         if constexpr (!G::OUT) {
             // state-only mode with decay: warp 0 forms every chunk's decay cumsum
-            // ahead of the key warps (each once its stage's L slot is free)
+            // ahead of the key warps.  Chunk c's L slot is free once both key
+            // warpgroups have finished the feature map of chunk c - NKV (its
+            // phi_done), so the cumsum does not wait for the chunk's data.
             float Aseg = 1.f;   // product of the chunk decays (the segment's A)
             if constexpr (DECAY) {
                 if (tw < 32) {
@@ -856,7 +858,11 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int h = 0; h < C / 32; ++h) apre[h] = 1.f;
                     float lam = 0.f;
                     for (int c = 0; ok && c < nch; ++c) {
-                        if (!mbar_wait(&bar[G::B_KV_FULL + c % G::NKV], (c / G::NKV) & 1, ab, 31)) { ok = false; break; }
+                        if (c >= G::NKV &&
+                            !mbar_wait(&bar[G::B_PHI + c % G::NKV], ((c - G::NKV) / G::NKV) & 1, ab, 31)) {
+                            ok = false;
+                            break;
+                        }
                         decay_cumsum<C, D, DECAY, MODE>(bar, Fsm, p, t_begin, t_end, bh, c, nch, lane, Aseg, apre, lam);
                     }
                 }
