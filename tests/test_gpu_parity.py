@@ -299,3 +299,21 @@ def test_noncausal_d32_native_out(la, orc, dtype):
     ro, _, _ = orc.noncausal(q, k, v)
     assert o.dtype == dtype
     assert row_rel_err(o.float().cpu().numpy(), ro) < 2e-2
+
+
+@pytest.mark.parametrize("dtype,d,chunk,decay", [(torch.bfloat16, 128, 128, False), (torch.bfloat16, 128, 64, True),
+                                                 (torch.float32, 64, 64, False)])
+def test_prefill_events_entry_point(la, dtype, d, chunk, decay):
+    """la_prefill_causal_ev: the same kernels as la_prefill_causal (bitwise equal
+    results) plus four events recorded around the passes, in order."""
+    q, k, v, a = _small_inputs(dtype, d, 3000, decay, 1, 2, seed=12)
+    o1, S1, _ = gpu_prefill(la, q, k, v, a, chunk, torch.float32)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    S = torch.zeros((1, 2, d, d), device=DEV)
+    z = torch.zeros((1, 2, d), device=DEV)
+    o2 = la.la_prefill_causal(q.to(DEV), k.to(DEV), v.to(DEV), decay=None if a is None else a.to(DEV),
+                              chunk=chunk, state_S=S, state_z=z, out_dtype=torch.float32, events=ev)
+    torch.cuda.synchronize()
+    assert np.array_equal(o1, o2.cpu().numpy()) and np.array_equal(S1, S.cpu().numpy())
+    times = [ev[j].elapsed_time(ev[j + 1]) for j in range(3)]
+    assert all(t >= 0 for t in times) and sum(times) > 0
