@@ -35,6 +35,13 @@ __device__ __forceinline__ float lg2_approx(float x) {
 }
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Programmatic dependent launch: pdl_wait blocks until the grids this one was
+// launched after have completed and their memory is visible (it returns at
+// once for a normal launch); pdl_trigger lets a dependent grid start launching
+// once every CTA of this grid has triggered or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // phi(x) = elu(x) + 1 (alpha = 1): x + 1 for x > 0, and e^x for x <= 0, which
 // equals (e^x - 1) + 1 without the cancellation.  ("Transformers are RNNs"
 // feature map, as given on the knowledge-base page, section 2, "Choice of phi".)

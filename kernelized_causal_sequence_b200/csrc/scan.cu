@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, cons
                                                            float *total) {
     __shared__ float tile[32][33];
     __shared__ float Atile[32];
+    pdl_wait();   // the segment states of the state pass
     const int bh = blockIdx.y, e0 = blockIdx.x * 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float *ws = ws_state + (size_t)bh * n_seg * E;
@@ -77,6 +78,7 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, cons
             else if (state_out_z) state_out_z[(size_t)bh * (E - dS) + (e - dS)] = carry[m];
         }
     }
+    pdl_trigger();
 }
 
 
@@ -94,6 +96,7 @@ __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, 
                                                                float *state_out_S, float *state_out_z,
                                                                float *total) {
     __shared__ float Ash[kSeqScanMaxSeg];
+    pdl_wait();   // the segment states of the state pass
     const int bh = blockIdx.y;
     const int e = blockIdx.x * 256 + threadIdx.x;
     if (threadIdx.x < n_seg) Ash[threadIdx.x] = ws_A[(size_t)bh * n_seg + threadIdx.x];
@@ -120,24 +123,39 @@ __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, 
     if (total) total[(size_t)bh * E + e] = carry;
     if (e < dS) { if (state_out_S) state_out_S[(size_t)bh * dS + e] = carry; }
     else if (state_out_z) state_out_z[(size_t)bh * (E - dS) + (e - dS)] = carry;
+    pdl_trigger();
 }
 
 la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n_seg, int D,
                               int mode, float *state_S, float *state_z, float *total,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool pdl) {
     const int E = D * D + D;
     const float *sin_S = mode == LA_STATE_INOUT ? state_S : nullptr;
     const float *sin_z = mode == LA_STATE_INOUT ? state_z : nullptr;
     float *sout_S = mode != LA_STATE_NONE ? state_S : nullptr;
     float *sout_z = mode != LA_STATE_NONE ? state_z : nullptr;
+    // with pdl, the scan may start launching while the state pass finishes
+    // (it waits for that pass's results before reading them)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t err;
     if (n_seg <= kSeqScanMaxSeg) {
-        segment_scan_seq_kernel<<<dim3((E + 255) / 256, (unsigned)BH), 256, 0, st>>>(
-            ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, total);
+        cfg.gridDim = dim3((E + 255) / 256, (unsigned)BH);
+        err = cudaLaunchKernelEx(&cfg, segment_scan_seq_kernel, ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z,
+                                 sout_S, sout_z, total);
     } else {
-        segment_scan_kernel<<<dim3((E + 31) / 32, (unsigned)BH), 256, 0, st>>>(
-            ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z, sout_S, sout_z, total);
+        cfg.gridDim = dim3((E + 31) / 32, (unsigned)BH);
+        err = cudaLaunchKernelEx(&cfg, segment_scan_kernel, ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z,
+                                 sout_S, sout_z, total);
     }
     count_launches(1);
+    if (err != cudaSuccess) return cuda_fail("segment_scan launch", err);
     return cuda_check("segment_scan launch", cudaGetLastError());
 }
 

@@ -13,6 +13,6 @@ void count_launches(int n);  // process-wide kernel launch counter (la_launch_co
 // goes to state_S/state_z (mode OUT/INOUT) and to `total` when non-null.
 la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n_seg, int D,
                               int mode, float *state_S, float *state_z, float *total,
-                              cudaStream_t st);
+                              cudaStream_t st, bool pdl = false);
 
 }  // namespace la

@@ -49,14 +49,28 @@ bool make_map(CUtensorMap *m, const void *base, la_dtype dt, long BH, int T, int
 
 template <int C, int D, bool DECAY, int MODE, typename InT, typename OutT>
 la_status launch_tc(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                    const CUtensorMap &mo, const tc::TcParams &p, long BH, int n_ctas_x, cudaStream_t st) {
+                    const CUtensorMap &mo, const tc::TcParams &p, long BH, int n_ctas_x, cudaStream_t st,
+                    bool pdl = false) {
     using G = tc::Cfg<C, D, DECAY, MODE>;
     auto kern = tc::tc_prefill_kernel<C, D, DECAY, MODE, InT, OutT>;
     la_status e = cuda_check("tensor-core kernel smem attribute",
                              cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES));
     if (e != LA_OK) return e;
-    kern<<<dim3(n_ctas_x, (unsigned)BH), tc::kThreads, G::SMEM_BYTES, st>>>(mq, mk, mv, mo, p);
+    // with pdl the kernel may start launching while the previous one (the
+    // segment scan) finishes; it waits for that kernel before reading its output
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(n_ctas_x, (unsigned)BH);
+    cfg.blockDim = dim3(tc::kThreads);
+    cfg.dynamicSmemBytes = G::SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, p);
     count_launches(1);
+    if (err != cudaSuccess) return cuda_fail("tensor-core kernel launch", err);
     return cuda_check("tensor-core kernel launch", cudaGetLastError());
 }
 
@@ -96,12 +110,15 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
     if (s != LA_OK) return s;
     if ((s = record_event(a.events, 1, st)) != LA_OK) return s;
     // K2: decayed exclusive scan over segments (+ state in/out)
+    // (programmatic dependent launches: each kernel's launch overlaps the end of
+    // the previous one; events between the passes, when asked for, serialise them)
+    const bool pdl = a.events == nullptr;
     s = launch_segment_scan(a.ws_state, a.ws_A, a.BH, a.n_seg, D, a.mode, a.state_S, a.state_z,
-                            nullptr, st);
+                            nullptr, st, pdl);
     if (s != LA_OK) return s;
     if ((s = record_event(a.events, 2, st)) != LA_OK) return s;
     // K3: chunked output from the segment-entry states
-    s = launch_tc<C, D, DECAY, tc::kOutput, InT, OutT>(mq, mk, mv, mo, p, a.BH, a.n_seg, st);
+    s = launch_tc<C, D, DECAY, tc::kOutput, InT, OutT>(mq, mk, mv, mo, p, a.BH, a.n_seg, st, pdl);
     if (s != LA_OK) return s;
     return record_event(a.events, 3, st);
 }

@@ -814,6 +814,8 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 g0 = Fsm[G::F_G + 0];
             }
             tc_fence_after();
+            // (output mode may have been launched before the segment scan ended)
+            if constexpr (G::OUT) pdl_wait();
             const float *st = p.ws_state + ((size_t)bh * p.n_seg + seg) * (D * D + D);
             if (ok) {
 #pragma unroll 1
@@ -1088,6 +1090,10 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     tc_fence_before();
     __syncthreads();
+    // the CTA's work is done (state-only: its segment state is written), so a
+    // dependent grid may start launching; it waits for this grid's completion
+    // before it reads anything this grid wrote
+    pdl_trigger();
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, G::TMEM_COLS);
