@@ -70,6 +70,28 @@ la_status cuda_fail(const char *where, cudaError_t e) {
 
 namespace {
 
+// Launches kern, with programmatic stream serialisation when pdl is set (the
+// kernel may start launching while the previous kernel in the stream ends; it
+// must call pdl_wait before reading that kernel's output).
+template <typename... KArgs, typename... Args>
+la_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                    const char *what, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    count_launches(1);
+    if (e != cudaSuccess) return cuda_fail(what, e);
+    return cuda_check(what, cudaGetLastError());
+}
+
 // ---------------------------------------------------------------- SIMT path
 template <typename InT, typename OutT, int D>
 la_status simt_causal(SimtParams p, cudaStream_t st) {
@@ -81,21 +103,23 @@ la_status simt_causal(SimtParams p, cudaStream_t st) {
         if (e != LA_OK) return e;
         k1<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p, p.T);
     }
+    count_launches(1);
+    la_status e = cuda_check("segment_state launch", cudaGetLastError());
+    if (e != LA_OK) return e;
     if (record_event(p.events, 1, st) != LA_OK) return LA_ERR_CUDA;
+    const bool pdl = p.events == nullptr;   // events between the passes serialise them
     if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, D, p.mode, p.state_S, p.state_z,
-                            nullptr, st) != LA_OK)
+                            nullptr, st, pdl) != LA_OK)
         return LA_ERR_CUDA;
     if (record_event(p.events, 2, st) != LA_OK) return LA_ERR_CUDA;
     {
         auto k3 = simt_chunk_output_kernel<InT, OutT, D>;
         const size_t sm = simt_output_smem<D>();
-        la_status e = cuda_check("chunk_output smem attribute", allow_smem(k3, sm));
+        e = cuda_check("chunk_output smem attribute", allow_smem(k3, sm));
         if (e != LA_OK) return e;
-        k3<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p);
+        e = launch_ex(k3, dim3(p.n_seg, p.BH), dim3(kSimtThreads), sm, st, pdl, "chunk_output launch", p);
+        if (e != LA_OK) return e;
     }
-    count_launches(2);
-    la_status e = cuda_check("causal kernel launch", cudaGetLastError());
-    if (e != LA_OK) return e;
     return record_event(p.events, 3, st);
 }
 
@@ -108,19 +132,21 @@ la_status simt_noncausal(SimtParams p, int Lk, cudaStream_t st) {
         if (e != LA_OK) return e;
         k1<<<dim3(p.n_seg, p.BH), kSimtThreads, sm, st>>>(p, Lk);
     }
+    count_launches(1);
+    la_status e = cuda_check("segment_state launch", cudaGetLastError());
+    if (e != LA_OK) return e;
     if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, D, p.mode, p.state_S, p.state_z,
-                            p.ws_total, st) != LA_OK)
+                            p.ws_total, st, true) != LA_OK)
         return LA_ERR_CUDA;
     if (p.Lq > 0) {
         auto k3 = simt_noncausal_readout_kernel<InT, OutT, D>;
         const size_t sm = simt_readout_smem<D>();
-        la_status e = cuda_check("readout smem attribute", allow_smem(k3, sm));
+        e = cuda_check("readout smem attribute", allow_smem(k3, sm));
         if (e != LA_OK) return e;
-        k3<<<dim3((p.Lq + kReadoutQueries - 1) / kReadoutQueries, p.BH), kSimtThreads, sm, st>>>(p);
-        count_launches(1);
+        e = launch_ex(k3, dim3((p.Lq + kReadoutQueries - 1) / kReadoutQueries, p.BH), dim3(kSimtThreads), sm, st,
+                      true, "readout launch", p);
     }
-    count_launches(1);
-    return cuda_check("non-causal kernel launch", cudaGetLastError());
+    return e;
 }
 
 // Dispatch over (in dtype, out dtype, head dim) for a functor template F.
@@ -158,16 +184,14 @@ la_status nc32_noncausal(SimtParams p, int Lk, cudaStream_t st) {
     la_status e = cuda_check("nc32 state launch", cudaGetLastError());
     if (e != LA_OK) return e;
     e = launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, 32, p.mode, p.state_S, p.state_z,
-                            p.ws_total, st);
+                            p.ws_total, st, true);
     if (e != LA_OK) return e;
     if (p.Lq > 0) {
         const int tpc = nc32_tiles_per_cta(p.BH, p.Lq);
         const long span = (long)tpc * kNc32Tile;
-        nc32_readout_kernel<InT, OutT>
-            <<<dim3((unsigned)((p.Lq + span - 1) / span), p.BH), kNc32Threads, 0, st>>>(
-                (const InT *)p.q, p.Lq, tpc, p.ws_total, p.eps, (OutT *)p.out);
-        count_launches(1);
-        e = cuda_check("nc32 read-out launch", cudaGetLastError());
+        e = launch_ex(nc32_readout_kernel<InT, OutT>, dim3((unsigned)((p.Lq + span - 1) / span), p.BH),
+                      dim3(kNc32Threads), 0, st, true, "nc32 read-out launch", (const InT *)p.q, p.Lq, tpc,
+                      (const float *)p.ws_total, p.eps, (OutT *)p.out);
     }
     return e;
 }

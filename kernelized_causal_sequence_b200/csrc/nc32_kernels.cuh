@@ -149,6 +149,8 @@ nc32_state_kernel(const InT *__restrict__ k, const InT *__restrict__ v, int Lk, 
         dst[32 * 32 + t] = zs;
     }
     if (t == 0) ws_A[(size_t)bh * n_seg + seg] = 1.f;
+    __syncthreads();
+    pdl_trigger();   // this segment's state is written: the scan may launch
 }
 
 
@@ -187,6 +189,7 @@ nc32_readout_kernel(const InT *__restrict__ q, int Lq, int tiles_per_cta, const 
     const int t = threadIdx.x, i0 = (t >> 3) * 4, b0 = (t & 7) * 4;
     const int bh = blockIdx.y;
     const float *tot = total + (size_t)bh * (32 * 32 + 32);
+    pdl_wait();   // the segment scan's head totals
     for (int e = t; e < 32 * 32; e += kNc32Threads) Ssm[e / 32][e % 32] = tot[e];
     if (t < 32) zsm[t] = tot[32 * 32 + t];
     const long span = (long)tiles_per_cta * kNc32Tile;

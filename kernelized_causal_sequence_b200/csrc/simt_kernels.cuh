@@ -153,6 +153,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_segment_state_kernel(SimtPa
         for (int c = 0; c < TR; ++c) dst[(ty * TR + r) * D + tx * TR + c] = acc[r][c];
     if (tid < D) dst[D * D + tid] = zacc;
     if (tid == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = Aseg;
+    __syncthreads();
+    pdl_trigger();   // this segment's state is written: the scan may launch
 }
 
 template <int D> __host__ __device__ constexpr size_t simt_output_smem() {
@@ -188,6 +190,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
     const float *A = p.decay ? p.decay + (size_t)bh * p.T : nullptr;
 
     const float *st = p.ws_state + ((size_t)bh * p.n_seg + seg) * (D * D + D);
+    pdl_wait();   // the segment scan's output
     for (int i = tid; i < D * D + D; i += kSimtThreads) S[i] = st[i];
     __syncthreads();
 
@@ -273,6 +276,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
                 for (int c = 0; c < CPT; ++c) o[c] = from_f32<OutT>(acc[c] / dn);
             }
         }
+        // the state after the segment's last chunk is never read (the scan
+        // forms the segment-entry states and the final state)
+        if (c0 + p.chunk >= t_end) break;
         // state update over the chunk's keys
         const float Lend = A ? Lc[n - 1] : 0.f;
         float sreg[TR][TR];
@@ -347,6 +353,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_noncausal_readout_kernel(Si
     const int bh = blockIdx.y, tid = threadIdx.x;
     const int row = tid / 8, cg = tid % 8;
     const float *tot = p.ws_total + (size_t)bh * (D * D + D);
+    pdl_wait();   // the segment scan's head totals
     for (int i = tid; i < D * D + D; i += kSimtThreads) S[i] = tot[i];
     const InT *Q = (const InT *)p.q + (size_t)bh * p.Lq * D;
     OutT *O = (OutT *)p.out + (size_t)bh * p.Lq * D;
