@@ -166,6 +166,32 @@ def test_empty_and_state_only(la):
     assert float(S.min()) == 2.0
 
 
+@pytest.mark.parametrize("dtype,d,T,chunk,decay", [(torch.bfloat16, 128, 3000, 128, True),
+                                                   (torch.bfloat16, 64, 2000, 64, False),
+                                                   (torch.float32, 64, 1000, 64, True)])
+def test_state_mode_none_matches_out(la, dtype, d, T, chunk, decay):
+    """Without a state output the output is bitwise the same, and no state
+    buffer is written (the last segment of the output pass writes the final
+    state only when one is asked for)."""
+    B, H = 1, 2
+    assert la.la_prefill_plan(B, H, T, d, chunk)[0] > 1   # several segments per head
+    q, k, v, a = _small_inputs(dtype, d, T, decay, B, H, seed=41)
+    qd, kd, vd = (x.to(DEV) for x in (q, k, v))
+    ad = None if a is None else a.to(DEV)
+    S = torch.full((B, H, d, d), 7.0, device=DEV)
+    z = torch.full((B, H, d), 7.0, device=DEV)
+    o_none = la.la_prefill_causal(qd, kd, vd, decay=ad, chunk=chunk, state_S=S, state_z=z,
+                                  mode=la.LA_STATE_NONE, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert float(S.min()) == 7.0 and float(S.max()) == 7.0
+    assert float(z.min()) == 7.0 and float(z.max()) == 7.0
+    o_out = la.la_prefill_causal(qd, kd, vd, decay=ad, chunk=chunk, state_S=S, state_z=z,
+                                 mode=la.LA_STATE_OUT, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(o_none, o_out)
+    assert float(z.min()) > 0.0   # phi > 0: the written normaliser is positive
+
+
 # -------------------------------------------------------- full-size workloads
 def test_workload_causal_f32(la, orc):
     w = W["causal_f32_t256_d64"]
