@@ -82,13 +82,19 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, cons
 }
 
 
-// K2 for few segments per head (the common case): one thread per state
-// element walks the head's segments in order, with the loads of eight
-// segments in flight at a time, so each block streams whole coalesced rows of
-// the workspace.  The segment factors A_s of the head are staged in shared
-// memory.  grid (ceil((D*D + D) / 256), BH), 256 threads.
+// K2 for few segments per head (the common case): one thread per four
+// consecutive state elements walks the head's segments in order.  Its loads
+// for the first eight segments are issued before the block waits for the
+// segment factors A_s (staged in shared memory), so both latencies overlap,
+// and a grid of 16-byte accesses fits in one wave at the usual head counts.
+// E (= D*D + D) and D*D are multiples of 4 for every supported head dim, and
+// the workspace and state pointers are 16-byte aligned.
+// grid (ceil(E / 1024), BH), 256 threads.
 constexpr int kSeqScanMaxSeg = 64;
 constexpr int kSeqScanBatch = 8;
+__device__ __forceinline__ float4 fma4(float a, const float4 &c, const float4 &x) {
+    return make_float4(fmaf(a, c.x, x.x), fmaf(a, c.y, x.y), fmaf(a, c.z, x.z), fmaf(a, c.w, x.w));
+}
 __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, const float *ws_A,
                                                                int n_seg, int E, int dS,
                                                                const float *state_in_S,
@@ -98,31 +104,40 @@ __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, 
     __shared__ float Ash[kSeqScanMaxSeg];
     pdl_wait();   // the segment states of the state pass
     const int bh = blockIdx.y;
-    const int e = blockIdx.x * 256 + threadIdx.x;
+    const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
+    const bool live = e < E;
+    float4 *ws = reinterpret_cast<float4 *>(ws_state + (size_t)bh * n_seg * E + (live ? e : 0));
+    const size_t E4 = (size_t)E / 4;   // segment stride in float4
+    float4 x[kSeqScanBatch];
+#pragma unroll
+    for (int i = 0; i < kSeqScanBatch; ++i)
+        x[i] = (live && i < n_seg) ? ws[i * E4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (live) {
+        if (e < dS) { if (state_in_S) carry = *reinterpret_cast<const float4 *>(state_in_S + (size_t)bh * dS + e); }
+        else if (state_in_z) carry = *reinterpret_cast<const float4 *>(state_in_z + (size_t)bh * (E - dS) + (e - dS));
+    }
     if (threadIdx.x < n_seg) Ash[threadIdx.x] = ws_A[(size_t)bh * n_seg + threadIdx.x];
     __syncthreads();
-    if (e >= E) return;
-    float *ws = ws_state + (size_t)bh * n_seg * E + e;
-    float carry = 0.f;
-    if (e < dS) { if (state_in_S) carry = state_in_S[(size_t)bh * dS + e]; }
-    else if (state_in_z) carry = state_in_z[(size_t)bh * (E - dS) + (e - dS)];
+    if (!live) return;
 #pragma unroll 1
     for (int s0 = 0; s0 < n_seg; s0 += kSeqScanBatch) {
-        float x[kSeqScanBatch];
+        if (s0 > 0) {
 #pragma unroll
-        for (int i = 0; i < kSeqScanBatch; ++i)
-            x[i] = (s0 + i < n_seg) ? ws[(size_t)(s0 + i) * E] : 0.f;
+            for (int i = 0; i < kSeqScanBatch; ++i)
+                if (s0 + i < n_seg) x[i] = ws[(size_t)(s0 + i) * E4];
+        }
 #pragma unroll
         for (int i = 0; i < kSeqScanBatch; ++i) {
             if (s0 + i < n_seg) {
-                ws[(size_t)(s0 + i) * E] = carry;   // state entering segment s0 + i
-                carry = fmaf(Ash[s0 + i], carry, x[i]);
+                ws[(size_t)(s0 + i) * E4] = carry;   // state entering segment s0 + i
+                carry = fma4(Ash[s0 + i], carry, x[i]);
             }
         }
     }
-    if (total) total[(size_t)bh * E + e] = carry;
-    if (e < dS) { if (state_out_S) state_out_S[(size_t)bh * dS + e] = carry; }
-    else if (state_out_z) state_out_z[(size_t)bh * (E - dS) + (e - dS)] = carry;
+    if (total) *reinterpret_cast<float4 *>(total + (size_t)bh * E + e) = carry;
+    if (e < dS) { if (state_out_S) *reinterpret_cast<float4 *>(state_out_S + (size_t)bh * dS + e) = carry; }
+    else if (state_out_z) *reinterpret_cast<float4 *>(state_out_z + (size_t)bh * (E - dS) + (e - dS)) = carry;
     pdl_trigger();
 }
 
@@ -145,8 +160,8 @@ la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t err;
-    if (n_seg <= kSeqScanMaxSeg) {
-        cfg.gridDim = dim3((E + 255) / 256, (unsigned)BH);
+    if (n_seg <= kSeqScanMaxSeg && E % 4 == 0 && D % 4 == 0) {   // float4 groups stay inside S or z
+        cfg.gridDim = dim3((E / 4 + 255) / 256, (unsigned)BH);
         err = cudaLaunchKernelEx(&cfg, segment_scan_seq_kernel, ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z,
                                  sout_S, sout_z, total);
     } else {
