@@ -108,7 +108,7 @@ la_status simt_causal(SimtParams p, cudaStream_t st) {
     if (e != LA_OK) return e;
     if (record_event(p.events, 1, st) != LA_OK) return LA_ERR_CUDA;
     const bool pdl = p.events == nullptr;   // events between the passes serialise them
-    if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, D, p.mode, p.state_S, p.state_z,
+    if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, p.n_seg, D, p.mode, p.state_S, p.state_z,
                             nullptr, st, pdl) != LA_OK)
         return LA_ERR_CUDA;
     if (record_event(p.events, 2, st) != LA_OK) return LA_ERR_CUDA;
@@ -135,7 +135,7 @@ la_status simt_noncausal(SimtParams p, int Lk, cudaStream_t st) {
     count_launches(1);
     la_status e = cuda_check("segment_state launch", cudaGetLastError());
     if (e != LA_OK) return e;
-    if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, D, p.mode, p.state_S, p.state_z,
+    if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, p.n_seg, D, p.mode, p.state_S, p.state_z,
                             p.ws_total, st, true) != LA_OK)
         return LA_ERR_CUDA;
     if (p.Lq > 0) {
@@ -183,7 +183,7 @@ la_status nc32_noncausal(SimtParams p, int Lk, cudaStream_t st) {
     count_launches(1);
     la_status e = cuda_check("nc32 state launch", cudaGetLastError());
     if (e != LA_OK) return e;
-    e = launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, 32, p.mode, p.state_S, p.state_z,
+    e = launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, p.n_seg, 32, p.mode, p.state_S, p.state_z,
                             p.ws_total, st, true);
     if (e != LA_OK) return e;
     if (p.Lq > 0) {

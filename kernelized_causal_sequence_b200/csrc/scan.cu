@@ -13,10 +13,11 @@ namespace la {
 // and the final state is S_in(n_seg).  A block takes 32 state elements of one
 // head; a 32-segment x 32-element tile is staged through shared memory so
 // global accesses stay coalesced, and each warp scans one element across the
-// 32 segments of the tile with shuffles (lanes = segments).
+// 32 segments of the tile with shuffles (lanes = segments).  Segments from
+// n_dx on contribute nothing (A = 1, dX = 0).
 // grid (ceil((D*D + D) / 32), BH), 256 threads.
 __global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, const float *ws_A,
-                                                           int n_seg, int E, int dS,
+                                                           int n_seg, int n_dx, int E, int dS,
                                                            const float *state_in_S,
                                                            const float *state_in_z,
                                                            float *state_out_S, float *state_out_z,
@@ -45,9 +46,9 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, cons
         __syncthreads();
         for (int i = warp; i < 32; i += 8) {
             const int s = s0 + i, e = e0 + lane;
-            tile[i][lane] = (s < n_seg && e < E) ? ws[(size_t)s * E + e] : 0.f;
+            tile[i][lane] = (s < n_dx && e < E) ? ws[(size_t)s * E + e] : 0.f;
         }
-        if (tid < 32) Atile[tid] = (s0 + tid < n_seg) ? Ah[s0 + tid] : 1.f;
+        if (tid < 32) Atile[tid] = (s0 + tid < n_dx) ? Ah[s0 + tid] : 1.f;
         __syncthreads();
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, cons
             if (s < n_seg && e < E) ws[(size_t)s * E + e] = tile[i][lane];
         }
     }
-    if (lane == 0) {
+    if (lane == 0 && n_dx == n_seg) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const int e = e0 + warp + 8 * m;
@@ -96,7 +97,7 @@ __device__ __forceinline__ float4 fma4(float a, const float4 &c, const float4 &x
     return make_float4(fmaf(a, c.x, x.x), fmaf(a, c.y, x.y), fmaf(a, c.z, x.z), fmaf(a, c.w, x.w));
 }
 __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, const float *ws_A,
-                                                               int n_seg, int E, int dS,
+                                                               int n_seg, int n_dx, int E, int dS,
                                                                const float *state_in_S,
                                                                const float *state_in_z,
                                                                float *state_out_S, float *state_out_z,
@@ -111,13 +112,13 @@ __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, 
     float4 x[kSeqScanBatch];
 #pragma unroll
     for (int i = 0; i < kSeqScanBatch; ++i)
-        x[i] = (live && i < n_seg) ? ws[i * E4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[i] = (live && i < n_dx) ? ws[i * E4] : make_float4(0.f, 0.f, 0.f, 0.f);
     float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
     if (live) {
         if (e < dS) { if (state_in_S) carry = *reinterpret_cast<const float4 *>(state_in_S + (size_t)bh * dS + e); }
         else if (state_in_z) carry = *reinterpret_cast<const float4 *>(state_in_z + (size_t)bh * (E - dS) + (e - dS));
     }
-    if (threadIdx.x < n_seg) Ash[threadIdx.x] = ws_A[(size_t)bh * n_seg + threadIdx.x];
+    if (threadIdx.x < n_dx) Ash[threadIdx.x] = ws_A[(size_t)bh * n_seg + threadIdx.x];
     __syncthreads();
     if (!live) return;
 #pragma unroll 1
@@ -125,15 +126,19 @@ __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, 
         if (s0 > 0) {
 #pragma unroll
             for (int i = 0; i < kSeqScanBatch; ++i)
-                if (s0 + i < n_seg) x[i] = ws[(size_t)(s0 + i) * E4];
+                if (s0 + i < n_dx) x[i] = ws[(size_t)(s0 + i) * E4];
         }
 #pragma unroll
         for (int i = 0; i < kSeqScanBatch; ++i) {
             if (s0 + i < n_seg) {
                 ws[(size_t)(s0 + i) * E4] = carry;   // state entering segment s0 + i
-                carry = fma4(Ash[s0 + i], carry, x[i]);
+                if (s0 + i < n_dx) carry = fma4(Ash[s0 + i], carry, x[i]);
             }
         }
+    }
+    if (n_dx != n_seg) {   // the output pass forms the final state
+        pdl_trigger();
+        return;
     }
     if (total) *reinterpret_cast<float4 *>(total + (size_t)bh * E + e) = carry;
     if (e < dS) { if (state_out_S) *reinterpret_cast<float4 *>(state_out_S + (size_t)bh * dS + e) = carry; }
@@ -141,7 +146,7 @@ __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, 
     pdl_trigger();
 }
 
-la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n_seg, int D,
+la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n_seg, int n_dx, int D,
                               int mode, float *state_S, float *state_z, float *total,
                               cudaStream_t st, bool pdl) {
     const int E = D * D + D;
@@ -162,11 +167,11 @@ la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n
     cudaError_t err;
     if (n_seg <= kSeqScanMaxSeg && E % 4 == 0 && D % 4 == 0) {   // float4 groups stay inside S or z
         cfg.gridDim = dim3((E / 4 + 255) / 256, (unsigned)BH);
-        err = cudaLaunchKernelEx(&cfg, segment_scan_seq_kernel, ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z,
+        err = cudaLaunchKernelEx(&cfg, segment_scan_seq_kernel, ws_state, ws_A, n_seg, n_dx, E, D * D, sin_S, sin_z,
                                  sout_S, sout_z, total);
     } else {
         cfg.gridDim = dim3((E + 31) / 32, (unsigned)BH);
-        err = cudaLaunchKernelEx(&cfg, segment_scan_kernel, ws_state, ws_A, n_seg, E, D * D, sin_S, sin_z,
+        err = cudaLaunchKernelEx(&cfg, segment_scan_kernel, ws_state, ws_A, n_seg, n_dx, E, D * D, sin_S, sin_z,
                                  sout_S, sout_z, total);
     }
     count_launches(1);

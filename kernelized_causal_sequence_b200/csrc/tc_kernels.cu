@@ -86,6 +86,11 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
     p.out = a.out;
     p.ws_state = a.ws_state;
     p.ws_A = a.ws_A;
+    // the last segment's output pass forms the final state, so the state pass
+    // and the scan skip that segment's contribution
+    const int n_k1 = a.n_seg - 1;
+    p.fin_S = a.mode != LA_STATE_NONE ? a.state_S : nullptr;
+    p.fin_z = a.mode != LA_STATE_NONE ? a.state_z : nullptr;
     p.status = a.status;
     p.T = a.T;
     p.seg_len = a.seg_len;
@@ -95,17 +100,19 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
     if (e0 != LA_OK) return e0;
     la_status s = record_event(a.events, 0, st);
     if (s != LA_OK) return s;
-    // K1: per-segment state contributions.  A segment's contribution does not
-    // depend on the chunk, so K1 always walks it in 128-token tiles (fewer,
-    // longer pipeline steps); segments are whole 64-token chunks and the last
-    // tile of a segment may be a half tile.
-    if constexpr (C == 64) {
+    // K1: per-segment state contributions of segments 0 .. n_seg-2.  A
+    // segment's contribution does not depend on the chunk, so K1 always walks
+    // it in 128-token tiles (fewer, longer pipeline steps); segments are whole
+    // 64-token chunks and the last tile of a segment may be a half tile.
+    if (n_k1 == 0) {
+        s = LA_OK;
+    } else if constexpr (C == 64) {
         CUtensorMap mk1, mv1;
         if (!make_map(&mk1, a.k, a.in_dtype, a.BH, a.T, D, 128) || !make_map(&mv1, a.v, a.in_dtype, a.BH, a.T, D, 128))
             return cuda_fail_msg("cuTensorMapEncodeTiled", "tensor map encoding failed");
-        s = launch_tc<128, D, DECAY, tc::kStateOnly, InT, float>(mq, mk1, mv1, mo, p, a.BH, a.n_seg, st);
+        s = launch_tc<128, D, DECAY, tc::kStateOnly, InT, float>(mq, mk1, mv1, mo, p, a.BH, n_k1, st);
     } else {
-        s = launch_tc<C, D, DECAY, tc::kStateOnly, InT, float>(mq, mk, mv, mo, p, a.BH, a.n_seg, st);
+        s = launch_tc<C, D, DECAY, tc::kStateOnly, InT, float>(mq, mk, mv, mo, p, a.BH, n_k1, st);
     }
     if (s != LA_OK) return s;
     if ((s = record_event(a.events, 1, st)) != LA_OK) return s;
@@ -113,8 +120,8 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
     // (programmatic dependent launches: each kernel's launch overlaps the end of
     // the previous one; events between the passes, when asked for, serialise them)
     const bool pdl = a.events == nullptr;
-    s = launch_segment_scan(a.ws_state, a.ws_A, a.BH, a.n_seg, D, a.mode, a.state_S, a.state_z,
-                            nullptr, st, pdl);
+    s = launch_segment_scan(a.ws_state, a.ws_A, a.BH, a.n_seg, n_k1, D, a.mode, a.state_S, a.state_z,
+                            nullptr, st, pdl && n_k1 > 0);
     if (s != LA_OK) return s;
     if ((s = record_event(a.events, 2, st)) != LA_OK) return s;
     // K3: chunked output from the segment-entry states

@@ -134,6 +134,8 @@ struct TcParams {
     void *out;            // [BH, T, D]
     float *ws_state;      // [BH, n_seg, D*D + D]
     float *ws_A;          // [BH, n_seg]
+    float *fin_S;         // [BH, D, D] or null: output mode writes the final state
+    float *fin_z;         // [BH, D]      from the last segment (the scan does not)
     int *status;          // status word (0 = ok)
     int T, seg_len, n_seg;
     float eps;
@@ -162,6 +164,30 @@ template <> __device__ __forceinline__ void store_row32<f16>(f16 *dst, const flo
     for (int i = 0; i < 4; ++i)
         d4[i] = make_uint4(pack_f16x2(o[8 * i], o[8 * i + 1]), pack_f16x2(o[8 * i + 2], o[8 * i + 3]),
                            pack_f16x2(o[8 * i + 4], o[8 * i + 5]), pack_f16x2(o[8 * i + 6], o[8 * i + 7]));
+}
+
+// The state (S, z) held in TMEM (rows = feature index, one row per thread)
+// to fp32 global memory: S row-major [D][D], z [D].  Out of line: it runs
+// once per CTA and keeps the chunk loop's code small.
+template <int D>
+__device__ __noinline__ void write_final_state(uint32_t t_s, uint32_t t_z, float *S, float *z, int a_row,
+                                               bool row_ok) {
+    uint32_t zbits;
+    tmem_ld1(t_z, zbits);
+#pragma unroll 1
+    for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t u[32];
+        tmem_ld32(t_s + cb * 32, u);
+        tmem_ld_wait();
+        if (row_ok) {
+            float4 *d4 = reinterpret_cast<float4 *>(S + (size_t)a_row * D + cb * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                d4[i] = make_float4(__uint_as_float(u[4 * i]), __uint_as_float(u[4 * i + 1]),
+                                    __uint_as_float(u[4 * i + 2]), __uint_as_float(u[4 * i + 3]));
+        }
+    }
+    if (row_ok) z[a_row] = __uint_as_float(zbits);
 }
 
 // Unpack 8 input elements (one 16-byte chunk) to fp32.
@@ -901,7 +927,17 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, c + 1, tw);
                     if (!ok) break;
                 }
-                if (c == nch - 1) break;   // the final state of a segment is produced by the scan
+                if (c == nch - 1) {
+                    // the state after a segment's last chunk is read only as the
+                    // final state, which the last segment writes out
+                    if (p.fin_S && seg == p.n_seg - 1 && mbar_wait(&bar[G::B_DS_FULL], c & 1, ab, 19)) {
+                        tc_fence_after();
+                        write_final_state<D>(tmem + lane_base + G::T_S, tmem + lane_base + G::T_Z,
+                                             p.fin_S + (size_t)bh * D * D, p.fin_z + (size_t)bh * D, a_row,
+                                             srow_ok);
+                    }
+                    break;
+                }
                 if (!mbar_wait(&bar[G::B_DS_FULL], c & 1, ab, 11)) { ok = false; break; }
                 float gnext = 1.f;   // decay of chunk c+1
                 if constexpr (DECAY) {
