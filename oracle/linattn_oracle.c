@@ -23,9 +23,16 @@
  *                                               (normalised read-out with the
  *                                                 1e-6 of the section 3 sketch)
  *
+ * Gated form: an optional per-token gain b_t scales the new term,
+ *   S_t = a_t S_{t-1} + b_t phi(k_t) v_t^T,  z_t = a_t z_{t-1} + b_t phi(k_t).
+ * Random Feature Attention's sigmoid gate g_t is a_t = g_t, b_t = 1 - g_t
+ * (concept card "Linear attention": RFA variant and the closing paragraph of
+ * its "Implementation sketch", RFA eq. 7); b_t = 1 is the plain form.
+ *
  * Layouts (all row-major, C order, fp64):
  *   q, k     [B, H, T, d_k]      v [B, H, T, d_v]      out [B, H, T, d_v]
  *   decay    [B, H, T] (causal) or [B, H] (decode); NULL = no decay
+ *   gain     same layout as decay; NULL = 1
  *   S        [B, H, d_k, d_v]    z [B, H, d_k]
  *
  * Parallelism: independent (b, h) heads are spread over OpenMP threads; the
@@ -62,14 +69,17 @@ int orc_max_threads(void)
 #endif
 }
 
-/* One head of the causal recurrence.  fk/fq are scratch of length dk. */
+/* One head of the causal recurrence.  fk/fq are scratch of length dk.  The
+ * gain multiplies the new key's features once (b * phi(k_t)), so it reaches
+ * both the state and the normaliser; b = 1 leaves every value unchanged. */
 static void causal_head(const double *q, const double *k, const double *v,
-                        const double *decay, long T, int dk, int dv, double eps,
-                        double *S, double *z, double *out, double *fk, double *fq)
+                        const double *decay, const double *gain, long T, int dk, int dv,
+                        double eps, double *S, double *z, double *out, double *fk, double *fq)
 {
     for (long t = 0; t < T; ++t) {
         const double *qt = q + t * dk, *kt = k + t * dk, *vt = v + t * dv;
-        for (int i = 0; i < dk; ++i) { fk[i] = phi(kt[i]); fq[i] = phi(qt[i]); }
+        const double b = gain ? gain[t] : 1.0;
+        for (int i = 0; i < dk; ++i) { fk[i] = b * phi(kt[i]); fq[i] = phi(qt[i]); }
         if (decay) {
             /* decayed form: the old state is scaled first, the new token
              * enters undecayed */
@@ -102,10 +112,10 @@ static void causal_head(const double *q, const double *k, const double *v,
  *   S_out/z_out: final state, or NULL to discard.
  * Returns 0, or -1 on a bad argument / allocation failure.
  */
-int orc_causal(const double *q, const double *k, const double *v, const double *decay,
-               int B, int H, long T, int dk, int dv, double eps,
-               const double *S_in, const double *z_in,
-               double *out, double *S_out, double *z_out)
+int orc_causal_gated(const double *q, const double *k, const double *v, const double *decay,
+                     const double *gain, int B, int H, long T, int dk, int dv, double eps,
+                     const double *S_in, const double *z_in,
+                     double *out, double *S_out, double *z_out)
 {
     if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
     const long BH = (long)B * H;
@@ -127,8 +137,8 @@ int orc_causal(const double *q, const double *k, const double *v, const double *
                 if (z_in) memcpy(z, z_in + bh * dk, sizeof(double) * (size_t)dk);
                 else memset(z, 0, sizeof(double) * (size_t)dk);
                 causal_head(q + bh * T * dk, k + bh * T * dk, v + bh * T * dv,
-                            decay ? decay + bh * T : NULL, T, dk, dv, eps,
-                            S, z, out + bh * T * dv, fk, fq);
+                            decay ? decay + bh * T : NULL, gain ? gain + bh * T : NULL, T, dk, dv,
+                            eps, S, z, out + bh * T * dv, fk, fq);
                 if (S_out) memcpy(S_out + bh * dk * dv, S, sizeof(double) * (size_t)dk * dv);
                 if (z_out) memcpy(z_out + bh * dk, z, sizeof(double) * (size_t)dk);
             }
@@ -136,6 +146,14 @@ int orc_causal(const double *q, const double *k, const double *v, const double *
         free(S); free(z); free(fk); free(fq);
     }
     return err ? -1 : 0;
+}
+
+int orc_causal(const double *q, const double *k, const double *v, const double *decay,
+               int B, int H, long T, int dk, int dv, double eps,
+               const double *S_in, const double *z_in,
+               double *out, double *S_out, double *z_out)
+{
+    return orc_causal_gated(q, k, v, decay, NULL, B, H, T, dk, dv, eps, S_in, z_in, out, S_out, z_out);
 }
 
 /*
@@ -200,11 +218,11 @@ int orc_noncausal(const double *q, const double *k, const double *v,
 /*
  * One constant-state decode step per head: the causal loop body applied once
  * to a carried (S, z), which are updated in place.
- *   q, k [B, H, dk], v [B, H, dv], decay [B, H] or NULL, out [B, H, dv].
+ *   q, k [B, H, dk], v [B, H, dv], decay and gain [B, H] or NULL, out [B, H, dv].
  */
-int orc_decode_step(const double *q, const double *k, const double *v, const double *decay,
-                    int B, int H, int dk, int dv, double eps,
-                    double *S, double *z, double *out)
+int orc_decode_step_gated(const double *q, const double *k, const double *v, const double *decay,
+                          const double *gain, int B, int H, int dk, int dv, double eps,
+                          double *S, double *z, double *out)
 {
     if (B < 0 || H < 0 || dk <= 0 || dv <= 0 || !S || !z) return -1;
     const long BH = (long)B * H;
@@ -220,11 +238,18 @@ int orc_decode_step(const double *q, const double *k, const double *v, const dou
 #pragma omp for schedule(static)
             for (long bh = 0; bh < BH; ++bh) {
                 causal_head(q + bh * dk, k + bh * dk, v + bh * dv,
-                            decay ? decay + bh : NULL, 1, dk, dv, eps,
+                            decay ? decay + bh : NULL, gain ? gain + bh : NULL, 1, dk, dv, eps,
                             S + bh * dk * dv, z + bh * dk, out + bh * dv, fk, fq);
             }
         }
         free(fk); free(fq);
     }
     return err ? -1 : 0;
+}
+
+int orc_decode_step(const double *q, const double *k, const double *v, const double *decay,
+                    int B, int H, int dk, int dv, double eps,
+                    double *S, double *z, double *out)
+{
+    return orc_decode_step_gated(q, k, v, decay, NULL, B, H, dk, dv, eps, S, z, out);
 }

@@ -289,3 +289,98 @@ def test_oracle_thread_count_invariance(orc):
     o2, _, _ = orc.causal(q, k, v)
     orc.set_threads(n)
     assert np.array_equal(o1, o2)
+
+
+# ------------------------------------------------------------------ gated form
+# A per-token gain b_t on the new term, S_t = a_t S_{t-1} + b_t phi(k_t) v_t^T
+# (and z alike).  Random Feature Attention's sigmoid gate is a_t = g_t,
+# b_t = 1 - g_t (concept card, RFA variant and the closing paragraph of its
+# implementation sketch; RFA eq. 7).
+
+@pytest.mark.parametrize("seed,T,d", [(81, 9, 3), (82, 40, 4), (83, 64, 6)])
+def test_gated_quadratic(orc, seed, T, d):
+    """The gated recurrence equals the quadratic form weighted by
+    W_ij = (prod_{l=j+1..i} a_l) * b_j: the gain belongs to the key's token and
+    is not decayed at its own step."""
+    rng = np.random.default_rng(seed)
+    q, k, v = (rng.standard_normal((1, 2, T, d)) for _ in range(3))
+    a = 1.0 / (1.0 + np.exp(-(rng.standard_normal((1, 2, T)) + 2.0)))
+    b = rng.uniform(0.0, 2.0, (1, 2, T))
+    b[0, 0, T // 3] = 0.0   # a key that enters with weight zero
+    out, S, z = orc.causal(q, k, v, decay=a, eps=1e-6, gain=b)
+    for h in range(2):
+        W = _semiseparable(a[0, h]) * b[0, h][None, :]
+        ref = quad_causal(q[0, h], k[0, h], v[0, h], 1e-6, weights=W)
+        np.testing.assert_allclose(out[0, h], ref, rtol=1e-11, atol=1e-12)
+        fk = phi_ref(k[0, h])
+        np.testing.assert_allclose(S[0, h], (fk * W[-1][:, None]).T @ v[0, h], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(z[0, h], (fk * W[-1][:, None]).sum(0), rtol=1e-11, atol=1e-12)
+    # the gain is not the decay: moving it onto the query index changes the result
+    W_wrong = _semiseparable(a[0, 1]) * b[0, 1][:, None]
+    assert np.abs(out[0, 1] - quad_causal(q[0, 1], k[0, 1], v[0, 1], 1e-6, weights=W_wrong)).max() > 1e-3
+
+
+def test_rfa_gate_closed_form(orc):
+    """Constant gate g, all keys equal (w = phi(q_t).phi(k) per query): the
+    gated sums are geometric, z_t = (1 - g^(t+1)) phi(k) and
+    o_t = w (1-g) sum_{j<=t} g^(t-j) v_j / (w (1 - g^(t+1)) + eps)."""
+    rng = np.random.default_rng(91)
+    T, d, e, g, eps = 30, 4, 3, 0.8, 1e-3
+    q = rng.standard_normal((1, 1, T, d))
+    kk = np.broadcast_to(rng.standard_normal((1, 1, 1, d)), (1, 1, T, d)).copy()
+    v = rng.standard_normal((1, 1, T, e))
+    out, S, z = orc.causal(q, kk, v, decay=np.full((1, 1, T), g), eps=eps, gain=np.full((1, 1, T), 1.0 - g))
+    fk = phi_ref(kk[0, 0, 0])
+    w = phi_ref(q[0, 0]) @ fk
+    t = np.arange(T)
+    num = np.stack([(1.0 - g) * (g ** (tt - np.arange(tt + 1)))[:, None].T @ v[0, 0, :tt + 1] for tt in t])[:, 0]
+    ref = (w[:, None] * num) / (w * (1.0 - g ** (t + 1)) + eps)[:, None]
+    np.testing.assert_allclose(out[0, 0], ref, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(z[0, 0], (1.0 - g ** T) * fk, rtol=1e-12)
+
+
+@pytest.mark.parametrize("with_decay", [False, True])
+def test_gain_one_is_plain_bitwise(orc, with_decay):
+    rng = np.random.default_rng(95 + with_decay)
+    q, k, v = (rng.standard_normal((2, 2, 50, 6)) for _ in range(3))
+    a = rng.uniform(0.5, 1.0, (2, 2, 50)) if with_decay else None
+    o1, S1, z1 = orc.causal(q, k, v, decay=a, eps=1e-6)
+    o2, S2, z2 = orc.causal(q, k, v, decay=a, eps=1e-6, gain=np.ones((2, 2, 50)))
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2) and np.array_equal(z1, z2)
+
+
+def test_gain_scale_invariance(orc):
+    """With eps = 0 the read-out is a ratio, so scaling every gain by c leaves
+    the outputs unchanged while the state scales by c."""
+    rng = np.random.default_rng(97)
+    q, k, v = (rng.standard_normal((1, 2, 33, 5)) for _ in range(3))
+    a = rng.uniform(0.6, 1.0, (1, 2, 33))
+    b = rng.uniform(0.1, 1.0, (1, 2, 33))
+    o1, S1, z1 = orc.causal(q, k, v, decay=a, eps=0.0, gain=b)
+    o2, S2, z2 = orc.causal(q, k, v, decay=a, eps=0.0, gain=3.0 * b)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S2, 3.0 * S1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(z2, 3.0 * z1, rtol=1e-12)
+
+
+def test_gated_split_and_decode_handoff(orc):
+    rng = np.random.default_rng(99)
+    B, H, T1, T2, d, e = 1, 2, 11, 17, 4, 3
+    T = T1 + T2
+    q = rng.standard_normal((B, H, T + 1, d))
+    k = rng.standard_normal((B, H, T + 1, d))
+    v = rng.standard_normal((B, H, T + 1, e))
+    g = 1.0 / (1.0 + np.exp(-(rng.standard_normal((B, H, T + 1)) + 2.0)))
+    a, b = g, 1.0 - g
+    o_full, S_full, z_full = orc.causal(q[:, :, :T], k[:, :, :T], v[:, :, :T], a[:, :, :T], gain=b[:, :, :T])
+    o1, S1, z1 = orc.causal(q[:, :, :T1], k[:, :, :T1], v[:, :, :T1], a[:, :, :T1], gain=b[:, :, :T1])
+    o2, S2, z2 = orc.causal(q[:, :, T1:T], k[:, :, T1:T], v[:, :, T1:T], a[:, :, T1:T], S_in=S1, z_in=z1,
+                            gain=b[:, :, T1:T])
+    np.testing.assert_allclose(np.concatenate([o1, o2], 2), o_full, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S2, S_full, rtol=1e-12, atol=1e-12)
+    od, Sd, zd = orc.decode_step(q[:, :, T], k[:, :, T], v[:, :, T], S_full, z_full, decay=a[:, :, T],
+                                 gain=b[:, :, T])
+    o_next, S_next, z_next = orc.causal(q, k, v, a, gain=b)
+    np.testing.assert_allclose(od, o_next[:, :, T], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(Sd, S_next, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(zd, z_next, rtol=1e-12)
