@@ -60,10 +60,11 @@ def elem_bytes(dtype: str) -> int:
 
 
 def prefill_algorithmic_bytes(w) -> int:
-    """Minimum bytes any implementation moves: Q, K, V (and decay) read once,
-    O written once.  The fp32 state in/out is excluded (it is per head)."""
+    """Minimum bytes any implementation moves: Q, K, V (and decay, gain) read
+    once, O written once.  The fp32 state in/out is excluded (it is per head)."""
     ht = w.B * w.H * w.T
-    per = 3 * w.d * elem_bytes(w.dtype) + w.d * elem_bytes(w.out_dtype) + (4 if w.decay else 0)
+    per = (3 * w.d * elem_bytes(w.dtype) + w.d * elem_bytes(w.out_dtype) + (4 if w.decay else 0)
+           + (4 if w.gated else 0))
     return ht * per
 
 
@@ -261,7 +262,9 @@ def measure_workloads(dev, peaks, iters=10, only=None):
     rows = [("causal_f32_t256_d64", None), ("causal_bf16_b4h8_t2048_d64", None),
             ("ssd_decay_bf16_b2h16_t8192_d128", None),
             # the same SSD inputs with 128-token chunks (equal results up to rounding)
-            ("ssd_decay_bf16_b2h16_t8192_d128", 128)]
+            ("ssd_decay_bf16_b2h16_t8192_d128", 128),
+            # the gated form (RFA gate) at the SSD shape
+            ("rfa_gated_bf16_b2h16_t8192_d128", None)]
     for name, chunk in rows:
         if only is not None and name != only:
             continue
@@ -270,22 +273,27 @@ def measure_workloads(dev, peaks, iters=10, only=None):
             w = dataclasses.replace(w, chunk=chunk)
         key = name if chunk is None else f"{name}@chunk{chunk}"
         q, k, v, a = (None if x is None else x.to(dev) for x in inputs.qkv(w))
+        gn = inputs.gate_gain(w, None if a is None else a.cpu())
+        gn = None if gn is None else gn.to(dev)
         out = torch.empty((w.B, w.H, w.T, w.d), dtype=w.torch_out_dtype, device=dev)
         S = torch.zeros((w.B, w.H, w.d, w.d), device=dev)
         z = torch.zeros((w.B, w.H, w.d), device=dev)
         ws = torch.empty(max(1, la.la_prefill_workspace_size(w.B, w.H, w.T, w.d, w.d, w.chunk)),
                          dtype=torch.uint8, device=dev)
         fn = lambda: la.la_prefill_causal(q, k, v, decay=a, eps=w.eps, chunk=w.chunk, state_S=S,
-                                          state_z=z, out=out, workspace=ws)
+                                          state_z=z, out=out, workspace=ws, gain=gn)
         fn()
         ms = time_calls(fn, iters, flush)
         # per-pass split of one more (flushed) call, from the library's events
-        kev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        flush()
-        la.la_prefill_causal(q, k, v, decay=a, eps=w.eps, chunk=w.chunk, state_S=S, state_z=z,
-                             out=out, workspace=ws, events=kev)
-        torch.cuda.synchronize(dev)
-        split = {nm: kev[j].elapsed_time(kev[j + 1]) for j, nm in enumerate(("K1_ms", "K2_ms", "K3_ms"))}
+        # (the gated entry point records no events: whole-call time only)
+        split = None
+        if gn is None:
+            kev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            flush()
+            la.la_prefill_causal(q, k, v, decay=a, eps=w.eps, chunk=w.chunk, state_S=S, state_z=z,
+                                 out=out, workspace=ws, events=kev)
+            torch.cuda.synchronize(dev)
+            split = {nm: kev[j].elapsed_time(kev[j + 1]) for j, nm in enumerate(("K1_ms", "K2_ms", "K3_ms"))}
         b = prefill_algorithmic_bytes(w)
         res[key] = {"ms": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3), "algorithmic_bytes": b,
                     "hbm_frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "chunk": w.chunk,

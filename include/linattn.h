@@ -102,6 +102,27 @@ la_status la_prefill_causal_ev(const void *q, const void *k, const void *v, la_d
                                void *workspace, size_t workspace_bytes, void *stream,
                                void *const *events);
 
+/*
+ * la_prefill_causal_gated — the causal prefill with a per-token gain b_t on
+ * the new term (the gated form):
+ *   S_t = a_t S_{t-1} + b_t phi(k_t) v_t^T,   z_t = a_t z_{t-1} + b_t phi(k_t),
+ *   out_t = phi(q_t)^T S_t / (phi(q_t)^T z_t + eps).
+ * Random Feature Attention's sigmoid gate g_t (concept card "Linear
+ * attention", RFA variant and the closing paragraph of its implementation
+ * sketch; RFA eq. 7) is decay = g, gain = 1 - g; NodeFormer's per-key
+ * multiplier is a gain without decay.
+ *   gain   [B, H, T] fp32, finite and >= 0 (a documented precondition, not
+ *          checked on the device), 16-byte aligned, or NULL (b = 1: this is
+ *          la_prefill_causal).
+ * Every other argument, the workspace size and the error behaviour are those
+ * of la_prefill_causal.
+ */
+la_status la_prefill_causal_gated(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                                  const float *decay, const float *gain, int B, int H, int T,
+                                  int d_k, int d_v, float eps, int chunk, float *state_S,
+                                  float *state_z, la_state_mode mode, void *out, la_dtype out_dtype,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of workspace la_prefill_causal needs for these sizes (0 if none). */
 size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chunk);
 
@@ -167,6 +188,17 @@ la_status la_decode_step(const void *q, const void *k, const void *v, la_dtype i
                          const float *decay, int B, int H, int d_k, int d_v, float eps,
                          float *state_S, float *state_z, void *out, la_dtype out_dtype,
                          void *stream);
+
+/*
+ * One gated decode step: S <- a S + b phi(k) v^T, z <- a z + b phi(k), then
+ * the read-out of la_decode_step.  gain [B, H] fp32 (b >= 0, 16-byte aligned)
+ * or NULL (b = 1: this is la_decode_step); the RFA gate is decay = g,
+ * gain = 1 - g.  Other arguments as la_decode_step.
+ */
+la_status la_decode_step_gated(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                               const float *decay, const float *gain, int B, int H, int d_k,
+                               int d_v, float eps, float *state_S, float *state_z, void *out,
+                               la_dtype out_dtype, void *stream);
 
 /* Static description of a status code (never NULL). */
 const char *la_status_string(la_status s);

@@ -63,6 +63,9 @@ def lib() -> ctypes.CDLL:
         L.la_prefill_causal_ev.restype = _i
         L.la_prefill_causal_ev.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _i, _vp,
                                            _vp, _i, _vp, _i, _vp, _sz, _vp, _vp]
+        L.la_prefill_causal_gated.restype = _i
+        L.la_prefill_causal_gated.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _f, _i,
+                                              _vp, _vp, _i, _vp, _i, _vp, _sz, _vp]
         L.la_prefill_workspace_size.restype = _sz
         L.la_prefill_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
         L.la_forward_noncausal.restype = _i
@@ -73,6 +76,9 @@ def lib() -> ctypes.CDLL:
         L.la_decode_step.restype = _i
         L.la_decode_step.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp,
                                      _i, _vp]
+        L.la_decode_step_gated.restype = _i
+        L.la_decode_step_gated.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp,
+                                           _vp, _i, _vp]
         L.la_status_string.restype = ctypes.c_char_p
         L.la_status_string.argtypes = [_i]
         L.la_prefill_plan.restype = _i
@@ -137,13 +143,15 @@ def _workspace(nbytes, device):
 
 def la_prefill_causal(q, k, v, decay=None, eps=1e-6, chunk=64, state_S=None, state_z=None,
                       mode=None, out=None, out_dtype=None, workspace=None, stream=None,
-                      events=None):
+                      events=None, gain=None):
     """Causal chunked prefill.  q, k: [B,H,T,d_k]; v: [B,H,T,d_v] (f32/bf16/f16, CUDA,
     contiguous); decay: [B,H,T] fp32 or None.  state_S [B,H,d_k,d_v] / state_z [B,H,d_k]
     fp32 with ``mode`` LA_STATE_NONE/OUT/INOUT (default: OUT if given, else NONE).
+    ``gain``: [B,H,T] fp32 (>= 0) or None — the gated form, token t's new term
+    scaled by gain[t] (la_prefill_causal_gated; the RFA gate is decay=g, gain=1-g).
     ``events``: None, or 4 recorded-once ``torch.cuda.Event(enable_timing=True)``
     objects that la_prefill_causal_ev records around the state pass, the scan and
-    the output pass.  Returns ``out`` [B,H,T,d_v]."""
+    the output pass (not with ``gain``).  Returns ``out`` [B,H,T,d_v]."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     out_dtype = q.dtype if out_dtype is None else out_dtype
@@ -156,7 +164,12 @@ def la_prefill_causal(q, k, v, decay=None, eps=1e-6, chunk=64, state_S=None, sta
     args = (_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(decay), B, H, T, dk, dv, float(eps),
             int(chunk), _ptr(state_S), _ptr(state_z), int(mode), _ptr(out), _DT[out.dtype],
             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
-    if events is None:
+    if gain is not None:
+        if events is not None:
+            raise ValueError("events are not recorded by the gated prefill")
+        st = lib().la_prefill_causal_gated(*args[:5], _ptr(gain), *args[5:])
+        _check("la_prefill_causal_gated", st)
+    elif events is None:
         st = lib().la_prefill_causal(*args)
         _check("la_prefill_causal", st)
     else:
@@ -192,15 +205,16 @@ def la_forward_noncausal(q, k, v, eps=1e-6, state_S=None, state_z=None, mode=Non
 
 
 def la_decode_step(q, k, v, state_S, state_z, decay=None, eps=1e-6, out=None, out_dtype=None,
-                   stream=None):
-    """One decode step; q, k: [B,H,d_k]; v: [B,H,d_v]; state updated in place."""
+                   stream=None, gain=None):
+    """One decode step; q, k: [B,H,d_k]; v: [B,H,d_v]; state updated in place.
+    ``decay``, ``gain``: [B,H] fp32 or None (gated step: S <- a S + b phi(k) v^T)."""
     B, H, dk = q.shape
     dv = v.shape[-1]
     out_dtype = q.dtype if out_dtype is None else out_dtype
     if out is None:
         out = torch.empty((B, H, dv), dtype=out_dtype, device=q.device)
-    st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(decay), B, H, dk, dv,
-                              float(eps), _ptr(state_S), _ptr(state_z), _ptr(out), _DT[out.dtype],
-                              _stream(stream))
-    _check("la_decode_step", st)
+    st = lib().la_decode_step_gated(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(decay), _ptr(gain), B, H,
+                                    dk, dv, float(eps), _ptr(state_S), _ptr(state_z), _ptr(out),
+                                    _DT[out.dtype], _stream(stream))
+    _check("la_decode_step_gated" if gain is not None else "la_decode_step", st)
     return out

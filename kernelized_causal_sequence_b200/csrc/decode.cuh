@@ -1,6 +1,8 @@
 // decode.cuh — the constant-state decode step (knowledge-base page, section 2
 // "Causal recurrence"; concept card "Implementation sketch" with the optional
-// scalar decay):  S <- a S + phi(k) v^T,  z <- a z + phi(k),
+// scalar decay and, for the gated form, a gain b on the new term — the RFA
+// gate is a = g, b = 1 - g):
+//                 S <- a S + b phi(k) v^T,  z <- a z + b phi(k),
 //                 out = phi(q)^T S / (phi(q)^T z + eps).
 //
 // Memory-bound: each head's fp32 state (d_k x d_v + d_k) is read once and
@@ -18,7 +20,8 @@ constexpr int kDecodeThreads = 256;
 template <typename InT, typename OutT, int D>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k, const InT *__restrict__ v,
-                   const float *__restrict__ decay, float eps, float *__restrict__ S,
+                   const float *__restrict__ decay, const float *__restrict__ gain, float eps,
+                   float *__restrict__ S,
                    float *__restrict__ z, OutT *__restrict__ out) {
     constexpr int CG = D / 4;                     // float4 column groups per row
     constexpr int RSTEP = kDecodeThreads / CG;    // rows handled concurrently
@@ -27,8 +30,9 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k, const I
     __shared__ float den_part[kDecodeThreads / 32];
     const int bh = blockIdx.x, tid = threadIdx.x;
     const float a = decay ? decay[bh] : 1.f;
+    const float b = gain ? gain[bh] : 1.f;
     if (tid < D) {
-        fk[tid] = phi_fast(to_f32(k[(size_t)bh * D + tid]));
+        fk[tid] = b * phi_fast(to_f32(k[(size_t)bh * D + tid]));
         fq[tid] = phi_fast(to_f32(q[(size_t)bh * D + tid]));
     }
     const int cg = tid % CG, r0 = tid / CG;

@@ -203,10 +203,10 @@ template <typename IT, typename OT, int D> struct SimtNoncausalF {
     }
 };
 template <typename IT, typename OT, int D> struct DecodeF {
-    static la_status run(const void *q, const void *k, const void *v, const float *decay,
+    static la_status run(const void *q, const void *k, const void *v, const float *decay, const float *gain,
                          float eps, float *S, float *z, void *out, long BH, cudaStream_t st) {
         decode_step_kernel<IT, OT, D><<<(unsigned)BH, kDecodeThreads, 0, st>>>(
-            (const IT *)q, (const IT *)k, (const IT *)v, decay, eps, S, z, (OT *)out);
+            (const IT *)q, (const IT *)k, (const IT *)v, decay, gain, eps, S, z, (OT *)out);
         count_launches(1);
         return cuda_check("decode_step launch", cudaGetLastError());
     }
@@ -228,6 +228,65 @@ la_status check_state(la_state_mode mode, const float *S, const float *z) {
     if (mode != LA_STATE_NONE && (!S || !z || !aligned16(S) || !aligned16(z)))
         return LA_ERR_INVALID_ARG;
     return LA_OK;
+}
+
+// The causal prefill behind every prefill entry point: decay and gain are
+// optional per-token [BH, T] arrays, events optional (4 cudaEvent_t).
+la_status prefill_impl(const void *q, const void *k, const void *v, la_dtype in_dtype, const float *decay,
+                       const float *gain, int B, int H, int T, int d_k, int d_v, float eps, int chunk,
+                       float *state_S, float *state_z, la_state_mode mode, void *out, la_dtype out_dtype,
+                       void *workspace, size_t workspace_bytes, void *stream, void *const *events) {
+    la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0 || T < 0) return LA_ERR_INVALID_ARG;
+    if (chunk != 64 && chunk != 128) return LA_ERR_UNSUPPORTED;
+    if ((s = check_state(mode, state_S, state_z)) != LA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    const long BH = (long)B * H;
+    if (BH == 0) return LA_OK;
+    if (T == 0) {
+        if (mode == LA_STATE_OUT) {
+            la_status e = cuda_check("state memset", cudaMemsetAsync(state_S, 0, sizeof(float) * BH * d_k * d_v, st));
+            if (e == LA_OK) e = cuda_check("state memset", cudaMemsetAsync(state_z, 0, sizeof(float) * BH * d_k, st));
+            if (e != LA_OK) return e;
+        }
+        return LA_OK;
+    }
+    if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    if (decay && !aligned16(decay)) return LA_ERR_INVALID_ARG;
+    if (gain && !aligned16(gain)) return LA_ERR_INVALID_ARG;
+    if (BH > 65535L) return LA_ERR_UNSUPPORTED;   // heads run along grid y
+    const Plan pl = make_plan(BH, T, chunk, d_k);
+    const WsLayout wl = ws_layout(BH, pl.n_seg, d_k, false);
+    if (!workspace || workspace_bytes < wl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return LA_ERR_INVALID_ARG;
+    char *ws = (char *)workspace;
+
+    if (tc_supported(in_dtype, d_k, chunk, decay != nullptr)) {
+        TcCausalArgs a;
+        a.q = q; a.k = k; a.v = v; a.decay = decay; a.gain = gain; a.out = out;
+        a.in_dtype = in_dtype; a.out_dtype = out_dtype;
+        a.ws_state = (float *)(ws + wl.state_off);
+        a.ws_A = (float *)(ws + wl.A_off);
+        a.status = (int *)(ws + wl.status_off);
+        a.state_S = state_S; a.state_z = state_z; a.mode = mode;
+        a.BH = BH; a.T = T; a.D = d_k; a.chunk = chunk; a.seg_len = pl.seg_len;
+        a.n_seg = pl.n_seg; a.eps = eps;
+        a.events = events;
+        return tc_causal(a, st);
+    }
+    SimtParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k; p.v = v; p.decay = decay; p.gain = gain; p.out = out;
+    p.ws_state = (float *)(ws + wl.state_off);
+    p.ws_A = (float *)(ws + wl.A_off);
+    p.ws_total = nullptr;
+    p.state_S = state_S; p.state_z = state_z; p.mode = mode;
+    p.BH = (int)BH; p.T = T; p.Lq = T; p.chunk = chunk; p.seg_len = pl.seg_len; p.n_seg = pl.n_seg;
+    p.eps = eps;
+    p.events = events;
+    return dispatch3<SimtCausalF>(in_dtype, out_dtype, d_k, p, st);
 }
 
 }  // namespace
@@ -294,56 +353,17 @@ la_status la_prefill_causal_ev(const void *q, const void *k, const void *v, la_d
                                int chunk, float *state_S, float *state_z, la_state_mode mode,
                                void *out, la_dtype out_dtype, void *workspace,
                                size_t workspace_bytes, void *stream, void *const *events) {
-    la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
-    if (s != LA_OK) return s;
-    if (B < 0 || H < 0 || T < 0) return LA_ERR_INVALID_ARG;
-    if (chunk != 64 && chunk != 128) return LA_ERR_UNSUPPORTED;
-    if ((s = check_state(mode, state_S, state_z)) != LA_OK) return s;
-    cudaStream_t st = (cudaStream_t)stream;
-    const long BH = (long)B * H;
-    if (BH == 0) return LA_OK;
-    if (T == 0) {
-        if (mode == LA_STATE_OUT) {
-            la_status e = cuda_check("state memset", cudaMemsetAsync(state_S, 0, sizeof(float) * BH * d_k * d_v, st));
-            if (e == LA_OK) e = cuda_check("state memset", cudaMemsetAsync(state_z, 0, sizeof(float) * BH * d_k, st));
-            if (e != LA_OK) return e;
-        }
-        return LA_OK;
-    }
-    if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_INVALID_ARG;
-    if (decay && !aligned16(decay)) return LA_ERR_INVALID_ARG;
-    if (BH > 65535L) return LA_ERR_UNSUPPORTED;   // heads run along grid y
-    const Plan pl = make_plan(BH, T, chunk, d_k);
-    const WsLayout wl = ws_layout(BH, pl.n_seg, d_k, false);
-    if (!workspace || workspace_bytes < wl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-        return LA_ERR_INVALID_ARG;
-    char *ws = (char *)workspace;
+    return prefill_impl(q, k, v, in_dtype, decay, nullptr, B, H, T, d_k, d_v, eps, chunk, state_S, state_z,
+                        mode, out, out_dtype, workspace, workspace_bytes, stream, events);
+}
 
-    if (tc_supported(in_dtype, d_k, chunk, decay != nullptr)) {
-        TcCausalArgs a;
-        a.q = q; a.k = k; a.v = v; a.decay = decay; a.out = out;
-        a.in_dtype = in_dtype; a.out_dtype = out_dtype;
-        a.ws_state = (float *)(ws + wl.state_off);
-        a.ws_A = (float *)(ws + wl.A_off);
-        a.status = (int *)(ws + wl.status_off);
-        a.state_S = state_S; a.state_z = state_z; a.mode = mode;
-        a.BH = BH; a.T = T; a.D = d_k; a.chunk = chunk; a.seg_len = pl.seg_len;
-        a.n_seg = pl.n_seg; a.eps = eps;
-        a.events = events;
-        return tc_causal(a, st);
-    }
-    SimtParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.q = q; p.k = k; p.v = v; p.decay = decay; p.out = out;
-    p.ws_state = (float *)(ws + wl.state_off);
-    p.ws_A = (float *)(ws + wl.A_off);
-    p.ws_total = nullptr;
-    p.state_S = state_S; p.state_z = state_z; p.mode = mode;
-    p.BH = (int)BH; p.T = T; p.Lq = T; p.chunk = chunk; p.seg_len = pl.seg_len; p.n_seg = pl.n_seg;
-    p.eps = eps;
-    p.events = events;
-    return dispatch3<SimtCausalF>(in_dtype, out_dtype, d_k, p, st);
+la_status la_prefill_causal_gated(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                                  const float *decay, const float *gain, int B, int H, int T, int d_k,
+                                  int d_v, float eps, int chunk, float *state_S, float *state_z,
+                                  la_state_mode mode, void *out, la_dtype out_dtype, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+    return prefill_impl(q, k, v, in_dtype, decay, gain, B, H, T, d_k, d_v, eps, chunk, state_S, state_z,
+                        mode, out, out_dtype, workspace, workspace_bytes, stream, nullptr);
 }
 
 la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_dtype in_dtype,
@@ -392,10 +412,10 @@ la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_d
     return dispatch3<SimtNoncausalF>(in_dtype, out_dtype, d_k, p, Lk, st);
 }
 
-la_status la_decode_step(const void *q, const void *k, const void *v, la_dtype in_dtype,
-                         const float *decay, int B, int H, int d_k, int d_v, float eps,
-                         float *state_S, float *state_z, void *out, la_dtype out_dtype,
-                         void *stream) {
+la_status la_decode_step_gated(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                               const float *decay, const float *gain, int B, int H, int d_k, int d_v,
+                               float eps, float *state_S, float *state_z, void *out, la_dtype out_dtype,
+                               void *stream) {
     la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
     if (s != LA_OK) return s;
     if (B < 0 || H < 0) return LA_ERR_INVALID_ARG;
@@ -403,11 +423,20 @@ la_status la_decode_step(const void *q, const void *k, const void *v, la_dtype i
     if (BH == 0) return LA_OK;
     if (!q || !k || !v || !out || !state_S || !state_z) return LA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-        !aligned16(state_S) || !aligned16(state_z) || (decay && !aligned16(decay)))
+        !aligned16(state_S) || !aligned16(state_z) || (decay && !aligned16(decay)) ||
+        (gain && !aligned16(gain)))
         return LA_ERR_INVALID_ARG;
     if (BH > 0x7fffffffL) return LA_ERR_UNSUPPORTED;
-    return dispatch3<DecodeF>(in_dtype, out_dtype, d_k, q, k, v, decay, eps, state_S, state_z, out,
+    return dispatch3<DecodeF>(in_dtype, out_dtype, d_k, q, k, v, decay, gain, eps, state_S, state_z, out,
                               BH, (cudaStream_t)stream);
+}
+
+la_status la_decode_step(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                         const float *decay, int B, int H, int d_k, int d_v, float eps,
+                         float *state_S, float *state_z, void *out, la_dtype out_dtype,
+                         void *stream) {
+    return la_decode_step_gated(q, k, v, in_dtype, decay, nullptr, B, H, d_k, d_v, eps, state_S, state_z, out,
+                                out_dtype, stream);
 }
 
 }  // extern "C"

@@ -26,6 +26,7 @@ namespace la {
 struct SimtParams {
     const void *q, *k, *v;
     const float *decay;     // [BH, T] or nullptr
+    const float *gain;      // [BH, T] or nullptr: gain b_t on token t's new term (causal only)
     void *out;
     float *ws_state;        // [BH, n_seg, D*D + D]
     float *ws_A;            // [BH, n_seg]
@@ -88,6 +89,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_segment_state_kernel(SimtPa
     const InT *K = (const InT *)p.k + (size_t)bh * T_keys * D;
     const InT *V = (const InT *)p.v + (size_t)bh * T_keys * D;
     const float *A = p.decay ? p.decay + (size_t)bh * T_keys : nullptr;
+    const float *Gk = p.gain ? p.gain + (size_t)bh * T_keys : nullptr;   // per-token gains
 
     float acc[TR][TR];
 #pragma unroll
@@ -124,6 +126,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_segment_state_kernel(SimtPa
                     if (j0 + j < n) {
                         f = phi_precise(kx[u]);
                         if (A) f *= expf(Lend - Lc[j0 + j]);
+                        if (Gk) f *= Gk[c0 + j0 + j];
                     }
                     fk[idx] = f;
                     vv[idx] = vx[u];
@@ -188,6 +191,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
     const InT *V = (const InT *)p.v + (size_t)bh * p.T * D;
     OutT *O = (OutT *)p.out + (size_t)bh * p.T * D;
     const float *A = p.decay ? p.decay + (size_t)bh * p.T : nullptr;
+    const float *Gk = p.gain ? p.gain + (size_t)bh * p.T : nullptr;   // per-token gains
 
     const float *st = p.ws_state + ((size_t)bh * p.n_seg + seg) * (D * D + D);
     pdl_wait();   // the segment scan's output
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
 #pragma unroll
                     for (int u = 0; u < simt_per_thread(D); ++u) {
                         const int idx = tid + u * kSimtThreads, j = idx / D, a = idx % D;
-                        fk[j * RS + a] = (k0 + j < n) ? phi_precise(kx[u]) : 0.f;
+                        fk[j * RS + a] = (k0 + j < n) ? phi_precise(kx[u]) * (Gk ? Gk[c0 + k0 + j] : 1.f) : 0.f;
                         vv[idx] = vx[u];
                     }
                 }
@@ -304,6 +308,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
                     if (k0 + j < n) {
                         f = phi_precise(kx[u]);
                         if (A) f *= expf(Lend - Lc[k0 + j]);
+                        if (Gk) f *= Gk[c0 + k0 + j];
                     }
                     fk[j * RS + a] = f;
                     vv[idx] = vx[u];

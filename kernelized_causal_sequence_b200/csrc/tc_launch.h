@@ -9,6 +9,7 @@ namespace la {
 struct TcCausalArgs {
     const void *q, *k, *v;
     const float *decay;
+    const float *gain;     // per-token gain on the new term, or null
     void *out;
     la_dtype in_dtype, out_dtype;
     float *ws_state, *ws_A;

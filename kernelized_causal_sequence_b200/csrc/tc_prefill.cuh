@@ -90,7 +90,9 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int STG = OUT ? 4 * ROWS_PER_WARP * 128 : 0;
     static constexpr int OFF_F = OFF_STG + STG;                      // fp32 scratch
     static constexpr int F_L = 0;                                    // [NKV][C] log2-decay cumsum
-    static constexpr int F_G = F_L + (DECAY ? NKV * C : 0);          // [NKV] chunk decay
+    // [NKV][C] key-side log2 weights L_j - log2 b_j when a per-token gain b is given
+    static constexpr int F_LK = F_L + (DECAY ? NKV * C : 0);
+    static constexpr int F_G = F_LK + (DECAY ? NKV * C : 0);         // [NKV] chunk decay
     static constexpr int F_LE = F_G + NKV;                           // [NKV] log2 weight origin
     static constexpr int F_END = F_LE + NKV;
     static constexpr int OFF_BAR = (OFF_F + F_END * 4 + 7) / 8 * 8;
@@ -131,6 +133,7 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
 
 struct TcParams {
     const float *decay;   // [BH, T] or null
+    const float *gain;    // [BH, T] or null: per-token gain b_t >= 0 on the new term
     void *out;            // [BH, T, D]
     float *ws_state;      // [BH, n_seg, D*D + D]
     float *ws_A;          // [BH, n_seg]
@@ -351,33 +354,42 @@ template <bool OUT> __device__ __forceinline__ int chunk_at(int c, int nch) { re
 
 // Decay cumsum of chunk c by one warp: L_j (chunk-local inclusive cumsum of
 // log2 a) to shared memory, the chunk decay g = 2^(L_end) and the weight
-// origin; arrives on l_ready.  The decays of chunk c were loaded into
-// registers during chunk c-1; the loads of the next chunk start here so their
-// latency is hidden.  The caller has waited until the stage's L slot is free.
+// origin; arrives on l_ready.  With a per-token gain b (which scales key j's
+// new term), the key-side weights use Lk_j = L_j - log2 b_j instead of L_j:
+// every weight a key receives, 2^(x - L_j), becomes b_j 2^(x - L_j)
+// (b_j = 0 gives Lk_j = +inf and the weight 0).  Without decay (gain only)
+// a = 1.  The decays (and gains) of chunk c were loaded into registers
+// during chunk c-1; the loads of the next chunk start here so their latency
+// is hidden.  The caller has waited until the stage's L slot is free.
 template <int C, int D, bool DECAY, int MODE>
 __device__ __forceinline__ void decay_cumsum(uint64_t *bar, float *Fsm, const TcParams &p, long t_begin,
                                              long t_end, int bh, int c, int nch, int lane, float &Aseg,
-                                             float (&apre)[C / 32], float &lam) {
+                                             float (&apre)[C / 32], float (&bpre)[C / 32], float &lam) {
     using G = Cfg<C, D, DECAY, MODE>;
     const int s = c % G::NKV;
     const long t0 = t_begin + (long)chunk_at<G::OUT>(c, nch) * C;
     const int n = (int)min((long)C, t_end - t0);
     float *L = Fsm + G::F_L + s * C;
-    const float *a = p.decay + (size_t)bh * p.T + t0;
-    float cur[C / 32];
+    const bool has_a = p.decay != nullptr, has_b = p.gain != nullptr;
+    const float *a = has_a ? p.decay + (size_t)bh * p.T + t0 : nullptr;
+    const float *bg = has_b ? p.gain + (size_t)bh * p.T + t0 : nullptr;
+    float cur[C / 32], bcur[C / 32];
 #pragma unroll
     for (int h = 0; h < C / 32; ++h) {
         const int j = h * 32 + lane;
-        cur[h] = (c == 0) ? ((j < n) ? a[j] : 1.f) : apre[h];
+        cur[h] = (c == 0) ? ((has_a && j < n) ? a[j] : 1.f) : apre[h];
+        bcur[h] = (c == 0) ? ((has_b && j < n) ? bg[j] : 1.f) : bpre[h];
     }
     if (c + 1 < nch) {
         const long t1 = t_begin + (long)chunk_at<G::OUT>(c + 1, nch) * C;
         const int n1 = (int)min((long)C, t_end - t1);
-        const float *a1 = p.decay + (size_t)bh * p.T + t1;
+        const float *a1 = has_a ? p.decay + (size_t)bh * p.T + t1 : nullptr;
+        const float *b1 = has_b ? p.gain + (size_t)bh * p.T + t1 : nullptr;
 #pragma unroll
         for (int h = 0; h < C / 32; ++h) {
             const int j = h * 32 + lane;
-            apre[h] = (j < n1) ? a1[j] : 1.f;
+            apre[h] = (has_a && j < n1) ? a1[j] : 1.f;
+            bpre[h] = (has_b && j < n1) ? b1[j] : 1.f;
         }
     }
     float carry = 0.f;
@@ -387,6 +399,7 @@ __device__ __forceinline__ void decay_cumsum(uint64_t *bar, float *Fsm, const Tc
         float x = (j < n) ? lg2_approx(cur[h]) : 0.f;   // log2 units
         x = warp_sum_scan(x, lane) + carry;
         L[j] = x;   // rows >= n repeat the chunk total (never used)
+        if (has_b) Fsm[G::F_LK + s * C + j] = x - lg2_approx(bcur[h]);
         carry = __shfl_sync(0xffffffffu, x, 31);
     }
     if (lane == 0) {
@@ -403,6 +416,13 @@ __device__ __forceinline__ void decay_cumsum(uint64_t *bar, float *Fsm, const Tc
     if (lane == 0) mbar_arrive(&bar[G::B_L_READY + s]);
 }
 
+// Key-side log2 weights of stage s: L, or L - log2 b with a gain.
+template <int C, int D, bool DECAY, int MODE>
+__device__ __forceinline__ const float *key_log_weights(const float *Fsm, const TcParams &p, int s) {
+    using G = Cfg<C, D, DECAY, MODE>;
+    return Fsm + (p.gain ? G::F_LK : G::F_L) + s * C;
+}
+
 // Keys of chunk c (K warpgroup, thread index tk = 0..127): phi(K) in place (in
 // output mode all key rows, in state-only mode the first half, weighted by
 // the decay to the segment end; warps 0-3 take the rest); in output mode
@@ -411,14 +431,15 @@ __device__ __forceinline__ void decay_cumsum(uint64_t *bar, float *Fsm, const Tc
 template <int C, int D, bool DECAY, int MODE, typename InT>
 __device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm, const AbortCtx ab,
                                         const TcParams &p, long t_begin, long t_end, int bh, int c,
-                                        int nch, int tk, float &Aseg, float (&apre)[C / 32], float &lam) {
+                                        int nch, int tk, float &Aseg, float (&apre)[C / 32],
+                                        float (&bpre)[C / 32], float &lam) {
     using G = Cfg<C, D, DECAY, MODE>;
     const int lane = tk & 31;
     const int s = c % G::NKV;
     const long t0 = t_begin + (long)chunk_at<G::OUT>(c, nch) * C;
     const int n = (int)min((long)C, t_end - t0);
     if (!mbar_wait(&bar[G::B_KV_FULL + s], (c / G::NKV) & 1, ab, 8)) return false;
-    float *L = Fsm + G::F_L + s * C;
+    const float *Lk = key_log_weights<C, D, DECAY, MODE>(Fsm, p, s);
     // state-only mode: the weights need the decay cumsum, which the idle phi(Q)
     // warps compute ahead of the key warps
     if constexpr (DECAY && !G::OUT)
@@ -429,15 +450,16 @@ __device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm
     // output mode: plain phi(K) (MMA1 needs it; the decay weights are applied
     // in place after MMA1, see k_weight); state-only: w o phi(K) directly
     if constexpr (G::OUT)
-        phi_tile<InT, C, D, false, CONV, 0, 1, 1>(kt, kt + G::TILE, tk, n, L, Lend);
+        phi_tile<InT, C, D, false, CONV, 0, 1, 1>(kt, kt + G::TILE, tk, n, Lk, Lend);
     else
-        phi_tile<InT, C, D, DECAY, CONV, 0, 2, 4>(kt, kt + G::TILE, tk, n, L, Lend);
+        phi_tile<InT, C, D, DECAY, CONV, 0, 2, 4>(kt, kt + G::TILE, tk, n, Lk, Lend);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
     // output mode: phi(K) did not need the decays; the cumsum follows it (warp 0)
     if constexpr (DECAY && G::OUT)
-        if (tk < 32) decay_cumsum<C, D, DECAY, MODE>(bar, Fsm, p, t_begin, t_end, bh, c, nch, lane, Aseg, apre, lam);
+        if (tk < 32)
+            decay_cumsum<C, D, DECAY, MODE>(bar, Fsm, p, t_begin, t_end, bh, c, nch, lane, Aseg, apre, bpre, lam);
     return true;
 }
 
@@ -506,13 +528,14 @@ __device__ __forceinline__ bool q_stage(uint8_t *smem, uint64_t *bar, const Abor
 // becomes w o phi(K) in place (w_j = 2^(L_end - L_j)) for MMA3; arrives on
 // kw_ready.  False if aborting.
 template <int C, int D, bool DECAY, int MODE>
-__device__ __forceinline__ bool k_weight(uint8_t *smem, uint64_t *bar, float *Fsm, const AbortCtx ab, int c,
-                                         int tk) {
+__device__ __forceinline__ bool k_weight(uint8_t *smem, uint64_t *bar, float *Fsm, const TcParams &p,
+                                         const AbortCtx ab, int c, int tk) {
     using G = Cfg<C, D, DECAY, MODE>;
     const int s = c % G::NKV;
     if (!mbar_wait(&bar[G::B_SC_FULL], c & 1, ab, 21)) return false;
     if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 30)) return false;
-    scale_rows<C, D, true>(smem + G::OFF_KV + s * G::KV_STAGE, tk, Fsm + G::F_L + s * C, Fsm[G::F_LE + s]);
+    scale_rows<C, D, true>(smem + G::OFF_KV + s * G::KV_STAGE, tk, key_log_weights<C, D, DECAY, MODE>(Fsm, p, s),
+                           Fsm[G::F_LE + s]);
     fence_proxy_async_smem();
     __syncwarp();
     if ((tk & 31) == 0) mbar_arrive(&bar[G::B_KW_READY]);
@@ -562,14 +585,14 @@ __device__ __forceinline__ bool q_weight(uint8_t *smem, uint64_t *bar, float *Fs
 // 0-3 (thread index et = 0..127); arrives on phi_done.  False if aborting.
 template <int C, int D, bool DECAY, int MODE, typename InT>
 __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *bar, float *Fsm,
-                                                     const AbortCtx ab, long t_begin, long t_end, int c,
-                                                     int nch, int et) {
+                                                     const TcParams &p, const AbortCtx ab, long t_begin,
+                                                     long t_end, int c, int nch, int et) {
     using G = Cfg<C, D, DECAY, MODE>;
     const int s = c % G::NKV;
     const long t0 = t_begin + (long)chunk_at<G::OUT>(c, nch) * C;
     const int n = (int)min((long)C, t_end - t0);
     if (!mbar_wait(&bar[G::B_KV_FULL + s], (c / G::NKV) & 1, ab, 15)) return false;
-    const float *L = Fsm + G::F_L + s * C;
+    const float *L = key_log_weights<C, D, DECAY, MODE>(Fsm, p, s);
     if constexpr (DECAY)
         if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 16)) return false;
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
@@ -807,15 +830,15 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // ================= keys: decay cumsum and phi(K) (warps 10-13)
         const int tk = threadIdx.x - kKWarp0 * 32;   // 0..127
         float Aseg = 1.f;                            // product of chunk decays (state-only mode)
-        float apre[C / 32];                          // decays of the next chunk (warp kKWarp0)
+        float apre[C / 32], bpre[C / 32];            // decays and gains of the next chunk (warp kKWarp0)
 #pragma unroll
-        for (int h = 0; h < C / 32; ++h) apre[h] = 1.f;
+        for (int h = 0; h < C / 32; ++h) apre[h] = bpre[h] = 1.f;
         float lam = 0.f;   // log2 decay of the chunks already processed (state-only mode)
         bool ok = true;
         for (int c = 0; ok && c < nch; ++c) {
             ok = k_stage<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, p, t_begin, t_end, bh, c, nch, tk, Aseg,
-                                                 apre, lam);
-            if constexpr (G::QS) if (ok) ok = k_weight<C, D, DECAY, MODE>(smem, bar, Fsm, ab, c, tk);
+                                                 apre, bpre, lam);
+            if constexpr (G::QS) if (ok) ok = k_weight<C, D, DECAY, MODE>(smem, bar, Fsm, p, ab, c, tk);
         }
     } else if (warp >= kPhiWarp0) {
         // ================= phi(Q) and the state epilogue (warps 6-9)
@@ -881,9 +904,9 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             float Aseg = 1.f;   // product of the chunk decays (the segment's A)
             if constexpr (DECAY) {
                 if (tw < 32) {
-                    float apre[C / 32];
+                    float apre[C / 32], bpre[C / 32];
 #pragma unroll
-                    for (int h = 0; h < C / 32; ++h) apre[h] = 1.f;
+                    for (int h = 0; h < C / 32; ++h) apre[h] = bpre[h] = 1.f;
                     float lam = 0.f;
                     for (int c = 0; ok && c < nch; ++c) {
                         if (c >= G::NKV &&
@@ -891,7 +914,8 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             ok = false;
                             break;
                         }
-                        decay_cumsum<C, D, DECAY, MODE>(bar, Fsm, p, t_begin, t_end, bh, c, nch, lane, Aseg, apre, lam);
+                        decay_cumsum<C, D, DECAY, MODE>(bar, Fsm, p, t_begin, t_end, bh, c, nch, lane, Aseg, apre,
+                                                        bpre, lam);
                     }
                 }
             }
@@ -981,7 +1005,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     } else if constexpr (!G::OUT) {
         // ================= warps 0-3 in state-only mode: second half of phi(K)
         for (int c = 0; c < nch; ++c)
-            if (!phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, ab, t_begin, t_end, c, nch,
+            if (!phi_keys_second_half<C, D, DECAY, MODE, InT>(smem, bar, Fsm, p, ab, t_begin, t_end, c, nch,
                                                               threadIdx.x))
                 break;
     } else {
@@ -998,6 +1022,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (DECAY && !mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 28)) break;
             tc_fence_after();
             const float *L = Fsm + G::F_L + s * C;
+            const float *Lk = key_log_weights<C, D, DECAY, MODE>(Fsm, p, s);   // key side (gain folded in)
             const float Li = (DECAY && rvalid_lane) ? L[min(i, C - 1)] : 0.f;
             // scores -> P, one 32-column block per TMEM round trip (small code;
             // measured faster than two).  For this warp's rows [r0, r0 + R) a
@@ -1029,8 +1054,8 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             const int j = cb * 32 + 2 * k;
                             float v0 = __uint_as_float(u[h][2 * k]), v1 = __uint_as_float(u[h][2 * k + 1]);
                             if constexpr (DECAY) {
-                                v0 *= ex2_approx(Li - L[j]);
-                                v1 *= ex2_approx(Li - L[j + 1]);
+                                v0 *= ex2_approx(Li - Lk[j]);
+                                v1 *= ex2_approx(Li - Lk[j + 1]);
                             }
                             v0 = (full || j <= i) ? v0 : 0.f;
                             v1 = (full || j + 1 <= i) ? v1 : 0.f;

@@ -34,6 +34,7 @@ class Workload:
     out_dtype: str
     chunk: int = 64
     decay: bool = False
+    gated: bool = False   # RFA gate: decay a_t = g_t and gain b_t = 1 - g_t on the new term
     eps: float = 1e-6
     Lk: int = 0         # non-causal only
     qk_scale: float = 1.0
@@ -66,6 +67,12 @@ WORKLOADS = {
                                                 8192, 128, "bf16", "bf16", chunk=64, decay=True,
                                                 qk_scale=1 / math.sqrt(128),
                                                 v_scale=1 / math.sqrt(128), seed=1003),
+    # the gated form (RFA's sigmoid gate g_t = sigmoid(N(2, 1)), decay g_t and gain 1 - g_t)
+    # at the SSD workload's shape and chunk
+    "rfa_gated_bf16_b2h16_t8192_d128": Workload("rfa_gated_bf16_b2h16_t8192_d128", "causal", 2, 16,
+                                                8192, 128, "bf16", "bf16", chunk=64, decay=True,
+                                                gated=True, qk_scale=1 / math.sqrt(128),
+                                                v_scale=1 / math.sqrt(128), seed=1006),
     # non-causal, LoFTR-coarse shape: B=8, H=8, L=4800, d=32, fp16, V pre-scaled by 1/Lk
     "noncausal_f16_b8h8_l4800_d32": Workload("noncausal_f16_b8h8_l4800_d32", "noncausal", 8, 8,
                                              4800, 32, "f16", "f32", chunk=128, Lk=4800,
@@ -113,6 +120,14 @@ def qkv(w: Workload, seed: int | None = None, T: int | None = None, B: int | Non
         a = (np.float32(1.0) / (np.float32(1.0) + np.exp(-g))).astype(np.float32)
         decay = torch.from_numpy(a)
     return q, k, v, decay
+
+
+def gate_gain(w: Workload, decay: torch.Tensor | None) -> torch.Tensor | None:
+    """The gain input of a gated workload: 1 - g for the gate g drawn as its
+    decay (fp32, rounded once), else None."""
+    if not w.gated or decay is None:
+        return None
+    return torch.from_numpy((np.float32(1.0) - decay.numpy()).astype(np.float32))
 
 
 def cross_kv(w: Workload, Lk: int | None = None, B: int | None = None, H: int | None = None):

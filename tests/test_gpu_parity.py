@@ -343,3 +343,109 @@ def test_prefill_events_entry_point(la, dtype, d, chunk, decay):
     assert np.array_equal(o1, o2.cpu().numpy()) and np.array_equal(S1, S.cpu().numpy())
     times = [ev[j].elapsed_time(ev[j + 1]) for j in range(3)]
     assert all(t >= 0 for t in times) and sum(times) > 0
+
+
+# ------------------------------------------------------------- gated form
+# Per-token gain b_t on the new term (S_t = a_t S_{t-1} + b_t phi(k_t) v_t^T);
+# the RFA gate is a = g, b = 1 - g.
+GATED = [
+    # (dtype, d, T, chunk, kind, B, H)
+    (torch.bfloat16, 128, 1000, 128, "rfa", 1, 2),
+    (torch.bfloat16, 128, 1500, 64, "rfa", 2, 1),
+    (torch.bfloat16, 64, 777, 64, "gain", 1, 3),
+    (torch.bfloat16, 64, 777, 128, "decay_gain", 2, 1),
+    (torch.float16, 128, 513, 64, "gain", 1, 2),
+    (torch.float32, 64, 1000, 64, "rfa", 1, 2),
+    (torch.float32, 32, 300, 128, "gain", 2, 2),
+    (torch.bfloat16, 128, 5000, 64, "rfa", 1, 1),   # > 64 segments per head
+]
+
+
+def _gated_inputs(dtype, d, T, kind, B, H, seed):
+    q, k, v, a = _small_inputs(dtype, d, T, kind != "gain", B, H, seed)
+    rng = np.random.default_rng(seed + 1)
+    if kind == "rfa":
+        b = (1.0 - a.numpy()).astype(np.float32)
+    else:
+        b = rng.uniform(0.0, 2.0, (B, H, T)).astype(np.float32)
+        b[..., T // 3] = 0.0     # keys that enter with weight zero
+        b[..., T // 2] = 0.0
+    return q, k, v, a, torch.from_numpy(b)
+
+
+def gpu_prefill_gated(la, q, k, v, a, b, chunk, out_dtype):
+    B, H, T, d = q.shape
+    S = torch.zeros((B, H, d, d), dtype=torch.float32, device=DEV)
+    z = torch.zeros((B, H, d), dtype=torch.float32, device=DEV)
+    out = la.la_prefill_causal(q.to(DEV), k.to(DEV), v.to(DEV), decay=None if a is None else a.to(DEV),
+                               chunk=chunk, state_S=S, state_z=z, out_dtype=out_dtype, gain=b.to(DEV))
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), S.cpu().numpy(), z.cpu().numpy()
+
+
+@pytest.mark.parametrize("dtype,d,T,chunk,kind,B,H", GATED)
+def test_gated_prefill_small(la, orc, dtype, d, T, chunk, kind, B, H):
+    q, k, v, a, b = _gated_inputs(dtype, d, T, kind, B, H, seed=T * 5 + d)
+    ro, rS, rz = orc.causal(q, k, v, a, 1e-6, gain=b)
+    tol = tol_for(dtype)
+    for out_dtype in ([torch.float32] if dtype == torch.float32 else [torch.float32, dtype]):
+        o, S, z = gpu_prefill_gated(la, q, k, v, a, b, chunk, out_dtype)
+        assert row_rel_err(o, ro) < tol, f"output rel err {row_rel_err(o, ro)}"
+        assert row_rel_err(S.reshape(B, H, -1), rS.reshape(B, H, -1)) < tol
+        assert row_rel_err(z, rz) < tol
+
+
+def test_gain_one_matches_ungated(la):
+    """b = 1 is the ungated form: the CUDA-core path multiplies by 1.0 (bitwise
+    equal); on the tensor-core path the gain enters the key weights through
+    log2(1) = 0 (equal up to the exponent approximation)."""
+    q, k, v, a = _small_inputs(torch.float32, 64, 700, True, 1, 2, seed=12)
+    ones = torch.ones((1, 2, 700), dtype=torch.float32)
+    o1, S1, _ = gpu_prefill(la, q, k, v, a, 64, torch.float32)
+    o2, S2, _ = gpu_prefill_gated(la, q, k, v, a, ones, 64, torch.float32)
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
+    q, k, v, a = _small_inputs(torch.bfloat16, 128, 1000, True, 1, 2, seed=12)
+    ones = torch.ones((1, 2, 1000), dtype=torch.float32)
+    o1, S1, _ = gpu_prefill(la, q, k, v, a, 128, torch.float32)
+    o2, S2, _ = gpu_prefill_gated(la, q, k, v, a, ones, 128, torch.float32)
+    assert row_rel_err(o2, o1) < 1e-5
+    assert row_rel_err(S2.reshape(1, 2, -1), S1.reshape(1, 2, -1)) < 1e-5
+
+
+def test_workload_rfa_gated(la, orc):
+    """The RFA-gated workload at full size, launched as the bench launches it;
+    whole heads are compared with the oracle (heads are independent)."""
+    w = W["rfa_gated_bf16_b2h16_t8192_d128"]
+    q, k, v, a = inputs.qkv(w)
+    b = inputs.gate_gain(w, a)
+    S = torch.zeros((w.B, w.H, w.d, w.d), device=DEV)
+    z = torch.zeros((w.B, w.H, w.d), device=DEV)
+    o = la.la_prefill_causal(q.to(DEV), k.to(DEV), v.to(DEV), decay=a.to(DEV), chunk=w.chunk, state_S=S,
+                             state_z=z, gain=b.to(DEV)).float().cpu().numpy()
+    S = S.cpu().numpy()
+    for bb, h in ((0, 0), (1, 15)):
+        sl = (slice(bb, bb + 1), slice(h, h + 1))
+        ro, rS, _ = orc.causal(q[sl], k[sl], v[sl], a[sl], w.eps, gain=b[sl])
+        assert row_rel_err(o[sl], ro) < 2e-2
+        assert row_rel_err(S[sl].reshape(1, 1, -1), rS.reshape(1, 1, -1)) < 2e-2
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64), (torch.float16, 32)])
+def test_gated_decode(la, orc, dtype, d):
+    rng = np.random.default_rng(d)
+    B, H = 3, 4
+    q, k, v = (torch.from_numpy(rng.standard_normal((B, H, d), dtype=np.float32) / np.sqrt(d)).to(dtype)
+               for _ in range(3))
+    g = torch.from_numpy((1 / (1 + np.exp(-(rng.standard_normal((B, H)) + 2)))).astype(np.float32))
+    b = 1.0 - g
+    S0 = torch.from_numpy(rng.uniform(0, 1, (B, H, d, d)).astype(np.float32))
+    z0 = torch.from_numpy(rng.uniform(1, 2, (B, H, d)).astype(np.float32))
+    S, z = S0.to(DEV), z0.to(DEV)
+    o = la.la_decode_step(q.to(DEV), k.to(DEV), v.to(DEV), S, z, decay=g.to(DEV), gain=b.to(DEV),
+                          out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ro, rS, rz = orc.decode_step(q, k, v, S0, z0, decay=g, gain=b)
+    tol = tol_for(dtype)
+    assert row_rel_err(o.cpu().numpy(), ro) < tol
+    assert row_rel_err(S.cpu().numpy().reshape(B, H, -1), rS.reshape(B, H, -1)) < 1e-5
+    assert row_rel_err(z.cpu().numpy(), rz) < 1e-5
