@@ -37,10 +37,10 @@ METRIC = "causal linear-attn prefill tokens/s on 1 B200 and % of roofline; decod
 
 # DRAM bytes (read + write) of one launch of the output pass (K3) at the
 # long-context workload, from an ncu capture of the same kernel at T = 32768
-# (412.23 MB read + 109.00 MB written) scaled by the tokens processed (x4);
+# (412.25 MB read + 108.39 MB written) scaled by the tokens processed (x4);
 # see profiles/tc_prefill_k1_k3_b1h16_t32768_d128.md.  Only valid for that
 # workload and for the kernel source it was captured from.
-K3_TRAFFIC_LONG_CONTEXT = 4 * (412.23e6 + 109.00e6)
+K3_TRAFFIC_LONG_CONTEXT = 4 * (412.25e6 + 108.39e6)
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
