@@ -12,7 +12,8 @@ arrays to it.  Inputs of any float dtype are converted to float64 exactly
 
 Pinned by ``tests/test_oracle_pins.py`` against the masked quadratic form, the
 decayed (1-semiseparable) quadratic form, the gated form's weighted quadratic
-form and its constant-gate closed form, associativity of the non-causal
+form and its constant-gate closed form, the mLSTM read-out's weighted
+quadratic form with the max(|.|, 1) normaliser, associativity of the non-causal
 bracketing, closed forms on constructed inputs and the linear-attention
 lesson's printed N=8, d=4 example.
 """
@@ -50,16 +51,17 @@ def _load():
     global _lib
     if _lib is None:
         lib = ctypes.CDLL(build())
-        lib.orc_causal_gated.restype = ctypes.c_int
-        lib.orc_causal_gated.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_long,
-                                         ctypes.c_int, ctypes.c_int, ctypes.c_double, _D, _D, _D, _D, _D]
+        lib.orc_causal_form.restype = ctypes.c_int
+        lib.orc_causal_form.argtypes = [ctypes.c_int, _D, _D, _D, _D, _D, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                        _D, _D, _D, _D, _D]
         lib.orc_noncausal.restype = ctypes.c_int
         lib.orc_noncausal.argtypes = [_D, _D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_long,
                                       ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                       _D, _D, _D, _D, _D]
-        lib.orc_decode_step_gated.restype = ctypes.c_int
-        lib.orc_decode_step_gated.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                              ctypes.c_int, ctypes.c_double, _D, _D, _D]
+        lib.orc_decode_step_form.restype = ctypes.c_int
+        lib.orc_decode_step_form.argtypes = [ctypes.c_int, _D, _D, _D, _D, _D, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_double, _D, _D, _D]
         lib.orc_max_threads.restype = ctypes.c_int
         lib.orc_set_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -87,9 +89,11 @@ def max_threads() -> int:
     return int(_load().orc_max_threads())
 
 
-def causal(q, k, v, decay=None, eps=1e-6, S_in=None, z_in=None, gain=None):
+def causal(q, k, v, decay=None, eps=1e-6, S_in=None, z_in=None, gain=None, mlstm=False):
     """Causal recurrence.  q, k: [B,H,T,dk]; v: [B,H,T,dv]; decay, gain: [B,H,T] or
     None (gain b_t scales the new term: S_t = a_t S_{t-1} + b_t phi(k_t) v_t^T).
+    ``mlstm``: the identity feature map and the max(|q^T z|, 1) read-out (decay =
+    forget gate, gain = input gate; eps unused).
     Returns (out [B,H,T,dv], S [B,H,dk,dv], z [B,H,dk]) in fp64."""
     q, k, v, decay, S_in, z_in, gain = map(_f64, (q, k, v, decay, S_in, z_in, gain))
     B, H, T, dk = q.shape
@@ -106,8 +110,8 @@ def causal(q, k, v, decay=None, eps=1e-6, S_in=None, z_in=None, gain=None):
     out = np.zeros((B, H, T, dv))
     S = np.zeros((B, H, dk, dv))
     z = np.zeros((B, H, dk))
-    rc = _load().orc_causal_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(gain), B, H, T, dk, dv,
-                                  float(eps), _ptr(S_in), _ptr(z_in), _ptr(out), _ptr(S), _ptr(z))
+    rc = _load().orc_causal_form(int(bool(mlstm)), _ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(gain), B, H,
+                                 T, dk, dv, float(eps), _ptr(S_in), _ptr(z_in), _ptr(out), _ptr(S), _ptr(z))
     if rc != 0:
         raise RuntimeError("orc_causal failed")
     return out, S, z
@@ -130,17 +134,18 @@ def noncausal(q, k, v, eps=1e-6, S_in=None, z_in=None):
     return out, S, z
 
 
-def decode_step(q, k, v, S, z, decay=None, eps=1e-6, gain=None):
+def decode_step(q, k, v, S, z, decay=None, eps=1e-6, gain=None, mlstm=False):
     """One decode step.  q, k: [B,H,dk]; v: [B,H,dv]; S: [B,H,dk,dv]; z: [B,H,dk];
-    decay, gain: [B,H] or None.  Returns (out [B,H,dv], S_new, z_new); inputs untouched."""
+    decay, gain: [B,H] or None; ``mlstm`` as in causal().
+    Returns (out [B,H,dv], S_new, z_new); inputs untouched."""
     q, k, v, decay, gain = map(_f64, (q, k, v, decay, gain))
     S = _f64(S).copy()
     z = _f64(z).copy()
     B, H, dk = q.shape
     dv = v.shape[-1]
     out = np.zeros((B, H, dv))
-    rc = _load().orc_decode_step_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(gain), B, H, dk, dv,
-                                       float(eps), _ptr(S), _ptr(z), _ptr(out))
+    rc = _load().orc_decode_step_form(int(bool(mlstm)), _ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(gain),
+                                      B, H, dk, dv, float(eps), _ptr(S), _ptr(z), _ptr(out))
     if rc != 0:
         raise RuntimeError("orc_decode_step failed")
     return out, S, z

@@ -29,6 +29,13 @@
  * (concept card "Linear attention": RFA variant and the closing paragraph of
  * its "Implementation sketch", RFA eq. 7); b_t = 1 is the plain form.
  *
+ * mLSTM read-out (concept card, "Matrix memory with exponential gates
+ * (mLSTM)"; its implementation sketch: the identity as the feature map,
+ * input-dependent gates and a normaliser read-out): C_t = f_t C_{t-1} +
+ * i_t v_t k_t^T, n_t = f_t n_{t-1} + i_t k_t, h_t = C_t q_t / max(|n_t^T q_t|, 1).
+ * With S = C^T this is the gated recurrence above with phi = identity,
+ * a = f, b = i, and the denominator max(|q^T z|, 1) in place of q^T z + eps.
+ *
  * Layouts (all row-major, C order, fp64):
  *   q, k     [B, H, T, d_k]      v [B, H, T, d_v]      out [B, H, T, d_v]
  *   decay    [B, H, T] (causal) or [B, H] (decode); NULL = no decay
@@ -51,6 +58,12 @@
  * the -1/+1 pair.  At x = 0 both branches give 1. */
 static double phi(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
 
+/* Feature map and read-out of one call: elu(x)+1 with (den + eps), or the
+ * mLSTM form: the identity with max(|den|, 1). */
+typedef struct { int mlstm; } form_t;
+static double fmap(form_t f, double x) { return f.mlstm ? x : phi(x); }
+static double denom(form_t f, double den, double eps) { return f.mlstm ? fmax(fabs(den), 1.0) : den + eps; }
+
 void orc_set_threads(int n)
 {
 #ifdef _OPENMP
@@ -72,14 +85,14 @@ int orc_max_threads(void)
 /* One head of the causal recurrence.  fk/fq are scratch of length dk.  The
  * gain multiplies the new key's features once (b * phi(k_t)), so it reaches
  * both the state and the normaliser; b = 1 leaves every value unchanged. */
-static void causal_head(const double *q, const double *k, const double *v,
+static void causal_head(form_t form, const double *q, const double *k, const double *v,
                         const double *decay, const double *gain, long T, int dk, int dv,
                         double eps, double *S, double *z, double *out, double *fk, double *fq)
 {
     for (long t = 0; t < T; ++t) {
         const double *qt = q + t * dk, *kt = k + t * dk, *vt = v + t * dv;
         const double b = gain ? gain[t] : 1.0;
-        for (int i = 0; i < dk; ++i) { fk[i] = b * phi(kt[i]); fq[i] = phi(qt[i]); }
+        for (int i = 0; i < dk; ++i) { fk[i] = b * fmap(form, kt[i]); fq[i] = fmap(form, qt[i]); }
         if (decay) {
             /* decayed form: the old state is scaled first, the new token
              * enters undecayed */
@@ -97,11 +110,12 @@ static void causal_head(const double *q, const double *k, const double *v,
         }
         double den = 0.0;
         for (int i = 0; i < dk; ++i) den += fq[i] * z[i];
+        den = denom(form, den, eps);
         double *ot = out + t * dv;
         for (int j = 0; j < dv; ++j) {
             double num = 0.0;
             for (int i = 0; i < dk; ++i) num += fq[i] * S[i * dv + j];
-            ot[j] = num / (den + eps);
+            ot[j] = num / den;
         }
     }
 }
@@ -112,11 +126,12 @@ static void causal_head(const double *q, const double *k, const double *v,
  *   S_out/z_out: final state, or NULL to discard.
  * Returns 0, or -1 on a bad argument / allocation failure.
  */
-int orc_causal_gated(const double *q, const double *k, const double *v, const double *decay,
-                     const double *gain, int B, int H, long T, int dk, int dv, double eps,
-                     const double *S_in, const double *z_in,
-                     double *out, double *S_out, double *z_out)
+int orc_causal_form(int mlstm, const double *q, const double *k, const double *v, const double *decay,
+                    const double *gain, int B, int H, long T, int dk, int dv, double eps,
+                    const double *S_in, const double *z_in,
+                    double *out, double *S_out, double *z_out)
 {
+    const form_t form = {mlstm};
     if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
     const long BH = (long)B * H;
     int err = 0;
@@ -136,7 +151,7 @@ int orc_causal_gated(const double *q, const double *k, const double *v, const do
                 else memset(S, 0, sizeof(double) * (size_t)dk * dv);
                 if (z_in) memcpy(z, z_in + bh * dk, sizeof(double) * (size_t)dk);
                 else memset(z, 0, sizeof(double) * (size_t)dk);
-                causal_head(q + bh * T * dk, k + bh * T * dk, v + bh * T * dv,
+                causal_head(form, q + bh * T * dk, k + bh * T * dk, v + bh * T * dv,
                             decay ? decay + bh * T : NULL, gain ? gain + bh * T : NULL, T, dk, dv,
                             eps, S, z, out + bh * T * dv, fk, fq);
                 if (S_out) memcpy(S_out + bh * dk * dv, S, sizeof(double) * (size_t)dk * dv);
@@ -148,12 +163,20 @@ int orc_causal_gated(const double *q, const double *k, const double *v, const do
     return err ? -1 : 0;
 }
 
+int orc_causal_gated(const double *q, const double *k, const double *v, const double *decay,
+                     const double *gain, int B, int H, long T, int dk, int dv, double eps,
+                     const double *S_in, const double *z_in,
+                     double *out, double *S_out, double *z_out)
+{
+    return orc_causal_form(0, q, k, v, decay, gain, B, H, T, dk, dv, eps, S_in, z_in, out, S_out, z_out);
+}
+
 int orc_causal(const double *q, const double *k, const double *v, const double *decay,
                int B, int H, long T, int dk, int dv, double eps,
                const double *S_in, const double *z_in,
                double *out, double *S_out, double *z_out)
 {
-    return orc_causal_gated(q, k, v, decay, NULL, B, H, T, dk, dv, eps, S_in, z_in, out, S_out, z_out);
+    return orc_causal_form(0, q, k, v, decay, NULL, B, H, T, dk, dv, eps, S_in, z_in, out, S_out, z_out);
 }
 
 /*
@@ -220,10 +243,11 @@ int orc_noncausal(const double *q, const double *k, const double *v,
  * to a carried (S, z), which are updated in place.
  *   q, k [B, H, dk], v [B, H, dv], decay and gain [B, H] or NULL, out [B, H, dv].
  */
-int orc_decode_step_gated(const double *q, const double *k, const double *v, const double *decay,
-                          const double *gain, int B, int H, int dk, int dv, double eps,
-                          double *S, double *z, double *out)
+int orc_decode_step_form(int mlstm, const double *q, const double *k, const double *v,
+                         const double *decay, const double *gain, int B, int H, int dk, int dv,
+                         double eps, double *S, double *z, double *out)
 {
+    const form_t form = {mlstm};
     if (B < 0 || H < 0 || dk <= 0 || dv <= 0 || !S || !z) return -1;
     const long BH = (long)B * H;
     int err = 0;
@@ -237,7 +261,7 @@ int orc_decode_step_gated(const double *q, const double *k, const double *v, con
         } else {
 #pragma omp for schedule(static)
             for (long bh = 0; bh < BH; ++bh) {
-                causal_head(q + bh * dk, k + bh * dk, v + bh * dv,
+                causal_head(form, q + bh * dk, k + bh * dk, v + bh * dv,
                             decay ? decay + bh : NULL, gain ? gain + bh : NULL, 1, dk, dv, eps,
                             S + bh * dk * dv, z + bh * dk, out + bh * dv, fk, fq);
             }
@@ -247,9 +271,16 @@ int orc_decode_step_gated(const double *q, const double *k, const double *v, con
     return err ? -1 : 0;
 }
 
+int orc_decode_step_gated(const double *q, const double *k, const double *v, const double *decay,
+                          const double *gain, int B, int H, int dk, int dv, double eps,
+                          double *S, double *z, double *out)
+{
+    return orc_decode_step_form(0, q, k, v, decay, gain, B, H, dk, dv, eps, S, z, out);
+}
+
 int orc_decode_step(const double *q, const double *k, const double *v, const double *decay,
                     int B, int H, int dk, int dv, double eps,
                     double *S, double *z, double *out)
 {
-    return orc_decode_step_gated(q, k, v, decay, NULL, B, H, dk, dv, eps, S, z, out);
+    return orc_decode_step_form(0, q, k, v, decay, NULL, B, H, dk, dv, eps, S, z, out);
 }

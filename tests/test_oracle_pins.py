@@ -384,3 +384,82 @@ def test_gated_split_and_decode_handoff(orc):
     np.testing.assert_allclose(od, o_next[:, :, T], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(Sd, S_next, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(zd, z_next, rtol=1e-12)
+
+
+# ------------------------------------------------------------- mLSTM read-out
+# Concept card, "Matrix memory with exponential gates (mLSTM)":
+# C_t = f_t C_{t-1} + i_t v_t k_t^T, n_t = f_t n_{t-1} + i_t k_t, and the
+# read-out C_t q_t / max(|n_t^T q_t|, 1); its implementation sketch places it
+# in the running-sum loop with the identity as the feature map.
+
+def _mlstm_quadratic(q, k, v, f, i):
+    """Quadratic form of one head: raw scores q_t.k_j weighted by
+    (prod_{l=j+1..t} f_l) i_j for j <= t; numerator = weighted scores @ v,
+    denominator max(|row sum|, 1)."""
+    W = _semiseparable(f) * i[None, :]
+    sc = (q @ k.T) * W
+    den = np.maximum(np.abs(sc.sum(-1)), 1.0)
+    return (sc @ v) / den[:, None], sc.sum(-1)
+
+
+@pytest.mark.parametrize("seed,T,d,qs", [(101, 12, 3, 1.0), (102, 48, 4, 0.7), (103, 64, 8, 1.5)])
+def test_mlstm_quadratic(orc, seed, T, d, qs):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, 2, T, d)) * qs
+    k, v = (rng.standard_normal((1, 2, T, d)) for _ in range(2))
+    f = 1.0 / (1.0 + np.exp(-(rng.standard_normal((1, 2, T)) + 2.0)))
+    i = np.exp(rng.standard_normal((1, 2, T)) * 0.5)
+    out, S, z = orc.causal(q, k, v, decay=f, gain=i, mlstm=True)
+    seen_small = seen_large = False
+    for h in range(2):
+        ref, den = _mlstm_quadratic(q[0, h], k[0, h], v[0, h], f[0, h], i[0, h])
+        np.testing.assert_allclose(out[0, h], ref, rtol=1e-11, atol=1e-12)
+        seen_small |= bool((np.abs(den) < 1).any())
+        seen_large |= bool((np.abs(den) > 1).any())
+        # the memory holds the raw keys: S = sum_j w_j k_j v_j^T, z = sum_j w_j k_j
+        w = _semiseparable(f[0, h])[-1] * i[0, h]
+        np.testing.assert_allclose(S[0, h], (k[0, h] * w[:, None]).T @ v[0, h], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(z[0, h], (k[0, h] * w[:, None]).sum(0), rtol=1e-11, atol=1e-12)
+    assert seen_small and seen_large   # both sides of the max(|.|, 1) are exercised
+
+
+def test_mlstm_normaliser_homogeneity(orc):
+    """Rows with |n^T q| < 1 are divided by 1, so they scale linearly with q;
+    rows with |n^T q| > 1 are divided by |n^T q|, so scaling q by c only
+    flips their sign with c."""
+    rng = np.random.default_rng(105)
+    T, d = 40, 4
+    q, k, v = (rng.standard_normal((1, 1, T, d)) for _ in range(3))
+    f = np.full((1, 1, T), 0.9)
+    tiny = 1e-3 * q
+    o1, _, z = orc.causal(tiny, k, v, decay=f, mlstm=True)
+    o2, _, _ = orc.causal(0.5 * tiny, k, v, decay=f, mlstm=True)
+    np.testing.assert_allclose(o2, 0.5 * o1, rtol=1e-12, atol=1e-16)
+    big = 1e3 * q
+    o3, _, _ = orc.causal(big, k, v, decay=f, mlstm=True)
+    o4, _, _ = orc.causal(-2.0 * big, k, v, decay=f, mlstm=True)
+    np.testing.assert_allclose(o4, -o3, rtol=1e-12, atol=1e-12)
+    # the elu+1 form is a different read-out on the same inputs
+    o5, _, _ = orc.causal(big, k, v, decay=f)
+    assert np.abs(o5 - o3).max() > 1e-3
+
+
+def test_mlstm_split_and_decode_handoff(orc):
+    rng = np.random.default_rng(107)
+    B, H, T1, T2, d, e = 1, 2, 9, 14, 4, 3
+    T = T1 + T2
+    q, k = (rng.standard_normal((B, H, T + 1, d)) for _ in range(2))
+    v = rng.standard_normal((B, H, T + 1, e))
+    f = 1.0 / (1.0 + np.exp(-(rng.standard_normal((B, H, T + 1)) + 2.0)))
+    i = np.exp(rng.standard_normal((B, H, T + 1)) * 0.5)
+    kw = dict(mlstm=True)
+    o_full, S_full, z_full = orc.causal(q[:, :, :T], k[:, :, :T], v[:, :, :T], f[:, :, :T], gain=i[:, :, :T], **kw)
+    o1, S1, z1 = orc.causal(q[:, :, :T1], k[:, :, :T1], v[:, :, :T1], f[:, :, :T1], gain=i[:, :, :T1], **kw)
+    o2, S2, z2 = orc.causal(q[:, :, T1:T], k[:, :, T1:T], v[:, :, T1:T], f[:, :, T1:T], S_in=S1, z_in=z1,
+                            gain=i[:, :, T1:T], **kw)
+    np.testing.assert_allclose(np.concatenate([o1, o2], 2), o_full, rtol=1e-12, atol=1e-13)
+    od, Sd, zd = orc.decode_step(q[:, :, T], k[:, :, T], v[:, :, T], S_full, z_full, decay=f[:, :, T],
+                                 gain=i[:, :, T], **kw)
+    o_next, S_next, z_next = orc.causal(q, k, v, f, gain=i, **kw)
+    np.testing.assert_allclose(od, o_next[:, :, T], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(Sd, S_next, rtol=1e-12, atol=1e-12)
