@@ -60,11 +60,12 @@ def elem_bytes(dtype: str) -> int:
 
 
 def prefill_algorithmic_bytes(w) -> int:
-    """Minimum bytes any implementation moves: Q, K, V (and decay, gain) read
-    once, O written once.  The fp32 state in/out is excluded (it is per head)."""
+    """Minimum bytes any implementation moves: Q, K, V (and decay, gain or input
+    gate) read once, O written once.  The fp32 state in/out is excluded (it is
+    per head)."""
     ht = w.B * w.H * w.T
     per = (3 * w.d * elem_bytes(w.dtype) + w.d * elem_bytes(w.out_dtype) + (4 if w.decay else 0)
-           + (4 if w.gated else 0))
+           + (4 if (w.gated or w.mlstm) else 0))
     return ht * per
 
 
@@ -263,8 +264,9 @@ def measure_workloads(dev, peaks, iters=10, only=None):
             ("ssd_decay_bf16_b2h16_t8192_d128", None),
             # the same SSD inputs with 128-token chunks (equal results up to rounding)
             ("ssd_decay_bf16_b2h16_t8192_d128", 128),
-            # the gated form (RFA gate) at the SSD shape
-            ("rfa_gated_bf16_b2h16_t8192_d128", None)]
+            # the gated form (RFA gate) and the mLSTM read-out at the SSD shape
+            ("rfa_gated_bf16_b2h16_t8192_d128", None),
+            ("mlstm_bf16_b2h16_t8192_d128", None)]
     for name, chunk in rows:
         if only is not None and name != only:
             continue
@@ -280,14 +282,19 @@ def measure_workloads(dev, peaks, iters=10, only=None):
         z = torch.zeros((w.B, w.H, w.d), device=dev)
         ws = torch.empty(max(1, la.la_prefill_workspace_size(w.B, w.H, w.T, w.d, w.d, w.chunk)),
                          dtype=torch.uint8, device=dev)
-        fn = lambda: la.la_prefill_causal(q, k, v, decay=a, eps=w.eps, chunk=w.chunk, state_S=S,
-                                          state_z=z, out=out, workspace=ws, gain=gn)
+        if w.mlstm:
+            ig = inputs.input_gate(w).to(dev)
+            fn = lambda: la.la_prefill_causal_mlstm(q, k, v, forget=a, input_gate=ig, chunk=w.chunk, state_S=S,
+                                                    state_z=z, out=out, workspace=ws)
+        else:
+            fn = lambda: la.la_prefill_causal(q, k, v, decay=a, eps=w.eps, chunk=w.chunk, state_S=S,
+                                              state_z=z, out=out, workspace=ws, gain=gn)
         fn()
         ms = time_calls(fn, iters, flush)
         # per-pass split of one more (flushed) call, from the library's events
-        # (the gated entry point records no events: whole-call time only)
+        # (the gated and mLSTM entry points record no events: whole-call time only)
         split = None
-        if gn is None:
+        if gn is None and not w.mlstm:
             kev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
             flush()
             la.la_prefill_causal(q, k, v, decay=a, eps=w.eps, chunk=w.chunk, state_S=S, state_z=z,

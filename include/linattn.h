@@ -123,6 +123,28 @@ la_status la_prefill_causal_gated(const void *q, const void *k, const void *v, l
                                   float *state_z, la_state_mode mode, void *out, la_dtype out_dtype,
                                   void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * la_prefill_causal_mlstm — the causal prefill with the mLSTM read-out
+ * (concept card "Linear attention", "Matrix memory with exponential gates
+ * (mLSTM)": C_t = f_t C_{t-1} + i_t v_t k_t^T, n_t = f_t n_{t-1} + i_t k_t,
+ * h_t = C_t q_t / max(|n_t^T q_t|, 1); the card's implementation sketch fits
+ * it to the running-sum loop with the identity as the feature map).  In this
+ * library's terms, with S = C^T and z = n:
+ *   S_t = f_t S_{t-1} + i_t k_t v_t^T,   z_t = f_t z_{t-1} + i_t k_t,
+ *   out_t = q_t^T S_t / max(|q_t^T z_t|, 1)          (no feature map, no eps)
+ *   forget      [B, H, T] fp32 in (0, 1], or NULL (f = 1)
+ *   input_gate  [B, H, T] fp32, finite and >= 0 (an exponential gate's value;
+ *               the stabiliser state of exponential gating is the caller's),
+ *               or NULL (i = 1)
+ * Both are 16-byte aligned; the state carries the raw keys.  Other arguments,
+ * the workspace size and the error behaviour are those of la_prefill_causal.
+ */
+la_status la_prefill_causal_mlstm(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                                  const float *forget, const float *input_gate, int B, int H, int T,
+                                  int d_k, int d_v, int chunk, float *state_S, float *state_z,
+                                  la_state_mode mode, void *out, la_dtype out_dtype, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
 /* Bytes of workspace la_prefill_causal needs for these sizes (0 if none). */
 size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chunk);
 
@@ -199,6 +221,17 @@ la_status la_decode_step_gated(const void *q, const void *k, const void *v, la_d
                                const float *decay, const float *gain, int B, int H, int d_k,
                                int d_v, float eps, float *state_S, float *state_z, void *out,
                                la_dtype out_dtype, void *stream);
+
+/*
+ * One mLSTM decode step (see la_prefill_causal_mlstm):
+ *   S <- f S + i k v^T, z <- f z + i k, out = q^T S / max(|q^T z|, 1)
+ * forget, input_gate: [B, H] fp32 or NULL (1).  Other arguments as
+ * la_decode_step.
+ */
+la_status la_decode_step_mlstm(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                               const float *forget, const float *input_gate, int B, int H, int d_k,
+                               int d_v, float *state_S, float *state_z, void *out, la_dtype out_dtype,
+                               void *stream);
 
 /* Static description of a status code (never NULL). */
 const char *la_status_string(la_status s);

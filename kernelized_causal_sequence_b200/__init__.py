@@ -22,6 +22,7 @@ import torch
 
 __all__ = [
     "LinAttnError", "lib", "la_prefill_causal", "la_forward_noncausal", "la_decode_step",
+    "la_prefill_causal_mlstm", "la_decode_step_mlstm",
     "la_prefill_workspace_size", "la_noncausal_workspace_size", "la_status_string",
     "la_prefill_path", "la_launch_count", "LA_F32", "LA_BF16", "LA_F16", "LA_STATE_NONE", "LA_STATE_OUT",
     "LA_STATE_INOUT", "LIB_PATH",
@@ -66,6 +67,9 @@ def lib() -> ctypes.CDLL:
         L.la_prefill_causal_gated.restype = _i
         L.la_prefill_causal_gated.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _f, _i,
                                               _vp, _vp, _i, _vp, _i, _vp, _sz, _vp]
+        L.la_prefill_causal_mlstm.restype = _i
+        L.la_prefill_causal_mlstm.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                              _vp, _vp, _i, _vp, _i, _vp, _sz, _vp]
         L.la_prefill_workspace_size.restype = _sz
         L.la_prefill_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
         L.la_forward_noncausal.restype = _i
@@ -78,6 +82,9 @@ def lib() -> ctypes.CDLL:
                                      _i, _vp]
         L.la_decode_step_gated.restype = _i
         L.la_decode_step_gated.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp,
+                                           _vp, _i, _vp]
+        L.la_decode_step_mlstm.restype = _i
+        L.la_decode_step_mlstm.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _vp, _vp,
                                            _vp, _i, _vp]
         L.la_status_string.restype = ctypes.c_char_p
         L.la_status_string.argtypes = [_i]
@@ -181,6 +188,43 @@ def la_prefill_causal(q, k, v, decay=None, eps=1e-6, chunk=64, state_S=None, sta
         arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(int(e.cuda_event)) for e in events])
         st = lib().la_prefill_causal_ev(*args, arr)
         _check("la_prefill_causal_ev", st)
+    return out
+
+
+def la_prefill_causal_mlstm(q, k, v, forget=None, input_gate=None, chunk=64, state_S=None, state_z=None,
+                            mode=None, out=None, out_dtype=None, workspace=None, stream=None):
+    """Causal prefill with the mLSTM read-out: identity feature map, forget gate
+    f and input gate i (``[B,H,T]`` fp32 or None), out = q^T S / max(|q^T z|, 1)."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
+    if mode is None:
+        mode = LA_STATE_OUT if state_S is not None else LA_STATE_NONE
+    if workspace is None:
+        workspace = _workspace(la_prefill_workspace_size(B, H, T, dk, dv, chunk), q.device)
+    st = lib().la_prefill_causal_mlstm(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(forget), _ptr(input_gate),
+                                       B, H, T, dk, dv, int(chunk), _ptr(state_S), _ptr(state_z), int(mode),
+                                       _ptr(out), _DT[out.dtype], _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("la_prefill_causal_mlstm", st)
+    return out
+
+
+def la_decode_step_mlstm(q, k, v, state_S, state_z, forget=None, input_gate=None, out=None,
+                         out_dtype=None, stream=None):
+    """One mLSTM decode step (``forget``, ``input_gate``: [B,H] fp32 or None);
+    the state is updated in place."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=out_dtype, device=q.device)
+    st = lib().la_decode_step_mlstm(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(forget), _ptr(input_gate),
+                                    B, H, dk, dv, _ptr(state_S), _ptr(state_z), _ptr(out), _DT[out.dtype],
+                                    _stream(stream))
+    _check("la_decode_step_mlstm", st)
     return out
 
 

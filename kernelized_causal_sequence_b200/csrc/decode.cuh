@@ -3,7 +3,8 @@
 // scalar decay and, for the gated form, a gain b on the new term — the RFA
 // gate is a = g, b = 1 - g):
 //                 S <- a S + b phi(k) v^T,  z <- a z + b phi(k),
-//                 out = phi(q)^T S / (phi(q)^T z + eps).
+//                 out = phi(q)^T S / (phi(q)^T z + eps);
+// the mLSTM read-out takes phi = identity and divides by max(|q^T z|, 1).
 //
 // Memory-bound: each head's fp32 state (d_k x d_v + d_k) is read once and
 // written once; q, k, v and out are a few hundred bytes.  One CTA per head;
@@ -20,8 +21,8 @@ constexpr int kDecodeThreads = 256;
 template <typename InT, typename OutT, int D>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k, const InT *__restrict__ v,
-                   const float *__restrict__ decay, const float *__restrict__ gain, float eps,
-                   float *__restrict__ S,
+                   const float *__restrict__ decay, const float *__restrict__ gain, int mlstm,
+                   float eps, float *__restrict__ S,
                    float *__restrict__ z, OutT *__restrict__ out) {
     constexpr int CG = D / 4;                     // float4 column groups per row
     constexpr int RSTEP = kDecodeThreads / CG;    // rows handled concurrently
@@ -32,8 +33,9 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k, const I
     const float a = decay ? decay[bh] : 1.f;
     const float b = gain ? gain[bh] : 1.f;
     if (tid < D) {
-        fk[tid] = b * phi_fast(to_f32(k[(size_t)bh * D + tid]));
-        fq[tid] = phi_fast(to_f32(q[(size_t)bh * D + tid]));
+        const float kx = to_f32(k[(size_t)bh * D + tid]), qx = to_f32(q[(size_t)bh * D + tid]);
+        fk[tid] = b * (mlstm ? kx : phi_fast(kx));
+        fq[tid] = mlstm ? qx : phi_fast(qx);
     }
     const int cg = tid % CG, r0 = tid / CG;
     float4 vv;
@@ -79,7 +81,7 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k, const I
         }
         float den = 0.f;
         for (int w = 0; w < kDecodeThreads / 32; ++w) den += den_part[w];
-        den += eps;
+        den = mlstm ? fmaxf(fabsf(den), 1.f) : den + eps;
         OutT *o = out + (size_t)bh * D + tid * 4;
         o[0] = from_f32<OutT>(t.x / den);
         o[1] = from_f32<OutT>(t.y / den);

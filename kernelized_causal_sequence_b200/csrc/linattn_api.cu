@@ -204,9 +204,9 @@ template <typename IT, typename OT, int D> struct SimtNoncausalF {
 };
 template <typename IT, typename OT, int D> struct DecodeF {
     static la_status run(const void *q, const void *k, const void *v, const float *decay, const float *gain,
-                         float eps, float *S, float *z, void *out, long BH, cudaStream_t st) {
+                         int mlstm, float eps, float *S, float *z, void *out, long BH, cudaStream_t st) {
         decode_step_kernel<IT, OT, D><<<(unsigned)BH, kDecodeThreads, 0, st>>>(
-            (const IT *)q, (const IT *)k, (const IT *)v, decay, gain, eps, S, z, (OT *)out);
+            (const IT *)q, (const IT *)k, (const IT *)v, decay, gain, mlstm, eps, S, z, (OT *)out);
         count_launches(1);
         return cuda_check("decode_step launch", cudaGetLastError());
     }
@@ -231,9 +231,10 @@ la_status check_state(la_state_mode mode, const float *S, const float *z) {
 }
 
 // The causal prefill behind every prefill entry point: decay and gain are
-// optional per-token [BH, T] arrays, events optional (4 cudaEvent_t).
+// optional per-token [BH, T] arrays, mlstm selects the identity feature map
+// and the max(|den|, 1) read-out, events optional (4 cudaEvent_t).
 la_status prefill_impl(const void *q, const void *k, const void *v, la_dtype in_dtype, const float *decay,
-                       const float *gain, int B, int H, int T, int d_k, int d_v, float eps, int chunk,
+                       const float *gain, int mlstm, int B, int H, int T, int d_k, int d_v, float eps, int chunk,
                        float *state_S, float *state_z, la_state_mode mode, void *out, la_dtype out_dtype,
                        void *workspace, size_t workspace_bytes, void *stream, void *const *events) {
     la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
@@ -265,7 +266,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, la_dtype in_
 
     if (tc_supported(in_dtype, d_k, chunk, decay != nullptr)) {
         TcCausalArgs a;
-        a.q = q; a.k = k; a.v = v; a.decay = decay; a.gain = gain; a.out = out;
+        a.q = q; a.k = k; a.v = v; a.decay = decay; a.gain = gain; a.mlstm = mlstm; a.out = out;
         a.in_dtype = in_dtype; a.out_dtype = out_dtype;
         a.ws_state = (float *)(ws + wl.state_off);
         a.ws_A = (float *)(ws + wl.A_off);
@@ -278,7 +279,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, la_dtype in_
     }
     SimtParams p;
     std::memset(&p, 0, sizeof(p));
-    p.q = q; p.k = k; p.v = v; p.decay = decay; p.gain = gain; p.out = out;
+    p.q = q; p.k = k; p.v = v; p.decay = decay; p.gain = gain; p.mlstm = mlstm; p.out = out;
     p.ws_state = (float *)(ws + wl.state_off);
     p.ws_A = (float *)(ws + wl.A_off);
     p.ws_total = nullptr;
@@ -287,6 +288,25 @@ la_status prefill_impl(const void *q, const void *k, const void *v, la_dtype in_
     p.eps = eps;
     p.events = events;
     return dispatch3<SimtCausalF>(in_dtype, out_dtype, d_k, p, st);
+}
+
+// Every decode entry point: gain optional, mlstm as for the prefill.
+la_status decode_impl(const void *q, const void *k, const void *v, la_dtype in_dtype, const float *decay,
+                      const float *gain, int mlstm, int B, int H, int d_k, int d_v, float eps, float *state_S,
+                      float *state_z, void *out, la_dtype out_dtype, void *stream) {
+    la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
+    if (s != LA_OK) return s;
+    if (B < 0 || H < 0) return LA_ERR_INVALID_ARG;
+    const long BH = (long)B * H;
+    if (BH == 0) return LA_OK;
+    if (!q || !k || !v || !out || !state_S || !state_z) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(state_S) || !aligned16(state_z) || (decay && !aligned16(decay)) ||
+        (gain && !aligned16(gain)))
+        return LA_ERR_INVALID_ARG;
+    if (BH > 0x7fffffffL) return LA_ERR_UNSUPPORTED;
+    return dispatch3<DecodeF>(in_dtype, out_dtype, d_k, q, k, v, decay, gain, mlstm, eps, state_S, state_z,
+                              out, BH, (cudaStream_t)stream);
 }
 
 }  // namespace
@@ -353,7 +373,7 @@ la_status la_prefill_causal_ev(const void *q, const void *k, const void *v, la_d
                                int chunk, float *state_S, float *state_z, la_state_mode mode,
                                void *out, la_dtype out_dtype, void *workspace,
                                size_t workspace_bytes, void *stream, void *const *events) {
-    return prefill_impl(q, k, v, in_dtype, decay, nullptr, B, H, T, d_k, d_v, eps, chunk, state_S, state_z,
+    return prefill_impl(q, k, v, in_dtype, decay, nullptr, 0, B, H, T, d_k, d_v, eps, chunk, state_S, state_z,
                         mode, out, out_dtype, workspace, workspace_bytes, stream, events);
 }
 
@@ -362,8 +382,17 @@ la_status la_prefill_causal_gated(const void *q, const void *k, const void *v, l
                                   int d_v, float eps, int chunk, float *state_S, float *state_z,
                                   la_state_mode mode, void *out, la_dtype out_dtype, void *workspace,
                                   size_t workspace_bytes, void *stream) {
-    return prefill_impl(q, k, v, in_dtype, decay, gain, B, H, T, d_k, d_v, eps, chunk, state_S, state_z,
+    return prefill_impl(q, k, v, in_dtype, decay, gain, 0, B, H, T, d_k, d_v, eps, chunk, state_S, state_z,
                         mode, out, out_dtype, workspace, workspace_bytes, stream, nullptr);
+}
+
+la_status la_prefill_causal_mlstm(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                                  const float *forget, const float *input_gate, int B, int H, int T,
+                                  int d_k, int d_v, int chunk, float *state_S, float *state_z,
+                                  la_state_mode mode, void *out, la_dtype out_dtype, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+    return prefill_impl(q, k, v, in_dtype, forget, input_gate, 1, B, H, T, d_k, d_v, 0.f, chunk, state_S,
+                        state_z, mode, out, out_dtype, workspace, workspace_bytes, stream, nullptr);
 }
 
 la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_dtype in_dtype,
@@ -416,27 +445,24 @@ la_status la_decode_step_gated(const void *q, const void *k, const void *v, la_d
                                const float *decay, const float *gain, int B, int H, int d_k, int d_v,
                                float eps, float *state_S, float *state_z, void *out, la_dtype out_dtype,
                                void *stream) {
-    la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
-    if (s != LA_OK) return s;
-    if (B < 0 || H < 0) return LA_ERR_INVALID_ARG;
-    const long BH = (long)B * H;
-    if (BH == 0) return LA_OK;
-    if (!q || !k || !v || !out || !state_S || !state_z) return LA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-        !aligned16(state_S) || !aligned16(state_z) || (decay && !aligned16(decay)) ||
-        (gain && !aligned16(gain)))
-        return LA_ERR_INVALID_ARG;
-    if (BH > 0x7fffffffL) return LA_ERR_UNSUPPORTED;
-    return dispatch3<DecodeF>(in_dtype, out_dtype, d_k, q, k, v, decay, gain, eps, state_S, state_z, out,
-                              BH, (cudaStream_t)stream);
+    return decode_impl(q, k, v, in_dtype, decay, gain, 0, B, H, d_k, d_v, eps, state_S, state_z, out, out_dtype,
+                       stream);
+}
+
+la_status la_decode_step_mlstm(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                               const float *forget, const float *input_gate, int B, int H, int d_k,
+                               int d_v, float *state_S, float *state_z, void *out, la_dtype out_dtype,
+                               void *stream) {
+    return decode_impl(q, k, v, in_dtype, forget, input_gate, 1, B, H, d_k, d_v, 0.f, state_S, state_z, out,
+                       out_dtype, stream);
 }
 
 la_status la_decode_step(const void *q, const void *k, const void *v, la_dtype in_dtype,
                          const float *decay, int B, int H, int d_k, int d_v, float eps,
                          float *state_S, float *state_z, void *out, la_dtype out_dtype,
                          void *stream) {
-    return la_decode_step_gated(q, k, v, in_dtype, decay, nullptr, B, H, d_k, d_v, eps, state_S, state_z, out,
-                                out_dtype, stream);
+    return decode_impl(q, k, v, in_dtype, decay, nullptr, 0, B, H, d_k, d_v, eps, state_S, state_z, out,
+                       out_dtype, stream);
 }
 
 }  // extern "C"

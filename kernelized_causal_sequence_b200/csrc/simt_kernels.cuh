@@ -27,6 +27,7 @@ struct SimtParams {
     const void *q, *k, *v;
     const float *decay;     // [BH, T] or nullptr
     const float *gain;      // [BH, T] or nullptr: gain b_t on token t's new term (causal only)
+    int mlstm;              // causal only: identity feature map, read-out / max(|den|, 1)
     void *out;
     float *ws_state;        // [BH, n_seg, D*D + D]
     float *ws_A;            // [BH, n_seg]
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_segment_state_kernel(SimtPa
                     const int idx = tid + u * kSimtThreads, j = idx / D;
                     float f = 0.f;
                     if (j0 + j < n) {
-                        f = phi_precise(kx[u]);
+                        f = p.mlstm ? kx[u] : phi_precise(kx[u]);
                         if (A) f *= expf(Lend - Lc[j0 + j]);
                         if (Gk) f *= Gk[c0 + j0 + j];
                     }
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
 #pragma unroll
                 for (int u = 0; u < simt_per_thread(D); ++u) {
                     const int idx = tid + u * kSimtThreads, j = idx / D, a = idx % D;
-                    fq[j * RS + a] = (q0 + j < n) ? phi_precise(qx[u]) : 0.f;
+                    fq[j * RS + a] = (q0 + j < n) ? (p.mlstm ? qx[u] : phi_precise(qx[u])) : 0.f;
                 }
             }
             __syncthreads();
@@ -241,7 +242,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
 #pragma unroll
                     for (int u = 0; u < simt_per_thread(D); ++u) {
                         const int idx = tid + u * kSimtThreads, j = idx / D, a = idx % D;
-                        fk[j * RS + a] = (k0 + j < n) ? phi_precise(kx[u]) * (Gk ? Gk[c0 + k0 + j] : 1.f) : 0.f;
+                        fk[j * RS + a] =
+                            (k0 + j < n) ? (p.mlstm ? kx[u] : phi_precise(kx[u])) * (Gk ? Gk[c0 + k0 + j] : 1.f) : 0.f;
                         vv[idx] = vx[u];
                     }
                 }
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
                 __syncthreads();
             }
             if (il < n) {
-                const float dn = den + p.eps;
+                const float dn = p.mlstm ? fmaxf(fabsf(den), 1.f) : den + p.eps;
                 OutT *o = O + (size_t)(c0 + il) * D + cg * CPT;
 #pragma unroll
                 for (int c = 0; c < CPT; ++c) o[c] = from_f32<OutT>(acc[c] / dn);
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_output_kernel(SimtPar
                     const int idx = tid + u * kSimtThreads, j = idx / D, a = idx % D;
                     float f = 0.f;
                     if (k0 + j < n) {
-                        f = phi_precise(kx[u]);
+                        f = p.mlstm ? kx[u] : phi_precise(kx[u]);
                         if (A) f *= expf(Lend - Lc[k0 + j]);
                         if (Gk) f *= Gk[c0 + k0 + j];
                     }

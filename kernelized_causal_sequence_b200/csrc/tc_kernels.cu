@@ -84,6 +84,7 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
     tc::TcParams p;
     p.decay = a.decay;
     p.gain = a.gain;
+    p.mlstm = a.mlstm;
     p.out = a.out;
     p.ws_state = a.ws_state;
     p.ws_A = a.ws_A;
@@ -133,9 +134,9 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
 
 template <typename InT, typename OutT>
 la_status dispatch_cd(const TcCausalArgs &a, cudaStream_t st) {
-    // a gain runs the decay kernels (its weights share the decay's log2 form;
-    // without decay a = 1)
-    const bool dec = a.decay != nullptr || a.gain != nullptr;
+    // a gain or the mLSTM form runs the decay kernels (the gain's weights share
+    // the decay's log2 form; without decay a = 1)
+    const bool dec = a.decay != nullptr || a.gain != nullptr || a.mlstm;
     if (a.D == 128) {
         if (a.chunk == 128)
             return dec ? run_causal<128, 128, true, InT, OutT>(a, st) : run_causal<128, 128, false, InT, OutT>(a, st);

@@ -10,6 +10,7 @@ struct TcCausalArgs {
     const void *q, *k, *v;
     const float *decay;
     const float *gain;     // per-token gain on the new term, or null
+    int mlstm;             // identity feature map, max(|den|, 1) read-out
     void *out;
     la_dtype in_dtype, out_dtype;
     float *ws_state, *ws_A;

@@ -134,6 +134,7 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
 struct TcParams {
     const float *decay;   // [BH, T] or null
     const float *gain;    // [BH, T] or null: per-token gain b_t >= 0 on the new term
+    int mlstm;            // 1: identity feature map and the max(|den|, 1) read-out (decay kernels only)
     void *out;            // [BH, T, D]
     float *ws_state;      // [BH, n_seg, D*D + D]
     float *ws_A;          // [BH, n_seg]
@@ -191,6 +192,19 @@ __device__ __noinline__ void write_final_state(uint32_t t_s, uint32_t t_z, float
         }
     }
     if (row_ok) z[a_row] = __uint_as_float(zbits);
+}
+
+// z (row a of the normaliser) as the B operand of MMAd, K-major without
+// swizzle, [16][D] bf16: row n = 0 holds bf16(z).  The decay kernels (which
+// also serve the gated and mLSTM forms) add row n = 1 = bf16(z - bf16(z)), so
+// column 0 + column 1 of the product is phi(q).z to about 16 mantissa bits:
+// with the identity feature map q.z can cancel, and one bf16 rounding of z
+// would be amplified by it.  Element (n, a) sits at (a / 8) * 64 + 8 n + a % 8.
+template <bool HILO>
+__device__ __forceinline__ void write_z_operand(bf16 *zb, int a, float z) {
+    const bf16 hi = __float2bfloat16_rn(z);
+    zb[(a / 8) * 64 + (a % 8)] = hi;
+    if constexpr (HILO) zb[(a / 8) * 64 + 8 + (a % 8)] = __float2bfloat16_rn(z - __bfloat162float(hi));
 }
 
 // Unpack 8 input elements (one 16-byte chunk) to fp32.
@@ -263,8 +277,11 @@ __device__ __forceinline__ void write_state_row(uint8_t *sbf, int a, int col0, c
 // all its rows, and all loads of a batch are issued before any arithmetic.
 // The tile's rows are split into NPART equal parts; this call does parts
 // [PB, PE) (the two warpgroups of the state-only pass each take half).
+// With ident the feature map is the identity (the mLSTM read-out): rows are
+// only weighted, zeroed past n and converted to bf16.
 template <typename InT, int C, int D, bool WEIGHT, bool CONVERT_V, int PB = 0, int PE = 1, int NPART = 1>
-__device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *vt, int tw, int n, const float *L, float Lend) {
+__device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *vt, int tw, int n, const float *L, float Lend,
+                                         bool ident = false) {
     constexpr int KB = D / 64, BOXB = C * 128;
     constexpr int PH = 128 / (8 * KB);
     constexpr int NIT = C / PH;
@@ -286,7 +303,7 @@ __device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *vt, int tw, int
             const uint32_t off = base + (i0 + i) * PH * 128;
             const bool valid = r < n;
             if constexpr (std::is_same<InT, bf16>::value) {
-                uint4 f = phi_bf16x8(raw[i]);
+                uint4 f = ident ? raw[i] : phi_bf16x8(raw[i]);
                 if (!valid) f = make_uint4(0u, 0u, 0u, 0u);
                 if constexpr (WEIGHT) {
                     const float w = valid ? ex2_approx(Lend - L[r]) : 0.f;
@@ -300,7 +317,7 @@ __device__ __forceinline__ void phi_tile(uint8_t *tile, uint8_t *vt, int tw, int
                 unpack8<InT>(raw[i], x);
                 const float w = WEIGHT ? (valid ? ex2_approx(Lend - L[r]) : 0.f) : 1.f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = valid ? phi_fast(x[e]) * w : 0.f;
+                for (int e = 0; e < 8; ++e) x[e] = valid ? (ident ? x[e] : phi_fast(x[e])) * w : 0.f;
                 *reinterpret_cast<uint4 *>(tile + off) = pack8_bf16(x);
             }
         }
@@ -450,9 +467,9 @@ __device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm
     // output mode: plain phi(K) (MMA1 needs it; the decay weights are applied
     // in place after MMA1, see k_weight); state-only: w o phi(K) directly
     if constexpr (G::OUT)
-        phi_tile<InT, C, D, false, CONV, 0, 1, 1>(kt, kt + G::TILE, tk, n, Lk, Lend);
+        phi_tile<InT, C, D, false, CONV, 0, 1, 1>(kt, kt + G::TILE, tk, n, Lk, Lend, DECAY && p.mlstm);
     else
-        phi_tile<InT, C, D, DECAY, CONV, 0, 2, 4>(kt, kt + G::TILE, tk, n, Lk, Lend);
+        phi_tile<InT, C, D, DECAY, CONV, 0, 2, 4>(kt, kt + G::TILE, tk, n, Lk, Lend, DECAY && p.mlstm);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
@@ -468,7 +485,7 @@ __device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm
 // or in place in shared memory (chunk 64).  Arrives on phi_done.
 template <int C, int D, bool DECAY, int MODE, typename InT>
 __device__ __forceinline__ bool q_stage(uint8_t *smem, uint64_t *bar, const AbortCtx ab, uint32_t tmem,
-                                        int c, int tw) {
+                                        int c, int tw, bool ident) {
     using G = Cfg<C, D, DECAY, MODE>;
     const int lane = tw & 31, q = (kPhiWarp0 + (tw >> 5)) & 3;
     const int s = c % G::NKV;
@@ -489,7 +506,7 @@ __device__ __forceinline__ bool q_stage(uint8_t *smem, uint64_t *bar, const Abor
 #pragma unroll
             for (int lc = 0; lc < 8; ++lc) {
                 if constexpr (std::is_same<InT, bf16>::value) {
-                    const uint4 f = phi_bf16x8(raw[lc]);
+                    const uint4 f = ident ? raw[lc] : phi_bf16x8(raw[lc]);
                     packed[lc * 4 + 0] = f.x;
                     packed[lc * 4 + 1] = f.y;
                     packed[lc * 4 + 2] = f.z;
@@ -499,7 +516,8 @@ __device__ __forceinline__ bool q_stage(uint8_t *smem, uint64_t *bar, const Abor
                     unpack8<InT>(raw[lc], x);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        packed[lc * 4 + e] = pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
+                        packed[lc * 4 + e] = ident ? pack_bf16x2(x[2 * e], x[2 * e + 1])
+                                                   : pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
                 }
             }
             if (b == G::KB - 1) {
@@ -515,7 +533,7 @@ __device__ __forceinline__ bool q_stage(uint8_t *smem, uint64_t *bar, const Abor
         }
         tmem_st_wait();
     } else {
-        phi_tile<InT, C, D, false, false>(qs, nullptr, tw, C, nullptr, 0.f);
+        phi_tile<InT, C, D, false, false>(qs, nullptr, tw, C, nullptr, 0.f, ident);
         fence_proxy_async_smem();
     }
     tc_fence_before();
@@ -597,7 +615,8 @@ __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *ba
         if (!mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 16)) return false;
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
     constexpr bool CONV = !std::is_same<InT, bf16>::value;
-    phi_tile<InT, C, D, DECAY, CONV, 2, 4, 4>(kt, kt + G::TILE, et, n, L, DECAY ? Fsm[G::F_LE + s] : 0.f);
+    phi_tile<InT, C, D, DECAY, CONV, 2, 4, 4>(kt, kt + G::TILE, et, n, L, DECAY ? Fsm[G::F_LE + s] : 0.f,
+                                              DECAY && p.mlstm);
     fence_proxy_async_smem();
     __syncwarp();
     if ((et & 31) == 0) mbar_arrive(&bar[G::B_PHI + s]);
@@ -854,7 +873,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int a_row = q * SROWS + lane;   // state row (feature index)
 
         if constexpr (G::OUT)
-            if (nch > 0) ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, 0, tw);
+            if (nch > 0) ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, 0, tw, DECAY && p.mlstm);
         // ---- segment start: state entering the segment -> TMEM (and operands)
         if (ok && nch > 0) {
             float g0 = 1.f;   // decay of chunk 0 (the state is rescaled before its update)
@@ -885,7 +904,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if (srow_ok) {
                         // z operand: row n = 0 of the [16][D] K-major no-swizzle layout
                         bf16 *zb = reinterpret_cast<bf16 *>(smem + G::OFF_ZB);
-                        zb[(a_row / 8) * 64 + (a_row % 8)] = __float2bfloat16_rn(zin);
+                        write_z_operand<DECAY>(zb, a_row, zin);
                     }
                 }
                 tmem_st_wait();
@@ -948,7 +967,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if (!ok) break;
                 }
                 if (c + 1 < nch) {
-                    ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, c + 1, tw);
+                    ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, c + 1, tw, DECAY && p.mlstm);
                     if (!ok) break;
                 }
                 if (c == nch - 1) {
@@ -990,7 +1009,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 if (srow_ok) {
                     bf16 *zb = reinterpret_cast<bf16 *>(smem + G::OFF_ZB);
-                    zb[(a_row / 8) * 64 + (a_row % 8)] = __float2bfloat16_rn(__uint_as_float(zbits));
+                    write_z_operand<DECAY>(zb, a_row, __uint_as_float(zbits));
                 }
                 if constexpr (DECAY) {
                     tmem_st1(tmem + lane_base + G::T_Z, __float_as_uint(__uint_as_float(zbits) * gnext));
@@ -1095,12 +1114,19 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int bx = g / GPB, gb = g % GPB;
                 float o[32];
                 {
-                    uint32_t u[32], ud = 0u;
-                    if (g == 0) tmem_ld1(tmem + lane_base + G::T_DEN, ud);
+                    uint32_t u[32], ud = 0u, ud_lo = 0u;
+                    if (g == 0) {
+                        tmem_ld1(tmem + lane_base + G::T_DEN, ud);
+                        if constexpr (DECAY) tmem_ld1(tmem + lane_base + G::T_DEN + 1, ud_lo);   // phi(q).z_lo
+                    }
                     tmem_ld32(tmem + lane_base + G::T_O + g * 32, u);
                     tmem_ld_wait();
                     // denominator: (decayed) phi(q).z of the carried state + row sum of P + eps
-                    if (g == 0) inv = 1.f / (__uint_as_float(ud) + rowsum + p.eps);
+                    if (g == 0) {
+                        const float den = (__uint_as_float(ud) + __uint_as_float(ud_lo)) + rowsum;
+                        // mLSTM read-out: divide by max(|den|, 1) (decay kernels only)
+                        inv = (DECAY && p.mlstm) ? 1.f / fmaxf(fabsf(den), 1.f) : 1.f / (den + p.eps);
+                    }
 #pragma unroll
                     for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(u[k]) * inv;
                 }

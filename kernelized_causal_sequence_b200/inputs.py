@@ -35,6 +35,8 @@ class Workload:
     chunk: int = 64
     decay: bool = False
     gated: bool = False   # RFA gate: decay a_t = g_t and gain b_t = 1 - g_t on the new term
+    mlstm: bool = False   # mLSTM read-out: decay = forget gate, plus an input gate (input_gate())
+    k_scale: float = 0.0  # keys' scale when it differs from qk_scale (0: qk_scale)
     eps: float = 1e-6
     Lk: int = 0         # non-causal only
     qk_scale: float = 1.0
@@ -73,6 +75,12 @@ WORKLOADS = {
                                                 8192, 128, "bf16", "bf16", chunk=64, decay=True,
                                                 gated=True, qk_scale=1 / math.sqrt(128),
                                                 v_scale=1 / math.sqrt(128), seed=1006),
+    # the mLSTM read-out at the same shape: q ~ N(0,1), k and v ~ N(0,1)/sqrt(128),
+    # forget gate sigmoid(N(2, 1)), input gate exp(0.5 N(0, 1) - 0.5)
+    "mlstm_bf16_b2h16_t8192_d128": Workload("mlstm_bf16_b2h16_t8192_d128", "causal", 2, 16, 8192, 128,
+                                            "bf16", "bf16", chunk=64, decay=True, mlstm=True,
+                                            qk_scale=1.0, k_scale=1 / math.sqrt(128),
+                                            v_scale=1 / math.sqrt(128), seed=1007),
     # non-causal, LoFTR-coarse shape: B=8, H=8, L=4800, d=32, fp16, V pre-scaled by 1/Lk
     "noncausal_f16_b8h8_l4800_d32": Workload("noncausal_f16_b8h8_l4800_d32", "noncausal", 8, 8,
                                              4800, 32, "f16", "f32", chunk=128, Lk=4800,
@@ -112,7 +120,7 @@ def qkv(w: Workload, seed: int | None = None, T: int | None = None, B: int | Non
     rng = np.random.default_rng(seed)
     shape = (B, H, T, w.d)
     q = _cast(_normals(rng, shape) * np.float32(w.qk_scale), w.dtype)
-    k = _cast(_normals(rng, shape) * np.float32(w.qk_scale), w.dtype)
+    k = _cast(_normals(rng, shape) * np.float32(w.k_scale or w.qk_scale), w.dtype)
     v = _cast(_normals(rng, shape) * np.float32(w.v_scale), w.dtype)
     decay = None
     if w.decay:
@@ -128,6 +136,20 @@ def gate_gain(w: Workload, decay: torch.Tensor | None) -> torch.Tensor | None:
     if not w.gated or decay is None:
         return None
     return torch.from_numpy((np.float32(1.0) - decay.numpy()).astype(np.float32))
+
+
+def input_gate(w: Workload, T: int | None = None, B: int | None = None,
+               H: int | None = None) -> torch.Tensor | None:
+    """The input gate of an mLSTM workload, exp(0.5 x - 0.5) with x ~ N(0, 1)
+    drawn from its own stream (seed + 50), [B,H,T] fp32; else None."""
+    if not w.mlstm:
+        return None
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    T = w.T if T is None else T
+    rng = np.random.default_rng(w.seed + 50)
+    x = _normals(rng, (B, H, T))
+    return torch.from_numpy(np.exp(np.float32(0.5) * x - np.float32(0.5)).astype(np.float32))
 
 
 def cross_kv(w: Workload, Lk: int | None = None, B: int | None = None, H: int | None = None):
