@@ -134,7 +134,6 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
 struct TcParams {
     const float *decay;   // [BH, T] or null
     const float *gain;    // [BH, T] or null: per-token gain b_t >= 0 on the new term
-    int mlstm;            // 1: identity feature map and the max(|den|, 1) read-out (decay kernels only)
     void *out;            // [BH, T, D]
     float *ws_state;      // [BH, n_seg, D*D + D]
     float *ws_A;          // [BH, n_seg]
@@ -143,6 +142,7 @@ struct TcParams {
     int *status;          // status word (0 = ok)
     int T, seg_len, n_seg;
     float eps;
+    int mlstm;            // 1: identity feature map and the max(|den|, 1) read-out (decay kernels only)
 };
 
 template <typename OutT> __device__ __forceinline__ void store_row32(OutT *dst, const float (&o)[32]);
@@ -1123,9 +1123,13 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     tmem_ld_wait();
                     // denominator: (decayed) phi(q).z of the carried state + row sum of P + eps
                     if (g == 0) {
-                        const float den = (__uint_as_float(ud) + __uint_as_float(ud_lo)) + rowsum;
-                        // mLSTM read-out: divide by max(|den|, 1) (decay kernels only)
-                        inv = (DECAY && p.mlstm) ? 1.f / fmaxf(fabsf(den), 1.f) : 1.f / (den + p.eps);
+                        if constexpr (DECAY) {
+                            const float den = (__uint_as_float(ud) + __uint_as_float(ud_lo)) + rowsum;
+                            // mLSTM read-out: divide by max(|den|, 1)
+                            inv = p.mlstm ? 1.f / fmaxf(fabsf(den), 1.f) : 1.f / (den + p.eps);
+                        } else {
+                            inv = 1.f / (__uint_as_float(ud) + rowsum + p.eps);
+                        }
                     }
 #pragma unroll
                     for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(u[k]) * inv;
