@@ -59,7 +59,7 @@ def test_prefill_path_selection(L):
     assert la.la_prefill_path(la.LA_F32, 64, 64, 64) == 0
     assert la.la_prefill_path(la.LA_BF16, 64, 64, 96) == -1
     assert la.la_prefill_path(la.LA_BF16, 48, 48, 64) == -1
-    # 16-bit inputs with d in {64, 128} run on tensor cores, except chunk 128 with decay
+    # 16-bit inputs with d in {64, 128} run on tensor cores, either chunk, with or without decay
     assert la.la_prefill_path(la.LA_BF16, 128, 128, 128) == 1
     assert la.la_prefill_path(la.LA_F16, 64, 64, 64, has_decay=True) == 1
     assert la.la_prefill_path(la.LA_BF16, 128, 128, 128, has_decay=True) == 1
@@ -130,3 +130,46 @@ def test_prefill_plan(L):
     assert n * sl >= 5000 and (n - 1) * sl < 5000 and sl % 64 == 0
     with pytest.raises(la.LinAttnError):
         la.la_prefill_plan(1, 1, 100, 64, 96)
+
+
+def test_gated_and_mlstm_reject_bad_arguments(L):
+    """The gated and mLSTM entry points share the prefill's and the decode
+    step's host checks, and add the alignment of the gain / gate arrays."""
+    E_ARG, E_UNS = la.LA_ERR_INVALID_ARG, la.LA_ERR_UNSUPPORTED
+
+    def gated(gain=P, decay=None, B=1, T=128, dk=64, dv=64, chunk=64, eps=1e-6):
+        return L.la_prefill_causal_gated(P, P, P, la.LA_BF16, decay, gain, B, 2, T, dk, dv, eps, chunk, P, P,
+                                         la.LA_STATE_OUT, P, la.LA_BF16, P, 1 << 30, None)
+
+    def mlstm(forget=None, igate=P, B=1, T=128, dk=64, dv=64, chunk=64):
+        return L.la_prefill_causal_mlstm(P, P, P, la.LA_BF16, forget, igate, B, 2, T, dk, dv, chunk, P, P,
+                                         la.LA_STATE_OUT, P, la.LA_BF16, P, 1 << 30, None)
+
+    assert gated(gain=P_ODD) == E_ARG
+    assert gated(decay=P_ODD) == E_ARG
+    assert gated(B=-1) == E_ARG
+    assert gated(chunk=96) == E_UNS
+    assert gated(dk=64, dv=128) == E_UNS
+    assert gated(eps=-1.0) == E_ARG
+    assert gated(B=0) == la.LA_OK              # nothing to do, nothing launched
+    assert mlstm(igate=P_ODD) == E_ARG
+    assert mlstm(forget=P_ODD) == E_ARG
+    assert mlstm(B=-1) == E_ARG
+    assert mlstm(chunk=32) == E_UNS
+    assert mlstm(dk=48, dv=48) == E_UNS
+    assert mlstm(B=0) == la.LA_OK
+
+    def dec_gated(gain=P, S=P, z=P, B=2):
+        return L.la_decode_step_gated(P, P, P, la.LA_BF16, None, gain, B, 2, 64, 64, 1e-6, S, z, P, la.LA_BF16,
+                                      None)
+
+    def dec_mlstm(igate=P, S=P, z=P, B=2, d=64):
+        return L.la_decode_step_mlstm(P, P, P, la.LA_BF16, None, igate, B, 2, d, d, S, z, P, la.LA_BF16, None)
+
+    assert dec_gated(gain=P_ODD) == E_ARG
+    assert dec_gated(S=None) == E_ARG
+    assert dec_gated(B=0) == la.LA_OK
+    assert dec_mlstm(igate=P_ODD) == E_ARG
+    assert dec_mlstm(z=None) == E_ARG
+    assert dec_mlstm(d=96) == E_UNS
+    assert dec_mlstm(B=0) == la.LA_OK
