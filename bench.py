@@ -197,6 +197,12 @@ def oracle_prefill_sample(w, q, k, v, a, tokens: int, threads: int | None = None
     return w.B * tokens / dt, dt, oracle.max_threads()
 
 
+def oracle_threads(n: int) -> None:
+    """Restore the oracle's thread count after a timed sample."""
+    import oracle
+    oracle.set_threads(n)
+
+
 def run_reference(args, w):
     """--impl reference: the fp64 oracle on the host cores, bounded samples."""
     import torch
@@ -557,6 +563,13 @@ def run_ours(args, w):
         line["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": f"first {tok} of {w.T} tokens of all {w.B * w.H} heads "
                                           f"(the whole prefill when equal), fp64 recurrence, {dt:.1f} s"}
+        # the same oracle on one host core, on a bounded sample (~1/16 of the work)
+        tok1 = max(1, min(w.T, tok // 16))
+        r1, dt1, _ = oracle_prefill_sample(w, q_h, k_h, v_h, a_h, tok1, threads=1)
+        oracle_threads(cores)
+        line["cpu_baseline"]["single_core"] = {
+            "value": r1, "unit": UNIT, "cores": 1,
+            "sample": f"first {tok1} of {w.T} tokens of all {w.B * w.H} heads, fp64 recurrence, {dt1:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
