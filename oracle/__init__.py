@@ -62,6 +62,9 @@ def _load():
         lib.orc_decode_step_form.restype = ctypes.c_int
         lib.orc_decode_step_form.argtypes = [ctypes.c_int, _D, _D, _D, _D, _D, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, ctypes.c_int, ctypes.c_double, _D, _D, _D]
+        lib.orc_flash.restype = ctypes.c_int
+        lib.orc_flash.argtypes = [_D, _D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_long, ctypes.c_int,
+                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, _D, _D]
         lib.orc_max_threads.restype = ctypes.c_int
         lib.orc_set_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -149,3 +152,22 @@ def decode_step(q, k, v, S, z, decay=None, eps=1e-6, gain=None, mlstm=False):
     if rc != 0:
         raise RuntimeError("orc_decode_step failed")
     return out, S, z
+
+
+def flash(q, k, v, chunk, scaled=False):
+    """FLASH chunk form (causal): exact squared-ReLU attention inside each chunk
+    plus a linear term over the earlier chunks' summaries; no feature map, no
+    normaliser.  ``scaled``: the listings' convention (scores and summaries
+    divided by the chunk length) instead of the equations'.  q, k: [B,H,T,dk];
+    v: [B,H,T,dv].  Returns (out [B,H,T,dv], S [B,H,dk,dv] = all summaries)."""
+    q, k, v = map(_f64, (q, k, v))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    out = np.zeros((B, H, T, dv))
+    S = np.zeros((B, H, dk, dv))
+    rc = _load().orc_flash(_ptr(q), _ptr(k), _ptr(v), B, H, T, dk, dv, int(chunk), int(bool(scaled)),
+                           _ptr(out), _ptr(S))
+    if rc != 0:
+        raise RuntimeError("orc_flash failed")
+    return out, S
+

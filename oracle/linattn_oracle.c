@@ -284,3 +284,75 @@ int orc_decode_step(const double *q, const double *k, const double *v, const dou
 {
     return orc_decode_step_form(0, q, k, v, decay, NULL, B, H, dk, dv, eps, S, z, out);
 }
+
+/*
+ * FLASH chunk form, causal (concept card "Linear attention", "Chunked
+ * attention: exact inside blocks, linear across them (FLASH)", and the
+ * closing paragraph of its implementation sketch): the sequence is cut into
+ * non-overlapping chunks of `chunk` tokens; inside a chunk, exact
+ * squared-ReLU attention over the chunk's earlier tokens (j <= t); across
+ * chunks, a linear term read from the summaries of the earlier chunks only,
+ * the summary of chunk g being sum_{j in g} k_j v_j^T, added to the running
+ * sum once the chunk is done.  Softmax-free: no feature map, no normaliser.
+ *   scaled = 0: the equations' form, weight relu(q.k)^2, summaries unscaled;
+ *   scaled = 1: the listings' form, scores divided by the chunk length before
+ *               the squared ReLU and each summary divided by the chunk length
+ *               (the nominal chunk, also for a shorter last chunk).
+ * S_out (or NULL) receives the sum of every chunk's summary.
+ */
+int orc_flash(const double *q, const double *k, const double *v, int B, int H, long T, int dk, int dv,
+              int chunk, int scaled, double *out, double *S_out)
+{
+    if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0 || chunk <= 0) return -1;
+    const long BH = (long)B * H;
+    const double sc = scaled ? (double)chunk : 1.0;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *M = (double *)malloc(sizeof(double) * (size_t)dk * dv);   /* earlier chunks' summaries */
+        double *dM = (double *)malloc(sizeof(double) * (size_t)dk * dv);  /* this chunk's summary */
+        if (!M || !dM) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bh = 0; bh < BH; ++bh) {
+                const double *qh = q + bh * T * dk, *kh = k + bh * T * dk, *vh = v + bh * T * dv;
+                double *oh = out + bh * T * dv;
+                memset(M, 0, sizeof(double) * (size_t)dk * dv);
+                for (long g0 = 0; g0 < T; g0 += chunk) {
+                    const long g1 = g0 + chunk < T ? g0 + chunk : T;
+                    for (long t = g0; t < g1; ++t) {
+                        const double *qt = qh + t * dk;
+                        double *ot = oh + t * dv;
+                        /* linear term: the summaries of the earlier chunks */
+                        for (int c = 0; c < dv; ++c) {
+                            double acc = 0.0;
+                            for (int i = 0; i < dk; ++i) acc += qt[i] * M[i * dv + c];
+                            ot[c] = acc;
+                        }
+                        /* exact squared-ReLU attention inside the chunk */
+                        for (long j = g0; j <= t; ++j) {
+                            double s = 0.0;
+                            for (int i = 0; i < dk; ++i) s += qt[i] * kh[j * dk + i];
+                            s /= sc;
+                            const double r = s > 0.0 ? s : 0.0;
+                            const double w = r * r;
+                            for (int c = 0; c < dv; ++c) ot[c] += w * vh[j * dv + c];
+                        }
+                    }
+                    /* the chunk's summary joins the running sum */
+                    memset(dM, 0, sizeof(double) * (size_t)dk * dv);
+                    for (long j = g0; j < g1; ++j)
+                        for (int i = 0; i < dk; ++i)
+                            for (int c = 0; c < dv; ++c) dM[i * dv + c] += kh[j * dk + i] * vh[j * dv + c];
+                    for (long e = 0; e < (long)dk * dv; ++e) M[e] += dM[e] / sc;
+                }
+                if (S_out) memcpy(S_out + bh * dk * dv, M, sizeof(double) * (size_t)dk * dv);
+            }
+        }
+        free(M); free(dM);
+    }
+    return err ? -1 : 0;
+}
+

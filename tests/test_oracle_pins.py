@@ -463,3 +463,72 @@ def test_mlstm_split_and_decode_handoff(orc):
     o_next, S_next, z_next = orc.causal(q, k, v, f, gain=i, **kw)
     np.testing.assert_allclose(od, o_next[:, :, T], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(Sd, S_next, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------ FLASH chunk form
+# Concept card, "Chunked attention: exact inside blocks, linear across them
+# (FLASH)" and the closing paragraph of its implementation sketch: exact
+# squared-ReLU attention inside each chunk, a linear term over the earlier
+# chunks' summaries, no normaliser; equations vs listings differ by the
+# chunk-length factors, so both are checked.
+
+def _flash_dense(q, k, v, C, scaled):
+    """Token-level form of one head: a T x T weight matrix with
+    relu(q_t.k_j / s)^2 for j <= t in t's chunk and (q_t.k_j) / s for j in an
+    earlier chunk (s = C in the listings' form, 1 in the equations')."""
+    T = q.shape[0]
+    s = float(C) if scaled else 1.0
+    raw = q @ k.T
+    ch = np.arange(T) // C
+    same = (ch[:, None] == ch[None, :]) & (np.arange(T)[None, :] <= np.arange(T)[:, None])
+    earlier = ch[None, :] < ch[:, None]
+    W = np.where(same, np.maximum(raw / s, 0.0) ** 2, 0.0) + np.where(earlier, raw / s, 0.0)
+    return W @ v
+
+
+@pytest.mark.parametrize("seed,T,d,C", [(111, 10, 3, 4), (112, 37, 4, 8), (113, 64, 5, 16)])
+@pytest.mark.parametrize("scaled", [False, True])
+def test_flash_dense_form(orc, seed, T, d, C, scaled):
+    rng = np.random.default_rng(seed)
+    q, k, v = (rng.standard_normal((1, 2, T, d)) for _ in range(3))
+    out, S = orc.flash(q, k, v, C, scaled=scaled)
+    s = float(C) if scaled else 1.0
+    for h in range(2):
+        np.testing.assert_allclose(out[0, h], _flash_dense(q[0, h], k[0, h], v[0, h], C, scaled),
+                                   rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(S[0, h], k[0, h].T @ v[0, h] / s, rtol=1e-11, atol=1e-12)
+
+
+def test_flash_special_chunks(orc):
+    rng = np.random.default_rng(115)
+    T, d = 20, 4
+    q, k, v = (rng.standard_normal((1, 1, T, d)) for _ in range(3))
+    # one chunk covering the sequence: causal squared-ReLU attention (torch's relu)
+    out, _ = orc.flash(q, k, v, T)
+    sc = torch.relu(torch.as_tensor(q[0, 0] @ k[0, 0].T)) ** 2 * torch.tril(torch.ones(T, T, dtype=torch.float64))
+    np.testing.assert_allclose(out[0, 0], (sc @ torch.as_tensor(v[0, 0])).numpy(), rtol=1e-12, atol=1e-12)
+    # chunk 1: linear attention over the earlier tokens plus relu(q_t.k_t)^2 v_t;
+    # both conventions coincide
+    o_eq, _ = orc.flash(q, k, v, 1)
+    o_ls, _ = orc.flash(q, k, v, 1, scaled=True)
+    assert np.array_equal(o_eq, o_ls)
+    raw = q[0, 0] @ k[0, 0].T
+    ref = np.tril(raw, -1) @ v[0, 0] + (np.maximum(np.diag(raw), 0) ** 2)[:, None] * v[0, 0]
+    np.testing.assert_allclose(o_eq[0, 0], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_flash_causal_and_linear_in_v(orc):
+    rng = np.random.default_rng(117)
+    T, d, C = 30, 4, 8
+    q, k, v = (rng.standard_normal((1, 1, T, d)) for _ in range(3))
+    out, _ = orc.flash(q, k, v, C, scaled=True)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[..., 17:, :] += 1.0
+    k2[..., 17:, :] -= 2.0
+    v2[..., 17:, :] *= 3.0
+    out2, _ = orc.flash(q2, k2, v2, C, scaled=True)
+    assert np.array_equal(out[..., :17, :], out2[..., :17, :])
+    v3 = rng.standard_normal(v.shape)
+    o3, _ = orc.flash(q, k, v3, C, scaled=True)
+    o4, _ = orc.flash(q, k, 2.0 * v - v3, C, scaled=True)
+    np.testing.assert_allclose(o4, 2.0 * out - o3, rtol=1e-11, atol=1e-12)
