@@ -23,6 +23,16 @@
 // 2^(L_i) for MMA2/MMAd, rows of phi(K) by w_j for MMA3/MMAz), so a single
 // accumulator holds the inter and intra terms and no second K tile is needed.
 //
+// The decay instantiations also serve two forms of the concept card:
+// - a per-token gain b_j on the new term (the RFA gate's 1 - g): it folds
+//   into the key-side log weights, Lk_j = L_j - log2 b_j, which the mask,
+//   w o phi(K) and the state pass read in place of L;
+// - the mLSTM read-out (flag mlstm): phi = identity and
+//   out = O / max(|den|, 1).
+// Their z operand of MMAd carries a hi and a lo bf16 row, so that a cancelling
+// q.z keeps about 16 mantissa bits.  The state-only pass covers every segment
+// but a head's last; the output pass of that segment writes the final state.
+//
 // Warp roles (448 threads; at most four warps share a scheduler, which caps
 // registers at 128 per thread):
 //   warps 0-3    epilogue: scores -> P (mask, decay, row sums), output division
