@@ -132,6 +132,17 @@ def test_prefill_plan(L):
         la.la_prefill_plan(1, 1, 100, 64, 96)
 
 
+@pytest.mark.parametrize("B,H,T,d,C", [(1, 1, 1 << 30, 128, 128), (1, 1, (1 << 31) - 1, 128, 64),
+                                       (1024, 64, 1 << 20, 128, 128), (1, 65535, 1 << 16, 128, 64)])
+def test_plan_and_workspace_at_extreme_sizes(L, B, H, T, d, C):
+    """Sizes near the ABI's limits: the plan still covers every token with
+    whole chunks, and the workspace size is computed in 64 bits."""
+    n, sl = la.la_prefill_plan(B, H, T, d, C)
+    assert n >= 1 and sl % C == 0 and n * sl >= T and (n - 1) * sl < T
+    ws = la.la_prefill_workspace_size(B, H, T, d, d, C)
+    assert ws >= 4 * B * H * n * (d * d + d)
+
+
 def test_gated_and_mlstm_reject_bad_arguments(L):
     """The gated and mLSTM entry points share the prefill's and the decode
     step's host checks, and add the alignment of the gain / gate arrays."""
