@@ -20,11 +20,20 @@
  * Conventions common to every entry point
  *   - All tensor pointers are DEVICE pointers to contiguous row-major arrays,
  *     16-byte aligned.  The caller owns every buffer, including the workspace;
- *     the library never allocates device memory and never synchronises.
+ *     the library never allocates device memory and never synchronises
+ *     (except la_workspace_status and la_noalloc_status, which read a status
+ *     word back to the host).
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream).  Every argument error detectable on
  *     the host is reported before anything is launched, and nothing is then
  *     written.  A failed launch returns LA_ERR_CUDA.
+ *   - Every wait inside the tensor-core kernels (on a copy, a tensor-core
+ *     product or another warp of the same block) is bounded (~2 s, see
+ *     la_set_wait_limit_ns).  A wait that runs out ends its block early and
+ *     leaves LA_ERR_TIMEOUT in the call's status word, at the start of the
+ *     workspace; the output and state of that call are then incomplete.  The
+ *     entry point itself has already returned LA_OK by then (calls are
+ *     asynchronous): read the status with la_workspace_status.
  *   - Heads are independent: q, k [B, H, T, d_k], v [B, H, T, d_v],
  *     out [B, H, T, d_v]; state S [B, H, d_k, d_v] and z [B, H, d_k], fp32.
  *   - Supported: d_k == d_v in {32, 64, 128}; in_dtype in {F32, BF16, F16};
@@ -145,6 +154,75 @@ la_status la_prefill_causal_mlstm(const void *q, const void *k, const void *v, l
                                   la_state_mode mode, void *out, la_dtype out_dtype, void *workspace,
                                   size_t workspace_bytes, void *stream);
 
+/*
+ * la_prefill_causal_flash — the FLASH chunk form (concept card "Linear
+ * attention", "Chunked attention: exact inside blocks, linear across them
+ * (FLASH)", and the closing paragraph of its implementation sketch): the
+ * sequence is cut into chunks of `chunk` tokens; inside a chunk, exact
+ * squared-ReLU attention over the chunk's earlier tokens; across chunks, a
+ * linear term read from the summaries of the earlier chunks.  For token t in
+ * chunk g, with s = 1 (scaled = 0: the card's equations) or s = chunk
+ * (scaled = 1: its listings, also for a shorter last chunk):
+ *   out_t = sum_{j <= t, j in g} relu(q_t . k_j / s)^2 v_j
+ *         + q_t^T (sum_{j in chunks before g} k_j v_j^T) / s
+ * No feature map and no normaliser (softmax-free); the chunk is part of the
+ * definition here, not only a blocking choice.  The state is the raw running
+ * sum over every token processed:
+ *   state_S = sum_j k_j v_j^T   [B, H, d_k, d_v],   state_z = sum_j k_j   [B, H, d_k]
+ * (the read-out divides it by s), so a hand-off through the state continues
+ * the same chunking when the earlier part's length is a multiple of `chunk`.
+ * Tensor-core path only: in_dtype BF16 or F16, d_k = d_v in {64, 128},
+ * chunk 64 or 128; otherwise LA_ERR_UNSUPPORTED.  scaled not 0 or 1:
+ * LA_ERR_INVALID_ARG.  The workspace size and every other argument and error
+ * are those of la_prefill_causal.
+ */
+la_status la_prefill_causal_flash(const void *q, const void *k, const void *v, la_dtype in_dtype,
+                                  int B, int H, int T, int d_k, int d_v, int chunk, int scaled,
+                                  float *state_S, float *state_z, la_state_mode mode, void *out,
+                                  la_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
+ * Sequence sharding (one sequence's tokens split over several GPUs, in
+ * order).  The causal recurrence is affine in the state: a shard maps an
+ * entry state X to A X + dX, with
+ *   dS = sum_j w_j b_j phi(k_j) v_j^T,  dz = sum_j w_j b_j phi(k_j),
+ *   A = prod_t a_t over the shard,  w_j = prod_{t > j in the shard} a_t
+ * (concept card "Linear attention", SSD variant: the chunked algorithm's
+ * recurrence between blocks, here between shards).  Each rank summarises
+ * its shard (la_prefill_causal_summary), the ranks exchange the summaries
+ * (an all-gather, done by the caller, e.g. NCCL), each rank folds the
+ * summaries of the shards before its own into its entry state
+ * (la_state_combine), and runs la_prefill_causal on its shard with that
+ * state as LA_STATE_INOUT.
+ *
+ * la_prefill_causal_summary: dS -> sum_S [B, H, d_k, d_v], dz -> sum_z
+ * [B, H, d_k], A -> sum_A [B, H] (fp32, 16-byte aligned, required) for the
+ * elu+1 forms (decay and gain optional, as in la_prefill_causal_gated).
+ * Takes no queries and writes no output; the workspace is
+ * la_prefill_workspace_size(B, H, T, d_k, d_v, chunk) bytes (T == 0 gives
+ * (0, 0, 1) and needs 256 bytes).  Other arguments and errors as
+ * la_prefill_causal.
+ */
+la_status la_prefill_causal_summary(const void *k, const void *v, la_dtype in_dtype, const float *decay,
+                                    const float *gain, int B, int H, int T, int d_k, int d_v, int chunk,
+                                    float *sum_S, float *sum_z, float *sum_A, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+
+/*
+ * la_state_combine: the entry state of shard r of R from the gathered
+ * summaries, X_0 = (S_in, z_in) or zeros (both NULL), X_{i+1} = A_i X_i + dX_i,
+ * written to (S_out, z_out) = X_r.
+ *   S_all [R, B, H, d_k, d_v], z_all [R, B, H, d_k], A_all [R, B, H]: fp32,
+ *   the shards' la_prefill_causal_summary outputs in shard order (may be NULL
+ *   when r == 0).  S_out [B, H, d_k, d_v], z_out [B, H, d_k] must not overlap
+ *   the inputs.  Errors: LA_ERR_INVALID_ARG for r outside [0, R) or missing
+ *   buffers, LA_ERR_UNSUPPORTED for head dims other than 32, 64, 128.
+ */
+la_status la_state_combine(const float *S_all, const float *z_all, const float *A_all, int R, int r, int B,
+                           int H, int d_k, int d_v, const float *S_in, const float *z_in, float *S_out,
+                           float *z_out, void *stream);
+
 /* Bytes of workspace la_prefill_causal needs for these sizes (0 if none). */
 size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chunk);
 
@@ -166,9 +244,12 @@ size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chun
  * allocating library routine).
  *   - Sizes whose la_prefill_workspace_size exceeds LA_NOALLOC_SCRATCH_BYTES
  *     return LA_ERR_UNSUPPORTED before anything is launched.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current and caches it; make that
- *     first call before any stream capture.  LA_ERR_CUDA if the lookup fails.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress,
+ *     which allocates nothing) with the call's device current, so the address
+ *     stays right across a teardown of the primary context.  The first call on
+ *     a device may load the library's device code; make it before any stream
+ *     capture.  LA_ERR_CUDA if the lookup fails.
+ *   - The call's status word is in the array: read it with la_noalloc_status.
  *   - All calls share the one array, which keeps the last call's contents;
  *     nothing in it needs to start at zero (every entry is written before it
  *     is read).  Calls that overlap on the GPU (e.g. on two streams at once)
@@ -232,6 +313,34 @@ la_status la_decode_step_mlstm(const void *q, const void *k, const void *v, la_d
                                const float *forget, const float *input_gate, int B, int H, int d_k,
                                int d_v, float *state_S, float *state_z, void *out, la_dtype out_dtype,
                                void *stream);
+
+/*
+ * Status of the last call that used `workspace` (a workspace passed to
+ * la_prefill_causal*, la_forward_noncausal or la_prefill_causal_noalloc's
+ * array): LA_OK, or LA_ERR_TIMEOUT if a bounded device-side wait of that call
+ * gave up (its output and state are then incomplete).  *waiter (if non-NULL)
+ * receives the id of the first wait that gave up (0 if none), for diagnosis.
+ * Unlike every other entry point this one synchronises `stream`: it copies
+ * the 8-byte status word to the host on `stream` and waits for it.  Call it on
+ * the stream of the call it checks.  LA_ERR_INVALID_ARG for a null or
+ * misaligned workspace, LA_ERR_CUDA if the copy fails.  Each call clears the
+ * status word of its own workspace before launching anything.
+ */
+la_status la_workspace_status(const void *workspace, int *waiter, void *stream);
+
+/* la_workspace_status for la_prefill_causal_noalloc, whose status word lives
+ * in the library's scratch array (this device's copy). */
+la_status la_noalloc_status(int *waiter, void *stream);
+
+/*
+ * Sets the limit, in nanoseconds, of every bounded device-side wait of the
+ * calls launched after it, process-wide, and returns the previous limit.  The
+ * default is 2e9 (2 s).  0 makes every wait that is not already satisfied at
+ * its first poll give up at once: a test of the timeout path, not a setting
+ * for production.  The drain waits through which a block lets its copies and
+ * products in flight complete before it exits keep their own fixed bound.
+ */
+uint64_t la_set_wait_limit_ns(uint64_t ns);
 
 /* Static description of a status code (never NULL). */
 const char *la_status_string(la_status s);

@@ -22,9 +22,10 @@ import torch
 
 __all__ = [
     "LinAttnError", "lib", "la_prefill_causal", "la_forward_noncausal", "la_decode_step",
-    "la_prefill_causal_mlstm", "la_decode_step_mlstm",
+    "la_prefill_causal_mlstm", "la_decode_step_mlstm", "la_prefill_causal_flash",
+    "la_prefill_causal_summary", "la_state_combine",
     "la_prefill_workspace_size", "la_noncausal_workspace_size", "la_status_string",
-    "la_prefill_path", "la_launch_count", "LA_F32", "LA_BF16", "LA_F16", "LA_STATE_NONE", "LA_STATE_OUT",
+    "la_prefill_path", "la_launch_count", "la_workspace_status", "la_set_wait_limit_ns", "LA_F32", "LA_BF16", "LA_F16", "LA_STATE_NONE", "LA_STATE_OUT",
     "LA_STATE_INOUT", "LIB_PATH",
 ]
 
@@ -70,6 +71,14 @@ def lib() -> ctypes.CDLL:
         L.la_prefill_causal_mlstm.restype = _i
         L.la_prefill_causal_mlstm.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                               _vp, _vp, _i, _vp, _i, _vp, _sz, _vp]
+        L.la_prefill_causal_flash.restype = _i
+        L.la_prefill_causal_flash.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _i,
+                                              _vp, _i, _vp, _sz, _vp]
+        L.la_prefill_causal_summary.restype = _i
+        L.la_prefill_causal_summary.argtypes = [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                                                _vp, _sz, _vp]
+        L.la_state_combine.restype = _i
+        L.la_state_combine.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]
         L.la_prefill_workspace_size.restype = _sz
         L.la_prefill_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
         L.la_forward_noncausal.restype = _i
@@ -96,12 +105,35 @@ def lib() -> ctypes.CDLL:
         L.la_launch_count.argtypes = []
         L.la_last_error_string.restype = ctypes.c_char_p
         L.la_last_error_string.argtypes = []
+        L.la_workspace_status.restype = _i
+        L.la_workspace_status.argtypes = [_vp, ctypes.POINTER(_i), _vp]
+        L.la_noalloc_status.restype = _i
+        L.la_noalloc_status.argtypes = [ctypes.POINTER(_i), _vp]
+        L.la_set_wait_limit_ns.restype = ctypes.c_uint64
+        L.la_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = L
     return _lib
 
 
 def la_launch_count() -> int:
     return int(lib().la_launch_count())
+
+
+def la_workspace_status(workspace, stream=None):
+    """(status, waiter) of the last call that used ``workspace``: status is
+    LA_OK or LA_ERR_TIMEOUT (a bounded device-side wait of that call gave up),
+    waiter the id of the first wait that gave up.  Synchronises the stream."""
+    w = ctypes.c_int(0)
+    st = lib().la_workspace_status(_ptr(workspace), ctypes.byref(w), _stream(stream))
+    if st not in (LA_OK, LA_ERR_TIMEOUT):
+        raise LinAttnError("la_workspace_status", st)
+    return st, w.value
+
+
+def la_set_wait_limit_ns(ns: int) -> int:
+    """Limit of every bounded device-side wait of later calls (process-wide);
+    returns the previous limit."""
+    return int(lib().la_set_wait_limit_ns(int(ns)))
 
 
 def la_status_string(status: int) -> str:
@@ -210,6 +242,63 @@ def la_prefill_causal_mlstm(q, k, v, forget=None, input_gate=None, chunk=64, sta
                                        workspace.numel() * workspace.element_size(), _stream(stream))
     _check("la_prefill_causal_mlstm", st)
     return out
+
+
+def la_prefill_causal_flash(q, k, v, chunk=64, scaled=False, state_S=None, state_z=None, mode=None, out=None,
+                            out_dtype=None, workspace=None, stream=None):
+    """The FLASH chunk form: exact relu(q.k / s)^2 attention inside each chunk
+    plus q^T (sum of the earlier chunks' k v^T) / s; s = chunk if ``scaled``
+    (the listings' convention) else 1.  The state is the raw sum of k v^T
+    (and of k) over all tokens.  Returns ``out`` [B,H,T,d_v]."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=out_dtype, device=q.device)
+    if mode is None:
+        mode = LA_STATE_OUT if state_S is not None else LA_STATE_NONE
+    if workspace is None:
+        workspace = _workspace(la_prefill_workspace_size(B, H, T, dk, dv, chunk), q.device)
+    st = lib().la_prefill_causal_flash(_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], B, H, T, dk, dv, int(chunk),
+                                       int(bool(scaled)), _ptr(state_S), _ptr(state_z), int(mode), _ptr(out),
+                                       _DT[out.dtype], _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("la_prefill_causal_flash",
+    "la_prefill_causal_summary", "la_state_combine", st)
+    return out
+
+
+def la_prefill_causal_summary(k, v, decay=None, gain=None, chunk=64, sum_S=None, sum_z=None, sum_A=None,
+                              workspace=None, stream=None):
+    """A shard's summary: (dS [B,H,dk,dv], dz [B,H,dk], A [B,H]) fp32, the
+    shard's contribution to the state from a zero entry state and its decay
+    product (la_prefill_causal_summary)."""
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    dev = k.device
+    sum_S = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if sum_S is None else sum_S
+    sum_z = torch.empty((B, H, dk), dtype=torch.float32, device=dev) if sum_z is None else sum_z
+    sum_A = torch.empty((B, H), dtype=torch.float32, device=dev) if sum_A is None else sum_A
+    if workspace is None:
+        workspace = _workspace(max(256, la_prefill_workspace_size(B, H, max(T, 1), dk, dv, chunk)), dev)
+    st = lib().la_prefill_causal_summary(_ptr(k), _ptr(v), _DT[k.dtype], _ptr(decay), _ptr(gain), B, H, T, dk, dv,
+                                         int(chunk), _ptr(sum_S), _ptr(sum_z), _ptr(sum_A), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("la_prefill_causal_summary", st)
+    return sum_S, sum_z, sum_A
+
+
+def la_state_combine(S_all, z_all, A_all, r, S_in=None, z_in=None, S_out=None, z_out=None, stream=None):
+    """Entry state of shard r from the gathered summaries [R, B, H, ...]
+    (la_state_combine).  Returns (S_out, z_out)."""
+    R, B, H, dk, dv = S_all.shape
+    dev = S_all.device
+    S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if S_out is None else S_out
+    z_out = torch.empty((B, H, dk), dtype=torch.float32, device=dev) if z_out is None else z_out
+    st = lib().la_state_combine(_ptr(S_all), _ptr(z_all), _ptr(A_all), R, int(r), B, H, dk, dv, _ptr(S_in),
+                                _ptr(z_in), _ptr(S_out), _ptr(z_out), _stream(stream))
+    _check("la_state_combine", st)
+    return S_out, z_out
 
 
 def la_decode_step_mlstm(q, k, v, state_S, state_z, forget=None, input_gate=None, out=None,

@@ -28,21 +28,32 @@ inline bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
 inline bool dtype_ok(la_dtype t) { return t == LA_F32 || t == LA_BF16 || t == LA_F16; }
 
 // Workspace layout of the segment-scan paths:
-//   [ws_state: BH * n_seg * (D*D + D) fp32][ws_A: BH * n_seg fp32]
-//   [ws_total: BH * (D*D + D) fp32, non-causal only][status word, 256 bytes]
+//   [status word: 2 ints, 256 bytes][ws_state: BH * n_seg * (D*D + D) fp32]
+//   [ws_A: BH * n_seg fp32][ws_total: BH * (D*D + D) fp32, non-causal only]
+// The status word sits at offset 0 so that la_workspace_status can read it
+// without knowing the sizes of the call.
 struct WsLayout {
-    size_t state_off, A_off, total_off, status_off, bytes;
+    size_t status_off, state_off, A_off, total_off, bytes;
 };
 
 WsLayout ws_layout(long BH, int n_seg, int D, bool with_total) {
     WsLayout w;
     const size_t E = (size_t)D * D + D;
-    w.state_off = 0;
+    w.status_off = 0;
+    w.state_off = kAlign;
     w.A_off = align_up(w.state_off + sizeof(float) * (size_t)BH * n_seg * E);
     w.total_off = align_up(w.A_off + sizeof(float) * (size_t)BH * n_seg);
-    w.status_off = with_total ? align_up(w.total_off + sizeof(float) * (size_t)BH * E) : w.total_off;
-    w.bytes = w.status_off + kAlign;
+    w.bytes = with_total ? align_up(w.total_off + sizeof(float) * (size_t)BH * E) : w.total_off;
     return w;
+}
+
+// Limit of every bounded device-side wait of the calls that follow
+// (la_set_wait_limit_ns), process-wide.
+std::atomic<unsigned long long> g_wait_ns{2000000000ull};
+
+// Clears the call's status word (2 ints at the start of the workspace).
+la_status clear_status(void *workspace, cudaStream_t st) {
+    return cuda_check("status memset", cudaMemsetAsync(workspace, 0, 2 * sizeof(int), st));
 }
 
 // Per-(kernel, device) opt-in to large dynamic shared memory.
@@ -109,8 +120,9 @@ la_status simt_causal(SimtParams p, cudaStream_t st) {
     if (record_event(p.events, 1, st) != LA_OK) return LA_ERR_CUDA;
     const bool pdl = p.events == nullptr;   // events between the passes serialise them
     if (launch_segment_scan(p.ws_state, p.ws_A, p.BH, p.n_seg, p.n_seg, D, p.mode, p.state_S, p.state_z,
-                            nullptr, st, pdl) != LA_OK)
+                            nullptr, st, pdl, p.sum_A) != LA_OK)
         return LA_ERR_CUDA;
+    if (p.sum_A) return record_event(p.events, 3, st);   // shard summary: no output pass
     if (record_event(p.events, 2, st) != LA_OK) return LA_ERR_CUDA;
     {
         auto k3 = simt_chunk_output_kernel<InT, OutT, D>;
@@ -236,15 +248,29 @@ la_status check_state(la_state_mode mode, const float *S, const float *z) {
 la_status prefill_impl(const void *q, const void *k, const void *v, la_dtype in_dtype, const float *decay,
                        const float *gain, int mlstm, int B, int H, int T, int d_k, int d_v, float eps, int chunk,
                        float *state_S, float *state_z, la_state_mode mode, void *out, la_dtype out_dtype,
-                       void *workspace, size_t workspace_bytes, void *stream, void *const *events) {
+                       void *workspace, size_t workspace_bytes, void *stream, void *const *events,
+                       int flash = 0, float inv_s = 1.f, float *sum_A = nullptr) {
+    // sum_A non-null: the shard summary (state pass + scan, no output pass):
+    // state_S/state_z receive the total contribution, sum_A the decay product
     la_status s = check_common(in_dtype, out_dtype, d_k, d_v, eps);
     if (s != LA_OK) return s;
     if (B < 0 || H < 0 || T < 0) return LA_ERR_INVALID_ARG;
     if (chunk != 64 && chunk != 128) return LA_ERR_UNSUPPORTED;
+    if (flash && !tc_supported(in_dtype, d_k, chunk, false)) return LA_ERR_UNSUPPORTED;
     if ((s = check_state(mode, state_S, state_z)) != LA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
     const long BH = (long)B * H;
     if (BH == 0) return LA_OK;
+    const bool summary = sum_A != nullptr;
+    if (T == 0 && summary) {
+        // nothing to summarise: (0, 0) and a decay product of 1, from the scan over no segments
+        if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < kAlign)
+            return LA_ERR_INVALID_ARG;
+        la_status e = clear_status(workspace, st);
+        if (e != LA_OK) return e;
+        return launch_segment_scan(nullptr, nullptr, BH, 0, 0, d_k, LA_STATE_OUT, state_S, state_z, nullptr, st,
+                                   false, sum_A);
+    }
     if (T == 0) {
         if (mode == LA_STATE_OUT) {
             la_status e = cuda_check("state memset", cudaMemsetAsync(state_S, 0, sizeof(float) * BH * d_k * d_v, st));
@@ -253,8 +279,14 @@ la_status prefill_impl(const void *q, const void *k, const void *v, la_dtype in_
         }
         return LA_OK;
     }
+    if (summary) {   // no queries, no output: the maps of the unused operands point at the keys
+        q = k;
+        out = const_cast<void *>(k);
+        out_dtype = in_dtype;
+    }
     if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    if (summary && !aligned16(sum_A)) return LA_ERR_INVALID_ARG;
     if (decay && !aligned16(decay)) return LA_ERR_INVALID_ARG;
     if (gain && !aligned16(gain)) return LA_ERR_INVALID_ARG;
     if (BH > 65535L) return LA_ERR_UNSUPPORTED;   // heads run along grid y
@@ -263,14 +295,18 @@ la_status prefill_impl(const void *q, const void *k, const void *v, la_dtype in_
     if (!workspace || workspace_bytes < wl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return LA_ERR_INVALID_ARG;
     char *ws = (char *)workspace;
+    if ((s = clear_status(ws, st)) != LA_OK) return s;
 
     if (tc_supported(in_dtype, d_k, chunk, decay != nullptr)) {
         TcCausalArgs a;
         a.q = q; a.k = k; a.v = v; a.decay = decay; a.gain = gain; a.mlstm = mlstm; a.out = out;
+        a.flash = flash; a.inv_s = inv_s;
+        a.summary = summary; a.sum_A = sum_A;
         a.in_dtype = in_dtype; a.out_dtype = out_dtype;
         a.ws_state = (float *)(ws + wl.state_off);
         a.ws_A = (float *)(ws + wl.A_off);
         a.status = (int *)(ws + wl.status_off);
+        a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
         a.state_S = state_S; a.state_z = state_z; a.mode = mode;
         a.BH = BH; a.T = T; a.D = d_k; a.chunk = chunk; a.seg_len = pl.seg_len;
         a.n_seg = pl.n_seg; a.eps = eps;
@@ -287,6 +323,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, la_dtype in_
     p.BH = (int)BH; p.T = T; p.Lq = T; p.chunk = chunk; p.seg_len = pl.seg_len; p.n_seg = pl.n_seg;
     p.eps = eps;
     p.events = events;
+    p.sum_A = sum_A;
     return dispatch3<SimtCausalF>(in_dtype, out_dtype, d_k, p, st);
 }
 
@@ -314,6 +351,19 @@ la_status decode_impl(const void *q, const void *k, const void *v, la_dtype in_d
 extern "C" {
 
 uint64_t la_launch_count(void) { return la::g_launches.load(std::memory_order_relaxed); }
+
+uint64_t la_set_wait_limit_ns(uint64_t ns) { return g_wait_ns.exchange(ns); }
+
+la_status la_workspace_status(const void *workspace, int *waiter, void *stream) {
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA_ERR_INVALID_ARG;
+    int host[2] = {0, 0};
+    cudaStream_t st = (cudaStream_t)stream;
+    la_status e = cuda_check("status read", cudaMemcpyAsync(host, workspace, sizeof(host), cudaMemcpyDeviceToHost, st));
+    if (e == LA_OK) e = cuda_check("status read", cudaStreamSynchronize(st));
+    if (e != LA_OK) return e;
+    if (waiter) *waiter = host[1];
+    return (la_status)host[0];
+}
 
 const char *la_last_error_string(void) { return la::g_last_error; }
 
@@ -354,8 +404,14 @@ size_t la_prefill_workspace_size(int B, int H, int T, int d_k, int d_v, int chun
 size_t la_noncausal_workspace_size(int B, int H, int Lk, int d_k, int d_v) {
     if (B <= 0 || H <= 0 || Lk < 0 || d_k != d_v || !dim_ok(d_k)) return 0;
     const long BH = (long)B * H;
+    // enough for either path (the dtype is not an argument here)
     const Plan pl = make_nc_plan(BH, Lk, d_k);
-    return ws_layout(BH, pl.n_seg, d_k, true).bytes;
+    int n_seg = pl.n_seg;
+    if (d_k == 32) {
+        const Plan pt = make_nc_tc_plan(BH, Lk);
+        if (pt.n_seg > n_seg) n_seg = pt.n_seg;
+    }
+    return ws_layout(BH, n_seg, d_k, true).bytes;
 }
 
 la_status la_prefill_causal(const void *q, const void *k, const void *v, la_dtype in_dtype,
@@ -395,6 +451,39 @@ la_status la_prefill_causal_mlstm(const void *q, const void *k, const void *v, l
                         state_z, mode, out, out_dtype, workspace, workspace_bytes, stream, nullptr);
 }
 
+la_status la_prefill_causal_summary(const void *k, const void *v, la_dtype in_dtype, const float *decay,
+                                    const float *gain, int B, int H, int T, int d_k, int d_v, int chunk,
+                                    float *sum_S, float *sum_z, float *sum_A, void *workspace,
+                                    size_t workspace_bytes, void *stream) {
+    if (!sum_A || !sum_S || !sum_z) return LA_ERR_INVALID_ARG;
+    return prefill_impl(nullptr, k, v, in_dtype, decay, gain, 0, B, H, T, d_k, d_v, 0.f, chunk, sum_S, sum_z,
+                        LA_STATE_OUT, nullptr, in_dtype, workspace, workspace_bytes, stream, nullptr, 0, 1.f,
+                        sum_A);
+}
+
+la_status la_state_combine(const float *S_all, const float *z_all, const float *A_all, int R, int r, int B,
+                           int H, int d_k, int d_v, const float *S_in, const float *z_in, float *S_out,
+                           float *z_out, void *stream) {
+    if (B < 0 || H < 0 || R < 1 || r < 0 || r >= R || d_k <= 0 || d_v <= 0) return LA_ERR_INVALID_ARG;
+    if (d_k != d_v || !dim_ok(d_k)) return LA_ERR_UNSUPPORTED;
+    const long BH = (long)B * H;
+    if (BH == 0) return LA_OK;
+    if (BH > 65535L) return LA_ERR_UNSUPPORTED;
+    if (!S_out || !z_out || (r > 0 && (!S_all || !z_all || !A_all)) || ((S_in == nullptr) != (z_in == nullptr)))
+        return LA_ERR_INVALID_ARG;
+    return launch_state_combine(S_all, z_all, A_all, r, BH, d_k, S_in, z_in, S_out, z_out, (cudaStream_t)stream);
+}
+
+la_status la_prefill_causal_flash(const void *q, const void *k, const void *v, la_dtype in_dtype, int B, int H,
+                                  int T, int d_k, int d_v, int chunk, int scaled, float *state_S, float *state_z,
+                                  la_state_mode mode, void *out, la_dtype out_dtype, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+    if (scaled != 0 && scaled != 1) return LA_ERR_INVALID_ARG;
+    const float inv_s = scaled ? 1.f / (float)chunk : 1.f;   // chunk is 64 or 128: exact
+    return prefill_impl(q, k, v, in_dtype, nullptr, nullptr, 0, B, H, T, d_k, d_v, 0.f, chunk, state_S, state_z,
+                        mode, out, out_dtype, workspace, workspace_bytes, stream, nullptr, 1, inv_s);
+}
+
 la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_dtype in_dtype,
                                const float *decay, int B, int H, int Lq, int Lk, int d_k, int d_v,
                                float eps, float *state_S, float *state_z, la_state_mode mode,
@@ -411,19 +500,23 @@ la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_d
     if (Lq > 0 && (!q || !out || !aligned16(q) || !aligned16(out))) return LA_ERR_INVALID_ARG;
     if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return LA_ERR_INVALID_ARG;
     if (BH > 65535L) return LA_ERR_UNSUPPORTED;   // heads run along grid y
-    const Plan pl = make_nc_plan(BH, Lk, d_k);
+    const bool tc = tc_noncausal_supported(in_dtype, d_k);
+    const Plan pl = tc ? make_nc_tc_plan(BH, Lk) : make_nc_plan(BH, Lk, d_k);
     const WsLayout wl = ws_layout(BH, pl.n_seg, d_k, true);
     if (!workspace || workspace_bytes < wl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return LA_ERR_INVALID_ARG;
     char *ws = (char *)workspace;
+    if ((s = clear_status(ws, st)) != LA_OK) return s;
 
-    if (tc_noncausal_supported(in_dtype, d_k)) {
+    if (tc) {
         TcNoncausalArgs a;
         a.q = q; a.k = k; a.v = v; a.out = out;
         a.in_dtype = in_dtype; a.out_dtype = out_dtype;
         a.ws_state = (float *)(ws + wl.state_off);
         a.ws_A = (float *)(ws + wl.A_off);
         a.ws_total = (float *)(ws + wl.total_off);
+        a.status = (int *)(ws + wl.status_off);
+        a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
         a.state_S = state_S; a.state_z = state_z; a.mode = mode;
         a.BH = BH; a.Lq = Lq; a.Lk = Lk; a.D = d_k; a.seg_len = pl.seg_len; a.n_seg = pl.n_seg;
         a.eps = eps;

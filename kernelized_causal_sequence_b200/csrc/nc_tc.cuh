@@ -1,0 +1,583 @@
+// nc_tc.cuh — tcgen05 tensor-core kernels of the non-causal form at head
+// dimension 32 (16-bit inputs, bf16 tensor-core operands, fp32 accumulation):
+//
+//   S = phi(K)^T V,  z = phi(K)^T 1,  out_i = phi(q_i)^T S / (phi(q_i)^T z + eps)
+//
+// ("Linear Attention" knowledge-base page, section 3, non-causal sketch: the
+// key-value summary is formed once and every query reads it; the linear-
+// attention lesson's developer snippet, step 1, the regrouping
+// (phi(Q) phi(K)^T) V = phi(Q) (phi(K)^T V).)
+//
+// Two kernels, chained by programmatic dependent launch:
+//
+// nc_state_kernel — one CTA per (group of 4 heads, key segment).  The
+//   4 heads' [128 keys x 32] K and V tiles arrive by TMA (64-byte swizzle, one
+//   slab per head); phi(K) is applied in place (rows past the segment zeroed)
+//   and fp16 V converted to bf16 in place.  With the 4 heads' feature columns
+//   stacked along M (MN-major A, the next head's slab one 32-element block
+//   further), one M=128, N=128 MMA per 16 keys accumulates phi(K_g)^T V_h for
+//   every head pair (g, h) of the group; the diagonal 32 x 32 blocks are the
+//   heads' states, the rest is discarded (d = 32 is below the tensor core's
+//   M >= 64, and the extra products are free beside the memory traffic).  A
+//   second MMA against a ones operand gives z.  The CTA writes its partial
+//   (S, z) per head to the workspace.
+//
+// nc_readout_kernel — a persistent pass over 128-query tiles (every CTA a
+//   contiguous range of (head, tile) pairs).  Its set-up and first query
+//   loads overlap the state kernel; before it reads the partial states it
+//   waits for that grid (griddepcontrol.wait).  At each new head the
+//   epilogue warps sum the head's partials in a fixed order (deterministic)
+//   and write S and z as a bf16 hi + lo pair of K-major operands [48][32]
+//   (rows 0-31 the columns of S, row 32 z, the rest 0), so the read-out keeps
+//   about 16 mantissa bits of the state.  Per tile: phi(Q) rows go to TMEM as
+//   the A operand (one thread per query row), four M=128, N=48, K=16 MMAs
+//   form [phi(q) S | phi(q) z] in TMEM, and the epilogue divides, stages the
+//   rows swizzled and stores them by TMA (rows past Lq clipped).
+//
+// Every wait is bounded (tc_ptx.cuh); on expiry the CTA raises the call's
+// status word (LA_ERR_TIMEOUT), drains its copies and products and exits.
+#pragma once
+#include <type_traits>
+
+#include "common.cuh"
+#include "tc_prefill.cuh"
+#include "tc_ptx.cuh"
+
+namespace la {
+namespace nctc {
+
+using namespace la::tc;
+
+constexpr int kD = 32;               // head dimension of these kernels
+constexpr int kHP = 4;               // heads per state CTA: M = 4 x 32 = 128
+constexpr int kRows = 128;           // keys per state tile, queries per read-out tile
+constexpr int kRowBytes = kD * 2;    // one 16-bit row of 32 features
+constexpr int kE = kD * kD + kD;     // floats of one (S, z) state
+
+struct NcStateParams {
+    float *ws_state;                 // [BH][n_seg][kE] partial states
+    float *ws_A;                     // [BH][n_seg] (1: no decay; read by the segment scan)
+    const float *state_in_S;         // [BH][32][32] added to segment 0's partial, or null
+    const float *state_in_z;         // [BH][32]
+    int *status;                     // the call's status word [2]
+    unsigned long long wait_ns;
+    int BH, Lk, seg_len, n_seg;      // seg_len: a multiple of kRows
+};
+
+struct SCfg {
+    static constexpr int HEAD_TILE = kRows * kRowBytes;   // 8 KB: one head's [128][32] tile
+    static constexpr int TILE = kHP * HEAD_TILE;          // 32 KB: the group's 4 slabs
+    static constexpr int STAGE = 2 * TILE;                // K, then V
+    static constexpr int NST = 2;
+    static constexpr int OFF_KV = 0;
+    static constexpr int OFF_ONES = NST * STAGE;          // ones operand [16][128] bf16
+    static constexpr int ONES = 16 * kRows * 2;
+    static constexpr int OFF_BAR = OFF_ONES + ONES;
+    static constexpr int B_FULL = 0, B_EMPTY = NST, B_PHI = 2 * NST, B_DONE = 3 * NST, B_DRAIN = B_DONE + 1;
+    static constexpr int NBAR = B_DRAIN + 1;
+    static constexpr int OFF_TMEMADDR = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_ABORT = OFF_TMEMADDR + 4;
+    static constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;   // + alignment slack
+    static constexpr int T_S = 0, T_Z = 128, TMEM_COLS = 256;
+    static constexpr int THREADS = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 phi and epilogue
+    static_assert(STAGE % 1024 == 0 && OFF_ONES % 16 == 0, "layout");
+};
+
+// phi in place on the [4 heads][128 rows][64 B] K tile (rows >= nvalid zeroed),
+// and the V tile converted to bf16 (fp16 inputs).  Thread tw (0..127) takes
+// the 16-byte chunks u = tw + 128 i: the swizzle only permutes chunks inside
+// a 64-byte row, so chunk u lies in row (u / 4) % 128 whatever its position.
+template <typename InT>
+__device__ __forceinline__ void phi_key_tile(uint8_t *kt, uint8_t *vt, int tw, int nvalid) {
+    constexpr int NCH = SCfg::TILE / 16;        // 2048 chunks
+    constexpr int PER = NCH / 128;              // 16 per thread
+    constexpr int BATCH = 8;
+#pragma unroll 1
+    for (int i0 = 0; i0 < PER; i0 += BATCH) {
+        uint4 raw[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) raw[i] = reinterpret_cast<const uint4 *>(kt)[tw + 128 * (i0 + i)];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            const int u = tw + 128 * (i0 + i);
+            const bool valid = ((u >> 2) & (kRows - 1)) < nvalid;
+            uint4 f;
+            if constexpr (std::is_same<InT, bf16>::value) {
+                f = phi_bf16x8(raw[i]);
+            } else {
+                float x[8];
+                unpack8<InT>(raw[i], x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = phi_fast(x[e]);
+                f = pack8_bf16(x);
+            }
+            if (!valid) f = make_uint4(0u, 0u, 0u, 0u);
+            reinterpret_cast<uint4 *>(kt)[u] = f;
+        }
+        if constexpr (!std::is_same<InT, bf16>::value) {
+            uint4 rv[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) rv[i] = reinterpret_cast<const uint4 *>(vt)[tw + 128 * (i0 + i)];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                float y[8];
+                unpack8<InT>(rv[i], y);
+                reinterpret_cast<uint4 *>(vt)[tw + 128 * (i0 + i)] = pack8_bf16(y);
+            }
+        }
+    }
+}
+
+// grid (n_seg, ceil(BH / 4)), 192 threads.
+template <typename InT>
+__global__ void __launch_bounds__(SCfg::THREADS, 1)
+nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                NcStateParams p) {
+    using G = SCfg;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + G::OFF_BAR);
+    uint32_t *tmem_addr_smem = reinterpret_cast<uint32_t *>(smem + G::OFF_TMEMADDR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + G::OFF_ABORT);
+    const AbortCtx ab{abort_flag, p.status, p.wait_ns};
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int seg = blockIdx.x, grp = blockIdx.y;
+    const long j0 = (long)seg * p.seg_len;
+    const long j1 = min((long)p.Lk, j0 + p.seg_len);
+    const int ntiles = (int)((j1 - j0 + kRows - 1) / kRows);
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < G::NST; ++s) {
+            mbar_init(&bar[G::B_FULL + s], 1);
+            mbar_init(&bar[G::B_EMPTY + s], 1);
+            mbar_init(&bar[G::B_PHI + s], 4);
+        }
+        mbar_init(&bar[G::B_DONE], 1);
+        mbar_init(&bar[G::B_DRAIN], 1);
+        fence_mbar_init();
+    }
+    {
+        uint32_t *ones = reinterpret_cast<uint32_t *>(smem + G::OFF_ONES);
+        for (int i = threadIdx.x; i < G::ONES / 4; i += G::THREADS) ones[i] = 0x3F803F80u;   // bf16 1.0 pairs
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) tmem_alloc(tmem_addr_smem, G::TMEM_COLS);
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_addr_smem;
+    if ((smem_u32(smem) & 1023u) != 0) raise_abort(ab, 99, kStatusLayout);
+    // the read-out kernel may be scheduled now: its set-up and query loads do
+    // not depend on this grid, and it waits for this grid before reading the
+    // partial states
+    pdl_trigger();
+
+    if (warp == 0) {
+        // ================= TMA producer
+        if (lane == 0 && !*abort_flag) {
+            int issued[G::NST] = {};
+            for (int t = 0; t < ntiles; ++t) {
+                const int s = t % G::NST, use = t / G::NST;
+                if (use > 0 && !mbar_wait(&bar[G::B_EMPTY + s], (use - 1) & 1, ab, 1)) break;
+                uint8_t *kd = smem + G::OFF_KV + s * G::STAGE;
+                mbar_expect_tx(&bar[G::B_FULL + s], 2 * G::TILE);
+                const int y = (int)(j0 + (long)t * kRows), z = grp * kHP;
+                tma_load_3d(kd, &tm_k, &bar[G::B_FULL + s], 0, y, z);
+                tma_load_3d(kd + G::TILE, &tm_v, &bar[G::B_FULL + s], 0, y, z);
+                issued[s] = use + 1;
+            }
+            if (*abort_flag) {
+                volatile int never = 0;
+                AbortCtx timed{&never, nullptr, kDrainLimitNs};
+                for (int s = 0; s < G::NST; ++s)
+                    if (issued[s] > 0) mbar_wait(&bar[G::B_FULL + s], (issued[s] - 1) & 1, timed, 0);
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer
+        if (lane == 0 && !*abort_flag) {
+            constexpr uint32_t ID_S = idesc_bf16(128, 128, true, true);
+            constexpr uint32_t ID_Z = idesc_bf16(128, 16, true, false);
+            const uint32_t sb = smem_u32(smem);
+            const uint64_t dOnes = sdesc_nosw(sb + G::OFF_ONES, 128, (kRows / 8) * 128);
+            bool done = true;
+            for (int t = 0; t < ntiles; ++t) {
+                const int s = t % G::NST;
+                if (!mbar_wait(&bar[G::B_PHI + s], (t / G::NST) & 1, ab, 3)) { done = false; break; }
+                tc_fence_after();
+                const uint32_t kt = sb + G::OFF_KV + s * G::STAGE;
+                // MN-major operands: 4 head slabs of 32 columns (lbo = one slab),
+                // 8-row groups 512 bytes apart; 16 keys = 1024 bytes per K step
+                const uint64_t dK = sdesc_sw64(kt, G::HEAD_TILE, 512);
+                const uint64_t dV = sdesc_sw64(kt + G::TILE, G::HEAD_TILE, 512);
+#pragma unroll
+                for (int kk = 0; kk < kRows / 16; ++kk)
+                    mma_ss(tmem + G::T_S, dK + (uint64_t)((kk * 1024) >> 4), dV + (uint64_t)((kk * 1024) >> 4), ID_S,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < kRows / 16; ++kk)
+                    mma_ss(tmem + G::T_Z, dK + (uint64_t)((kk * 1024) >> 4), dOnes + (uint64_t)((kk * 256) >> 4), ID_Z,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&bar[G::B_EMPTY + s]);
+            }
+            if (done) mma_commit(&bar[G::B_DONE]);
+            volatile int never = 0;
+            AbortCtx timed{&never, nullptr, kDrainLimitNs};
+            mma_commit(&bar[G::B_DRAIN]);
+            mbar_wait(&bar[G::B_DRAIN], 0, timed, 0);
+        }
+    } else {
+        // ================= warps 2-5: phi(K), then the partial state out
+        const int tw = threadIdx.x - 64;
+        bool ok = true;
+        for (int t = 0; t < ntiles; ++t) {
+            const int s = t % G::NST;
+            if (!mbar_wait(&bar[G::B_FULL + s], (t / G::NST) & 1, ab, 4)) { ok = false; break; }
+            const long y0 = j0 + (long)t * kRows;
+            const int nvalid = (int)min((long)kRows, j1 - y0);
+            uint8_t *kt = smem + G::OFF_KV + s * G::STAGE;
+            phi_key_tile<InT>(kt, kt + G::TILE, tw, nvalid);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
+        }
+        if (ok && ntiles > 0 && mbar_wait(&bar[G::B_DONE], 0, ab, 5)) {
+            tc_fence_after();
+            // TMEM lane quarter q = head q of the group; lane = feature a
+            const int q = warp & 3, a = lane;
+            const long bh = (long)grp * kHP + q;
+            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+            uint32_t u[32], zb;
+            tmem_ld32(tmem + lane_base + G::T_S + q * 32, u);   // the diagonal block: S_q[a][0..31]
+            tmem_ld1(tmem + lane_base + G::T_Z, zb);
+            tmem_ld_wait();
+            if (bh < p.BH && !*abort_flag) {
+                float *dst = p.ws_state + ((size_t)bh * p.n_seg + seg) * kE;
+                float vals[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) vals[i] = __uint_as_float(u[i]);
+                float zv = __uint_as_float(zb);
+                if (seg == 0 && p.state_in_S) {   // the state-in joins the first segment's partial
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) vals[i] += p.state_in_S[(size_t)bh * kD * kD + a * kD + i];
+                    zv += p.state_in_z[(size_t)bh * kD + a];
+                }
+                float4 *d4 = reinterpret_cast<float4 *>(dst + a * kD);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    d4[i] = make_float4(vals[4 * i], vals[4 * i + 1], vals[4 * i + 2], vals[4 * i + 3]);
+                dst[kD * kD + a] = zv;
+                if (lane == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = 1.f;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, G::TMEM_COLS);
+    }
+}
+
+// --------------------------------------------------------------------------
+struct NcReadParams {
+    const float *ws_state;           // [BH][n_seg][kE] partials (n_seg may be 0)
+    const float *state_in_S;         // used only when n_seg == 0 (no keys): [BH][32][32], or null
+    const float *state_in_z;
+    float *state_out_S;              // the head totals, or null
+    float *state_out_z;
+    int *status;
+    unsigned long long wait_ns;
+    int BH, Lq, n_seg, tiles_per_head;
+    long total_tiles;                // BH * tiles_per_head
+    float eps;
+};
+
+template <typename OutT> struct RCfg {
+    static constexpr int QT = kRows * kRowBytes;            // 8 KB query tile
+    static constexpr int NQ = 6;
+    static constexpr int OFF_Q = 0;
+    static constexpr int STG_WARP = 4096;                   // one warp's 32 output rows (<= 128 B each)
+    static constexpr int OFF_STG = NQ * QT;                 // 2 buffers x 4 warps
+    static constexpr int OFF_B = OFF_STG + 2 * 4 * STG_WARP;
+    static constexpr int BN = 48;                           // B operand rows: 32 of S, 1 of z, 15 zero
+    static constexpr int BOP = BN * kD * 2;                 // 3 KB
+    static constexpr int OFF_BAR = OFF_B + 2 * BOP;         // hi, lo
+    static constexpr int B_QFULL = 0, B_QEMPTY = NQ, B_AFULL = 2 * NQ, B_AEMPTY = B_AFULL + 2,
+                         B_DFULL = B_AEMPTY + 2, B_DEMPTY = B_DFULL + 2, B_BREADY = B_DEMPTY + 2,
+                         B_DRAIN = B_BREADY + 1, NBAR = B_DRAIN + 1;
+    static constexpr int OFF_TMEMADDR = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_ABORT = OFF_TMEMADDR + 4;
+    static constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;
+    static constexpr int T_D0 = 0, T_D1 = 64, T_A0 = 128, T_A1 = 160, TMEM_COLS = 256;
+    static constexpr int THREADS = 320;   // warp 0 TMA, 1 MMA, 2-5 phi(Q), 6-9 epilogue
+    static constexpr int ROWB = kD * (int)sizeof(OutT);     // output row bytes: 128 (fp32) or 64
+    static_assert(OFF_STG % 1024 == 0 && OFF_B % 16 == 0, "layout");
+};
+
+// Byte offset of element (n, k) of a K-major no-swizzle [48][32] operand:
+// core matrices (8 rows x 8 k) of 128 bytes, 4 along K (128 bytes apart),
+// groups of 8 rows 512 bytes apart.
+__device__ __forceinline__ int bop_off(int n, int k) {
+    return (n >> 3) * 512 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
+}
+
+// 16-byte chunk c of output row r in a warp's staging rows, swizzled as the
+// output tensor map (128-byte rows: 128-byte swizzle; 64-byte rows: 64-byte).
+template <int ROWB> __device__ __forceinline__ int stg_off(int r, int c) {
+    if constexpr (ROWB == 128) return r * 128 + ((c ^ (r & 7)) << 4);
+    else return r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+}
+
+// grid (G), 320 threads; CTA b takes the flattened (head, tile) range
+// [b * total / G, (b + 1) * total / G).
+template <typename InT, typename OutT>
+__global__ void __launch_bounds__(RCfg<OutT>::THREADS, 1)
+nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+                  NcReadParams p) {
+    using G = RCfg<OutT>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + G::OFF_BAR);
+    uint32_t *tmem_addr_smem = reinterpret_cast<uint32_t *>(smem + G::OFF_TMEMADDR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + G::OFF_ABORT);
+    const AbortCtx ab{abort_flag, p.status, p.wait_ns};
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long f0 = (long)blockIdx.x * p.total_tiles / gridDim.x;
+    const long f1 = (long)(blockIdx.x + 1) * p.total_tiles / gridDim.x;
+    const int n = (int)(f1 - f0);
+    const int tph = p.tiles_per_head;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < G::NQ; ++s) {
+            mbar_init(&bar[G::B_QFULL + s], 1);
+            mbar_init(&bar[G::B_QEMPTY + s], 4);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[G::B_AFULL + s], 4);
+            mbar_init(&bar[G::B_AEMPTY + s], 1);
+            mbar_init(&bar[G::B_DFULL + s], 1);
+            mbar_init(&bar[G::B_DEMPTY + s], 4);
+        }
+        mbar_init(&bar[G::B_BREADY], 4);
+        mbar_init(&bar[G::B_DRAIN], 1);
+        fence_mbar_init();
+    }
+    {   // B operands start zeroed (rows 33-47 stay zero)
+        uint32_t *b = reinterpret_cast<uint32_t *>(smem + G::OFF_B);
+        for (int i = threadIdx.x; i < 2 * G::BOP / 4; i += G::THREADS) b[i] = 0u;
+    }
+    if (warp == 1) tmem_alloc(tmem_addr_smem, G::TMEM_COLS);
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_o);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_addr_smem;
+    if ((smem_u32(smem) & 1023u) != 0) raise_abort(ab, 99, kStatusLayout);
+
+    if (warp == 0) {
+        // ================= TMA producer: query tiles (independent of the state kernel)
+        if (lane == 0 && !*abort_flag) {
+            int issued[G::NQ] = {};
+            for (int i = 0; i < n; ++i) {
+                const int s = i % G::NQ, use = i / G::NQ;
+                if (use > 0 && !mbar_wait(&bar[G::B_QEMPTY + s], (use - 1) & 1, ab, 1)) break;
+                const long f = f0 + i;
+                const int bh = (int)(f / tph), t = (int)(f % tph);
+                mbar_expect_tx(&bar[G::B_QFULL + s], G::QT);
+                tma_load_3d(smem + G::OFF_Q + s * G::QT, &tm_q, &bar[G::B_QFULL + s], 0, t * kRows, bh);
+                issued[s] = use + 1;
+            }
+            if (*abort_flag) {
+                volatile int never = 0;
+                AbortCtx timed{&never, nullptr, kDrainLimitNs};
+                for (int s = 0; s < G::NQ; ++s)
+                    if (issued[s] > 0) mbar_wait(&bar[G::B_QFULL + s], (issued[s] - 1) & 1, timed, 0);
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer
+        if (lane == 0 && !*abort_flag) {
+            constexpr uint32_t ID = idesc_bf16(128, G::BN, false, false);
+            const uint32_t sb = smem_u32(smem);
+            const uint64_t dBhi = sdesc_nosw(sb + G::OFF_B, 128, 512);
+            const uint64_t dBlo = sdesc_nosw(sb + G::OFF_B + G::BOP, 128, 512);
+            int cur = -1, hc = -1;
+            for (int i = 0; i < n; ++i) {
+                const int a = i & 1;
+                const int bh = (int)((f0 + i) / tph);
+                if (!mbar_wait(&bar[G::B_AFULL + a], (i >> 1) & 1, ab, 2)) break;
+                if (i >= 2 && !mbar_wait(&bar[G::B_DEMPTY + a], ((i >> 1) - 1) & 1, ab, 3)) break;
+                if (bh != cur) {
+                    cur = bh;
+                    ++hc;
+                    if (!mbar_wait(&bar[G::B_BREADY], hc & 1, ab, 4)) break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem + (a ? G::T_D1 : G::T_D0), at = tmem + (a ? G::T_A1 : G::T_A0);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    mma_ts(d, at + kk * 8, dBhi + (uint64_t)((kk * 256) >> 4), ID, kk > 0 ? 1u : 0u);
+                    mma_ts(d, at + kk * 8, dBlo + (uint64_t)((kk * 256) >> 4), ID, 1u);
+                }
+                mma_commit(&bar[G::B_DFULL + a]);
+                mma_commit(&bar[G::B_AEMPTY + a]);
+            }
+            volatile int never = 0;
+            AbortCtx timed{&never, nullptr, kDrainLimitNs};
+            mma_commit(&bar[G::B_DRAIN]);
+            mbar_wait(&bar[G::B_DRAIN], 0, timed, 0);
+        }
+    } else if (warp < 6) {
+        // ================= phi(Q) into TMEM (warps 2-5, one thread per query row)
+        const int q = warp & 3, r = q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        for (int i = 0; i < n; ++i) {
+            const int s = i % G::NQ, a = i & 1;
+            if (!mbar_wait(&bar[G::B_QFULL + s], (i / G::NQ) & 1, ab, 5)) break;
+            const uint8_t *qs = smem + G::OFF_Q + s * G::QT;
+            uint4 raw[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                raw[c] = *reinterpret_cast<const uint4 *>(qs + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[G::B_QEMPTY + s]);
+            uint32_t packed[16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if constexpr (std::is_same<InT, bf16>::value) {
+                    const uint4 f = phi_bf16x8(raw[c]);
+                    packed[4 * c + 0] = f.x;
+                    packed[4 * c + 1] = f.y;
+                    packed[4 * c + 2] = f.z;
+                    packed[4 * c + 3] = f.w;
+                } else {
+                    float x[8];
+                    unpack8<InT>(raw[c], x);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) packed[4 * c + e] = pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
+                }
+            }
+            if (i >= 2 && !mbar_wait(&bar[G::B_AEMPTY + a], ((i >> 1) - 1) & 1, ab, 6)) break;
+            tc_fence_after();
+            tmem_st16(tmem + lane_base + (a ? G::T_A1 : G::T_A0), packed);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[G::B_AFULL + a]);
+        }
+    } else {
+        // ================= epilogue (warps 6-9): head state -> B operands, output
+        const int q = warp & 3, et = threadIdx.x - 192;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        bool waited = false;
+        int cur = -1;
+        for (int i = 0; i < n; ++i) {
+            const int a = i & 1;
+            const long f = f0 + i;
+            const int bh = (int)(f / tph), t = (int)(f % tph);
+            if (bh != cur) {
+                cur = bh;
+                if (!waited) {
+                    pdl_wait();   // the state kernel's partials are complete and visible
+                    waited = true;
+                }
+                // the head's total: sum of its partials in segment order (or the
+                // state-in when there are no keys); the CTA holding the head's
+                // first tile writes it as the state output
+                const bool owner = t == 0 && p.state_out_S != nullptr;
+                uint8_t *bhi = smem + G::OFF_B, *blo = smem + G::OFF_B + G::BOP;
+                for (int e = et; e < kE; e += 128) {
+                    float acc = 0.f;
+                    if (p.n_seg == 0) {
+                        if (p.state_in_S)
+                            acc = e < kD * kD ? p.state_in_S[(size_t)bh * kD * kD + e]
+                                              : p.state_in_z[(size_t)bh * kD + (e - kD * kD)];
+                    } else {
+                        const float *src = p.ws_state + (size_t)bh * p.n_seg * kE + e;
+                        for (int s = 0; s < p.n_seg; ++s) acc += src[(size_t)s * kE];
+                    }
+                    if (owner) {
+                        if (e < kD * kD) p.state_out_S[(size_t)bh * kD * kD + e] = acc;
+                        else p.state_out_z[(size_t)bh * kD + (e - kD * kD)] = acc;
+                    }
+                    // S[k][nn] -> element (nn, k); z[k] -> element (32, k)
+                    const int nn = e < kD * kD ? e % kD : kD;
+                    const int k = e < kD * kD ? e / kD : e - kD * kD;
+                    const bf16 hi = __float2bfloat16_rn(acc);
+                    *reinterpret_cast<bf16 *>(bhi + bop_off(nn, k)) = hi;
+                    *reinterpret_cast<bf16 *>(blo + bop_off(nn, k)) = __float2bfloat16_rn(acc - __bfloat162float(hi));
+                }
+                // each warp's writes are complete and visible to the tensor core
+                // before its arrival; the MMA waits for all four
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[G::B_BREADY]);
+            }
+            if (!mbar_wait(&bar[G::B_DFULL + a], (i >> 1) & 1, ab, 7)) break;
+            tc_fence_after();
+            uint32_t u[32], ud;
+            const uint32_t d = tmem + lane_base + (a ? G::T_D1 : G::T_D0);
+            tmem_ld32(d, u);
+            tmem_ld1(d + kD, ud);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[G::B_DEMPTY + a]);
+            const float inv = 1.f / (__uint_as_float(ud) + p.eps);
+            uint8_t *stg = smem + G::OFF_STG + (a * 4 + (warp - 6)) * G::STG_WARP;
+            // this warp's store of two tiles ago must have read its staging rows
+            if (lane == 0) bulk_wait_read1();
+            __syncwarp();
+            if constexpr (sizeof(OutT) == 4) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<float4 *>(stg + stg_off<128>(lane, c)) =
+                        make_float4(__uint_as_float(u[4 * c]) * inv, __uint_as_float(u[4 * c + 1]) * inv,
+                                    __uint_as_float(u[4 * c + 2]) * inv, __uint_as_float(u[4 * c + 3]) * inv);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(u[8 * c + e]) * inv;
+                    uint4 w;
+                    if constexpr (std::is_same<OutT, bf16>::value) w = pack8_bf16(x);
+                    else
+                        w = make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]), pack_f16x2(x[4], x[5]),
+                                       pack_f16x2(x[6], x[7]));
+                    *reinterpret_cast<uint4 *>(stg + stg_off<64>(lane, c)) = w;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(&tm_o, stg, 0, t * kRows + q * 32, bh);
+                bulk_commit();
+            }
+        }
+        if (lane == 0) bulk_wait0();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, G::TMEM_COLS);
+    }
+}
+
+}  // namespace nctc
+}  // namespace la

@@ -11,10 +11,10 @@
 // The array is a file-scope __device__ variable: every GPU that loads this
 // library holds LA_NOALLOC_SCRATCH_BYTES of it until the process exits.  Host
 // code cannot use the variable's name as a device address (on the host it is
-// only a stand-in symbol), so the device address is looked up once per device
-// with cudaGetSymbolAddress and cached.
-#include <mutex>
-
+// only a stand-in symbol), so each call looks the device address up with
+// cudaGetSymbolAddress, with the call's device current.  The lookup allocates
+// nothing; repeating it on every call keeps the address right if the caller
+// has torn down and recreated the device's primary context in between.
 #include "linattn.h"
 #include <cuda_runtime.h>
 
@@ -22,22 +22,12 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRA
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (set-up on the
-// first call per device).  Returns nullptr on failure.
+// Device address of the scratch array on the current device, or nullptr if
+// the lookup fails.
 void *scratch_for_current_device() {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
-        g_scratch_ptr[dev] = p;
-    }
-    return g_scratch_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    return p;
 }
 
 }  // namespace
@@ -56,4 +46,10 @@ extern "C" la_status la_prefill_causal_noalloc(const void *q, const void *k, con
     return la_prefill_causal(q, k, v, in_dtype, decay, B, H, T, d_k, d_v, eps, chunk, state_S,
                              state_z, mode, out, out_dtype, scratch,
                              (size_t)LA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" la_status la_noalloc_status(int *waiter, void *stream) {
+    void *scratch = scratch_for_current_device();
+    if (!scratch) return LA_ERR_CUDA;
+    return la_workspace_status(scratch, waiter, stream);
 }

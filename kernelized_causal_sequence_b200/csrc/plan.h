@@ -69,6 +69,24 @@ inline Plan make_nc_plan(long BH, long Lk, int D) {
     return p;
 }
 
+// Key segments of the tensor-core non-causal form (head dimension 32): one
+// CTA per (group of 4 heads, segment of whole 128-key tiles), the segment
+// count chosen so that all CTAs fit in one wave on the SMs.
+constexpr int kNcTcHeads = 4;
+inline Plan make_nc_tc_plan(long BH, long Lk) {
+    Plan p;
+    p.chunk = kNc32TileRows;
+    const long groups = (BH + kNcTcHeads - 1) / kNcTcHeads;
+    const long tiles = Lk > 0 ? (Lk + kNc32TileRows - 1) / kNc32TileRows : 1;
+    long segs = kNumSMs / (groups > 0 ? groups : 1);
+    if (segs < 1) segs = 1;
+    if (segs > tiles) segs = tiles;
+    const long per = (tiles + segs - 1) / segs;
+    p.seg_len = (int)(per * kNc32TileRows);
+    p.n_seg = (int)((tiles + per - 1) / per);
+    return p;
+}
+
 // Query tiles per read-out CTA at head dimension 32: one wave of
 // 4 x 148 CTAs over all heads.
 inline int nc32_tiles_per_cta(long BH, long Lq) {

@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, cons
                                                            const float *state_in_S,
                                                            const float *state_in_z,
                                                            float *state_out_S, float *state_out_z,
-                                                           float *total) {
+                                                           float *total, float *total_A) {
     __shared__ float tile[32][33];
     __shared__ float Atile[32];
     pdl_wait();   // the segment states of the state pass
@@ -69,6 +69,11 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(float *ws_state, cons
             if (s < n_seg && e < E) ws[(size_t)s * E + e] = tile[i][lane];
         }
     }
+    if (total_A && blockIdx.x == 0 && threadIdx.x == 0) {   // the head's total decay product
+        float A = 1.f;
+        for (int i = 0; i < n_dx; ++i) A *= Ah[i];
+        total_A[bh] = A;
+    }
     if (lane == 0 && n_dx == n_seg) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, 
                                                                const float *state_in_S,
                                                                const float *state_in_z,
                                                                float *state_out_S, float *state_out_z,
-                                                               float *total) {
+                                                               float *total, float *total_A) {
     __shared__ float Ash[kSeqScanMaxSeg];
     pdl_wait();   // the segment states of the state pass
     const int bh = blockIdx.y;
@@ -120,6 +125,11 @@ __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, 
     }
     if (threadIdx.x < n_dx) Ash[threadIdx.x] = ws_A[(size_t)bh * n_seg + threadIdx.x];
     __syncthreads();
+    if (total_A && blockIdx.x == 0 && threadIdx.x == 0) {   // the head's total decay product
+        float A = 1.f;
+        for (int i = 0; i < n_dx; ++i) A *= Ash[i];
+        total_A[bh] = A;
+    }
     if (!live) return;
 #pragma unroll 1
     for (int s0 = 0; s0 < n_seg; s0 += kSeqScanBatch) {
@@ -148,7 +158,7 @@ __global__ void __launch_bounds__(256) segment_scan_seq_kernel(float *ws_state, 
 
 la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n_seg, int n_dx, int D,
                               int mode, float *state_S, float *state_z, float *total,
-                              cudaStream_t st, bool pdl) {
+                              cudaStream_t st, bool pdl, float *total_A) {
     const int E = D * D + D;
     const float *sin_S = mode == LA_STATE_INOUT ? state_S : nullptr;
     const float *sin_z = mode == LA_STATE_INOUT ? state_z : nullptr;
@@ -168,15 +178,49 @@ la_status launch_segment_scan(float *ws_state, const float *ws_A, long BH, int n
     if (n_seg <= kSeqScanMaxSeg && E % 4 == 0 && D % 4 == 0) {   // float4 groups stay inside S or z
         cfg.gridDim = dim3((E / 4 + 255) / 256, (unsigned)BH);
         err = cudaLaunchKernelEx(&cfg, segment_scan_seq_kernel, ws_state, ws_A, n_seg, n_dx, E, D * D, sin_S, sin_z,
-                                 sout_S, sout_z, total);
+                                 sout_S, sout_z, total, total_A);
     } else {
         cfg.gridDim = dim3((E + 31) / 32, (unsigned)BH);
         err = cudaLaunchKernelEx(&cfg, segment_scan_kernel, ws_state, ws_A, n_seg, n_dx, E, D * D, sin_S, sin_z,
-                                 sout_S, sout_z, total);
+                                 sout_S, sout_z, total, total_A);
     }
     count_launches(1);
     if (err != cudaSuccess) return cuda_fail("segment_scan launch", err);
     return cuda_check("segment_scan launch", cudaGetLastError());
+}
+
+// Entry state of shard r of a sequence split over R shards (in order): the
+// shards' summaries (dS_i, dz_i, A_i) fold as X_{i+1} = A_i X_i + dX_i from
+// X_0 = state-in (or 0); shard r starts from X_r.  One thread per element of
+// a head's state; layouts [R][BH][D*D] (S), [R][BH][D] (z), [R][BH] (A).
+__global__ void __launch_bounds__(256) state_combine_kernel(const float *S_all, const float *z_all,
+                                                            const float *A_all, int r, long BH, int D,
+                                                            const float *S_in, const float *z_in, float *S_out,
+                                                            float *z_out) {
+    const int E = D * D + D;
+    const long bh = blockIdx.y;
+    const int e = blockIdx.x * 256 + threadIdx.x;
+    if (e >= E) return;
+    const bool isS = e < D * D;
+    const int ez = e - D * D;
+    float x = 0.f;
+    if (isS) { if (S_in) x = S_in[bh * D * D + e]; }
+    else if (z_in) x = z_in[bh * D + ez];
+    for (int i = 0; i < r; ++i) {
+        const float dx = isS ? S_all[((size_t)i * BH + bh) * D * D + e] : z_all[((size_t)i * BH + bh) * D + ez];
+        x = fmaf(A_all[(size_t)i * BH + bh], x, dx);
+    }
+    if (isS) S_out[bh * D * D + e] = x;
+    else z_out[bh * D + ez] = x;
+}
+
+la_status launch_state_combine(const float *S_all, const float *z_all, const float *A_all, int r, long BH, int D,
+                               const float *S_in, const float *z_in, float *S_out, float *z_out, cudaStream_t st) {
+    const int E = D * D + D;
+    state_combine_kernel<<<dim3((E + 255) / 256, (unsigned)BH), 256, 0, st>>>(S_all, z_all, A_all, r, BH, D, S_in,
+                                                                               z_in, S_out, z_out);
+    count_launches(1);
+    return cuda_check("state_combine launch", cudaGetLastError());
 }
 
 }  // namespace la

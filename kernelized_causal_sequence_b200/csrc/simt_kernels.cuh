@@ -37,6 +37,7 @@ struct SimtParams {
     int BH, T, Lq, chunk, seg_len, n_seg;
     float eps;
     void *const *events;    // host only: 4 cudaEvent_t recorded around K1, K2, K3, or null
+    float *sum_A;           // host only: shard summary (no output pass), each head's decay product
 };
 
 constexpr int kSimtThreads = 256;

@@ -11,10 +11,15 @@ struct TcCausalArgs {
     const float *decay;
     const float *gain;     // per-token gain on the new term, or null
     int mlstm;             // identity feature map, max(|den|, 1) read-out
+    int flash;             // the FLASH chunk form (identity map, relu(score / s)^2, no normaliser)
+    float inv_s;           // FLASH: 1 / s
+    bool summary;          // state pass + scan only: the total contribution to state_S/state_z (mode OUT)
+    float *sum_A;          // summary: each head's decay product [BH]
     void *out;
     la_dtype in_dtype, out_dtype;
     float *ws_state, *ws_A;
-    int *status;
+    int *status;           // the call's status word [2] in the workspace (cleared by the caller)
+    unsigned long long wait_ns;   // limit of every bounded device-side wait
     float *state_S, *state_z;
     la_state_mode mode;
     long BH;
@@ -28,6 +33,8 @@ struct TcNoncausalArgs {
     void *out;
     la_dtype in_dtype, out_dtype;
     float *ws_state, *ws_A, *ws_total;
+    int *status;                  // the call's status word [2] (cleared by the caller)
+    unsigned long long wait_ns;
     float *state_S, *state_z;
     la_state_mode mode;
     long BH;

@@ -45,7 +45,8 @@
 //   warps 10-13  decay cumsum and phi(K) (then w o phi(K) in place).
 //
 // Every wait is bounded (see tc_ptx.cuh); on expiry the CTA raises its abort
-// flag and the status word, drains its copies and MMAs, frees TMEM, returns.
+// flag and the call's status word (LA_ERR_TIMEOUT and the id of the wait),
+// drains its copies and MMAs, frees TMEM and returns.
 #pragma once
 #include <type_traits>
 
@@ -149,10 +150,14 @@ struct TcParams {
     float *ws_A;          // [BH, n_seg]
     float *fin_S;         // [BH, D, D] or null: output mode writes the final state
     float *fin_z;         // [BH, D]      from the last segment (the scan does not)
-    int *status;          // status word (0 = ok)
+    int *status;          // status word [2]: code (0 = ok), id of the first wait that gave up
     int T, seg_len, n_seg;
     float eps;
     int mlstm;            // 1: identity feature map and the max(|den|, 1) read-out (decay kernels only)
+    unsigned long long wait_ns;   // limit of every working wait
+    int flash;            // 1: the FLASH chunk form (identity feature map; kernels of form 2 and
+                          //    the decay form's state-only pass)
+    float inv_s;          // FLASH: 1 / the score and summary scale (1 or 1 / chunk)
 };
 
 template <typename OutT> __device__ __forceinline__ void store_row32(OutT *dst, const float (&o)[32]);
@@ -477,9 +482,9 @@ __device__ __forceinline__ bool k_stage(uint8_t *smem, uint64_t *bar, float *Fsm
     // output mode: plain phi(K) (MMA1 needs it; the decay weights are applied
     // in place after MMA1, see k_weight); state-only: w o phi(K) directly
     if constexpr (G::OUT)
-        phi_tile<InT, C, D, false, CONV, 0, 1, 1>(kt, kt + G::TILE, tk, n, Lk, Lend, DECAY && p.mlstm);
+        phi_tile<InT, C, D, false, CONV, 0, 1, 1>(kt, kt + G::TILE, tk, n, Lk, Lend, DECAY && (p.mlstm || p.flash));
     else
-        phi_tile<InT, C, D, DECAY, CONV, 0, 2, 4>(kt, kt + G::TILE, tk, n, Lk, Lend, DECAY && p.mlstm);
+        phi_tile<InT, C, D, DECAY, CONV, 0, 2, 4>(kt, kt + G::TILE, tk, n, Lk, Lend, DECAY && (p.mlstm || p.flash));
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
@@ -626,7 +631,7 @@ __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *ba
     uint8_t *kt = smem + G::OFF_KV + s * G::KV_STAGE;
     constexpr bool CONV = !std::is_same<InT, bf16>::value;
     phi_tile<InT, C, D, DECAY, CONV, 2, 4, 4>(kt, kt + G::TILE, et, n, L, DECAY ? Fsm[G::F_LE + s] : 0.f,
-                                              DECAY && p.mlstm);
+                                              DECAY && (p.mlstm || p.flash));
     fence_proxy_async_smem();
     __syncwarp();
     if ((et & 31) == 0) mbar_arrive(&bar[G::B_PHI + s]);
@@ -634,11 +639,17 @@ __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *ba
 }
 
 // ---------------------------------------------------------------------------
-template <int C, int D, bool DECAY, int MODE, typename InT, typename OutT>
+// FORM: 0 = no decay, 1 = decay (also the gated and mLSTM forms), 2 = the
+// FLASH chunk form (the decay form's machinery with a = 1 and the identity
+// feature map; scores -> relu(score / s)^2 inside the chunk, the carried
+// summaries read as S / s, no normaliser).
+template <int C, int D, int FORM, int MODE, typename InT, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                   TcParams p) {
+    constexpr bool DECAY = FORM != 0;
+    constexpr bool FLASH = FORM == 2;
     using G = Cfg<C, D, DECAY, MODE>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -646,7 +657,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint32_t *tmem_addr_smem = reinterpret_cast<uint32_t *>(smem + G::OFF_TMEMADDR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + G::OFF_ABORT);
     float *Fsm = reinterpret_cast<float *>(smem + G::OFF_F);
-    const AbortCtx ab{abort_flag, p.status};
+    const AbortCtx ab{abort_flag, p.status, p.wait_ns};
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int seg = blockIdx.x, bh = blockIdx.y;
@@ -704,7 +715,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_addr_smem;
-    if ((smem_u32(smem) & 1023u) != 0) raise_abort(ab, 16);  // layout assumption violated
+    if ((smem_u32(smem) & 1023u) != 0) raise_abort(ab, 99, kStatusLayout);  // layout assumption violated
 
     if (warp == kTmaWarp) {
         // ================= TMA producer
@@ -737,14 +748,12 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             if (*abort_flag) {
                 // drain copies still in flight before the CTA may exit
-                AbortCtx drain{abort_flag, nullptr};
                 volatile int never = 0;
-                AbortCtx timed{&never, nullptr};
+                AbortCtx timed{&never, nullptr, kDrainLimitNs};
                 for (int s = 0; s < G::NKV; ++s)
                     if (issued_kv[s] > 0) mbar_wait(&bar[G::B_KV_FULL + s], (issued_kv[s] - 1) & 1, timed, 0);
                 for (int s = 0; s < 2; ++s)
                     if (issued_q[s] > 0) mbar_wait(&bar[G::B_Q_FULL + s], (issued_q[s] - 1) & 1, timed, 0);
-                (void)drain;
             }
         }
     } else if (warp == kMmaWarp) {
@@ -851,7 +860,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             // drain: every MMA issued by this thread has completed
             volatile int never = 0;
-            AbortCtx timed{&never, nullptr};
+            AbortCtx timed{&never, nullptr, kDrainLimitNs};
             mma_commit(&bar[G::B_DRAIN]);
             mbar_wait(&bar[G::B_DRAIN], 0, timed, 0);
         }
@@ -883,7 +892,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int a_row = q * SROWS + lane;   // state row (feature index)
 
         if constexpr (G::OUT)
-            if (nch > 0) ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, 0, tw, DECAY && p.mlstm);
+            if (nch > 0) ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, 0, tw, DECAY && (p.mlstm || p.flash));
         // ---- segment start: state entering the segment -> TMEM (and operands)
         if (ok && nch > 0) {
             float g0 = 1.f;   // decay of chunk 0 (the state is rescaled before its update)
@@ -904,6 +913,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int i = 0; i < 32; ++i) {
                         vals[i] = (G::OUT && srow_ok) ? st[(size_t)a_row * D + cb * 32 + i] : 0.f;
                         u[i] = __float_as_uint(vals[i] * g0);
+                        if constexpr (FLASH) vals[i] *= p.inv_s;   // operand: the summaries over s
                     }
                     tmem_st32(tmem + lane_base + G::T_S + cb * 32, u);
                     if constexpr (G::OUT) if (srow_ok) write_state_row<D>(smem + G::OFF_SBF, a_row, cb * 32, vals);
@@ -977,7 +987,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if (!ok) break;
                 }
                 if (c + 1 < nch) {
-                    ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, c + 1, tw, DECAY && p.mlstm);
+                    ok = q_stage<C, D, DECAY, MODE, InT>(smem, bar, ab, tmem, c + 1, tw, DECAY && (p.mlstm || p.flash));
                     if (!ok) break;
                 }
                 if (c == nch - 1) {
@@ -1010,8 +1020,13 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     float vals[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) vals[i] = __uint_as_float(u[i]);
+                    if constexpr (FLASH) {
+                        // the read-out sees the summaries over s; TMEM keeps the raw sum
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) vals[i] *= p.inv_s;
+                    }
                     if (srow_ok) write_state_row<D>(smem + G::OFF_SBF, a_row, cb * 32, vals);
-                    if constexpr (DECAY) {
+                    if constexpr (DECAY && !FLASH) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(vals[i] * gnext);
                         tmem_st32(tmem + lane_base + G::T_S + cb * 32, u);
@@ -1021,7 +1036,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     bf16 *zb = reinterpret_cast<bf16 *>(smem + G::OFF_ZB);
                     write_z_operand<DECAY>(zb, a_row, __uint_as_float(zbits));
                 }
-                if constexpr (DECAY) {
+                if constexpr (DECAY && !FLASH) {
                     tmem_st1(tmem + lane_base + G::T_Z, __float_as_uint(__uint_as_float(zbits) * gnext));
                     tmem_st_wait();
                 }
@@ -1082,7 +1097,13 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         for (int k = 0; k < 16; ++k) {
                             const int j = cb * 32 + 2 * k;
                             float v0 = __uint_as_float(u[h][2 * k]), v1 = __uint_as_float(u[h][2 * k + 1]);
-                            if constexpr (DECAY) {
+                            if constexpr (FLASH) {
+                                // exact squared-ReLU weight of the chunk form
+                                v0 = fmaxf(v0 * p.inv_s, 0.f);
+                                v1 = fmaxf(v1 * p.inv_s, 0.f);
+                                v0 *= v0;
+                                v1 *= v1;
+                            } else if constexpr (DECAY) {
                                 v0 *= ex2_approx(Li - Lk[j]);
                                 v1 *= ex2_approx(Li - Lk[j + 1]);
                             }
@@ -1133,7 +1154,9 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     tmem_ld_wait();
                     // denominator: (decayed) phi(q).z of the carried state + row sum of P + eps
                     if (g == 0) {
-                        if constexpr (DECAY) {
+                        if constexpr (FLASH) {
+                            inv = 1.f;   // no normaliser
+                        } else if constexpr (DECAY) {
                             const float den = (__uint_as_float(ud) + __uint_as_float(ud_lo)) + rowsum;
                             // mLSTM read-out: divide by max(|den|, 1)
                             inv = p.mlstm ? 1.f / fmaxf(fabsf(den), 1.f) : 1.f / (den + p.eps);

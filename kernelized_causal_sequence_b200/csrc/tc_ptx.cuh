@@ -38,31 +38,48 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
 // completes (or ~0.5 ms pass) instead of spinning, leaving issue slots to the
 // warps that work.
 constexpr uint32_t kSuspendHintNs = 500000;
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, uint32_t hint_ns = kSuspendHintNs) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
 
-// Wait limit of every spin in these kernels: ~2 s of wall time.  On expiry
-// the waiter raises the CTA's abort flag and the kernel's status word, and
-// every other waiter of the CTA gives up at its next poll.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Wait limits.  Every spin on an mbarrier is bounded: the working waits by
+// the launch's limit (~2 s by default, settable per process through
+// la_set_wait_limit_ns), the drain waits that let copies and MMAs in flight
+// complete before a CTA exits by a fixed bound of their own.  On expiry of a
+// working wait the waiter raises the CTA's abort flag and the call's status
+// word, and every other waiter of the CTA gives up at its next poll.
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
+
+// Status word of a call (two ints in the caller's workspace): [0] = 0 or the
+// la_status that ended the call early (LA_ERR_TIMEOUT for an expired wait),
+// [1] = the id of the first wait or check that gave up (for diagnosis).
+constexpr int kStatusTimeout = 4;    // LA_ERR_TIMEOUT
+constexpr int kStatusLayout = 3;     // LA_ERR_CUDA: a device-side layout check failed
 
 struct AbortCtx {
     volatile int *flag;    // shared memory, CTA-wide
-    int *status;           // global status word (may be null)
+    int *status;           // global status word [2] (may be null)
+    uint64_t limit_ns;     // wait limit
+    // suspend hint of each poll: kSuspendHintNs, or the limit when it is
+    // shorter (a limit of 0 makes every poll return at once)
+    __device__ uint32_t hint() const { return limit_ns < kSuspendHintNs ? (uint32_t)limit_ns : kSuspendHintNs; }
 };
 
-__device__ __forceinline__ void raise_abort(const AbortCtx &ab, int code) {
+__device__ __forceinline__ void raise_abort(const AbortCtx &ab, int code, int status = kStatusTimeout) {
     *ab.flag = 1;
-    if (ab.status) atomicExch(ab.status, code);
+    if (ab.status) {
+        atomicCAS(ab.status, 0, status);
+        atomicCAS(ab.status + 1, 0, code);
+    }
 }
 
 // Bounded wait on a phase parity.  Returns false if the CTA is aborting or
@@ -73,17 +90,18 @@ __device__ __forceinline__ void raise_abort(const AbortCtx &ab, int code) {
 __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, const AbortCtx ab, int code);
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const AbortCtx &ab,
                                           int code) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity, ab.hint())) return true;
     return mbar_wait_slow(bar, parity, ab, code);
 }
 __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, const AbortCtx ab, int code) {
     const uint64_t t0 = globaltimer_ns();
+    const uint32_t hint = ab.hint();
     uint32_t n = 0;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait(bar, parity, hint)) return true;
         if ((++n & 3u) == 0) {
             if (*ab.flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 >= ab.limit_ns) {
                 raise_abort(ab, code);
                 return false;
             }
@@ -129,6 +147,10 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // wait until the shared-memory sources of all committed stores have been read
 __device__ __forceinline__ void bulk_wait_read0() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// the same, allowing the most recent committed group to be still reading
+__device__ __forceinline__ void bulk_wait_read1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 // wait until all committed stores have completed
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -192,6 +214,21 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// The same with the 64-byte swizzle (layout type 4; atoms of 8 rows x 64 bytes,
+// 512-byte aligned): for an MN-major operand, lbo = the byte distance between
+// consecutive 32-element (64-byte) blocks along M or N, sbo = between
+// consecutive groups of 8 rows along K.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
+}
+// No swizzle, K-major (layout type 0): core matrices of 8 rows x 16 bytes
+// stored contiguously (128 bytes); lbo = the byte distance between core
+// matrices adjacent along K, sbo = between groups of 8 rows along M or N.
+__device__ __forceinline__ uint64_t sdesc_nosw(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
 // ------------------------------------------------------------------ TMEM ld/st

@@ -36,6 +36,7 @@ class Workload:
     decay: bool = False
     gated: bool = False   # RFA gate: decay a_t = g_t and gain b_t = 1 - g_t on the new term
     mlstm: bool = False   # mLSTM read-out: decay = forget gate, plus an input gate (input_gate())
+    flash: bool = False   # the FLASH chunk form (its own entry point)
     k_scale: float = 0.0  # keys' scale when it differs from qk_scale (0: qk_scale)
     eps: float = 1e-6
     Lk: int = 0         # non-causal only
@@ -81,6 +82,11 @@ WORKLOADS = {
                                             "bf16", "bf16", chunk=64, decay=True, mlstm=True,
                                             qk_scale=1.0, k_scale=1 / math.sqrt(128),
                                             v_scale=1 / math.sqrt(128), seed=1007),
+    # the FLASH chunk form at the same shape: q, k ~ N(0,1)/128^(1/4) (so q.k ~ N(0,1)),
+    # v ~ N(0,1)/sqrt(128); the chunk is part of the form's definition
+    "flash_bf16_b2h16_t8192_d128": Workload("flash_bf16_b2h16_t8192_d128", "causal", 2, 16, 8192, 128,
+                                            "bf16", "bf16", chunk=64, flash=True, qk_scale=128 ** -0.25,
+                                            v_scale=1 / math.sqrt(128), seed=1008),
     # non-causal, LoFTR-coarse shape: B=8, H=8, L=4800, d=32, fp16, V pre-scaled by 1/Lk
     "noncausal_f16_b8h8_l4800_d32": Workload("noncausal_f16_b8h8_l4800_d32", "noncausal", 8, 8,
                                              4800, 32, "f16", "f32", chunk=128, Lk=4800,
@@ -175,6 +181,19 @@ def decode_state(w: Workload, B: int | None = None, H: int | None = None):
     S = _normals(rng, (B, H, w.d, w.d)) * np.float32(math.sqrt(w.prompt) * w.v_scale)
     z = np.float32(w.prompt) * (np.float32(1.0) + np.float32(0.05) * _normals(rng, (B, H, w.d)))
     return torch.from_numpy(S.astype(np.float32)), torch.from_numpy(z.astype(np.float32))
+
+
+# Distinct per-step decode inputs; a longer decode loop cycles through them.
+DECODE_DISTINCT_INPUTS = 64
+
+
+def decode_prompt(w: Workload):
+    """The prompt whose prefill state starts a decode workload: q, k, v
+    [B, H, w.prompt, d] drawn like the long-context prefill's inputs (same
+    scales and dtype) from the decode workload's seed + 1."""
+    pw = WORKLOADS["prefill_bf16_h16_t131072_d128"]
+    q, k, v, _ = qkv(pw, T=w.prompt, B=w.B, H=w.H, seed=w.seed + 1)
+    return q, k, v
 
 
 def decode_inputs(w: Workload, step: int, B: int | None = None, H: int | None = None,

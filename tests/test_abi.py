@@ -30,6 +30,15 @@ def L():
     return la.lib()
 
 
+@pytest.fixture(autouse=True)
+def no_kernel_launched(L):
+    """Every call in this file must be settled on the host: the dummy device
+    addresses above are never dereferenced because no kernel is launched."""
+    before = L.la_launch_count()
+    yield
+    assert L.la_launch_count() == before, "a host-side check let a kernel launch"
+
+
 def test_exports_every_declared_symbol(L):
     names = declared_functions()
     assert {"la_prefill_causal", "la_forward_noncausal", "la_decode_step",
@@ -184,3 +193,18 @@ def test_gated_and_mlstm_reject_bad_arguments(L):
     assert dec_mlstm(z=None) == E_ARG
     assert dec_mlstm(d=96) == E_UNS
     assert dec_mlstm(B=0) == la.LA_OK
+
+
+def test_status_query_and_wait_limit(L):
+    """la_workspace_status rejects a null or misaligned workspace on the host;
+    la_set_wait_limit_ns returns the previous limit (default 2 s)."""
+    w = ctypes.c_int(0)
+    assert L.la_workspace_status(None, ctypes.byref(w), None) == la.LA_ERR_INVALID_ARG
+    assert L.la_workspace_status(ctypes.c_void_p(0x10010), ctypes.byref(w), None) == la.LA_ERR_INVALID_ARG
+    old = la.la_set_wait_limit_ns(12345)
+    try:
+        assert old == 2_000_000_000
+        assert la.la_set_wait_limit_ns(0) == 12345
+    finally:
+        la.la_set_wait_limit_ns(old)
+    assert la.la_set_wait_limit_ns(old) == old

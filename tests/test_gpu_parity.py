@@ -249,7 +249,11 @@ def test_workload_noncausal(la, orc, cross):
 @pytest.mark.parametrize("dtype,d,Lq,Lk", [(torch.float32, 64, 100, 333), (torch.bfloat16, 128, 17, 1000),
                                            (torch.float16, 32, 129, 0), (torch.bfloat16, 64, 0, 50),
                                            (torch.float32, 32, 300, 700), (torch.bfloat16, 32, 1000, 517),
-                                           (torch.float16, 32, 513, 5000)])
+                                           (torch.float16, 32, 513, 5000),
+                                           # tensor-core path at d = 32: no queries (state only),
+                                           # one key, one query, many heads per key segment
+                                           (torch.bfloat16, 32, 0, 700), (torch.float16, 32, 1, 1),
+                                           (torch.bfloat16, 32, 4800, 128), (torch.float16, 32, 257, 129)])
 def test_noncausal_small(la, orc, dtype, d, Lq, Lk):
     rng = np.random.default_rng(Lq + Lk)
     mk = lambda L: torch.from_numpy(rng.standard_normal((2, 3, L, d), dtype=np.float32)).to(dtype)
@@ -542,3 +546,246 @@ def test_mlstm_decode(la, orc, dtype, d):
     assert row_rel_err(o.cpu().numpy(), ro) < tol_for(dtype)
     assert row_rel_err(S.cpu().numpy().reshape(B, H, -1), rS.reshape(B, H, -1)) < 1e-5
     assert row_rel_err(z.cpu().numpy(), rz) < 1e-5
+
+
+# ------------------------------------------- decode exactly as the bench runs it
+def test_workload_decode_as_benched(la, orc):
+    """The long-context decode as the bench runs it: fp32 states from the
+    library's own prefill of the seeded 512-token prompt (B64 H16, chunk 128),
+    then all 1024 steps updating the states in place, the distinct step inputs
+    cycled.  The oracle receives the same fp32 states and runs its decode step
+    1024 times on sampled heads; every step's output and the final state are
+    compared.  The prompt's states are also checked against the oracle's
+    prefill of the prompt (the prefill -> decode hand-off)."""
+    wd = W["decode_bf16_b64h16_d128"]
+    B, H, d = wd.B, wd.H, wd.d
+    pq, pk, pv = inputs.decode_prompt(wd)
+    S = torch.zeros((B, H, d, d), device=DEV)
+    z = torch.zeros((B, H, d), device=DEV)
+    la.la_prefill_causal(pq.to(DEV), pk.to(DEV), pv.to(DEV), chunk=128, state_S=S, state_z=z,
+                         mode=la.LA_STATE_OUT)
+    torch.cuda.synchronize()
+    S0, z0 = S.cpu().numpy().astype(np.float64), z.cpu().numpy().astype(np.float64)
+    bidx = np.array([0, 17, 40, 63])
+    hidx = np.array([0, 5, 11, 15])
+    sel = lambda x: x[bidx, hidx][None]          # [1, n_sampled, ...]
+    _, rS_p, rz_p = orc.causal(sel(pq), sel(pk), sel(pv))
+    assert row_rel_err(sel(S0).reshape(1, len(bidx), -1), rS_p.reshape(1, len(bidx), -1)) < 2e-2
+    assert row_rel_err(sel(z0), rz_p) < 2e-2
+
+    n_in = inputs.DECODE_DISTINCT_INPUTS
+    steps_in = [inputs.decode_inputs(wd, i) for i in range(n_in)]
+    dq = torch.stack([s[0] for s in steps_in]).to(DEV)
+    dk = torch.stack([s[1] for s in steps_in]).to(DEV)
+    dv = torch.stack([s[2] for s in steps_in]).to(DEV)
+    outs = torch.empty((wd.steps, B, H, d), dtype=wd.torch_out_dtype, device=DEV)
+    for i in range(wd.steps):
+        j = i % n_in
+        la.la_decode_step(dq[j], dk[j], dv[j], S, z, eps=wd.eps, out=outs[i])
+    torch.cuda.synchronize()
+    got = outs[:, bidx, hidx].float().cpu().numpy()          # [steps, n_sampled, d]
+    rS, rz = sel(S0), sel(z0)
+    worst = 0.0
+    for i in range(wd.steps):
+        q, k, v, _ = steps_in[i % n_in]
+        ro, rS, rz = orc.decode_step(sel(q), sel(k), sel(v), rS, rz, eps=wd.eps)
+        worst = max(worst, row_rel_err(got[i][None], ro))
+    assert worst < 2e-2, f"worst step output rel err {worst}"
+    Sg, zg = S.cpu().numpy(), z.cpu().numpy()
+    assert row_rel_err(sel(Sg).reshape(1, len(bidx), -1), rS.reshape(1, len(bidx), -1)) < 2e-2
+    assert row_rel_err(sel(zg), rz) < 2e-2
+
+
+# ------------------------------------------------- feature-map and decay range
+def _scaled_inputs(dtype, d, T, B, H, seed, qk_std, decay=None):
+    rng = np.random.default_rng(seed)
+    mk = lambda s: torch.from_numpy((rng.standard_normal((B, H, T, d), dtype=np.float32) * s)).to(dtype)
+    q, k, v = mk(qk_std), mk(qk_std), mk(1.0 / np.sqrt(d))
+    return q, k, v
+
+
+# (dtype, d, chunk, qk_std): the workloads' N(0,1)/sqrt(d) scaled x4 and x8,
+# and unit-variance inputs x3, whose e^x branch reaches x < -10 (phi(x) of
+# order 1e-5) while the x + 1 branch reaches x > 10
+PHI_RANGE = [
+    (torch.bfloat16, 128, 128, 4.0 / np.sqrt(128)),
+    (torch.bfloat16, 128, 64, 8.0 / np.sqrt(128)),
+    (torch.bfloat16, 64, 64, 8.0 / np.sqrt(64)),
+    (torch.float16, 128, 128, 8.0 / np.sqrt(128)),
+    (torch.bfloat16, 128, 128, 3.0),
+    (torch.bfloat16, 64, 64, 3.0),
+    (torch.float16, 64, 128, 3.0),
+]
+
+
+@pytest.mark.parametrize("dtype,d,chunk,qk_std", PHI_RANGE)
+@pytest.mark.parametrize("decay", [False, True])
+def test_prefill_phi_range(la, orc, dtype, d, chunk, qk_std, decay):
+    """The tensor-core feature map on both branches far from 0: phi(x) = x + 1
+    for large x and e^x for x << 0 (2^(x log2 e) on the ex2 unit, rounded to
+    bf16)."""
+    B, H, T = 1, 2, 1100
+    q, k, v = _scaled_inputs(dtype, d, T, B, H, seed=int(qk_std * 1000) + d, qk_std=qk_std)
+    a = None
+    if decay:
+        rng = np.random.default_rng(d)
+        a = torch.from_numpy((1 / (1 + np.exp(-(rng.standard_normal((B, H, T)) + 2)))).astype(np.float32))
+    if qk_std >= 2.0:
+        assert float(q.float().min()) < -10 and float(k.float().max()) > 10
+    check_prefill(la, orc, q, k, v, a, chunk, torch.float32, 2e-2)
+
+
+@pytest.mark.parametrize("dtype,d,chunk", [(torch.bfloat16, 128, 64), (torch.bfloat16, 128, 128),
+                                           (torch.bfloat16, 64, 64), (torch.float32, 64, 64),
+                                           (torch.float16, 32, 128)])
+def test_prefill_decay_extremes(la, orc, dtype, d, chunk):
+    """Decays of 1 mixed inside every chunk with decays of 1e-6 and 1e-30,
+    where the in-chunk weights 2^(L_i - L_j) underflow to 0 and the carried
+    state is wiped; the exact answer is the recurrence's."""
+    B, H, T = 2, 2, 1500
+    q, k, v, _ = _small_inputs(dtype, d, T, False, B, H, seed=71 + d)
+    rng = np.random.default_rng(72 + d)
+    u = rng.uniform(size=(B, H, T))
+    a = np.ones((B, H, T), dtype=np.float32)
+    a[u < 0.08] = 1e-6
+    a[(u >= 0.08) & (u < 0.12)] = 1e-30
+    a[(u >= 0.12) & (u < 0.5)] = rng.uniform(0.2, 1.0, size=int(((u >= 0.12) & (u < 0.5)).sum()))
+    a = torch.from_numpy(a)
+    check_prefill(la, orc, q, k, v, a, chunk, torch.float32, tol_for(dtype))
+
+
+# ------------------------------------------------------------- timeout path
+@pytest.mark.parametrize("d,chunk,decay", [(128, 128, False), (128, 64, True)])
+def test_wait_timeout_is_reported_and_next_call_is_exact(la, d, chunk, decay):
+    """With the wait limit set to 0 every device-side wait that is not already
+    satisfied gives up at once: the blocks drain their copies and products,
+    free their tensor memory and exit, and the workspace's status word reports
+    LA_ERR_TIMEOUT with the id of the wait.  The next call with the default
+    limit is bitwise equal to the call before the timeout."""
+    B, H, T = 1, 2, 3000
+    q, k, v, a = _small_inputs(torch.bfloat16, d, T, decay, B, H, seed=81)
+    qd, kd, vd = (x.to(DEV) for x in (q, k, v))
+    ad = None if a is None else a.to(DEV)
+    ws = torch.empty(la.la_prefill_workspace_size(B, H, T, d, d, chunk), dtype=torch.uint8, device=DEV)
+
+    def call():
+        S = torch.zeros((B, H, d, d), device=DEV)
+        z = torch.zeros((B, H, d), device=DEV)
+        o = la.la_prefill_causal(qd, kd, vd, decay=ad, chunk=chunk, state_S=S, state_z=z,
+                                 out_dtype=torch.float32, workspace=ws)
+        return o, S
+
+    o1, S1 = call()
+    assert la.la_workspace_status(ws) == (la.LA_OK, 0)
+    old = la.la_set_wait_limit_ns(0)
+    try:
+        call()
+        st, waiter = la.la_workspace_status(ws)
+    finally:
+        la.la_set_wait_limit_ns(old)
+    assert st == la.LA_ERR_TIMEOUT and waiter > 0
+    o3, S3 = call()
+    assert la.la_workspace_status(ws) == (la.LA_OK, 0)
+    assert torch.equal(o1, o3) and torch.equal(S1, S3)
+
+
+@pytest.mark.parametrize("B,H,Lq,Lk", [(1, 3, 700, 900), (3, 7, 300, 2000), (1, 1, 128, 128)])
+def test_noncausal_tc_head_groups(la, orc, B, H, Lq, Lk):
+    """Head counts that leave the tensor-core state pass's last group of four
+    heads partly empty, in every state mode; the output is deterministic and
+    the same without a state output."""
+    rng = np.random.default_rng(B * 100 + H)
+    mk = lambda L: torch.from_numpy(rng.standard_normal((B, H, L, 32), dtype=np.float32) * 0.7).to(torch.float16)
+    q, k, v = mk(Lq), mk(Lk), mk(Lk)
+    S0 = torch.from_numpy(rng.standard_normal((B, H, 32, 32), dtype=np.float32))
+    z0 = torch.from_numpy(np.abs(rng.standard_normal((B, H, 32), dtype=np.float32)) + 1.0)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    ro, rS, rz = orc.noncausal(q, k, v, S_in=S0, z_in=z0)
+    S, z = S0.to(DEV).clone(), z0.to(DEV).clone()
+    o1 = la.la_forward_noncausal(qd, kd, vd, state_S=S, state_z=z, mode=la.LA_STATE_INOUT, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert row_rel_err(o1.cpu().numpy(), ro) < 2e-2
+    assert row_rel_err(S.cpu().numpy().reshape(B, H, -1), rS.reshape(B, H, -1)) < 2e-2
+    assert row_rel_err(z.cpu().numpy(), rz) < 2e-2
+    ro0, rS0, _ = orc.noncausal(q, k, v)
+    S2 = torch.full((B, H, 32, 32), 5.0, device=DEV)
+    z2 = torch.full((B, H, 32), 5.0, device=DEV)
+    o2 = la.la_forward_noncausal(qd, kd, vd, state_S=S2, state_z=z2, mode=la.LA_STATE_OUT, out_dtype=torch.float32)
+    o3 = la.la_forward_noncausal(qd, kd, vd, out_dtype=torch.float32)
+    o4 = la.la_forward_noncausal(qd, kd, vd, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert row_rel_err(o2.cpu().numpy(), ro0) < 2e-2
+    assert row_rel_err(S2.cpu().numpy().reshape(B, H, -1), rS0.reshape(B, H, -1)) < 2e-2
+    assert torch.equal(o2, o3) and torch.equal(o3, o4)
+
+
+# ------------------------------------------------------------- FLASH chunk form
+# Exact relu(q.k / s)^2 attention inside each chunk, q^T (earlier chunks'
+# summaries) / s across chunks; s = 1 (equations) or s = chunk (listings).
+FLASH = [
+    # (dtype, d, T, chunk, B, H)
+    (torch.bfloat16, 128, 1000, 128, 1, 2),    # ragged last chunk
+    (torch.bfloat16, 128, 1500, 64, 2, 1),
+    (torch.bfloat16, 64, 777, 64, 1, 3),
+    (torch.bfloat16, 64, 600, 128, 1, 2),
+    (torch.float16, 128, 513, 64, 1, 2),
+    (torch.bfloat16, 128, 5000, 64, 1, 1),     # > 64 segments per head
+    (torch.bfloat16, 128, 64, 64, 1, 1),       # one chunk: causal squared-ReLU attention alone
+]
+
+
+def _flash_inputs(dtype, d, T, B, H, seed):
+    rng = np.random.default_rng(seed)
+    s = d ** -0.25   # q.k ~ N(0, 1)
+    mk = lambda sc: torch.from_numpy(rng.standard_normal((B, H, T, d), dtype=np.float32) * sc).to(dtype)
+    return mk(s), mk(s), mk(1.0)
+
+
+@pytest.mark.parametrize("dtype,d,T,chunk,B,H", FLASH)
+@pytest.mark.parametrize("scaled", [False, True])
+def test_flash_prefill(la, orc, dtype, d, T, chunk, B, H, scaled):
+    q, k, v = _flash_inputs(dtype, d, T, B, H, seed=T + d + chunk)
+    ro, rS = orc.flash(q, k, v, chunk, scaled=scaled)
+    inv_s = 1.0 / chunk if scaled else 1.0
+    for out_dtype in (torch.float32, dtype):
+        S = torch.zeros((B, H, d, d), device=DEV)
+        z = torch.zeros((B, H, d), device=DEV)
+        o = la.la_prefill_causal_flash(q.to(DEV), k.to(DEV), v.to(DEV), chunk=chunk, scaled=scaled, state_S=S,
+                                       state_z=z, out_dtype=out_dtype)
+        torch.cuda.synchronize()
+        o = o.float().cpu().numpy()
+        err = row_rel_err(o, ro)
+        assert err < 2e-2, f"output rel err {err}"
+        Sg = S.cpu().numpy() * inv_s
+        assert row_rel_err(Sg.reshape(B, H, -1), rS.reshape(B, H, -1)) < 2e-2
+        rz = k.double().numpy().sum(axis=2)
+        assert row_rel_err(z.cpu().numpy(), rz) < 2e-2
+
+
+@pytest.mark.parametrize("scaled", [False, True])
+def test_flash_state_handoff(la, orc, scaled):
+    """A prefill split at a chunk boundary, the second part starting from the
+    first part's state, equals the whole prefill."""
+    d, T1, T2, chunk = 128, 640, 517, 64
+    q, k, v = _flash_inputs(torch.bfloat16, d, T1 + T2, 1, 2, seed=5)
+    ro, _ = orc.flash(q, k, v, chunk, scaled=scaled)
+    S = torch.zeros((1, 2, d, d), device=DEV)
+    z = torch.zeros((1, 2, d), device=DEV)
+    dv = lambda x, a, b: x[:, :, a:b].contiguous().to(DEV)
+    o1 = la.la_prefill_causal_flash(dv(q, 0, T1), dv(k, 0, T1), dv(v, 0, T1), chunk=chunk, scaled=scaled,
+                                    state_S=S, state_z=z, out_dtype=torch.float32)
+    o2 = la.la_prefill_causal_flash(dv(q, T1, T1 + T2), dv(k, T1, T1 + T2), dv(v, T1, T1 + T2), chunk=chunk,
+                                    scaled=scaled, state_S=S, state_z=z, mode=la.LA_STATE_INOUT,
+                                    out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    o = np.concatenate([o1.cpu().numpy(), o2.cpu().numpy()], axis=2)
+    assert row_rel_err(o, ro) < 2e-2
+
+
+def test_flash_rejects_unsupported(la):
+    q = torch.zeros((1, 1, 64, 32), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(la.LinAttnError):
+        la.la_prefill_causal_flash(q, q, q, chunk=64)          # d = 32: no tensor-core path
+    q = torch.zeros((1, 1, 64, 64), dtype=torch.float32, device=DEV)
+    with pytest.raises(la.LinAttnError):
+        la.la_prefill_causal_flash(q, q, q, chunk=64)          # fp32 inputs
