@@ -263,8 +263,7 @@ def la_prefill_causal_flash(q, k, v, chunk=64, scaled=False, state_S=None, state
                                        int(bool(scaled)), _ptr(state_S), _ptr(state_z), int(mode), _ptr(out),
                                        _DT[out.dtype], _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("la_prefill_causal_flash",
-    "la_prefill_causal_summary", "la_state_combine", st)
+    _check("la_prefill_causal_flash", st)
     return out
 
 

@@ -1,5 +1,6 @@
 // nc_tc.cuh — tcgen05 tensor-core kernels of the non-causal form at head
-// dimension 32 (16-bit inputs, bf16 tensor-core operands, fp32 accumulation):
+// dimension 32 (16-bit inputs; tensor-core operands in the input's type for
+// the state pass and in bf16 for the read-out; fp32 accumulation):
 //
 //   S = phi(K)^T V,  z = phi(K)^T 1,  out_i = phi(q_i)^T S / (phi(q_i)^T z + eps)
 //
@@ -12,8 +13,9 @@
 //
 // nc_state_kernel — one CTA per (group of 4 heads, key segment).  The
 //   4 heads' [128 keys x 32] K and V tiles arrive by TMA (64-byte swizzle, one
-//   slab per head); phi(K) is applied in place (rows past the segment zeroed)
-//   and fp16 V converted to bf16 in place.  With the 4 heads' feature columns
+//   slab per head); phi(K) is applied in place in the input's type (rows past
+//   the segment zeroed), so the MMA reads phi(K) and V as they are (bf16 or
+//   fp16 operands).  With the 4 heads' feature columns
 //   stacked along M (MN-major A, the next head's slab one 32-element block
 //   further), one M=128, N=128 MMA per 16 keys accumulates phi(K_g)^T V_h for
 //   every head pair (g, h) of the group; the diagonal 32 x 32 blocks are the
@@ -83,12 +85,28 @@ struct SCfg {
     static_assert(STAGE % 1024 == 0 && OFF_ONES % 16 == 0, "layout");
 };
 
-// phi in place on the [4 heads][128 rows][64 B] K tile (rows >= nvalid zeroed),
-// and the V tile converted to bf16 (fp16 inputs).  Thread tw (0..127) takes
+// phi on a packed pair of fp16 values, in fp16: max(x, 0) + 2^(min(x, 0) log2 e)
+// (x + 1 for x > 0, e^x for x <= 0), the exponential on the packed fp16 ex2
+// unit.  The exponent's fp16 rounding (2^-11 relative) moves e^x by under
+// 0.2% for |x| <= 3, below the tolerance of 16-bit inputs.
+__device__ __forceinline__ uint32_t phi_f16x2(uint32_t x2) {
+    constexpr uint32_t kLog2eH2 = 0x3DC53DC5u;   // log2(e) rounded to fp16, twice
+    uint32_t m, p, e, r;
+    asm("min.f16x2 %0, %1, %2;" : "=r"(m) : "r"(x2), "r"(0u));
+    asm("max.f16x2 %0, %1, %2;" : "=r"(p) : "r"(x2), "r"(0u));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(m) : "r"(m), "r"(kLog2eH2));
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(m));
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(p), "r"(e));
+    return r;
+}
+
+// phi in place on the [4 heads][128 rows][64 B] K tile (rows >= nvalid
+// zeroed), in the input's own 16-bit type: the state MMA then reads phi(K)
+// and V as they are (bf16 x bf16 or fp16 x fp16), and V needs no conversion.  Thread tw (0..127) takes
 // the 16-byte chunks u = tw + 128 i: the swizzle only permutes chunks inside
 // a 64-byte row, so chunk u lies in row (u / 4) % 128 whatever its position.
 template <typename InT>
-__device__ __forceinline__ void phi_key_tile(uint8_t *kt, uint8_t *vt, int tw, int nvalid) {
+__device__ __forceinline__ void phi_key_tile(uint8_t *kt, int tw, int nvalid) {
     constexpr int NCH = SCfg::TILE / 16;        // 2048 chunks
     constexpr int PER = NCH / 128;              // 16 per thread
     constexpr int BATCH = 8;
@@ -102,28 +120,12 @@ __device__ __forceinline__ void phi_key_tile(uint8_t *kt, uint8_t *vt, int tw, i
             const int u = tw + 128 * (i0 + i);
             const bool valid = ((u >> 2) & (kRows - 1)) < nvalid;
             uint4 f;
-            if constexpr (std::is_same<InT, bf16>::value) {
+            if constexpr (std::is_same<InT, bf16>::value)
                 f = phi_bf16x8(raw[i]);
-            } else {
-                float x[8];
-                unpack8<InT>(raw[i], x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = phi_fast(x[e]);
-                f = pack8_bf16(x);
-            }
+            else
+                f = make_uint4(phi_f16x2(raw[i].x), phi_f16x2(raw[i].y), phi_f16x2(raw[i].z), phi_f16x2(raw[i].w));
             if (!valid) f = make_uint4(0u, 0u, 0u, 0u);
             reinterpret_cast<uint4 *>(kt)[u] = f;
-        }
-        if constexpr (!std::is_same<InT, bf16>::value) {
-            uint4 rv[BATCH];
-#pragma unroll
-            for (int i = 0; i < BATCH; ++i) rv[i] = reinterpret_cast<const uint4 *>(vt)[tw + 128 * (i0 + i)];
-#pragma unroll
-            for (int i = 0; i < BATCH; ++i) {
-                float y[8];
-                unpack8<InT>(rv[i], y);
-                reinterpret_cast<uint4 *>(vt)[tw + 128 * (i0 + i)] = pack8_bf16(y);
-            }
         }
     }
 }
@@ -158,9 +160,10 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         mbar_init(&bar[G::B_DRAIN], 1);
         fence_mbar_init();
     }
-    {
+    {   // ones operand in the MMA's operand type
+        const uint32_t one2 = std::is_same<InT, f16>::value ? 0x3C003C00u : 0x3F803F80u;   // 1.0 pairs
         uint32_t *ones = reinterpret_cast<uint32_t *>(smem + G::OFF_ONES);
-        for (int i = threadIdx.x; i < G::ONES / 4; i += G::THREADS) ones[i] = 0x3F803F80u;   // bf16 1.0 pairs
+        for (int i = threadIdx.x; i < G::ONES / 4; i += G::THREADS) ones[i] = one2;
         fence_proxy_async_smem();
     }
     if (warp == 1) tmem_alloc(tmem_addr_smem, G::TMEM_COLS);
@@ -202,8 +205,9 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     } else if (warp == 1) {
         // ================= MMA issuer
         if (lane == 0 && !*abort_flag) {
-            constexpr uint32_t ID_S = idesc_bf16(128, 128, true, true);
-            constexpr uint32_t ID_Z = idesc_bf16(128, 16, true, false);
+            constexpr bool F16 = std::is_same<InT, f16>::value;
+            constexpr uint32_t ID_S = F16 ? idesc_f16(128, 128, true, true) : idesc_bf16(128, 128, true, true);
+            constexpr uint32_t ID_Z = F16 ? idesc_f16(128, 16, true, false) : idesc_bf16(128, 16, true, false);
             const uint32_t sb = smem_u32(smem);
             const uint64_t dOnes = sdesc_nosw(sb + G::OFF_ONES, 128, (kRows / 8) * 128);
             bool done = true;
@@ -242,7 +246,7 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const long y0 = j0 + (long)t * kRows;
             const int nvalid = (int)min((long)kRows, j1 - y0);
             uint8_t *kt = smem + G::OFF_KV + s * G::STAGE;
-            phi_key_tile<InT>(kt, kt + G::TILE, tw, nvalid);
+            phi_key_tile<InT>(kt, tw, nvalid);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
@@ -499,26 +503,68 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 // first tile writes it as the state output
                 const bool owner = t == 0 && p.state_out_S != nullptr;
                 uint8_t *bhi = smem + G::OFF_B, *blo = smem + G::OFF_B + G::BOP;
-                for (int e = et; e < kE; e += 128) {
-                    float acc = 0.f;
-                    if (p.n_seg == 0) {
-                        if (p.state_in_S)
-                            acc = e < kD * kD ? p.state_in_S[(size_t)bh * kD * kD + e]
-                                              : p.state_in_z[(size_t)bh * kD + (e - kD * kD)];
-                    } else {
-                        const float *src = p.ws_state + (size_t)bh * p.n_seg * kE + e;
-                        for (int s = 0; s < p.n_seg; ++s) acc += src[(size_t)s * kE];
+                // thread et sums float4 groups g = et, et + 128, et + 256 (< kE / 4)
+                // of the state; every load of a batch of segments is issued
+                // before any is used, so a head costs a few memory round trips
+                constexpr int NG = kE / 4;              // 264 groups of 4 floats
+                constexpr int GPT = (NG + 127) / 128;   // 3 per thread
+                constexpr int SB = 2;                   // segments per batch
+                float4 acc[GPT];
+#pragma unroll
+                for (int m = 0; m < GPT; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (p.n_seg == 0) {
+                    if (p.state_in_S) {
+#pragma unroll
+                        for (int m = 0; m < GPT; ++m) {
+                            const int g = et + 128 * m;
+                            if (g < kD * kD / 4)
+                                acc[m] = reinterpret_cast<const float4 *>(p.state_in_S + (size_t)bh * kD * kD)[g];
+                            else if (g < NG)
+                                acc[m] = reinterpret_cast<const float4 *>(p.state_in_z + (size_t)bh * kD)[g - kD * kD / 4];
+                        }
                     }
+                } else {
+                    const float4 *src = reinterpret_cast<const float4 *>(p.ws_state + (size_t)bh * p.n_seg * kE);
+                    for (int s0 = 0; s0 < p.n_seg; s0 += SB) {
+                        float4 x[SB][GPT];
+#pragma unroll
+                        for (int j = 0; j < SB; ++j)
+#pragma unroll
+                            for (int m = 0; m < GPT; ++m) {
+                                const int g = et + 128 * m;
+                                x[j][m] = (s0 + j < p.n_seg && g < NG) ? src[(size_t)(s0 + j) * NG + g]
+                                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                            }
+#pragma unroll
+                        for (int j = 0; j < SB; ++j)
+#pragma unroll
+                            for (int m = 0; m < GPT; ++m) {
+                                acc[m].x += x[j][m].x;
+                                acc[m].y += x[j][m].y;
+                                acc[m].z += x[j][m].z;
+                                acc[m].w += x[j][m].w;
+                            }
+                    }
+                }
+#pragma unroll
+                for (int m = 0; m < GPT; ++m) {
+                    const int g = et + 128 * m;
+                    if (g >= NG) continue;
                     if (owner) {
-                        if (e < kD * kD) p.state_out_S[(size_t)bh * kD * kD + e] = acc;
-                        else p.state_out_z[(size_t)bh * kD + (e - kD * kD)] = acc;
+                        if (g < kD * kD / 4) reinterpret_cast<float4 *>(p.state_out_S + (size_t)bh * kD * kD)[g] = acc[m];
+                        else reinterpret_cast<float4 *>(p.state_out_z + (size_t)bh * kD)[g - kD * kD / 4] = acc[m];
                     }
-                    // S[k][nn] -> element (nn, k); z[k] -> element (32, k)
-                    const int nn = e < kD * kD ? e % kD : kD;
-                    const int k = e < kD * kD ? e / kD : e - kD * kD;
-                    const bf16 hi = __float2bfloat16_rn(acc);
-                    *reinterpret_cast<bf16 *>(bhi + bop_off(nn, k)) = hi;
-                    *reinterpret_cast<bf16 *>(blo + bop_off(nn, k)) = __float2bfloat16_rn(acc - __bfloat162float(hi));
+                    const float v4[4] = {acc[m].x, acc[m].y, acc[m].z, acc[m].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        // S[k][nn] -> element (nn, k); z[k] -> element (32, k)
+                        const int e = 4 * g + j;
+                        const int nn = e < kD * kD ? e % kD : kD;
+                        const int k = e < kD * kD ? e / kD : e - kD * kD;
+                        const bf16 hi = __float2bfloat16_rn(v4[j]);
+                        *reinterpret_cast<bf16 *>(bhi + bop_off(nn, k)) = hi;
+                        *reinterpret_cast<bf16 *>(blo + bop_off(nn, k)) = __float2bfloat16_rn(v4[j] - __bfloat162float(hi));
+                    }
                 }
                 // each warp's writes are complete and visible to the tensor core
                 // before its arrival; the MMA waits for all four

@@ -188,7 +188,8 @@ def test_sharded_prefill_kernels_emulated_ranks(la, orc, dtype, d, chunk, shards
     # the decay products
     if a is not None:
         for i, (lo, hi) in enumerate(zip(bounds[:-1], bounds[1:])):
+            # products of ~900 decays of ~0.88 underflow fp32 to 0 (the exact ones are ~1e-60)
             np.testing.assert_allclose(A_all[i].cpu().numpy(), np.prod(a[:, :, lo:hi].double().numpy(), axis=-1),
-                                       rtol=1e-4)
+                                       rtol=1e-4, atol=1e-37)
     else:
         assert torch.all(A_all == 1)
