@@ -12,7 +12,7 @@
 // Two kernels, chained by programmatic dependent launch:
 //
 // nc_state_kernel — one CTA per (group of 4 heads, key segment).  The
-//   4 heads' [128 keys x 32] K and V tiles arrive by TMA (64-byte swizzle, one
+//   4 heads' [64 keys x 32] K and V tiles arrive by TMA (4 stages) (64-byte swizzle, one
 //   slab per head); phi(K) is applied in place in the input's type (rows past
 //   the segment zeroed), so the MMA reads phi(K) and V as they are (bf16 or
 //   fp16 operands).  With the 4 heads' feature columns
@@ -31,9 +31,10 @@
 //   epilogue warps sum the head's partials in a fixed order (deterministic)
 //   and write S and z as a bf16 hi + lo pair of K-major operands [48][32]
 //   (rows 0-31 the columns of S, row 32 z, the rest 0), so the read-out keeps
-//   about 16 mantissa bits of the state.  Per tile: phi(Q) rows go to TMEM as
-//   the A operand (one thread per query row), four M=128, N=48, K=16 MMAs
-//   form [phi(q) S | phi(q) z] in TMEM, and the epilogue divides, stages the
+//   about 16 mantissa bits of the state.  Per tile: phi(Q) is formed in place
+//   in the query tile (one thread per query row), which then serves as the
+//   K-major A operand; four M=128, N=48, K=16 MMAs form [phi(q) S | phi(q) z]
+//   in one of four TMEM accumulators, and the epilogue divides, stages the
 //   rows swizzled and stores them by TMA (rows past Lq clipped).
 //
 // Every wait is bounded (tc_ptx.cuh); on expiry the CTA raises the call's
@@ -52,7 +53,8 @@ using namespace la::tc;
 
 constexpr int kD = 32;               // head dimension of these kernels
 constexpr int kHP = 4;               // heads per state CTA: M = 4 x 32 = 128
-constexpr int kRows = 128;           // keys per state tile, queries per read-out tile
+constexpr int kRows = 128;           // queries per read-out tile
+constexpr int kSRows = 64;           // keys per state tile
 constexpr int kRowBytes = kD * 2;    // one 16-bit row of 32 features
 constexpr int kE = kD * kD + kD;     // floats of one (S, z) state
 
@@ -63,17 +65,17 @@ struct NcStateParams {
     const float *state_in_z;         // [BH][32]
     int *status;                     // the call's status word [2]
     unsigned long long wait_ns;
-    int BH, Lk, seg_len, n_seg;      // seg_len: a multiple of kRows
+    int BH, Lk, seg_len, n_seg;      // seg_len: a multiple of kSRows
 };
 
 struct SCfg {
-    static constexpr int HEAD_TILE = kRows * kRowBytes;   // 8 KB: one head's [128][32] tile
-    static constexpr int TILE = kHP * HEAD_TILE;          // 32 KB: the group's 4 slabs
+    static constexpr int HEAD_TILE = kSRows * kRowBytes;  // 4 KB: one head's [64][32] tile
+    static constexpr int TILE = kHP * HEAD_TILE;          // 16 KB: the group's 4 slabs
     static constexpr int STAGE = 2 * TILE;                // K, then V
-    static constexpr int NST = 2;
+    static constexpr int NST = 4;                         // 128 KB of keys and values in flight
     static constexpr int OFF_KV = 0;
-    static constexpr int OFF_ONES = NST * STAGE;          // ones operand [16][128] bf16
-    static constexpr int ONES = 16 * kRows * 2;
+    static constexpr int OFF_ONES = NST * STAGE;          // ones operand [16][64]
+    static constexpr int ONES = 16 * kSRows * 2;
     static constexpr int OFF_BAR = OFF_ONES + ONES;
     static constexpr int B_FULL = 0, B_EMPTY = NST, B_PHI = 2 * NST, B_DONE = 3 * NST, B_DRAIN = B_DONE + 1;
     static constexpr int NBAR = B_DRAIN + 1;
@@ -82,7 +84,7 @@ struct SCfg {
     static constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;   // + alignment slack
     static constexpr int T_S = 0, T_Z = 128, TMEM_COLS = 256;
     static constexpr int THREADS = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 phi and epilogue
-    static_assert(STAGE % 1024 == 0 && OFF_ONES % 16 == 0, "layout");
+    static_assert(STAGE % 1024 == 0 && HEAD_TILE % 512 == 0 && OFF_ONES % 16 == 0, "layout");
 };
 
 // phi on a packed pair of fp16 values, in fp16: max(x, 0) + 2^(min(x, 0) log2 e)
@@ -100,15 +102,15 @@ __device__ __forceinline__ uint32_t phi_f16x2(uint32_t x2) {
     return r;
 }
 
-// phi in place on the [4 heads][128 rows][64 B] K tile (rows >= nvalid
+// phi in place on the [4 heads][64 rows][64 B] K tile (rows >= nvalid
 // zeroed), in the input's own 16-bit type: the state MMA then reads phi(K)
 // and V as they are (bf16 x bf16 or fp16 x fp16), and V needs no conversion.  Thread tw (0..127) takes
 // the 16-byte chunks u = tw + 128 i: the swizzle only permutes chunks inside
-// a 64-byte row, so chunk u lies in row (u / 4) % 128 whatever its position.
+// a 64-byte row, so chunk u lies in row (u / 4) % 64 whatever its position.
 template <typename InT>
 __device__ __forceinline__ void phi_key_tile(uint8_t *kt, int tw, int nvalid) {
-    constexpr int NCH = SCfg::TILE / 16;        // 2048 chunks
-    constexpr int PER = NCH / 128;              // 16 per thread
+    constexpr int NCH = SCfg::TILE / 16;        // 1024 chunks
+    constexpr int PER = NCH / 128;              // 8 per thread
     constexpr int BATCH = 8;
 #pragma unroll 1
     for (int i0 = 0; i0 < PER; i0 += BATCH) {
@@ -118,7 +120,7 @@ __device__ __forceinline__ void phi_key_tile(uint8_t *kt, int tw, int nvalid) {
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
             const int u = tw + 128 * (i0 + i);
-            const bool valid = ((u >> 2) & (kRows - 1)) < nvalid;
+            const bool valid = ((u >> 2) & (kSRows - 1)) < nvalid;
             uint4 f;
             if constexpr (std::is_same<InT, bf16>::value)
                 f = phi_bf16x8(raw[i]);
@@ -147,7 +149,7 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int seg = blockIdx.x, grp = blockIdx.y;
     const long j0 = (long)seg * p.seg_len;
     const long j1 = min((long)p.Lk, j0 + p.seg_len);
-    const int ntiles = (int)((j1 - j0 + kRows - 1) / kRows);
+    const int ntiles = (int)((j1 - j0 + kSRows - 1) / kSRows);
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -190,7 +192,7 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 if (use > 0 && !mbar_wait(&bar[G::B_EMPTY + s], (use - 1) & 1, ab, 1)) break;
                 uint8_t *kd = smem + G::OFF_KV + s * G::STAGE;
                 mbar_expect_tx(&bar[G::B_FULL + s], 2 * G::TILE);
-                const int y = (int)(j0 + (long)t * kRows), z = grp * kHP;
+                const int y = (int)(j0 + (long)t * kSRows), z = grp * kHP;
                 tma_load_3d(kd, &tm_k, &bar[G::B_FULL + s], 0, y, z);
                 tma_load_3d(kd + G::TILE, &tm_v, &bar[G::B_FULL + s], 0, y, z);
                 issued[s] = use + 1;
@@ -209,7 +211,7 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             constexpr uint32_t ID_S = F16 ? idesc_f16(128, 128, true, true) : idesc_bf16(128, 128, true, true);
             constexpr uint32_t ID_Z = F16 ? idesc_f16(128, 16, true, false) : idesc_bf16(128, 16, true, false);
             const uint32_t sb = smem_u32(smem);
-            const uint64_t dOnes = sdesc_nosw(sb + G::OFF_ONES, 128, (kRows / 8) * 128);
+            const uint64_t dOnes = sdesc_nosw(sb + G::OFF_ONES, 128, (kSRows / 8) * 128);
             bool done = true;
             for (int t = 0; t < ntiles; ++t) {
                 const int s = t % G::NST;
@@ -221,11 +223,11 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const uint64_t dK = sdesc_sw64(kt, G::HEAD_TILE, 512);
                 const uint64_t dV = sdesc_sw64(kt + G::TILE, G::HEAD_TILE, 512);
 #pragma unroll
-                for (int kk = 0; kk < kRows / 16; ++kk)
+                for (int kk = 0; kk < kSRows / 16; ++kk)
                     mma_ss(tmem + G::T_S, dK + (uint64_t)((kk * 1024) >> 4), dV + (uint64_t)((kk * 1024) >> 4), ID_S,
                            (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < kRows / 16; ++kk)
+                for (int kk = 0; kk < kSRows / 16; ++kk)
                     mma_ss(tmem + G::T_Z, dK + (uint64_t)((kk * 1024) >> 4), dOnes + (uint64_t)((kk * 256) >> 4), ID_Z,
                            (t > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bar[G::B_EMPTY + s]);
@@ -243,8 +245,8 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int t = 0; t < ntiles; ++t) {
             const int s = t % G::NST;
             if (!mbar_wait(&bar[G::B_FULL + s], (t / G::NST) & 1, ab, 4)) { ok = false; break; }
-            const long y0 = j0 + (long)t * kRows;
-            const int nvalid = (int)min((long)kRows, j1 - y0);
+            const long y0 = j0 + (long)t * kSRows;
+            const int nvalid = (int)min((long)kSRows, j1 - y0);
             uint8_t *kt = smem + G::OFF_KV + s * G::STAGE;
             phi_key_tile<InT>(kt, tw, nvalid);
             fence_proxy_async_smem();
@@ -305,8 +307,9 @@ struct NcReadParams {
 };
 
 template <typename OutT> struct RCfg {
-    static constexpr int QT = kRows * kRowBytes;            // 8 KB query tile
-    static constexpr int NQ = 6;
+    static constexpr int QT = kRows * kRowBytes;            // 8 KB query tile (phi(Q) in place: the A operand)
+    static constexpr int NQ = 6;                            // query tiles in flight
+    static constexpr int ND = 4;                            // TMEM accumulators [128 x 48] in flight
     static constexpr int OFF_Q = 0;
     static constexpr int STG_WARP = 4096;                   // one warp's 32 output rows (<= 128 B each)
     static constexpr int OFF_STG = NQ * QT;                 // 2 buffers x 4 warps
@@ -314,16 +317,15 @@ template <typename OutT> struct RCfg {
     static constexpr int BN = 48;                           // B operand rows: 32 of S, 1 of z, 15 zero
     static constexpr int BOP = BN * kD * 2;                 // 3 KB
     static constexpr int OFF_BAR = OFF_B + 2 * BOP;         // hi, lo
-    static constexpr int B_QFULL = 0, B_QEMPTY = NQ, B_AFULL = 2 * NQ, B_AEMPTY = B_AFULL + 2,
-                         B_DFULL = B_AEMPTY + 2, B_DEMPTY = B_DFULL + 2, B_BREADY = B_DEMPTY + 2,
-                         B_DRAIN = B_BREADY + 1, NBAR = B_DRAIN + 1;
+    static constexpr int B_QFULL = 0, B_PHI = NQ, B_QEMPTY = 2 * NQ, B_DFULL = 3 * NQ, B_DEMPTY = B_DFULL + ND,
+                         B_BREADY = B_DEMPTY + ND, B_DRAIN = B_BREADY + 1, NBAR = B_DRAIN + 1;
     static constexpr int OFF_TMEMADDR = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEMADDR + 4;
     static constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;
-    static constexpr int T_D0 = 0, T_D1 = 64, T_A0 = 128, T_A1 = 160, TMEM_COLS = 256;
+    static constexpr int T_DSTRIDE = 64, TMEM_COLS = 256;   // accumulator a at columns 64 a .. 64 a + 47
     static constexpr int THREADS = 320;   // warp 0 TMA, 1 MMA, 2-5 phi(Q), 6-9 epilogue
     static constexpr int ROWB = kD * (int)sizeof(OutT);     // output row bytes: 128 (fp32) or 64
-    static_assert(OFF_STG % 1024 == 0 && OFF_B % 16 == 0, "layout");
+    static_assert(OFF_STG % 1024 == 0 && OFF_B % 16 == 0 && ND * T_DSTRIDE <= TMEM_COLS, "layout");
 };
 
 // Byte offset of element (n, k) of a K-major no-swizzle [48][32] operand:
@@ -364,13 +366,12 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         *abort_flag = 0;
         for (int s = 0; s < G::NQ; ++s) {
             mbar_init(&bar[G::B_QFULL + s], 1);
-            mbar_init(&bar[G::B_QEMPTY + s], 4);
+            mbar_init(&bar[G::B_PHI + s], 4);
+            mbar_init(&bar[G::B_QEMPTY + s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar[G::B_AFULL + s], 4);
-            mbar_init(&bar[G::B_AEMPTY + s], 1);
-            mbar_init(&bar[G::B_DFULL + s], 1);
-            mbar_init(&bar[G::B_DEMPTY + s], 4);
+        for (int a = 0; a < G::ND; ++a) {
+            mbar_init(&bar[G::B_DFULL + a], 1);
+            mbar_init(&bar[G::B_DEMPTY + a], 4);
         }
         mbar_init(&bar[G::B_BREADY], 4);
         mbar_init(&bar[G::B_DRAIN], 1);
@@ -420,24 +421,28 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint64_t dBlo = sdesc_nosw(sb + G::OFF_B + G::BOP, 128, 512);
             int cur = -1, hc = -1;
             for (int i = 0; i < n; ++i) {
-                const int a = i & 1;
+                const int s = i % G::NQ, a = i % G::ND;
                 const int bh = (int)((f0 + i) / tph);
-                if (!mbar_wait(&bar[G::B_AFULL + a], (i >> 1) & 1, ab, 2)) break;
-                if (i >= 2 && !mbar_wait(&bar[G::B_DEMPTY + a], ((i >> 1) - 1) & 1, ab, 3)) break;
+                if (!mbar_wait(&bar[G::B_PHI + s], (i / G::NQ) & 1, ab, 2)) break;
+                if (i >= G::ND && !mbar_wait(&bar[G::B_DEMPTY + a], ((i / G::ND) - 1) & 1, ab, 3)) break;
                 if (bh != cur) {
                     cur = bh;
                     ++hc;
                     if (!mbar_wait(&bar[G::B_BREADY], hc & 1, ab, 4)) break;
                 }
                 tc_fence_after();
-                const uint32_t d = tmem + (a ? G::T_D1 : G::T_D0), at = tmem + (a ? G::T_A1 : G::T_A0);
+                // A = phi(Q) in place in the query stage: K-major, 64-byte swizzle,
+                // 8-row groups 512 bytes apart; a K step of 16 is 32 bytes
+                const uint64_t dA = sdesc_sw64(sb + G::OFF_Q + s * G::QT, 16, 512);
+                const uint32_t d = tmem + a * G::T_DSTRIDE;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    mma_ts(d, at + kk * 8, dBhi + (uint64_t)((kk * 256) >> 4), ID, kk > 0 ? 1u : 0u);
-                    mma_ts(d, at + kk * 8, dBlo + (uint64_t)((kk * 256) >> 4), ID, 1u);
+                    mma_ss(d, dA + (uint64_t)((kk * 32) >> 4), dBhi + (uint64_t)((kk * 256) >> 4), ID,
+                           kk > 0 ? 1u : 0u);
+                    mma_ss(d, dA + (uint64_t)((kk * 32) >> 4), dBlo + (uint64_t)((kk * 256) >> 4), ID, 1u);
                 }
                 mma_commit(&bar[G::B_DFULL + a]);
-                mma_commit(&bar[G::B_AEMPTY + a]);
+                mma_commit(&bar[G::B_QEMPTY + s]);   // the query stage may be reloaded
             }
             volatile int never = 0;
             AbortCtx timed{&never, nullptr, kDrainLimitNs};
@@ -445,42 +450,33 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_wait(&bar[G::B_DRAIN], 0, timed, 0);
         }
     } else if (warp < 6) {
-        // ================= phi(Q) into TMEM (warps 2-5, one thread per query row)
+        // ================= phi(Q) in place (warps 2-5, one thread per query row)
         const int q = warp & 3, r = q * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         for (int i = 0; i < n; ++i) {
-            const int s = i % G::NQ, a = i & 1;
+            const int s = i % G::NQ;
             if (!mbar_wait(&bar[G::B_QFULL + s], (i / G::NQ) & 1, ab, 5)) break;
-            const uint8_t *qs = smem + G::OFF_Q + s * G::QT;
+            uint8_t *qs = smem + G::OFF_Q + s * G::QT;
             uint4 raw[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 raw[c] = *reinterpret_cast<const uint4 *>(qs + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[G::B_QEMPTY + s]);
-            uint32_t packed[16];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
+                uint4 f;
                 if constexpr (std::is_same<InT, bf16>::value) {
-                    const uint4 f = phi_bf16x8(raw[c]);
-                    packed[4 * c + 0] = f.x;
-                    packed[4 * c + 1] = f.y;
-                    packed[4 * c + 2] = f.z;
-                    packed[4 * c + 3] = f.w;
+                    f = phi_bf16x8(raw[c]);
                 } else {
                     float x[8];
                     unpack8<InT>(raw[c], x);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) packed[4 * c + e] = pack_bf16x2(phi_fast(x[2 * e]), phi_fast(x[2 * e + 1]));
+                    for (int e = 0; e < 8; ++e) x[e] = phi_fast(x[e]);
+                    f = pack8_bf16(x);
                 }
+                *reinterpret_cast<uint4 *>(qs + r * 64 + ((c ^ ((r >> 1) & 3)) << 4)) = f;
             }
-            if (i >= 2 && !mbar_wait(&bar[G::B_AEMPTY + a], ((i >> 1) - 1) & 1, ab, 6)) break;
-            tc_fence_after();
-            tmem_st16(tmem + lane_base + (a ? G::T_A1 : G::T_A0), packed);
-            tmem_st_wait();
-            tc_fence_before();
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[G::B_AFULL + a]);
+            if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
         }
     } else {
         // ================= epilogue (warps 6-9): head state -> B operands, output
@@ -489,7 +485,7 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         bool waited = false;
         int cur = -1;
         for (int i = 0; i < n; ++i) {
-            const int a = i & 1;
+            const int a = i % G::ND;
             const long f = f0 + i;
             const int bh = (int)(f / tph), t = (int)(f % tph);
             if (bh != cur) {
@@ -572,10 +568,10 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar[G::B_BREADY]);
             }
-            if (!mbar_wait(&bar[G::B_DFULL + a], (i >> 1) & 1, ab, 7)) break;
+            if (!mbar_wait(&bar[G::B_DFULL + a], (i / G::ND) & 1, ab, 7)) break;
             tc_fence_after();
             uint32_t u[32], ud;
-            const uint32_t d = tmem + lane_base + (a ? G::T_D1 : G::T_D0);
+            const uint32_t d = tmem + lane_base + a * G::T_DSTRIDE;
             tmem_ld32(d, u);
             tmem_ld1(d + kD, ud);
             tmem_ld_wait();
@@ -583,7 +579,7 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_DEMPTY + a]);
             const float inv = 1.f / (__uint_as_float(ud) + p.eps);
-            uint8_t *stg = smem + G::OFF_STG + (a * 4 + (warp - 6)) * G::STG_WARP;
+            uint8_t *stg = smem + G::OFF_STG + ((i & 1) * 4 + (warp - 6)) * G::STG_WARP;
             // this warp's store of two tiles ago must have read its staging rows
             if (lane == 0) bulk_wait_read1();
             __syncwarp();

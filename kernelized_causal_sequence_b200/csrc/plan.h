@@ -70,19 +70,20 @@ inline Plan make_nc_plan(long BH, long Lk, int D) {
 }
 
 // Key segments of the tensor-core non-causal form (head dimension 32): one
-// CTA per (group of 4 heads, segment of whole 128-key tiles), the segment
+// CTA per (group of 4 heads, segment of whole 64-key tiles), the segment
 // count chosen so that all CTAs fit in one wave on the SMs.
 constexpr int kNcTcHeads = 4;
+constexpr int kNcTcKeyTile = 64;
 inline Plan make_nc_tc_plan(long BH, long Lk) {
     Plan p;
-    p.chunk = kNc32TileRows;
+    p.chunk = kNcTcKeyTile;
     const long groups = (BH + kNcTcHeads - 1) / kNcTcHeads;
-    const long tiles = Lk > 0 ? (Lk + kNc32TileRows - 1) / kNc32TileRows : 1;
+    const long tiles = Lk > 0 ? (Lk + kNcTcKeyTile - 1) / kNcTcKeyTile : 1;
     long segs = kNumSMs / (groups > 0 ? groups : 1);
     if (segs < 1) segs = 1;
     if (segs > tiles) segs = tiles;
     const long per = (tiles + segs - 1) / segs;
-    p.seg_len = (int)(per * kNc32TileRows);
+    p.seg_len = (int)(per * kNcTcKeyTile);
     p.n_seg = (int)((tiles + per - 1) / per);
     return p;
 }

@@ -193,8 +193,8 @@ la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
     la_status s = LA_OK;
     if (keys) {
         CUtensorMap mk, mv;
-        if (!make_map_box(&mk, a.k, a.in_dtype, a.BH, a.Lk, kD, kRows, kHP, CU_TENSOR_MAP_SWIZZLE_64B) ||
-            !make_map_box(&mv, a.v, a.in_dtype, a.BH, a.Lk, kD, kRows, kHP, CU_TENSOR_MAP_SWIZZLE_64B))
+        if (!make_map_box(&mk, a.k, a.in_dtype, a.BH, a.Lk, kD, kSRows, kHP, CU_TENSOR_MAP_SWIZZLE_64B) ||
+            !make_map_box(&mv, a.v, a.in_dtype, a.BH, a.Lk, kD, kSRows, kHP, CU_TENSOR_MAP_SWIZZLE_64B))
             return cuda_fail_msg("cuTensorMapEncodeTiled", "tensor map encoding failed");
         NcStateParams sp;
         sp.ws_state = a.ws_state;

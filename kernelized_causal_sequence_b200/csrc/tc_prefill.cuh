@@ -785,6 +785,72 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const uint64_t dVm = sdesc_sw128(kt + G::TILE, G::BOXB, 1024);         // V, MN-major
                 if (!mbar_wait(&bar[G::B_PHI + s], (c / G::NKV) & 1, ab, 3)) break;
                 tc_fence_after();
+                if constexpr (G::OUT && !DECAY) {
+                    // No decay: the state update (MMA3, MMAz) is issued right after
+                    // the scores, ahead of the inter term, so it runs while the
+                    // previous chunk's output is still being read out of the O
+                    // accumulator.  The state epilogue then waits for MMA2/MMAd as
+                    // well (DS_FULL is committed after them): it rewrites the
+                    // operands they read.
+                    const uint64_t dQk = sdesc_sw128(sb + G::OFF_Q + (G::QT ? 0 : (c & 1)) * G::TILE, 16, 1024);
+                    // MMA1: scores = phi(Q) phi(K)^T (scores buffer free once MMA4 of c-1 is done)
+                    if (c > 0 && !mbar_wait(&bar[G::B_MMA4], (c - 1) & 1, ab, 4)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t koff = ((kk >> 2) * G::BOXB + (kk & 3) * 32) >> 4;
+                        if constexpr (G::QT)
+                            mma_ts(tmem + G::T_SC, tmem + G::T_Q + kk * 8, dKk + koff, ID_SC, kk > 0);
+                        else
+                            mma_ss(tmem + G::T_SC, dQk + koff, dKk + koff, ID_SC, kk > 0);
+                    }
+                    mma_commit(&bar[G::B_SC_FULL]);
+                    // MMA3 + MMAz: the state epilogue of c-1 has read the accumulators
+                    if (!mbar_wait(&bar[G::B_S_READY], c & 1, ab, 5)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        mma_ss(tmem + G::T_S, dKm + (uint64_t)((kk * 2048) >> 4),
+                               dVm + (uint64_t)((kk * 2048) >> 4), ID_DS, 1);
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        mma_ss(tmem + G::T_Z, dKm + (uint64_t)((kk * 2048) >> 4),
+                               dOnes + (uint64_t)((kk * 256) >> 4), ID_Z, 1);
+                    // MMA2 + MMAd: O is free once the output of c-1 has been read
+                    if (c > 0 && !mbar_wait(&bar[G::B_O_EMPTY], (c - 1) & 1, ab, 6)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t bS = dS0 + (uint64_t)((kk * 2048) >> 4);
+                        const uint64_t bZ = dZ0 + (uint64_t)((kk * 256) >> 4);
+                        if constexpr (G::QT) {
+                            mma_ts(tmem + G::T_O, tmem + G::T_Q + kk * 8, bS, ID_INT, kk > 0);
+                            mma_ts(tmem + G::T_DEN, tmem + G::T_Q + kk * 8, bZ, ID_DEN, kk > 0);
+                        } else {
+                            const uint64_t aQ = dQk + (uint64_t)(((kk >> 2) * G::BOXB + (kk & 3) * 32) >> 4);
+                            mma_ss(tmem + G::T_O, aQ, bS, ID_INT, kk > 0);
+                            mma_ss(tmem + G::T_DEN, aQ, bZ, ID_DEN, kk > 0);
+                        }
+                    }
+                    if constexpr (G::QT) mma_commit(&bar[G::B_QT_EMPTY]);
+                    else mma_commit(&bar[G::B_Q_EMPTY + (c & 1)]);
+                    mma_commit(&bar[G::B_DS_FULL]);
+                    // MMA4: exact intra-chunk product with the masked scores
+                    if (!mbar_wait(&bar[G::B_P_READY], c & 1, ab, 7)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk) {
+                        const uint64_t bV = dVm + (uint64_t)((kk * 2048) >> 4);
+                        if constexpr (G::PT)
+                            mma_ts(tmem + G::T_O, tmem + G::T_SC + kk * 8, bV, ID_PV, 1u);
+                        else
+                            mma_ss(tmem + G::T_O, dP0 + (uint64_t)((kk * 32) >> 4), bV, ID_PV, 1u);
+                    }
+                    mma_commit(&bar[G::B_MMA4]);
+                    mma_commit(&bar[G::B_O_FULL]);
+                    mma_commit(&bar[G::B_KV_EMPTY + s]);
+                    continue;
+                }
                 if constexpr (G::OUT) {
                     const uint64_t dQk = sdesc_sw128(sb + G::OFF_Q + (G::QT ? 0 : (c & 1)) * G::TILE, 16, 1024);
                     // MMA1: scores = phi(Q) phi(K)^T (scores buffer free once MMA4 of c-1 is done)
