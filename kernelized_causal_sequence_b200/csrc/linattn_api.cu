@@ -36,6 +36,9 @@ struct WsLayout {
     size_t status_off, state_off, A_off, total_off, bytes;
 };
 
+// (non-causal: the totals region also holds, at head dim 32, the tensor-core
+// read-out's operand images of 6144 bytes per head)
+constexpr size_t kBimgBytes = 6144;
 WsLayout ws_layout(long BH, int n_seg, int D, bool with_total) {
     WsLayout w;
     const size_t E = (size_t)D * D + D;
@@ -43,7 +46,9 @@ WsLayout ws_layout(long BH, int n_seg, int D, bool with_total) {
     w.state_off = kAlign;
     w.A_off = align_up(w.state_off + sizeof(float) * (size_t)BH * n_seg * E);
     w.total_off = align_up(w.A_off + sizeof(float) * (size_t)BH * n_seg);
-    w.bytes = with_total ? align_up(w.total_off + sizeof(float) * (size_t)BH * E) : w.total_off;
+    size_t per_head = sizeof(float) * E;
+    if (D == 32 && per_head < kBimgBytes) per_head = kBimgBytes;
+    w.bytes = with_total ? align_up(w.total_off + per_head * (size_t)BH) : w.total_off;
     return w;
 }
 
@@ -515,6 +520,7 @@ la_status la_forward_noncausal(const void *q, const void *k, const void *v, la_d
         a.ws_state = (float *)(ws + wl.state_off);
         a.ws_A = (float *)(ws + wl.A_off);
         a.ws_total = (float *)(ws + wl.total_off);
+        a.ws_bimg = (uint8_t *)(ws + wl.total_off);
         a.status = (int *)(ws + wl.status_off);
         a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
         a.state_S = state_S; a.state_z = state_z; a.mode = mode;

@@ -11,31 +11,34 @@
 //
 // Two kernels, chained by programmatic dependent launch:
 //
-// nc_state_kernel — one CTA per (group of 4 heads, key segment).  The
-//   4 heads' [64 keys x 32] K and V tiles arrive by TMA (4 stages) (64-byte swizzle, one
-//   slab per head); phi(K) is applied in place in the input's type (rows past
-//   the segment zeroed), so the MMA reads phi(K) and V as they are (bf16 or
-//   fp16 operands).  With the 4 heads' feature columns
+// nc_state_kernel — one CTA per (group of 4 heads, key segment); the
+//   segments of a group (at most 8) form one thread-block cluster.  The 4
+//   heads' [64 keys x 32] K and V tiles arrive by TMA (4 stages; 64-byte
+//   swizzle, one slab per head); phi(K) is applied in place in the input's
+//   type (rows past the segment zeroed), so the MMA reads phi(K) and V as
+//   they are (bf16 or fp16 operands).  With the 4 heads' feature columns
 //   stacked along M (MN-major A, the next head's slab one 32-element block
-//   further), one M=128, N=128 MMA per 16 keys accumulates phi(K_g)^T V_h for
-//   every head pair (g, h) of the group; the diagonal 32 x 32 blocks are the
-//   heads' states, the rest is discarded (d = 32 is below the tensor core's
-//   M >= 64, and the extra products are free beside the memory traffic).  A
-//   second MMA against a ones operand gives z.  The CTA writes its partial
-//   (S, z) per head to the workspace.
+//   further), one M=128, N=128 MMA per 16 keys accumulates phi(K_g)^T V_h
+//   for every head pair (g, h) of the group; the diagonal 32 x 32 blocks are
+//   the heads' states, the rest is discarded (d = 32 is below the tensor
+//   core's M >= 64, and the extra products are free beside the memory
+//   traffic).  A second MMA against a ones operand gives z.  Each CTA puts
+//   its partial (S, z) in its shared memory; across the cluster (distributed
+//   shared memory) every CTA sums its share of the elements over all the
+//   group's partials in a fixed order (deterministic), adds the state-in,
+//   writes the state-out and each head's read-out operands: S and z as a
+//   bf16 hi + lo pair of K-major [48][32] images (rows 0-31 the columns of S,
+//   row 32 z), so the read-out keeps about 16 mantissa bits of the state.
 //
 // nc_readout_kernel — a persistent pass over 128-query tiles (every CTA a
 //   contiguous range of (head, tile) pairs).  Its set-up and first query
-//   loads overlap the state kernel; before it reads the partial states it
-//   waits for that grid (griddepcontrol.wait).  At each new head the
-//   epilogue warps sum the head's partials in a fixed order (deterministic)
-//   and write S and z as a bf16 hi + lo pair of K-major operands [48][32]
-//   (rows 0-31 the columns of S, row 32 z, the rest 0), so the read-out keeps
-//   about 16 mantissa bits of the state.  Per tile: phi(Q) is formed in place
-//   in the query tile (one thread per query row), which then serves as the
-//   K-major A operand; four M=128, N=48, K=16 MMAs form [phi(q) S | phi(q) z]
-//   in one of four TMEM accumulators, and the epilogue divides, stages the
-//   rows swizzled and stores them by TMA (rows past Lq clipped).
+//   loads overlap the state kernel; at each new head one bulk copy brings the
+//   head's operand images (6 KB) in, after waiting for the state kernel
+//   (griddepcontrol.wait).  Per tile: phi(Q) is formed in place in the query
+//   tile (one thread per query row), which then serves as the K-major A
+//   operand; four M=128, N=48, K=16 MMAs form [phi(q) S | phi(q) z] in one
+//   of four TMEM accumulators, and the epilogue divides, stages the rows
+//   swizzled and stores them by TMA (rows past Lq clipped).
 //
 // Every wait is bounded (tc_ptx.cuh); on expiry the CTA raises the call's
 // status word (LA_ERR_TIMEOUT), drains its copies and products and exits.
@@ -58,14 +61,26 @@ constexpr int kSRows = 64;           // keys per state tile
 constexpr int kRowBytes = kD * 2;    // one 16-bit row of 32 features
 constexpr int kE = kD * kD + kD;     // floats of one (S, z) state
 
+constexpr int kBN = 48;                       // rows of the read-out's B operand: 32 of S, 1 of z, 15 unused
+constexpr int kBop = kBN * kD * 2;            // bytes of one [48][32] bf16 operand
+constexpr int kBimg = 2 * kBop;               // the hi and lo operands of one head: 6 KB
+
+// Byte offset of element (n, k) of a K-major no-swizzle [48][32] operand:
+// core matrices (8 rows x 8 k) of 128 bytes, 4 along K (128 bytes apart),
+// groups of 8 rows 512 bytes apart.
+__device__ __forceinline__ int bop_off(int n, int k) {
+    return (n >> 3) * 512 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
+}
+
 struct NcStateParams {
-    float *ws_state;                 // [BH][n_seg][kE] partial states
-    float *ws_A;                     // [BH][n_seg] (1: no decay; read by the segment scan)
-    const float *state_in_S;         // [BH][32][32] added to segment 0's partial, or null
+    uint8_t *ws_bimg;                // [BH][kBimg]: each head's total (S, z) as the read-out's B operands
+    const float *state_in_S;         // [BH][32][32] added to the sums, or null
     const float *state_in_z;         // [BH][32]
+    float *state_out_S;              // [BH][32][32] the totals, or null
+    float *state_out_z;              // [BH][32]
     int *status;                     // the call's status word [2]
     unsigned long long wait_ns;
-    int BH, Lk, seg_len, n_seg;      // seg_len: a multiple of kSRows
+    int BH, Lk, seg_len, n_seg;      // seg_len: a multiple of kSRows; n_seg <= 8 (the cluster)
 };
 
 struct SCfg {
@@ -253,36 +268,79 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
         }
+        // the CTA's partial (S, z) of its 4 heads -> its own shared memory
+        // [4][kE] fp32 (in the drained K/V stages); garbage if the CTA gave up
         if (ok && ntiles > 0 && mbar_wait(&bar[G::B_DONE], 0, ab, 5)) {
             tc_fence_after();
             // TMEM lane quarter q = head q of the group; lane = feature a
             const int q = warp & 3, a = lane;
-            const long bh = (long)grp * kHP + q;
             const uint32_t lane_base = (uint32_t)(q * 32) << 16;
             uint32_t u[32], zb;
             tmem_ld32(tmem + lane_base + G::T_S + q * 32, u);   // the diagonal block: S_q[a][0..31]
             tmem_ld1(tmem + lane_base + G::T_Z, zb);
             tmem_ld_wait();
-            if (bh < p.BH && !*abort_flag) {
-                float *dst = p.ws_state + ((size_t)bh * p.n_seg + seg) * kE;
-                float vals[32];
+            float *part = reinterpret_cast<float *>(smem + G::OFF_KV) + q * kE;
+            float4 *d4 = reinterpret_cast<float4 *>(part + a * kD);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) vals[i] = __uint_as_float(u[i]);
-                float zv = __uint_as_float(zb);
-                if (seg == 0 && p.state_in_S) {   // the state-in joins the first segment's partial
+            for (int i = 0; i < 8; ++i)
+                d4[i] = make_float4(__uint_as_float(u[4 * i]), __uint_as_float(u[4 * i + 1]),
+                                    __uint_as_float(u[4 * i + 2]), __uint_as_float(u[4 * i + 3]));
+            part[kD * kD + a] = __uint_as_float(zb);
+        }
+    }
+
+    // ---------------- the group's totals: the cluster is the group's n_seg
+    // CTAs; CTA r sums its share of the 4 heads' elements over every CTA's
+    // partial (distributed shared memory, fixed order), adds the state-in,
+    // writes the state-out and the read-out's B operand images (bf16 hi + lo)
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync();   // every partial is in shared memory
+    {
+        constexpr int NG = kE / 4;                       // 264 float4 groups per head
+        const int ncl = p.n_seg, rank = (int)cluster_ctarank();
+        const int f0 = rank * (kHP * NG) / ncl, f1 = (rank + 1) * (kHP * NG) / ncl;
+        const uint32_t part0 = smem_u32(smem + G::OFF_KV);
+        for (int f = f0 + (int)threadIdx.x; f < f1; f += G::THREADS) {
+            const int h = f / NG, g = f % NG;
+            const long bh = (long)grp * kHP + h;
+            const uint32_t off = part0 + (uint32_t)((h * kE + 4 * g) * 4);
+            float4 x[8];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) vals[i] += p.state_in_S[(size_t)bh * kD * kD + a * kD + i];
-                    zv += p.state_in_z[(size_t)bh * kD + a];
-                }
-                float4 *d4 = reinterpret_cast<float4 *>(dst + a * kD);
+            for (int r = 0; r < 8; ++r) x[r] = r < ncl ? ld_dsmem_f4(mapa_shared(off, r)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (bh < p.BH && p.state_in_S) {
+                acc = g < kD * kD / 4 ? reinterpret_cast<const float4 *>(p.state_in_S + (size_t)bh * kD * kD)[g]
+                                      : reinterpret_cast<const float4 *>(p.state_in_z + (size_t)bh * kD)[g - kD * kD / 4];
+            }
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    d4[i] = make_float4(vals[4 * i], vals[4 * i + 1], vals[4 * i + 2], vals[4 * i + 3]);
-                dst[kD * kD + a] = zv;
-                if (lane == 0) p.ws_A[(size_t)bh * p.n_seg + seg] = 1.f;
+            for (int r = 0; r < 8; ++r) {
+                acc.x += x[r].x;
+                acc.y += x[r].y;
+                acc.z += x[r].z;
+                acc.w += x[r].w;
+            }
+            if (bh >= p.BH || *abort_flag) continue;
+            if (p.state_out_S) {
+                if (g < kD * kD / 4) reinterpret_cast<float4 *>(p.state_out_S + (size_t)bh * kD * kD)[g] = acc;
+                else reinterpret_cast<float4 *>(p.state_out_z + (size_t)bh * kD)[g - kD * kD / 4] = acc;
+            }
+            uint8_t *img = p.ws_bimg + (size_t)bh * kBimg;
+            const float v4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                // S[k][nn] -> element (nn, k); z[k] -> element (32, k)
+                const int e = 4 * g + j;
+                const int nn = e < kD * kD ? e % kD : kD;
+                const int k = e < kD * kD ? e / kD : e - kD * kD;
+                const bf16 hi = __float2bfloat16_rn(v4[j]);
+                *reinterpret_cast<bf16 *>(img + bop_off(nn, k)) = hi;
+                *reinterpret_cast<bf16 *>(img + kBop + bop_off(nn, k)) = __float2bfloat16_rn(v4[j] - __bfloat162float(hi));
             }
         }
     }
+    __syncwarp();
+    cluster_sync();   // no CTA leaves while another reads its shared memory
 
     tc_fence_before();
     __syncthreads();
@@ -294,10 +352,11 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 // --------------------------------------------------------------------------
 struct NcReadParams {
-    const float *ws_state;           // [BH][n_seg][kE] partials (n_seg may be 0)
-    const float *state_in_S;         // used only when n_seg == 0 (no keys): [BH][32][32], or null
+    const uint8_t *ws_bimg;          // [BH][kBimg] the heads' B operand images (written by the state kernel),
+                                     // or null when there are no keys
+    const float *state_in_S;         // no keys only: [BH][32][32] (the totals), or null (zeros)
     const float *state_in_z;
-    float *state_out_S;              // the head totals, or null
+    float *state_out_S;              // no keys only: the head totals, or null
     float *state_out_z;
     int *status;
     unsigned long long wait_ns;
@@ -314,11 +373,12 @@ template <typename OutT> struct RCfg {
     static constexpr int STG_WARP = 4096;                   // one warp's 32 output rows (<= 128 B each)
     static constexpr int OFF_STG = NQ * QT;                 // 2 buffers x 4 warps
     static constexpr int OFF_B = OFF_STG + 2 * 4 * STG_WARP;
-    static constexpr int BN = 48;                           // B operand rows: 32 of S, 1 of z, 15 zero
-    static constexpr int BOP = BN * kD * 2;                 // 3 KB
+    static constexpr int BN = kBN;                          // B operand rows: 32 of S, 1 of z, 15 unused
+    static constexpr int BOP = kBop;                        // 3 KB
     static constexpr int OFF_BAR = OFF_B + 2 * BOP;         // hi, lo
     static constexpr int B_QFULL = 0, B_PHI = NQ, B_QEMPTY = 2 * NQ, B_DFULL = 3 * NQ, B_DEMPTY = B_DFULL + ND,
-                         B_BREADY = B_DEMPTY + ND, B_DRAIN = B_BREADY + 1, NBAR = B_DRAIN + 1;
+                         B_BREADY = B_DEMPTY + ND, B_BLOAD = B_BREADY + 1, B_DRAIN = B_BLOAD + 1,
+                         NBAR = B_DRAIN + 1;
     static constexpr int OFF_TMEMADDR = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEMADDR + 4;
     static constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;
@@ -327,13 +387,6 @@ template <typename OutT> struct RCfg {
     static constexpr int ROWB = kD * (int)sizeof(OutT);     // output row bytes: 128 (fp32) or 64
     static_assert(OFF_STG % 1024 == 0 && OFF_B % 16 == 0 && ND * T_DSTRIDE <= TMEM_COLS, "layout");
 };
-
-// Byte offset of element (n, k) of a K-major no-swizzle [48][32] operand:
-// core matrices (8 rows x 8 k) of 128 bytes, 4 along K (128 bytes apart),
-// groups of 8 rows 512 bytes apart.
-__device__ __forceinline__ int bop_off(int n, int k) {
-    return (n >> 3) * 512 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
-}
 
 // 16-byte chunk c of output row r in a warp's staging rows, swizzled as the
 // output tensor map (128-byte rows: 128-byte swizzle; 64-byte rows: 64-byte).
@@ -374,6 +427,7 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_init(&bar[G::B_DEMPTY + a], 4);
         }
         mbar_init(&bar[G::B_BREADY], 4);
+        mbar_init(&bar[G::B_BLOAD], 1);
         mbar_init(&bar[G::B_DRAIN], 1);
         fence_mbar_init();
     }
@@ -483,88 +537,54 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int q = warp & 3, et = threadIdx.x - 192;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         bool waited = false;
-        int cur = -1;
+        int cur = -1, hc = -1;
         for (int i = 0; i < n; ++i) {
             const int a = i % G::ND;
             const long f = f0 + i;
             const int bh = (int)(f / tph), t = (int)(f % tph);
             if (bh != cur) {
                 cur = bh;
-                if (!waited) {
-                    pdl_wait();   // the state kernel's partials are complete and visible
-                    waited = true;
-                }
-                // the head's total: sum of its partials in segment order (or the
-                // state-in when there are no keys); the CTA holding the head's
-                // first tile writes it as the state output
-                const bool owner = t == 0 && p.state_out_S != nullptr;
-                uint8_t *bhi = smem + G::OFF_B, *blo = smem + G::OFF_B + G::BOP;
-                // thread et sums float4 groups g = et, et + 128, et + 256 (< kE / 4)
-                // of the state; every load of a batch of segments is issued
-                // before any is used, so a head costs a few memory round trips
-                constexpr int NG = kE / 4;              // 264 groups of 4 floats
-                constexpr int GPT = (NG + 127) / 128;   // 3 per thread
-                constexpr int SB = 2;                   // segments per batch
-                float4 acc[GPT];
-#pragma unroll
-                for (int m = 0; m < GPT; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (p.n_seg == 0) {
-                    if (p.state_in_S) {
-#pragma unroll
-                        for (int m = 0; m < GPT; ++m) {
-                            const int g = et + 128 * m;
-                            if (g < kD * kD / 4)
-                                acc[m] = reinterpret_cast<const float4 *>(p.state_in_S + (size_t)bh * kD * kD)[g];
-                            else if (g < NG)
-                                acc[m] = reinterpret_cast<const float4 *>(p.state_in_z + (size_t)bh * kD)[g - kD * kD / 4];
+                ++hc;
+                if (p.ws_bimg) {
+                    // the state kernel wrote this head's B operands: one bulk
+                    // copy (the previous head's MMAs are complete: this warp
+                    // has consumed the accumulator of the previous tile)
+                    if (warp == 6 && lane == 0) {
+                        if (!waited) {
+                            pdl_wait();   // the state kernel's results are complete and visible
+                            waited = true;
                         }
+                        mbar_expect_tx(&bar[G::B_BLOAD], kBimg);
+                        bulk_load(smem + G::OFF_B, p.ws_bimg + (size_t)bh * kBimg, kBimg, &bar[G::B_BLOAD]);
                     }
+                    if (!mbar_wait(&bar[G::B_BLOAD], hc & 1, ab, 8)) break;
                 } else {
-                    const float4 *src = reinterpret_cast<const float4 *>(p.ws_state + (size_t)bh * p.n_seg * kE);
-                    for (int s0 = 0; s0 < p.n_seg; s0 += SB) {
-                        float4 x[SB][GPT];
-#pragma unroll
-                        for (int j = 0; j < SB; ++j)
-#pragma unroll
-                            for (int m = 0; m < GPT; ++m) {
-                                const int g = et + 128 * m;
-                                x[j][m] = (s0 + j < p.n_seg && g < NG) ? src[(size_t)(s0 + j) * NG + g]
-                                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-                            }
-#pragma unroll
-                        for (int j = 0; j < SB; ++j)
-#pragma unroll
-                            for (int m = 0; m < GPT; ++m) {
-                                acc[m].x += x[j][m].x;
-                                acc[m].y += x[j][m].y;
-                                acc[m].z += x[j][m].z;
-                                acc[m].w += x[j][m].w;
-                            }
+                    // no keys: the totals are the state-in (or zeros); the CTA
+                    // holding the head's first tile writes the state output
+                    if (!waited) {
+                        pdl_wait();
+                        waited = true;
                     }
-                }
-#pragma unroll
-                for (int m = 0; m < GPT; ++m) {
-                    const int g = et + 128 * m;
-                    if (g >= NG) continue;
-                    if (owner) {
-                        if (g < kD * kD / 4) reinterpret_cast<float4 *>(p.state_out_S + (size_t)bh * kD * kD)[g] = acc[m];
-                        else reinterpret_cast<float4 *>(p.state_out_z + (size_t)bh * kD)[g - kD * kD / 4] = acc[m];
-                    }
-                    const float v4[4] = {acc[m].x, acc[m].y, acc[m].z, acc[m].w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        // S[k][nn] -> element (nn, k); z[k] -> element (32, k)
-                        const int e = 4 * g + j;
+                    const bool owner = t == 0 && p.state_out_S != nullptr;
+                    uint8_t *bhi = smem + G::OFF_B, *blo = smem + G::OFF_B + G::BOP;
+                    for (int e = et; e < kE; e += 128) {
+                        float acc = 0.f;
+                        if (p.state_in_S)
+                            acc = e < kD * kD ? p.state_in_S[(size_t)bh * kD * kD + e]
+                                              : p.state_in_z[(size_t)bh * kD + (e - kD * kD)];
+                        if (owner) {
+                            if (e < kD * kD) p.state_out_S[(size_t)bh * kD * kD + e] = acc;
+                            else p.state_out_z[(size_t)bh * kD + (e - kD * kD)] = acc;
+                        }
                         const int nn = e < kD * kD ? e % kD : kD;
                         const int k = e < kD * kD ? e / kD : e - kD * kD;
-                        const bf16 hi = __float2bfloat16_rn(v4[j]);
+                        const bf16 hi = __float2bfloat16_rn(acc);
                         *reinterpret_cast<bf16 *>(bhi + bop_off(nn, k)) = hi;
-                        *reinterpret_cast<bf16 *>(blo + bop_off(nn, k)) = __float2bfloat16_rn(v4[j] - __bfloat162float(hi));
+                        *reinterpret_cast<bf16 *>(blo + bop_off(nn, k)) = __float2bfloat16_rn(acc - __bfloat162float(hi));
                     }
+                    // each warp's writes are complete and visible to the tensor core
+                    fence_proxy_async_smem();
                 }
-                // each warp's writes are complete and visible to the tensor core
-                // before its arrival; the MMA waits for all four
-                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar[G::B_BREADY]);
             }

@@ -188,7 +188,6 @@ template <typename InT, typename OutT>
 la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
     using namespace nctc;
     const bool keys = a.Lk > 0;
-    const int n_seg = keys ? a.n_seg : 0;
     const bool inout = a.mode == LA_STATE_INOUT;
     la_status s = LA_OK;
     if (keys) {
@@ -197,10 +196,11 @@ la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
             !make_map_box(&mv, a.v, a.in_dtype, a.BH, a.Lk, kD, kSRows, kHP, CU_TENSOR_MAP_SWIZZLE_64B))
             return cuda_fail_msg("cuTensorMapEncodeTiled", "tensor map encoding failed");
         NcStateParams sp;
-        sp.ws_state = a.ws_state;
-        sp.ws_A = a.ws_A;
+        sp.ws_bimg = a.ws_bimg;
         sp.state_in_S = inout ? a.state_S : nullptr;
         sp.state_in_z = inout ? a.state_z : nullptr;
+        sp.state_out_S = a.mode != LA_STATE_NONE ? a.state_S : nullptr;
+        sp.state_out_z = a.mode != LA_STATE_NONE ? a.state_z : nullptr;
         sp.status = a.status;
         sp.wait_ns = a.wait_ns;
         sp.BH = (int)a.BH;
@@ -211,17 +211,29 @@ la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
         s = cuda_check("non-causal state smem attribute",
                        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SCfg::SMEM_BYTES));
         if (s != LA_OK) return s;
-        const unsigned groups = (unsigned)((a.BH + kHP - 1) / kHP);
-        kern<<<dim3((unsigned)a.n_seg, groups), SCfg::THREADS, SCfg::SMEM_BYTES, st>>>(mk, mv, sp);
+        // one cluster per group of heads: its n_seg (<= 8) segment CTAs add
+        // their partial states through distributed shared memory
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)a.n_seg;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)a.n_seg, (unsigned)((a.BH + kHP - 1) / kHP));
+        cfg.blockDim = dim3(SCfg::THREADS);
+        cfg.dynamicSmemBytes = SCfg::SMEM_BYTES;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, mk, mv, sp);
         count_launches(1);
+        if (err != cudaSuccess) return cuda_fail("non-causal state launch", err);
         if ((s = cuda_check("non-causal state launch", cudaGetLastError())) != LA_OK) return s;
     }
     if (a.Lq == 0) {
-        if (a.mode == LA_STATE_NONE) return LA_OK;
-        // the state-in (INOUT) already joined segment 0's partial
-        const int mode = (keys && inout) ? LA_STATE_OUT : a.mode;
-        return launch_segment_scan(a.ws_state, a.ws_A, a.BH, n_seg, n_seg, kD, mode, a.state_S, a.state_z, nullptr,
-                                   st, keys);
+        if (keys || a.mode == LA_STATE_NONE) return LA_OK;   // the state kernel wrote the state output
+        // no keys and no queries: state-out = state-in (INOUT) or zeros (OUT), by the scan over no segments
+        return launch_segment_scan(nullptr, nullptr, a.BH, 0, 0, kD, a.mode, a.state_S, a.state_z, nullptr, st, false);
     }
     CUtensorMap mq, mo;
     if (!make_map_box(&mq, a.q, a.in_dtype, a.BH, a.Lq, kD, kRows, 1, CU_TENSOR_MAP_SWIZZLE_64B) ||
@@ -229,16 +241,16 @@ la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
                       a.out_dtype == LA_F32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
         return cuda_fail_msg("cuTensorMapEncodeTiled", "tensor map encoding failed");
     NcReadParams rp;
-    rp.ws_state = a.ws_state;
+    rp.ws_bimg = keys ? a.ws_bimg : nullptr;
     rp.state_in_S = (!keys && inout) ? a.state_S : nullptr;
     rp.state_in_z = (!keys && inout) ? a.state_z : nullptr;
-    rp.state_out_S = a.mode != LA_STATE_NONE ? a.state_S : nullptr;
-    rp.state_out_z = a.mode != LA_STATE_NONE ? a.state_z : nullptr;
+    rp.state_out_S = (!keys && a.mode != LA_STATE_NONE) ? a.state_S : nullptr;
+    rp.state_out_z = (!keys && a.mode != LA_STATE_NONE) ? a.state_z : nullptr;
     rp.status = a.status;
     rp.wait_ns = a.wait_ns;
     rp.BH = (int)a.BH;
     rp.Lq = a.Lq;
-    rp.n_seg = n_seg;
+    rp.n_seg = keys ? a.n_seg : 0;
     rp.tiles_per_head = (a.Lq + kRows - 1) / kRows;
     rp.total_tiles = a.BH * rp.tiles_per_head;
     rp.eps = a.eps;

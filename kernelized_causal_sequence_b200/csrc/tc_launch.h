@@ -33,6 +33,7 @@ struct TcNoncausalArgs {
     void *out;
     la_dtype in_dtype, out_dtype;
     float *ws_state, *ws_A, *ws_total;
+    uint8_t *ws_bimg;             // d 32 tensor-core path: [BH][6144] the heads' read-out operand images
     int *status;                  // the call's status word [2] (cleared by the caller)
     unsigned long long wait_ns;
     float *state_S, *state_z;

@@ -58,8 +58,8 @@ namespace tc {
 
 enum Mode { kStateOnly = 0, kOutput = 1 };
 
-constexpr int kThreads = 448;
-constexpr int kEpiWarp0 = 0, kTmaWarp = 4, kMmaWarp = 5, kPhiWarp0 = 6, kKWarp0 = 10;
+constexpr int kThreads = 480;
+constexpr int kEpiWarp0 = 0, kTmaWarp = 4, kMmaWarp = 5, kPhiWarp0 = 6, kKWarp0 = 10, kQTmaWarp = 14;
 
 constexpr int tmem_alloc_cols(int used) {
     return used <= 32 ? 32 : used <= 64 ? 64 : used <= 128 ? 128 : used <= 256 ? 256 : 512;
@@ -116,7 +116,8 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int B_DS_FULL = B_O_EMPTY + 1, B_S_READY = B_DS_FULL + 1;
     static constexpr int B_DRAIN = B_S_READY + 1, B_KW_READY = B_DRAIN + 1, B_QS_READY = B_KW_READY + 1;
     static constexpr int B_L_READY = B_QS_READY + 1;
-    static constexpr int NBAR = B_L_READY + NKV;
+    static constexpr int B_V_EMPTY = B_L_READY + NKV;   // V of a stage consumed (K: B_KV_EMPTY)
+    static constexpr int NBAR = B_V_EMPTY + NKV;
     static constexpr int OFF_TMEMADDR = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEMADDR + 4;
     static constexpr int OFF_END = OFF_ABORT + 4;
@@ -671,6 +672,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int s = 0; s < G::NKV; ++s) {
             mbar_init(&bar[G::B_KV_FULL + s], 1);
             mbar_init(&bar[G::B_KV_EMPTY + s], 1);
+            mbar_init(&bar[G::B_V_EMPTY + s], 1);
             mbar_init(&bar[G::B_PHI + s], 8);   // key warps + (query warps | warps 0-3)
             mbar_init(&bar[G::B_L_READY + s], 1);
         }
@@ -717,14 +719,15 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t tmem = *tmem_addr_smem;
     if ((smem_u32(smem) & 1023u) != 0) raise_abort(ab, 99, kStatusLayout);  // layout assumption violated
 
-    if (warp == kTmaWarp) {
-        // ================= TMA producer
-        if (lane == 0 && !*abort_flag) {
-            int issued_kv[G::NKV] = {}, issued_q[2] = {};
-            for (int c = 0; c < nch; ++c) {
-                const int s = c % G::NKV;
-                const int y = (int)(t_begin + (long)chunk_at<G::OUT>(c, nch) * C);
-                if constexpr (G::OUT) {
+    if (warp == kQTmaWarp) {
+        // ================= TMA producer of the query tiles (output mode): its
+        // own thread, so that a query slot that frees late does not hold back
+        // the key and value loads
+        if constexpr (G::OUT) {
+            if (lane == 0 && !*abort_flag) {
+                int issued_q[2] = {};
+                for (int c = 0; c < nch; ++c) {
+                    const int y = (int)(t_begin + (long)c * C);
                     const int sq = G::QT ? 0 : (c & 1);
                     const int use = G::QT ? c : (c >> 1);
                     if (use > 0 && !mbar_wait(&bar[G::B_Q_EMPTY + sq], (use - 1) & 1, ab, 1)) break;
@@ -735,25 +738,44 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         tma_load_3d(qd + b * G::BOXB, &tm_q, &bar[G::B_Q_FULL + sq], 64 * b, y, bh);
                     issued_q[sq] = use + 1;
                 }
+                if (*abort_flag) {
+                    volatile int never = 0;
+                    AbortCtx timed{&never, nullptr, kDrainLimitNs};
+                    for (int s = 0; s < 2; ++s)
+                        if (issued_q[s] > 0) mbar_wait(&bar[G::B_Q_FULL + s], (issued_q[s] - 1) & 1, timed, 0);
+                }
+            }
+        }
+    } else if (warp == kTmaWarp) {
+        // ================= TMA producer of the key and value tiles: a stage's
+        // K is reloaded once its last reader (MMA3/MMAz) is done, its V once
+        // MMA4 is; one full barrier counts both
+        if (lane == 0 && !*abort_flag) {
+            int issued_kv[G::NKV] = {};
+            for (int c = 0; c < nch; ++c) {
+                const int s = c % G::NKV;
+                const int y = (int)(t_begin + (long)chunk_at<G::OUT>(c, nch) * C);
                 const int use = c / G::NKV;
                 if (use > 0 && !mbar_wait(&bar[G::B_KV_EMPTY + s], (use - 1) & 1, ab, 2)) break;
                 uint8_t *kd = smem + G::OFF_KV + s * G::KV_STAGE;
                 mbar_expect_tx(&bar[G::B_KV_FULL + s], 2 * G::TILE);
-#pragma unroll
-                for (int b = 0; b < G::KB; ++b) {
-                    tma_load_3d(kd + b * G::BOXB, &tm_k, &bar[G::B_KV_FULL + s], 64 * b, y, bh);
-                    tma_load_3d(kd + G::TILE + b * G::BOXB, &tm_v, &bar[G::B_KV_FULL + s], 64 * b, y, bh);
-                }
                 issued_kv[s] = use + 1;
+#pragma unroll
+                for (int b = 0; b < G::KB; ++b)
+                    tma_load_3d(kd + b * G::BOXB, &tm_k, &bar[G::B_KV_FULL + s], 64 * b, y, bh);
+                if (use > 0 && !mbar_wait(&bar[G::B_V_EMPTY + s], (use - 1) & 1, ab, 26)) break;
+#pragma unroll
+                for (int b = 0; b < G::KB; ++b)
+                    tma_load_3d(kd + G::TILE + b * G::BOXB, &tm_v, &bar[G::B_KV_FULL + s], 64 * b, y, bh);
             }
             if (*abort_flag) {
-                // drain copies still in flight before the CTA may exit
+                // drain copies still in flight before the CTA may exit (a stage
+                // whose V was never issued completes no phase: its wait gives up
+                // after the fixed bound)
                 volatile int never = 0;
                 AbortCtx timed{&never, nullptr, kDrainLimitNs};
                 for (int s = 0; s < G::NKV; ++s)
                     if (issued_kv[s] > 0) mbar_wait(&bar[G::B_KV_FULL + s], (issued_kv[s] - 1) & 1, timed, 0);
-                for (int s = 0; s < 2; ++s)
-                    if (issued_q[s] > 0) mbar_wait(&bar[G::B_Q_FULL + s], (issued_q[s] - 1) & 1, timed, 0);
             }
         }
     } else if (warp == kMmaWarp) {
@@ -816,6 +838,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int kk = 0; kk < C / 16; ++kk)
                         mma_ss(tmem + G::T_Z, dKm + (uint64_t)((kk * 2048) >> 4),
                                dOnes + (uint64_t)((kk * 256) >> 4), ID_Z, 1);
+                    mma_commit(&bar[G::B_KV_EMPTY + s]);   // the keys' last readers are issued
                     // MMA2 + MMAd: O is free once the output of c-1 has been read
                     if (c > 0 && !mbar_wait(&bar[G::B_O_EMPTY], (c - 1) & 1, ab, 6)) break;
                     tc_fence_after();
@@ -848,7 +871,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                     mma_commit(&bar[G::B_MMA4]);
                     mma_commit(&bar[G::B_O_FULL]);
-                    mma_commit(&bar[G::B_KV_EMPTY + s]);
+                    mma_commit(&bar[G::B_V_EMPTY + s]);
                     continue;
                 }
                 if constexpr (G::OUT) {
@@ -923,6 +946,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     mma_commit(&bar[G::B_O_FULL]);
                 }
                 mma_commit(&bar[G::B_KV_EMPTY + s]);
+                mma_commit(&bar[G::B_V_EMPTY + s]);
             }
             // drain: every MMA issued by this thread has completed
             volatile int never = 0;
@@ -930,7 +954,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mma_commit(&bar[G::B_DRAIN]);
             mbar_wait(&bar[G::B_DRAIN], 0, timed, 0);
         }
-    } else if (warp >= kKWarp0) {
+    } else if (warp >= kKWarp0 && warp < kKWarp0 + 4) {
         // ================= keys: decay cumsum and phi(K) (warps 10-13)
         const int tk = threadIdx.x - kKWarp0 * 32;   // 0..127
         float Aseg = 1.f;                            // product of chunk decays (state-only mode)
