@@ -73,14 +73,10 @@ __device__ __forceinline__ int bop_off(int n, int k) {
 }
 
 struct NcStateParams {
-    uint8_t *ws_bimg;                // [BH][kBimg]: each head's total (S, z) as the read-out's B operands
-    const float *state_in_S;         // [BH][32][32] added to the sums, or null
-    const float *state_in_z;         // [BH][32]
-    float *state_out_S;              // [BH][32][32] the totals, or null
-    float *state_out_z;              // [BH][32]
+    float *ws_state;                 // [BH][n_seg][kE] partial states
     int *status;                     // the call's status word [2]
     unsigned long long wait_ns;
-    int BH, Lk, seg_len, n_seg;      // seg_len: a multiple of kSRows; n_seg <= 8 (the cluster)
+    int BH, Lk, seg_len, n_seg;      // seg_len: a multiple of kSRows
 };
 
 struct SCfg {
@@ -268,79 +264,28 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
         }
-        // the CTA's partial (S, z) of its 4 heads -> its own shared memory
-        // [4][kE] fp32 (in the drained K/V stages); garbage if the CTA gave up
+        // the CTA's partial (S, z) of each of its heads -> the workspace
         if (ok && ntiles > 0 && mbar_wait(&bar[G::B_DONE], 0, ab, 5)) {
             tc_fence_after();
             // TMEM lane quarter q = head q of the group; lane = feature a
             const int q = warp & 3, a = lane;
+            const long bh = (long)grp * kHP + q;
             const uint32_t lane_base = (uint32_t)(q * 32) << 16;
             uint32_t u[32], zb;
             tmem_ld32(tmem + lane_base + G::T_S + q * 32, u);   // the diagonal block: S_q[a][0..31]
             tmem_ld1(tmem + lane_base + G::T_Z, zb);
             tmem_ld_wait();
-            float *part = reinterpret_cast<float *>(smem + G::OFF_KV) + q * kE;
-            float4 *d4 = reinterpret_cast<float4 *>(part + a * kD);
+            if (bh < p.BH && !*abort_flag) {
+                float *dst = p.ws_state + ((size_t)bh * p.n_seg + seg) * kE;
+                float4 *d4 = reinterpret_cast<float4 *>(dst + a * kD);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                d4[i] = make_float4(__uint_as_float(u[4 * i]), __uint_as_float(u[4 * i + 1]),
-                                    __uint_as_float(u[4 * i + 2]), __uint_as_float(u[4 * i + 3]));
-            part[kD * kD + a] = __uint_as_float(zb);
-        }
-    }
-
-    // ---------------- the group's totals: the cluster is the group's n_seg
-    // CTAs; CTA r sums its share of the 4 heads' elements over every CTA's
-    // partial (distributed shared memory, fixed order), adds the state-in,
-    // writes the state-out and the read-out's B operand images (bf16 hi + lo)
-    __syncwarp();
-    tc_fence_before();
-    cluster_sync();   // every partial is in shared memory
-    {
-        constexpr int NG = kE / 4;                       // 264 float4 groups per head
-        const int ncl = p.n_seg, rank = (int)cluster_ctarank();
-        const int f0 = rank * (kHP * NG) / ncl, f1 = (rank + 1) * (kHP * NG) / ncl;
-        const uint32_t part0 = smem_u32(smem + G::OFF_KV);
-        for (int f = f0 + (int)threadIdx.x; f < f1; f += G::THREADS) {
-            const int h = f / NG, g = f % NG;
-            const long bh = (long)grp * kHP + h;
-            const uint32_t off = part0 + (uint32_t)((h * kE + 4 * g) * 4);
-            float4 x[8];
-#pragma unroll
-            for (int r = 0; r < 8; ++r) x[r] = r < ncl ? ld_dsmem_f4(mapa_shared(off, r)) : make_float4(0.f, 0.f, 0.f, 0.f);
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (bh < p.BH && p.state_in_S) {
-                acc = g < kD * kD / 4 ? reinterpret_cast<const float4 *>(p.state_in_S + (size_t)bh * kD * kD)[g]
-                                      : reinterpret_cast<const float4 *>(p.state_in_z + (size_t)bh * kD)[g - kD * kD / 4];
-            }
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                acc.x += x[r].x;
-                acc.y += x[r].y;
-                acc.z += x[r].z;
-                acc.w += x[r].w;
-            }
-            if (bh >= p.BH || *abort_flag) continue;
-            if (p.state_out_S) {
-                if (g < kD * kD / 4) reinterpret_cast<float4 *>(p.state_out_S + (size_t)bh * kD * kD)[g] = acc;
-                else reinterpret_cast<float4 *>(p.state_out_z + (size_t)bh * kD)[g - kD * kD / 4] = acc;
-            }
-            uint8_t *img = p.ws_bimg + (size_t)bh * kBimg;
-            const float v4[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                // S[k][nn] -> element (nn, k); z[k] -> element (32, k)
-                const int e = 4 * g + j;
-                const int nn = e < kD * kD ? e % kD : kD;
-                const int k = e < kD * kD ? e / kD : e - kD * kD;
-                const bf16 hi = __float2bfloat16_rn(v4[j]);
-                *reinterpret_cast<bf16 *>(img + bop_off(nn, k)) = hi;
-                *reinterpret_cast<bf16 *>(img + kBop + bop_off(nn, k)) = __float2bfloat16_rn(v4[j] - __bfloat162float(hi));
+                for (int i = 0; i < 8; ++i)
+                    d4[i] = make_float4(__uint_as_float(u[4 * i]), __uint_as_float(u[4 * i + 1]),
+                                        __uint_as_float(u[4 * i + 2]), __uint_as_float(u[4 * i + 3]));
+                dst[kD * kD + a] = __uint_as_float(zb);
             }
         }
     }
-    __syncwarp();
-    cluster_sync();   // no CTA leaves while another reads its shared memory
 
     tc_fence_before();
     __syncthreads();
@@ -351,13 +296,70 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 }
 
 // --------------------------------------------------------------------------
+// nc_combine_kernel — each head's total: the sum of its partial states in
+// segment order (deterministic) plus the state-in; writes the state-out and
+// the read-out's B operand images (bf16 hi and lo, K-major [48][32]: rows
+// 0-31 the columns of S, row 32 z; rows 33-47 are not written and only reach
+// output columns the read-out never reads).  One CTA per head, one thread
+// per 4 consecutive state elements; each thread's loads for up to 8 segments
+// are issued before any is used.  With no keys (n_seg = 0) the total is the
+// state-in or zeros.  grid (BH), kE / 4 = 264 threads.
+struct NcCombineParams {
+    const float *ws_state;           // [BH][n_seg][kE]
+    uint8_t *ws_bimg;                // [BH][kBimg]
+    const float *state_in_S, *state_in_z;   // or null
+    float *state_out_S, *state_out_z;       // or null
+    int n_seg;
+};
+constexpr int kCombineThreads = kE / 4;
+__global__ void __launch_bounds__(kCombineThreads) nc_combine_kernel(NcCombineParams p) {
+    const int g = threadIdx.x;
+    const long bh = blockIdx.x;
+    // the read-out kernel may be scheduled now (its set-up and query loads do
+    // not depend on this grid; it waits for this grid before reading the images)
+    pdl_trigger();
+    pdl_wait();   // the state kernel's partials
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p.state_in_S)
+        acc = g < kD * kD / 4 ? reinterpret_cast<const float4 *>(p.state_in_S + (size_t)bh * kD * kD)[g]
+                              : reinterpret_cast<const float4 *>(p.state_in_z + (size_t)bh * kD)[g - kD * kD / 4];
+    const float4 *src = reinterpret_cast<const float4 *>(p.ws_state + (size_t)bh * p.n_seg * kE) + g;
+    for (int s0 = 0; s0 < p.n_seg; s0 += 8) {
+        float4 x[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            x[j] = s0 + j < p.n_seg ? src[(size_t)(s0 + j) * (kE / 4)] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            acc.x += x[j].x;
+            acc.y += x[j].y;
+            acc.z += x[j].z;
+            acc.w += x[j].w;
+        }
+    }
+    if (p.state_out_S) {
+        if (g < kD * kD / 4) reinterpret_cast<float4 *>(p.state_out_S + (size_t)bh * kD * kD)[g] = acc;
+        else reinterpret_cast<float4 *>(p.state_out_z + (size_t)bh * kD)[g - kD * kD / 4] = acc;
+    }
+    if (p.ws_bimg) {
+        uint8_t *img = p.ws_bimg + (size_t)bh * kBimg;
+        const float v4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            // S[k][nn] -> element (nn, k); z[k] -> element (32, k)
+            const int e = 4 * g + j;
+            const int nn = e < kD * kD ? e % kD : kD;
+            const int k = e < kD * kD ? e / kD : e - kD * kD;
+            const bf16 hi = __float2bfloat16_rn(v4[j]);
+            *reinterpret_cast<bf16 *>(img + bop_off(nn, k)) = hi;
+            *reinterpret_cast<bf16 *>(img + kBop + bop_off(nn, k)) = __float2bfloat16_rn(v4[j] - __bfloat162float(hi));
+        }
+    }
+}
+
+// --------------------------------------------------------------------------
 struct NcReadParams {
-    const uint8_t *ws_bimg;          // [BH][kBimg] the heads' B operand images (written by the state kernel),
-                                     // or null when there are no keys
-    const float *state_in_S;         // no keys only: [BH][32][32] (the totals), or null (zeros)
-    const float *state_in_z;
-    float *state_out_S;              // no keys only: the head totals, or null
-    float *state_out_z;
+    const uint8_t *ws_bimg;          // [BH][kBimg] the heads' B operand images (the combine kernel's)
     int *status;
     unsigned long long wait_ns;
     int BH, Lq, n_seg, tiles_per_head;
@@ -545,46 +547,18 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (bh != cur) {
                 cur = bh;
                 ++hc;
-                if (p.ws_bimg) {
-                    // the state kernel wrote this head's B operands: one bulk
-                    // copy (the previous head's MMAs are complete: this warp
-                    // has consumed the accumulator of the previous tile)
-                    if (warp == 6 && lane == 0) {
-                        if (!waited) {
-                            pdl_wait();   // the state kernel's results are complete and visible
-                            waited = true;
-                        }
-                        mbar_expect_tx(&bar[G::B_BLOAD], kBimg);
-                        bulk_load(smem + G::OFF_B, p.ws_bimg + (size_t)bh * kBimg, kBimg, &bar[G::B_BLOAD]);
-                    }
-                    if (!mbar_wait(&bar[G::B_BLOAD], hc & 1, ab, 8)) break;
-                } else {
-                    // no keys: the totals are the state-in (or zeros); the CTA
-                    // holding the head's first tile writes the state output
+                // the combine kernel wrote this head's B operands: one bulk copy
+                // (the previous head's MMAs are complete: this warp has consumed
+                // the accumulator of the previous tile)
+                if (warp == 6 && lane == 0) {
                     if (!waited) {
-                        pdl_wait();
+                        pdl_wait();   // the combine kernel's results are complete and visible
                         waited = true;
                     }
-                    const bool owner = t == 0 && p.state_out_S != nullptr;
-                    uint8_t *bhi = smem + G::OFF_B, *blo = smem + G::OFF_B + G::BOP;
-                    for (int e = et; e < kE; e += 128) {
-                        float acc = 0.f;
-                        if (p.state_in_S)
-                            acc = e < kD * kD ? p.state_in_S[(size_t)bh * kD * kD + e]
-                                              : p.state_in_z[(size_t)bh * kD + (e - kD * kD)];
-                        if (owner) {
-                            if (e < kD * kD) p.state_out_S[(size_t)bh * kD * kD + e] = acc;
-                            else p.state_out_z[(size_t)bh * kD + (e - kD * kD)] = acc;
-                        }
-                        const int nn = e < kD * kD ? e % kD : kD;
-                        const int k = e < kD * kD ? e / kD : e - kD * kD;
-                        const bf16 hi = __float2bfloat16_rn(acc);
-                        *reinterpret_cast<bf16 *>(bhi + bop_off(nn, k)) = hi;
-                        *reinterpret_cast<bf16 *>(blo + bop_off(nn, k)) = __float2bfloat16_rn(acc - __bfloat162float(hi));
-                    }
-                    // each warp's writes are complete and visible to the tensor core
-                    fence_proxy_async_smem();
+                    mbar_expect_tx(&bar[G::B_BLOAD], kBimg);
+                    bulk_load(smem + G::OFF_B, p.ws_bimg + (size_t)bh * kBimg, kBimg, &bar[G::B_BLOAD]);
                 }
+                if (!mbar_wait(&bar[G::B_BLOAD], hc & 1, ab, 8)) break;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar[G::B_BREADY]);
             }

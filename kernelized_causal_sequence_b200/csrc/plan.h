@@ -71,18 +71,15 @@ inline Plan make_nc_plan(long BH, long Lk, int D) {
 
 // Key segments of the tensor-core non-causal form (head dimension 32): one
 // CTA per (group of 4 heads, segment of whole 64-key tiles), the segment
-// count chosen so that all CTAs fit in one wave on the SMs, at most 8 (the
-// group's segments form one cluster).
+// count chosen so that all CTAs fit in one wave on the SMs.
 constexpr int kNcTcHeads = 4;
 constexpr int kNcTcKeyTile = 64;
-constexpr int kNcTcMaxSegs = 8;   // the segments of a group form one thread-block cluster (portable size)
 inline Plan make_nc_tc_plan(long BH, long Lk) {
     Plan p;
     p.chunk = kNcTcKeyTile;
     const long groups = (BH + kNcTcHeads - 1) / kNcTcHeads;
     const long tiles = Lk > 0 ? (Lk + kNcTcKeyTile - 1) / kNcTcKeyTile : 1;
     long segs = kNumSMs / (groups > 0 ? groups : 1);
-    if (segs > kNcTcMaxSegs) segs = kNcTcMaxSegs;   // one cluster per group
     if (segs < 1) segs = 1;
     if (segs > tiles) segs = tiles;
     const long per = (tiles + segs - 1) / segs;

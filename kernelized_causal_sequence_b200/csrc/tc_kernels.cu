@@ -184,6 +184,29 @@ la_status dispatch_cd(const TcCausalArgs &a, cudaStream_t st) {
 // Non-causal form at head dim 32: the state kernel (per group of 4 heads and
 // key segment) and the read-out kernel, chained by programmatic dependent
 // launch.  With no queries the segment scan forms the state output instead.
+// Launches kern with programmatic stream serialisation when pdl is set.
+template <typename... KArgs, typename... Args>
+la_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                     const char *what, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, args...);
+    count_launches(1);
+    if (err != cudaSuccess) return cuda_fail(what, err);
+    return cuda_check(what, cudaGetLastError());
+}
+
+// Non-causal form at head dim 32: the state kernel (per group of 4 heads and
+// key segment), the combine kernel (per head: totals, state-out, read-out
+// operands) and the read-out kernel, chained by programmatic dependent launch.
 template <typename InT, typename OutT>
 la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
     using namespace nctc;
@@ -196,11 +219,7 @@ la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
             !make_map_box(&mv, a.v, a.in_dtype, a.BH, a.Lk, kD, kSRows, kHP, CU_TENSOR_MAP_SWIZZLE_64B))
             return cuda_fail_msg("cuTensorMapEncodeTiled", "tensor map encoding failed");
         NcStateParams sp;
-        sp.ws_bimg = a.ws_bimg;
-        sp.state_in_S = inout ? a.state_S : nullptr;
-        sp.state_in_z = inout ? a.state_z : nullptr;
-        sp.state_out_S = a.mode != LA_STATE_NONE ? a.state_S : nullptr;
-        sp.state_out_z = a.mode != LA_STATE_NONE ? a.state_z : nullptr;
+        sp.ws_state = a.ws_state;
         sp.status = a.status;
         sp.wait_ns = a.wait_ns;
         sp.BH = (int)a.BH;
@@ -211,41 +230,29 @@ la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
         s = cuda_check("non-causal state smem attribute",
                        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SCfg::SMEM_BYTES));
         if (s != LA_OK) return s;
-        // one cluster per group of heads: its n_seg (<= 8) segment CTAs add
-        // their partial states through distributed shared memory
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)a.n_seg;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.gridDim = dim3((unsigned)a.n_seg, (unsigned)((a.BH + kHP - 1) / kHP));
-        cfg.blockDim = dim3(SCfg::THREADS);
-        cfg.dynamicSmemBytes = SCfg::SMEM_BYTES;
-        cfg.stream = st;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, mk, mv, sp);
-        count_launches(1);
-        if (err != cudaSuccess) return cuda_fail("non-causal state launch", err);
-        if ((s = cuda_check("non-causal state launch", cudaGetLastError())) != LA_OK) return s;
+        s = launch_pdl(kern, dim3((unsigned)a.n_seg, (unsigned)((a.BH + kHP - 1) / kHP)), dim3(SCfg::THREADS),
+                       SCfg::SMEM_BYTES, st, false, "non-causal state launch", mk, mv, sp);
+        if (s != LA_OK) return s;
     }
-    if (a.Lq == 0) {
-        if (keys || a.mode == LA_STATE_NONE) return LA_OK;   // the state kernel wrote the state output
-        // no keys and no queries: state-out = state-in (INOUT) or zeros (OUT), by the scan over no segments
-        return launch_segment_scan(nullptr, nullptr, a.BH, 0, 0, kD, a.mode, a.state_S, a.state_z, nullptr, st, false);
-    }
+    if (a.Lq == 0 && a.mode == LA_STATE_NONE) return LA_OK;
+    NcCombineParams cp;
+    cp.ws_state = a.ws_state;
+    cp.ws_bimg = a.Lq > 0 ? a.ws_bimg : nullptr;
+    cp.state_in_S = inout ? a.state_S : nullptr;
+    cp.state_in_z = inout ? a.state_z : nullptr;
+    cp.state_out_S = a.mode != LA_STATE_NONE ? a.state_S : nullptr;
+    cp.state_out_z = a.mode != LA_STATE_NONE ? a.state_z : nullptr;
+    cp.n_seg = keys ? a.n_seg : 0;
+    s = launch_pdl(nc_combine_kernel, dim3((unsigned)a.BH), dim3(kCombineThreads), 0, st, keys,
+                   "non-causal combine launch", cp);
+    if (s != LA_OK || a.Lq == 0) return s;
     CUtensorMap mq, mo;
     if (!make_map_box(&mq, a.q, a.in_dtype, a.BH, a.Lq, kD, kRows, 1, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_map_box(&mo, a.out, a.out_dtype, a.BH, a.Lq, kD, 32, 1,
                       a.out_dtype == LA_F32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
         return cuda_fail_msg("cuTensorMapEncodeTiled", "tensor map encoding failed");
     NcReadParams rp;
-    rp.ws_bimg = keys ? a.ws_bimg : nullptr;
-    rp.state_in_S = (!keys && inout) ? a.state_S : nullptr;
-    rp.state_in_z = (!keys && inout) ? a.state_z : nullptr;
-    rp.state_out_S = (!keys && a.mode != LA_STATE_NONE) ? a.state_S : nullptr;
-    rp.state_out_z = (!keys && a.mode != LA_STATE_NONE) ? a.state_z : nullptr;
+    rp.ws_bimg = a.ws_bimg;
     rp.status = a.status;
     rp.wait_ns = a.wait_ns;
     rp.BH = (int)a.BH;
@@ -260,20 +267,9 @@ la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
                    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM));
     if (s != LA_OK) return s;
     const long grid = rp.total_tiles < kNumSMs ? rp.total_tiles : kNumSMs;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(RCfg<OutT>::THREADS);
-    cfg.dynamicSmemBytes = SM;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = keys ? 1 : 0;   // overlaps the state kernel's tail
-    const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, mq, mo, rp);
-    count_launches(1);
-    if (err != cudaSuccess) return cuda_fail("non-causal read-out launch", err);
-    return cuda_check("non-causal read-out launch", cudaGetLastError());
+    // its set-up and query loads overlap the combine kernel
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(RCfg<OutT>::THREADS), SM, st, true,
+                      "non-causal read-out launch", mq, mo, rp);
 }
 
 }  // namespace

@@ -211,11 +211,12 @@ __device__ __noinline__ void write_final_state(uint32_t t_s, uint32_t t_z, float
 }
 
 // z (row a of the normaliser) as the B operand of MMAd, K-major without
-// swizzle, [16][D] bf16: row n = 0 holds bf16(z).  The decay kernels (which
-// also serve the gated and mLSTM forms) add row n = 1 = bf16(z - bf16(z)), so
-// column 0 + column 1 of the product is phi(q).z to about 16 mantissa bits:
-// with the identity feature map q.z can cancel, and one bf16 rounding of z
-// would be amplified by it.  Element (n, a) sits at (a / 8) * 64 + 8 n + a % 8.
+// swizzle, [16][D] bf16: row n = 0 holds bf16(z) and row n = 1 bf16(z -
+// bf16(z)), so column 0 + column 1 of the product is phi(q).z to about 16
+// mantissa bits (with the identity feature map q.z can cancel, and one bf16
+// rounding of z would be amplified by it; without it the normaliser of a long
+// prefill still keeps its precision).  Element (n, a) sits at
+// (a / 8) * 64 + 8 n + a % 8.
 template <bool HILO>
 __device__ __forceinline__ void write_z_operand(bf16 *zb, int a, float z) {
     const bf16 hi = __float2bfloat16_rn(z);
@@ -1014,7 +1015,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if (srow_ok) {
                         // z operand: row n = 0 of the [16][D] K-major no-swizzle layout
                         bf16 *zb = reinterpret_cast<bf16 *>(smem + G::OFF_ZB);
-                        write_z_operand<DECAY>(zb, a_row, zin);
+                        write_z_operand<true>(zb, a_row, zin);
                     }
                 }
                 tmem_st_wait();
@@ -1124,7 +1125,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 if (srow_ok) {
                     bf16 *zb = reinterpret_cast<bf16 *>(smem + G::OFF_ZB);
-                    write_z_operand<DECAY>(zb, a_row, __uint_as_float(zbits));
+                    write_z_operand<true>(zb, a_row, __uint_as_float(zbits));
                 }
                 if constexpr (DECAY && !FLASH) {
                     tmem_st1(tmem + lane_base + G::T_Z, __float_as_uint(__uint_as_float(zbits) * gnext));
@@ -1238,7 +1239,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     uint32_t u[32], ud = 0u, ud_lo = 0u;
                     if (g == 0) {
                         tmem_ld1(tmem + lane_base + G::T_DEN, ud);
-                        if constexpr (DECAY) tmem_ld1(tmem + lane_base + G::T_DEN + 1, ud_lo);   // phi(q).z_lo
+                        tmem_ld1(tmem + lane_base + G::T_DEN + 1, ud_lo);   // phi(q).z_lo
                     }
                     tmem_ld32(tmem + lane_base + G::T_O + g * 32, u);
                     tmem_ld_wait();
@@ -1251,7 +1252,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             // mLSTM read-out: divide by max(|den|, 1)
                             inv = p.mlstm ? 1.f / fmaxf(fabsf(den), 1.f) : 1.f / (den + p.eps);
                         } else {
-                            inv = 1.f / (__uint_as_float(ud) + rowsum + p.eps);
+                            inv = 1.f / ((__uint_as_float(ud) + __uint_as_float(ud_lo)) + rowsum + p.eps);
                         }
                     }
 #pragma unroll

@@ -108,11 +108,10 @@ def test_prefill_state_inout_and_split(la, orc):
 def test_decay_one_matches_no_decay(la):
     """Decay 1 is the plain causal form.  On the fp32 CUDA-core path every
     decay factor is exactly 1 (2^0), so the results are bitwise equal.  On the
-    tensor-core path every decay weight is exactly 1 too, and the state is the
-    same up to fp32 summation order; the outputs differ by the normaliser
-    operand alone: the decay kernels carry z to the MMA as a hi + lo bf16 pair,
-    the plain kernels as one bf16 value, so they agree to bf16's unit
-    roundoff 2^-9."""
+    tensor-core path every decay weight is exactly 1 too and both kernel
+    families carry the normaliser as the same hi + lo bf16 pair, so the
+    results agree to fp32 rounding (the state is summed in a different order
+    of MMA issue)."""
     q, k, v, _ = _small_inputs(torch.float32, 64, 700, False, 1, 2, seed=9)
     ones = torch.ones((1, 2, 700), dtype=torch.float32)
     o1, S1, _ = gpu_prefill(la, q, k, v, None, 64, torch.float32)
@@ -122,7 +121,7 @@ def test_decay_one_matches_no_decay(la):
     ones = torch.ones((1, 2, 1000), dtype=torch.float32)
     o1, S1, _ = gpu_prefill(la, q, k, v, None, 64, torch.float32)
     o2, S2, _ = gpu_prefill(la, q, k, v, ones, 64, torch.float32)
-    assert row_rel_err(o2, o1) < 2.0 ** -9
+    assert row_rel_err(o2, o1) < 1e-5
     assert row_rel_err(S2.reshape(1, 2, -1), S1.reshape(1, 2, -1)) < 1e-5
 
 
