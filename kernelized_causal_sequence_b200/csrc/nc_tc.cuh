@@ -301,8 +301,8 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 // the read-out's B operand images (bf16 hi and lo, K-major [48][32]: rows
 // 0-31 the columns of S, row 32 z; rows 33-47 are not written and only reach
 // output columns the read-out never reads).  One CTA per head, one thread
-// per 4 consecutive state elements; each thread's loads for up to 8 segments
-// are issued before any is used.  With no keys (n_seg = 0) the total is the
+// per 4 consecutive state elements; each thread's loads for up to 16
+// segments are issued before any is used.  With no keys (n_seg = 0) the total is the
 // state-in or zeros.  grid (BH), kE / 4 = 264 threads.
 struct NcCombineParams {
     const float *ws_state;           // [BH][n_seg][kE]
@@ -324,13 +324,13 @@ __global__ void __launch_bounds__(kCombineThreads) nc_combine_kernel(NcCombinePa
         acc = g < kD * kD / 4 ? reinterpret_cast<const float4 *>(p.state_in_S + (size_t)bh * kD * kD)[g]
                               : reinterpret_cast<const float4 *>(p.state_in_z + (size_t)bh * kD)[g - kD * kD / 4];
     const float4 *src = reinterpret_cast<const float4 *>(p.ws_state + (size_t)bh * p.n_seg * kE) + g;
-    for (int s0 = 0; s0 < p.n_seg; s0 += 8) {
-        float4 x[8];
+    for (int s0 = 0; s0 < p.n_seg; s0 += 16) {
+        float4 x[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 16; ++j)
             x[j] = s0 + j < p.n_seg ? src[(size_t)(s0 + j) * (kE / 4)] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 16; ++j) {
             acc.x += x[j].x;
             acc.y += x[j].y;
             acc.z += x[j].z;
@@ -536,7 +536,7 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
     } else {
         // ================= epilogue (warps 6-9): head state -> B operands, output
-        const int q = warp & 3, et = threadIdx.x - 192;
+        const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         bool waited = false;
         int cur = -1, hc = -1;
