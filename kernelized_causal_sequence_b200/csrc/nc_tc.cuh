@@ -9,36 +9,40 @@
 // attention lesson's developer snippet, step 1, the regrouping
 // (phi(Q) phi(K)^T) V = phi(Q) (phi(K)^T V).)
 //
-// Two kernels, chained by programmatic dependent launch:
+// Three kernels, chained by programmatic dependent launch:
 //
-// nc_state_kernel — one CTA per (group of 4 heads, key segment); the
-//   segments of a group (at most 8) form one thread-block cluster.  The 4
-//   heads' [64 keys x 32] K and V tiles arrive by TMA (4 stages; 64-byte
-//   swizzle, one slab per head); phi(K) is applied in place in the input's
-//   type (rows past the segment zeroed), so the MMA reads phi(K) and V as
-//   they are (bf16 or fp16 operands).  With the 4 heads' feature columns
-//   stacked along M (MN-major A, the next head's slab one 32-element block
-//   further), one M=128, N=128 MMA per 16 keys accumulates phi(K_g)^T V_h
-//   for every head pair (g, h) of the group; the diagonal 32 x 32 blocks are
-//   the heads' states, the rest is discarded (d = 32 is below the tensor
-//   core's M >= 64, and the extra products are free beside the memory
-//   traffic).  A second MMA against a ones operand gives z.  Each CTA puts
-//   its partial (S, z) in its shared memory; across the cluster (distributed
-//   shared memory) every CTA sums its share of the elements over all the
-//   group's partials in a fixed order (deterministic), adds the state-in,
-//   writes the state-out and each head's read-out operands: S and z as a
-//   bf16 hi + lo pair of K-major [48][32] images (rows 0-31 the columns of S,
-//   row 32 z), so the read-out keeps about 16 mantissa bits of the state.
+// nc_state_kernel — one CTA per (group of 4 heads, key segment), the key
+//   tiles split evenly over the segments.  The 4 heads' [64 keys x 32] K and
+//   V tiles arrive by TMA (4 stages; 64-byte swizzle, one slab per head);
+//   eight warps apply phi(K) in place in the input's type (rows past the
+//   segment zeroed), so the MMA reads phi(K) and V as they are (bf16 or fp16
+//   operands).  With the 4 heads' feature columns stacked along M (MN-major
+//   A, the next head's slab one 32-element block further), one M=128, N=128
+//   MMA per 16 keys accumulates phi(K_g)^T V_h for every head pair (g, h) of
+//   the group; the diagonal 32 x 32 blocks are the heads' states, the rest
+//   is discarded (d = 32 is below the tensor core's M >= 64, and the extra
+//   products are free beside the memory traffic).  A second MMA against a
+//   ones operand gives z.  Each CTA writes its heads' partial (S, z) to the
+//   workspace.
+//
+// nc_combine_kernel — per head: the partials summed in segment order
+//   (deterministic) plus the state-in; writes the state-out and the head's
+//   read-out operands: S and z as a bf16 hi + lo pair of K-major [48][32]
+//   images (rows 0-31 the columns of S, row 32 z), so the read-out keeps
+//   about 16 mantissa bits of the state.
 //
 // nc_readout_kernel — a persistent pass over 128-query tiles (every CTA a
 //   contiguous range of (head, tile) pairs).  Its set-up and first query
-//   loads overlap the state kernel; at each new head one bulk copy brings the
-//   head's operand images (6 KB) in, after waiting for the state kernel
-//   (griddepcontrol.wait).  Per tile: phi(Q) is formed in place in the query
-//   tile (one thread per query row), which then serves as the K-major A
-//   operand; four M=128, N=48, K=16 MMAs form [phi(q) S | phi(q) z] in one
-//   of four TMEM accumulators, and the epilogue divides, stages the rows
-//   swizzled and stores them by TMA (rows past Lq clipped).
+//   loads overlap the state kernel (the largest shared-memory carveout lets
+//   a read-out CTA sit beside a state CTA).  After waiting for the combine
+//   kernel (griddepcontrol.wait) the query producer brings each head's
+//   operand images (6 KB) in by one bulk copy, into one of two buffers by
+//   the head's parity, ahead of the head's first tile.  Per tile: phi(Q) is
+//   formed in place in the query tile (one thread per query row), which then
+//   serves as the K-major A operand; four M=128, N=48, K=16 MMAs form
+//   [phi(q) S | phi(q) z] in one of four TMEM accumulators, and the epilogue
+//   divides, stages the rows swizzled and stores them by TMA (rows past Lq
+//   clipped).
 //
 // Every wait is bounded (tc_ptx.cuh); on expiry the CTA raises the call's
 // status word (LA_ERR_TIMEOUT), drains its copies and products and exits.
@@ -76,7 +80,7 @@ struct NcStateParams {
     float *ws_state;                 // [BH][n_seg][kE] partial states
     int *status;                     // the call's status word [2]
     unsigned long long wait_ns;
-    int BH, Lk, seg_len, n_seg;      // seg_len: a multiple of kSRows
+    int BH, Lk, n_seg;               // segment s: key tiles [s * tiles / n_seg, (s + 1) * tiles / n_seg)
 };
 
 struct SCfg {
@@ -94,7 +98,8 @@ struct SCfg {
     static constexpr int OFF_ABORT = OFF_TMEMADDR + 4;
     static constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;   // + alignment slack
     static constexpr int T_S = 0, T_Z = 128, TMEM_COLS = 256;
-    static constexpr int THREADS = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 phi and epilogue
+    static constexpr int THREADS = 320;   // warp 0 TMA, warp 1 MMA, warps 2-9 phi and epilogue
+    static constexpr int PHI_THREADS = 256;
     static_assert(STAGE % 1024 == 0 && HEAD_TILE % 512 == 0 && OFF_ONES % 16 == 0, "layout");
 };
 
@@ -115,22 +120,23 @@ __device__ __forceinline__ uint32_t phi_f16x2(uint32_t x2) {
 
 // phi in place on the [4 heads][64 rows][64 B] K tile (rows >= nvalid
 // zeroed), in the input's own 16-bit type: the state MMA then reads phi(K)
-// and V as they are (bf16 x bf16 or fp16 x fp16), and V needs no conversion.  Thread tw (0..127) takes
-// the 16-byte chunks u = tw + 128 i: the swizzle only permutes chunks inside
-// a 64-byte row, so chunk u lies in row (u / 4) % 64 whatever its position.
-template <typename InT>
+// and V as they are (bf16 x bf16 or fp16 x fp16), and V needs no conversion.
+// Thread tw (0..NT-1) takes the 16-byte chunks u = tw + NT i: the swizzle only
+// permutes chunks inside a 64-byte row, so chunk u lies in row (u / 4) % 64
+// whatever its position.
+template <typename InT, int NT>
 __device__ __forceinline__ void phi_key_tile(uint8_t *kt, int tw, int nvalid) {
     constexpr int NCH = SCfg::TILE / 16;        // 1024 chunks
-    constexpr int PER = NCH / 128;              // 8 per thread
-    constexpr int BATCH = 8;
+    constexpr int PER = NCH / NT;
+    constexpr int BATCH = PER < 8 ? PER : 8;
 #pragma unroll 1
     for (int i0 = 0; i0 < PER; i0 += BATCH) {
         uint4 raw[BATCH];
 #pragma unroll
-        for (int i = 0; i < BATCH; ++i) raw[i] = reinterpret_cast<const uint4 *>(kt)[tw + 128 * (i0 + i)];
+        for (int i = 0; i < BATCH; ++i) raw[i] = reinterpret_cast<const uint4 *>(kt)[tw + NT * (i0 + i)];
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
-            const int u = tw + 128 * (i0 + i);
+            const int u = tw + NT * (i0 + i);
             const bool valid = ((u >> 2) & (kSRows - 1)) < nvalid;
             uint4 f;
             if constexpr (std::is_same<InT, bf16>::value)
@@ -143,7 +149,7 @@ __device__ __forceinline__ void phi_key_tile(uint8_t *kt, int tw, int nvalid) {
     }
 }
 
-// grid (n_seg, ceil(BH / 4)), 192 threads.
+// grid (n_seg, ceil(BH / 4)), 320 threads.
 template <typename InT>
 __global__ void __launch_bounds__(SCfg::THREADS, 1)
 nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -158,8 +164,9 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int seg = blockIdx.x, grp = blockIdx.y;
-    const long j0 = (long)seg * p.seg_len;
-    const long j1 = min((long)p.Lk, j0 + p.seg_len);
+    const long n_tiles = ((long)p.Lk + kSRows - 1) / kSRows;
+    const long j0 = seg * n_tiles / p.n_seg * kSRows;
+    const long j1 = min((long)p.Lk, (seg + 1) * n_tiles / p.n_seg * kSRows);
     const int ntiles = (int)((j1 - j0 + kSRows - 1) / kSRows);
 
     if (threadIdx.x == 0) {
@@ -167,7 +174,7 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int s = 0; s < G::NST; ++s) {
             mbar_init(&bar[G::B_FULL + s], 1);
             mbar_init(&bar[G::B_EMPTY + s], 1);
-            mbar_init(&bar[G::B_PHI + s], 4);
+            mbar_init(&bar[G::B_PHI + s], G::PHI_THREADS / 32);
         }
         mbar_init(&bar[G::B_DONE], 1);
         mbar_init(&bar[G::B_DRAIN], 1);
@@ -250,7 +257,7 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_wait(&bar[G::B_DRAIN], 0, timed, 0);
         }
     } else {
-        // ================= warps 2-5: phi(K), then the partial state out
+        // ================= warps 2-9: phi(K), then the partial state out
         const int tw = threadIdx.x - 64;
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
@@ -259,7 +266,7 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const long y0 = j0 + (long)t * kSRows;
             const int nvalid = (int)min((long)kSRows, j1 - y0);
             uint8_t *kt = smem + G::OFF_KV + s * G::STAGE;
-            phi_key_tile<InT>(kt, tw, nvalid);
+            phi_key_tile<InT, G::PHI_THREADS>(kt, tw, nvalid);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
@@ -267,22 +274,24 @@ nc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // the CTA's partial (S, z) of each of its heads -> the workspace
         if (ok && ntiles > 0 && mbar_wait(&bar[G::B_DONE], 0, ab, 5)) {
             tc_fence_after();
-            // TMEM lane quarter q = head q of the group; lane = feature a
-            const int q = warp & 3, a = lane;
+            // TMEM lane quarter q = head q of the group; lane = feature a; warps
+            // 2-5 take columns 0-15 of the head's diagonal block (and z), warps
+            // 6-9 columns 16-31
+            const int q = warp & 3, a = lane, half = warp >= 6 ? 1 : 0;
             const long bh = (long)grp * kHP + q;
             const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-            uint32_t u[32], zb;
-            tmem_ld32(tmem + lane_base + G::T_S + q * 32, u);   // the diagonal block: S_q[a][0..31]
-            tmem_ld1(tmem + lane_base + G::T_Z, zb);
+            uint32_t u[16], zb = 0;
+            tmem_ld16(tmem + lane_base + G::T_S + q * 32 + half * 16, u);
+            if (!half) tmem_ld1(tmem + lane_base + G::T_Z, zb);
             tmem_ld_wait();
             if (bh < p.BH && !*abort_flag) {
                 float *dst = p.ws_state + ((size_t)bh * p.n_seg + seg) * kE;
-                float4 *d4 = reinterpret_cast<float4 *>(dst + a * kD);
+                float4 *d4 = reinterpret_cast<float4 *>(dst + a * kD + half * 16);
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < 4; ++i)
                     d4[i] = make_float4(__uint_as_float(u[4 * i]), __uint_as_float(u[4 * i + 1]),
                                         __uint_as_float(u[4 * i + 2]), __uint_as_float(u[4 * i + 3]));
-                dst[kD * kD + a] = __uint_as_float(zb);
+                if (!half) dst[kD * kD + a] = __uint_as_float(zb);
             }
         }
     }
@@ -369,7 +378,7 @@ struct NcReadParams {
 
 template <typename OutT> struct RCfg {
     static constexpr int QT = kRows * kRowBytes;            // 8 KB query tile (phi(Q) in place: the A operand)
-    static constexpr int NQ = 6;                            // query tiles in flight
+    static constexpr int NQ = 5;                            // query tiles in flight
     static constexpr int ND = 4;                            // TMEM accumulators [128 x 48] in flight
     static constexpr int OFF_Q = 0;
     static constexpr int STG_WARP = 4096;                   // one warp's 32 output rows (<= 128 B each)
@@ -377,9 +386,9 @@ template <typename OutT> struct RCfg {
     static constexpr int OFF_B = OFF_STG + 2 * 4 * STG_WARP;
     static constexpr int BN = kBN;                          // B operand rows: 32 of S, 1 of z, 15 unused
     static constexpr int BOP = kBop;                        // 3 KB
-    static constexpr int OFF_BAR = OFF_B + 2 * BOP;         // hi, lo
+    static constexpr int OFF_BAR = OFF_B + 2 * kBimg;       // two heads' operands (hi, lo), by head parity
     static constexpr int B_QFULL = 0, B_PHI = NQ, B_QEMPTY = 2 * NQ, B_DFULL = 3 * NQ, B_DEMPTY = B_DFULL + ND,
-                         B_BREADY = B_DEMPTY + ND, B_BLOAD = B_BREADY + 1, B_DRAIN = B_BLOAD + 1,
+                         B_BFREE = B_DEMPTY + ND, B_BLOAD = B_BFREE + 2, B_DRAIN = B_BLOAD + 2,
                          NBAR = B_DRAIN + 1;
     static constexpr int OFF_TMEMADDR = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEMADDR + 4;
@@ -428,14 +437,16 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_init(&bar[G::B_DFULL + a], 1);
             mbar_init(&bar[G::B_DEMPTY + a], 4);
         }
-        mbar_init(&bar[G::B_BREADY], 4);
-        mbar_init(&bar[G::B_BLOAD], 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar[G::B_BFREE + b], 1);
+            mbar_init(&bar[G::B_BLOAD + b], 1);
+        }
         mbar_init(&bar[G::B_DRAIN], 1);
         fence_mbar_init();
     }
     {   // B operands start zeroed (rows 33-47 stay zero)
         uint32_t *b = reinterpret_cast<uint32_t *>(smem + G::OFF_B);
-        for (int i = threadIdx.x; i < 2 * G::BOP / 4; i += G::THREADS) b[i] = 0u;
+        for (int i = threadIdx.x; i < 2 * kBimg / 4; i += G::THREADS) b[i] = 0u;
     }
     if (warp == 1) tmem_alloc(tmem_addr_smem, G::TMEM_COLS);
     if (warp == 0 && lane == 0) {
@@ -449,10 +460,30 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if ((smem_u32(smem) & 1023u) != 0) raise_abort(ab, 99, kStatusLayout);
 
     if (warp == 0) {
-        // ================= TMA producer: query tiles (independent of the state kernel)
+        // ================= TMA producer: query tiles (independent of the state kernel), and
+        // each head's operand images (the combine kernel's) into the buffer of the head's parity
         if (lane == 0 && !*abort_flag) {
-            int issued[G::NQ] = {};
-            for (int i = 0; i < n; ++i) {
+            int issued[G::NQ] = {}, issued_b[2] = {};
+            const int head0 = (int)(f0 / tph);
+            int next_img = 0;   // images issued so far (head index within this CTA's range)
+            bool ok = true;
+            // images of the heads up to index h: after the combine kernel (griddepcontrol.wait),
+            // each into its buffer once the MMAs of the head two before are complete
+            auto images_upto = [&](int h) {
+                for (; ok && next_img <= h; ++next_img) {
+                    const int b = next_img & 1;
+                    if (next_img == 0) pdl_wait();
+                    if (next_img >= 2 && !mbar_wait(&bar[G::B_BFREE + b], ((next_img >> 1) - 1) & 1, ab, 4)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(&bar[G::B_BLOAD + b], kBimg);
+                    bulk_load(smem + G::OFF_B + b * kBimg, p.ws_bimg + (size_t)(head0 + next_img) * kBimg, kBimg,
+                              &bar[G::B_BLOAD + b]);
+                    issued_b[b] = (next_img >> 1) + 1;
+                }
+            };
+            for (int i = 0; ok && i < n; ++i) {
                 const int s = i % G::NQ, use = i / G::NQ;
                 if (use > 0 && !mbar_wait(&bar[G::B_QEMPTY + s], (use - 1) & 1, ab, 1)) break;
                 const long f = f0 + i;
@@ -460,12 +491,16 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mbar_expect_tx(&bar[G::B_QFULL + s], G::QT);
                 tma_load_3d(smem + G::OFF_Q + s * G::QT, &tm_q, &bar[G::B_QFULL + s], 0, t * kRows, bh);
                 issued[s] = use + 1;
+                // once the first stages are filled: the images of the heads loaded so far
+                if (i >= G::NQ - 1 || i == n - 1) images_upto(bh - head0);
             }
             if (*abort_flag) {
                 volatile int never = 0;
                 AbortCtx timed{&never, nullptr, kDrainLimitNs};
                 for (int s = 0; s < G::NQ; ++s)
                     if (issued[s] > 0) mbar_wait(&bar[G::B_QFULL + s], (issued[s] - 1) & 1, timed, 0);
+                for (int b = 0; b < 2; ++b)
+                    if (issued_b[b] > 0) mbar_wait(&bar[G::B_BLOAD + b], (issued_b[b] - 1) & 1, timed, 0);
             }
         }
     } else if (warp == 1) {
@@ -473,8 +508,6 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (lane == 0 && !*abort_flag) {
             constexpr uint32_t ID = idesc_bf16(128, G::BN, false, false);
             const uint32_t sb = smem_u32(smem);
-            const uint64_t dBhi = sdesc_nosw(sb + G::OFF_B, 128, 512);
-            const uint64_t dBlo = sdesc_nosw(sb + G::OFF_B + G::BOP, 128, 512);
             int cur = -1, hc = -1;
             for (int i = 0; i < n; ++i) {
                 const int s = i % G::NQ, a = i % G::ND;
@@ -482,11 +515,15 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (!mbar_wait(&bar[G::B_PHI + s], (i / G::NQ) & 1, ab, 2)) break;
                 if (i >= G::ND && !mbar_wait(&bar[G::B_DEMPTY + a], ((i / G::ND) - 1) & 1, ab, 3)) break;
                 if (bh != cur) {
+                    // the previous head's operand buffer is free once its MMAs are complete
+                    if (hc >= 0) mma_commit(&bar[G::B_BFREE + (hc & 1)]);
                     cur = bh;
                     ++hc;
-                    if (!mbar_wait(&bar[G::B_BREADY], hc & 1, ab, 4)) break;
+                    if (!mbar_wait(&bar[G::B_BLOAD + (hc & 1)], (hc >> 1) & 1, ab, 6)) break;
                 }
                 tc_fence_after();
+                const uint64_t dBhi = sdesc_nosw(sb + G::OFF_B + (hc & 1) * kBimg, 128, 512);
+                const uint64_t dBlo = sdesc_nosw(sb + G::OFF_B + (hc & 1) * kBimg + G::BOP, 128, 512);
                 // A = phi(Q) in place in the query stage: K-major, 64-byte swizzle,
                 // 8-row groups 512 bytes apart; a K step of 16 is 32 bytes
                 const uint64_t dA = sdesc_sw64(sb + G::OFF_Q + s * G::QT, 16, 512);
@@ -535,33 +572,13 @@ nc_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (lane == 0) mbar_arrive(&bar[G::B_PHI + s]);
         }
     } else {
-        // ================= epilogue (warps 6-9): head state -> B operands, output
+        // ================= epilogue (warps 6-9): divide, stage, store
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        bool waited = false;
-        int cur = -1, hc = -1;
         for (int i = 0; i < n; ++i) {
             const int a = i % G::ND;
             const long f = f0 + i;
             const int bh = (int)(f / tph), t = (int)(f % tph);
-            if (bh != cur) {
-                cur = bh;
-                ++hc;
-                // the combine kernel wrote this head's B operands: one bulk copy
-                // (the previous head's MMAs are complete: this warp has consumed
-                // the accumulator of the previous tile)
-                if (warp == 6 && lane == 0) {
-                    if (!waited) {
-                        pdl_wait();   // the combine kernel's results are complete and visible
-                        waited = true;
-                    }
-                    mbar_expect_tx(&bar[G::B_BLOAD], kBimg);
-                    bulk_load(smem + G::OFF_B, p.ws_bimg + (size_t)bh * kBimg, kBimg, &bar[G::B_BLOAD]);
-                }
-                if (!mbar_wait(&bar[G::B_BLOAD], hc & 1, ab, 8)) break;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[G::B_BREADY]);
-            }
             if (!mbar_wait(&bar[G::B_DFULL + a], (i / G::ND) & 1, ab, 7)) break;
             tc_fence_after();
             uint32_t u[32], ud;

@@ -71,7 +71,9 @@ inline Plan make_nc_plan(long BH, long Lk, int D) {
 
 // Key segments of the tensor-core non-causal form (head dimension 32): one
 // CTA per (group of 4 heads, segment of whole 64-key tiles), the segment
-// count chosen so that all CTAs fit in one wave on the SMs.
+// count chosen so that all CTAs fit in one wave on the SMs.  The kernel splits
+// the tiles evenly: segment s takes tiles [s * tiles / n_seg, (s + 1) * tiles
+// / n_seg) (seg_len is the longest segment).
 constexpr int kNcTcHeads = 4;
 constexpr int kNcTcKeyTile = 64;
 inline Plan make_nc_tc_plan(long BH, long Lk) {
@@ -84,7 +86,7 @@ inline Plan make_nc_tc_plan(long BH, long Lk) {
     if (segs > tiles) segs = tiles;
     const long per = (tiles + segs - 1) / segs;
     p.seg_len = (int)(per * kNcTcKeyTile);
-    p.n_seg = (int)((tiles + per - 1) / per);
+    p.n_seg = (int)segs;
     return p;
 }
 

@@ -224,11 +224,15 @@ la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
         sp.wait_ns = a.wait_ns;
         sp.BH = (int)a.BH;
         sp.Lk = a.Lk;
-        sp.seg_len = a.seg_len;
         sp.n_seg = a.n_seg;
         auto kern = nc_state_kernel<InT>;
         s = cuda_check("non-causal state smem attribute",
                        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SCfg::SMEM_BYTES));
+        if (s != LA_OK) return s;
+        // the largest shared-memory carveout, so that a read-out CTA fits beside a state CTA
+        s = cuda_check("non-causal state carveout",
+                       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            (int)cudaSharedmemCarveoutMaxShared));
         if (s != LA_OK) return s;
         s = launch_pdl(kern, dim3((unsigned)a.n_seg, (unsigned)((a.BH + kHP - 1) / kHP)), dim3(SCfg::THREADS),
                        SCfg::SMEM_BYTES, st, false, "non-causal state launch", mk, mv, sp);
@@ -265,6 +269,10 @@ la_status run_noncausal32(const TcNoncausalArgs &a, cudaStream_t st) {
     constexpr int SM = RCfg<OutT>::SMEM_BYTES;
     s = cuda_check("non-causal read-out smem attribute",
                    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM));
+    if (s != LA_OK) return s;
+    s = cuda_check("non-causal read-out carveout",
+                   cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        (int)cudaSharedmemCarveoutMaxShared));
     if (s != LA_OK) return s;
     const long grid = rp.total_tiles < kNumSMs ? rp.total_tiles : kNumSMs;
     // its set-up and query loads overlap the combine kernel

@@ -688,6 +688,64 @@ def test_wait_timeout_is_reported_and_next_call_is_exact(la, d, chunk, decay):
     assert torch.equal(o1, o3) and torch.equal(S1, S3)
 
 
+@pytest.mark.parametrize("B,H,Lq,Lk", [(16, 16, 500, 2000), (16, 64, 129, 65), (2, 3, 1, 5000)])
+def test_noncausal_tc_many_heads(la, orc, B, H, Lq, Lk):
+    """The tensor-core non-causal path with many heads per SM (256 and 1024
+    heads), or one group of heads split into many key segments: equal to the
+    oracle with a state in and out, and bitwise repeatable."""
+    rng = np.random.default_rng(B * H + Lq)
+    mk = lambda L: torch.from_numpy(rng.standard_normal((B, H, L, 32), dtype=np.float32) * 0.6).to(torch.bfloat16)
+    q, k, v = mk(Lq), mk(Lk), mk(Lk)
+    S0 = torch.from_numpy(rng.standard_normal((B, H, 32, 32), dtype=np.float32))
+    z0 = torch.from_numpy(np.abs(rng.standard_normal((B, H, 32), dtype=np.float32)) + 1.0)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    ro, rS, rz = orc.noncausal(q, k, v, S_in=S0, z_in=z0)
+    outs = []
+    for _ in range(2):
+        S, z = S0.to(DEV).clone(), z0.to(DEV).clone()
+        o = la.la_forward_noncausal(qd, kd, vd, state_S=S, state_z=z, mode=la.LA_STATE_INOUT,
+                                    out_dtype=torch.float32)
+        outs.append((o, S, z))
+    torch.cuda.synchronize()
+    o, S, z = outs[0]
+    assert row_rel_err(o.cpu().numpy(), ro) < 2e-2
+    assert row_rel_err(S.cpu().numpy().reshape(B, H, -1), rS.reshape(B, H, -1)) < 2e-2
+    assert row_rel_err(z.cpu().numpy(), rz) < 2e-2
+    assert all(torch.equal(x, y) for x, y in zip(outs[0], outs[1]))
+
+
+def test_noncausal_wait_limit_zero(la):
+    """The non-causal tensor-core call under a wait limit of 0: every wait not
+    satisfied at once gives up, the blocks drain and exit, the status word
+    reports LA_ERR_TIMEOUT; the next call with the default limit is bitwise
+    equal to the call before."""
+    B, H, Lq, Lk = 2, 8, 3000, 3000
+    rng = np.random.default_rng(83)
+    mk = lambda L: torch.from_numpy(rng.standard_normal((B, H, L, 32), dtype=np.float32) * 0.6).to(DEV).half()
+    q, k, v = mk(Lq), mk(Lk), mk(Lk)
+    ws = torch.empty(la.la_noncausal_workspace_size(B, H, Lk, 32, 32), dtype=torch.uint8, device=DEV)
+
+    def call():
+        S = torch.zeros((B, H, 32, 32), device=DEV)
+        z = torch.zeros((B, H, 32), device=DEV)
+        o = la.la_forward_noncausal(q, k, v, state_S=S, state_z=z, mode=la.LA_STATE_OUT, out_dtype=torch.float32,
+                                    workspace=ws)
+        return o, S, z
+
+    r1 = call()
+    assert la.la_workspace_status(ws) == (la.LA_OK, 0)
+    old = la.la_set_wait_limit_ns(0)
+    try:
+        call()
+        st, waiter = la.la_workspace_status(ws)
+    finally:
+        la.la_set_wait_limit_ns(old)
+    assert st == la.LA_ERR_TIMEOUT and waiter > 0
+    r3 = call()
+    assert la.la_workspace_status(ws) == (la.LA_OK, 0)
+    assert all(torch.equal(x, y) for x, y in zip(r1, r3))
+
+
 @pytest.mark.parametrize("B,H,Lq,Lk", [(1, 3, 700, 900), (3, 7, 300, 2000), (1, 1, 128, 128)])
 def test_noncausal_tc_head_groups(la, orc, B, H, Lq, Lk):
     """Head counts that leave the tensor-core state pass's last group of four
