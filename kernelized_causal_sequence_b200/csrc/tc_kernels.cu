@@ -68,6 +68,25 @@ bool make_map_box(CUtensorMap *m, const void *base, la_dtype dt, long BH, long L
     return r == CUDA_SUCCESS;
 }
 
+// 3-D map over a [BH][L][D] tensor with a box of `cols` columns x rows x 1
+// head and the given swizzle.
+bool make_map_cols(CUtensorMap *m, const void *base, la_dtype dt, long BH, long L, int D, int cols, int rows,
+                   CUtensorMapSwizzle sw) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    const int es = dt == LA_F32 ? 4 : 2;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)L * D * es};
+    cuuint32_t box[3] = {(cuuint32_t)cols, (cuuint32_t)rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapDataType t = dt == LA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                  : dt == LA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    CUresult r = enc(m, t, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int C, int D, int FORM, int MODE, typename InT, typename OutT>
 la_status launch_tc(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                     const CUtensorMap &mo, const tc::TcParams &p, long BH, int n_ctas_x, cudaStream_t st,
@@ -102,7 +121,9 @@ la_status run_causal(const TcCausalArgs &a, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, a.q, a.in_dtype, a.BH, a.T, D, C) || !make_map(&mk, a.k, a.in_dtype, a.BH, a.T, D, C) ||
         !make_map(&mv, a.v, a.in_dtype, a.BH, a.T, D, C) ||
-        !make_map(&mo, a.out, a.out_dtype, a.BH, a.T, D, C == 128 ? 32 : 16))   // per-warp row blocks
+        // per-warp row blocks of 32 columns (64-byte rows, 16-bit outputs) or 128 bytes (fp32)
+        !make_map_cols(&mo, a.out, a.out_dtype, a.BH, a.T, D, 32, C == 128 ? 32 : 16,
+                       a.out_dtype == LA_F32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
         return cuda_fail_msg("cuTensorMapEncodeTiled", "tensor map encoding failed");
     tc::TcParams p;
     p.decay = a.decay;

@@ -1224,16 +1224,18 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (!mbar_wait(&bar[G::B_O_FULL], c & 1, ab, 14)) break;
             tc_fence_after();
             // output: 32 columns per TMEM round trip, scaled, converted and
-            // written swizzled to this warp's staging rows; each completed
-            // 128-byte-wide column box is stored by TMA (each warp stores its
-            // own rows; rows beyond T are clipped)
-            constexpr int CPB = 128 / (int)sizeof(OutT);     // columns per box
-            constexpr int GPB = CPB / 32;                    // 32-column groups per box
-            uint8_t *stg = smem + G::OFF_STG + q * (G::ROWS_PER_WARP * 128);   // this warp's rows
+            // written swizzled to this warp's staging rows, then stored by TMA
+            // (each warp stores its own rows; rows beyond T are clipped).  The
+            // O accumulator is released after its last TMEM read, before the
+            // last group is converted and stored.  16-bit outputs: one
+            // 32-column box (64-byte rows) per group, two staging buffers per
+            // warp, so a box waits only for the store two boxes back; fp32:
+            // one 128-byte-wide box per group, one buffer.
+            constexpr bool NARROW = sizeof(OutT) == 2;
+            uint8_t *stg_w = smem + G::OFF_STG + q * (G::ROWS_PER_WARP * 128);   // this warp's 4 KB (2 KB)
             float inv = 0.f;
 #pragma unroll 1
             for (int g = 0; g < D / 32; ++g) {
-                const int bx = g / GPB, gb = g % GPB;
                 float o[32];
                 {
                     uint32_t u[32], ud = 0u, ud_lo = 0u;
@@ -1243,6 +1245,12 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                     tmem_ld32(tmem + lane_base + G::T_O + g * 32, u);
                     tmem_ld_wait();
+                    if (g == D / 32 - 1) {
+                        // every TMEM read of O is complete: the next chunk's MMA2 may overwrite it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bar[G::B_O_EMPTY]);
+                    }
                     // denominator: (decayed) phi(q).z of the carried state + row sum of P + eps
                     if (g == 0) {
                         if constexpr (FLASH) {
@@ -1258,18 +1266,13 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                     for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(u[k]) * inv;
                 }
-                if (gb == 0) {
-                    // this warp's previous store must have read its staging rows
-                    if (lane == 0) bulk_wait_read0();
+                if constexpr (NARROW) {
+                    // buffer (c * D/32 + g) & 1 of this warp: [R][64 B], 64-byte swizzle
+                    const int nb = c * (D / 32) + g;
+                    uint8_t *stg = stg_w + (nb & 1) * (G::ROWS_PER_WARP * 64);
+                    if (lane == 0) bulk_wait_read1();   // the store that last used this buffer has read it
                     __syncwarp();
-                }
-                if (rvalid_lane) {
-                    if constexpr (sizeof(OutT) == 4) {
-#pragma unroll
-                        for (int m = 0; m < 8; ++m)
-                            *reinterpret_cast<float4 *>(stg + sw128_off(lane, m)) =
-                                make_float4(o[4 * m], o[4 * m + 1], o[4 * m + 2], o[4 * m + 3]);
-                    } else {
+                    if (rvalid_lane) {
 #pragma unroll
                         for (int m = 0; m < 4; ++m) {
                             float x[8];
@@ -1280,22 +1283,33 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             else
                                 w = make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]),
                                                pack_f16x2(x[4], x[5]), pack_f16x2(x[6], x[7]));
-                            *reinterpret_cast<uint4 *>(stg + sw128_off(lane, gb * 4 + m)) = w;
+                            *reinterpret_cast<uint4 *>(stg + lane * 64 + ((m ^ ((lane >> 1) & 3)) << 4)) = w;
                         }
                     }
-                }
-                if (gb == GPB - 1) {
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_3d(&tm_o, stg, bx * CPB, (int)t0 + q * G::ROWS_PER_WARP, bh);
+                        tma_store_3d(&tm_o, stg, g * 32, (int)t0 + q * G::ROWS_PER_WARP, bh);
+                        bulk_commit();
+                    }
+                } else {
+                    // this warp's previous store must have read its staging rows
+                    if (lane == 0) bulk_wait_read0();
+                    __syncwarp();
+                    if (rvalid_lane) {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m)
+                            *reinterpret_cast<float4 *>(stg_w + sw128_off(lane, m)) =
+                                make_float4(o[4 * m], o[4 * m + 1], o[4 * m + 2], o[4 * m + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tm_o, stg_w, g * 32, (int)t0 + q * G::ROWS_PER_WARP, bh);
                         bulk_commit();
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[G::B_O_EMPTY]);
         }
     }
 
