@@ -37,12 +37,11 @@ METRIC = "causal linear-attn prefill tokens/s on 1 B200 and % of roofline; decod
 
 # DRAM bytes (read + write) per launch at the long-context workload, from an
 # ncu capture of the same kernels at T = 32768 scaled to T = 131072 (K1 and K3
-# x4, the scan's segment states x1; profiles/dram_traffic_prefill_b1h16_t32768_d128.md
-# and profiles/tc_prefill_k1_k3_b1h16_t32768_d128.md):
+# x4, the scan's segment states x1; profiles/dram_traffic_prefill_b1h16_t32768_d128.md):
 # K3 alone, and the whole call (K1 + scan + K3).  Valid only for that workload
 # and the kernel source they were captured from.
-K3_TRAFFIC_LONG_CONTEXT = 4 * (412228352 + 108334336)
-CALL_TRAFFIC_LONG_CONTEXT = K3_TRAFFIC_LONG_CONTEXT + 4 * (243300352 + 4235264) + 8465408
+K3_TRAFFIC_LONG_CONTEXT = 4 * (412234240 + 105414912)
+CALL_TRAFFIC_LONG_CONTEXT = K3_TRAFFIC_LONG_CONTEXT + 4 * (243306752 + 3481856) + 8465152
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
