@@ -688,6 +688,34 @@ def test_wait_timeout_is_reported_and_next_call_is_exact(la, d, chunk, decay):
     assert torch.equal(o1, o3) and torch.equal(S1, S3)
 
 
+@pytest.mark.parametrize("dtype,d,chunk,decay,gain", [(torch.bfloat16, 128, 128, False, False),
+                                                       (torch.bfloat16, 64, 64, True, True),
+                                                       (torch.float32, 64, 64, True, False)])
+def test_prefill_from_host(la, orc, dtype, d, chunk, decay, gain):
+    """The host-input prefill (pinned host tensors, the sequence in pieces with
+    the copies overlapped, the state carried between the pieces): equal to the
+    oracle over the whole sequence, with a state in and out, the last piece
+    ragged."""
+    from kernelized_causal_sequence_b200 import hostio
+    B, H, T = 2, 3, 1000
+    q, k, v, a = _small_inputs(dtype, d, T, decay, B, H, seed=91)
+    rng = np.random.default_rng(92)
+    b = torch.from_numpy(rng.uniform(0.2, 1.5, (B, H, T)).astype(np.float32)) if gain else None
+    S0 = torch.from_numpy(rng.standard_normal((B, H, d, d), dtype=np.float32) * 0.1)
+    z0 = torch.from_numpy(np.abs(rng.standard_normal((B, H, d), dtype=np.float32)) + 1.0)
+    pin = lambda x: None if x is None else x.contiguous().pin_memory()
+    S, z = S0.to(DEV).clone(), z0.to(DEV).clone()
+    out, S, z = hostio.prefill_causal_from_host(pin(q), pin(k), pin(v), decay=pin(a), gain=pin(b), chunk=chunk,
+                                                out_dtype=torch.float32, state_S=S, state_z=z, piece_tokens=256)
+    torch.cuda.synchronize()
+    ro, rS, rz = orc.causal(q, k, v, a, 1e-6, S_in=S0.double().numpy(), z_in=z0.double().numpy(),
+                            gain=None if b is None else b.double().numpy())
+    tol = 1e-4 if dtype == torch.float32 else 2e-2
+    assert row_rel_err(out.numpy(), ro) < tol
+    assert row_rel_err(S.cpu().numpy().reshape(B, H, -1), rS.reshape(B, H, -1)) < tol
+    assert row_rel_err(z.cpu().numpy(), rz) < tol
+
+
 @pytest.mark.parametrize("B,H,Lq,Lk", [(16, 16, 500, 2000), (16, 64, 129, 65), (2, 3, 1, 5000)])
 def test_noncausal_tc_many_heads(la, orc, B, H, Lq, Lk):
     """The tensor-core non-causal path with many heads per SM (256 and 1024
