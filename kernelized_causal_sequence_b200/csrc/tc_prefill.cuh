@@ -78,6 +78,12 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     // rescaled in place once MMA1 has read them, so one accumulator holds
     // inter + intra; likewise phi(K) becomes w o phi(K) in place for MMA3.
     static constexpr bool QS = OUT && DECAY;
+    // Output pass, no decay, chunk 128: the P epilogue (scores -> P, row sums)
+    // runs on the state-epilogue warps, whose other work is light here, so the
+    // output warps only read out O and the intra-chunk product of chunk c does
+    // not wait for the read-out of chunk c - 1.  The row sums reach the output
+    // warps through TMEM (two columns, by chunk parity).
+    static constexpr bool PW = OUT && !DECAY && C == 128;
     // K/V stages: two in output mode (shared memory is full); the state-only
     // pass has room for more, which hides the load latency of its short chunks
     static constexpr int KV_BYTES = 2 * C * D * 2;
@@ -130,7 +136,8 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     static constexpr int T_Z = T_S + D;                       // z (column 0; MMAz accumulator)
     static constexpr int T_DEN = T_Z + 16;                    // phi(Q) z of the carried state
     static constexpr int T_Q = T_DEN + (OUT ? 16 : 0);
-    static constexpr int T_USED = T_Q + (QT ? D / 2 : 0);
+    static constexpr int T_RS = T_Q + (QT ? D / 2 : 0);      // row sums of P (PW), two columns
+    static constexpr int T_USED = T_RS + (PW ? 2 : 0);
     static constexpr int TMEM_COLS = tmem_alloc_cols(T_USED);
 
     static_assert(D == 64 || D == 128, "tensor-core path: D in {64, 128}");
@@ -645,6 +652,100 @@ __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *ba
 // FLASH chunk form (the decay form's machinery with a = 1 and the identity
 // feature map; scores -> relu(score / s)^2 inside the chunk, the carried
 // summaries read as S / s, no normaliser).
+// Scores -> P of chunk c for the TMEM lane quarter q (this warp's rows): the
+// mask (and decay, or FLASH's squared ReLU), P packed to bf16 (TMEM for chunk
+// 128, shared memory for chunk 64) and the row sums; arrives on p_ready.
+// With RS_TMEM the row sum also goes to TMEM column T_RS + (c & 1), for an
+// output epilogue run by other warps.  False if aborting.
+template <int C, int D, int FORM, int MODE, bool RS_TMEM>
+__device__ __forceinline__ bool p_epilogue(uint8_t *smem, uint64_t *bar, float *Fsm, const TcParams &p,
+                                           const AbortCtx ab, uint32_t tmem, int c, int q, int lane,
+                                           float &rowsum) {
+    constexpr bool DECAY = FORM != 0;
+    constexpr bool FLASH = FORM == 2;
+    using G = Cfg<C, D, DECAY, MODE>;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const bool rvalid_lane = lane < G::ROWS_PER_WARP;
+    const int i = q * G::ROWS_PER_WARP + lane;   // row of the chunk held by this thread
+    const int s = c % G::NKV;
+    rowsum = 0.f;
+    if (!mbar_wait(&bar[G::B_PHI + s], (c / G::NKV) & 1, ab, 12)) return false;
+    if (!mbar_wait(&bar[G::B_SC_FULL], c & 1, ab, 13)) return false;
+    if (DECAY && !mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 28)) return false;
+    tc_fence_after();
+    const float *L = Fsm + G::F_L + s * C;
+    const float *Lk = key_log_weights<C, D, DECAY, MODE>(Fsm, p, s);   // key side (gain folded in)
+    const float Li = (DECAY && rvalid_lane) ? L[min(i, C - 1)] : 0.f;
+    // scores -> P, one 32-column block per TMEM round trip (small code;
+    // measured faster than two).  For this warp's rows [r0, r0 + R) a
+    // block lies fully below the diagonal (no mask), fully above it
+    // (P = 0, scores not read) or on it.
+    const int r0 = q * G::ROWS_PER_WARP, r1 = r0 + G::ROWS_PER_WARP - 1;
+#pragma unroll 1
+    for (int cb0 = 0; cb0 < C / 32; cb0 += 1) {
+        uint32_t u[1][32];
+        bool live[1];
+#pragma unroll
+        for (int h = 0; h < 1; ++h) {
+            live[h] = (cb0 + h) * 32 <= r1;
+            if (live[h]) tmem_ld32(tmem + lane_base + G::T_SC + (cb0 + h) * 32, u[h]);
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 1; ++h) {
+            const int cb = cb0 + h;
+            uint32_t pk[16];
+            if (!live[h]) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) pk[k] = 0u;
+            } else {
+                const bool full = cb * 32 + 31 < r0;   // every j < every row of the warp
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int j = cb * 32 + 2 * k;
+                    float v0 = __uint_as_float(u[h][2 * k]), v1 = __uint_as_float(u[h][2 * k + 1]);
+                    if constexpr (FLASH) {
+                        // exact squared-ReLU weight of the chunk form
+                        v0 = fmaxf(v0 * p.inv_s, 0.f);
+                        v1 = fmaxf(v1 * p.inv_s, 0.f);
+                        v0 *= v0;
+                        v1 *= v1;
+                    } else if constexpr (DECAY) {
+                        v0 *= ex2_approx(Li - Lk[j]);
+                        v1 *= ex2_approx(Li - Lk[j + 1]);
+                    }
+                    v0 = (full || j <= i) ? v0 : 0.f;
+                    v1 = (full || j + 1 <= i) ? v1 : 0.f;
+                    rowsum += v0 + v1;
+                    pk[k] = pack_bf16x2(v0, v1);
+                }
+            }
+            if constexpr (G::PT) {
+                tmem_st16(tmem + lane_base + G::T_SC + cb * 16, pk);
+            } else if (rvalid_lane) {
+                uint8_t *pr = smem + G::OFF_P;
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4 *>(pr + sw128_off(i, cb * 4 + m)) =
+                        make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+            }
+        }
+    }
+    if constexpr (G::PT) tmem_st_wait();
+    else fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if constexpr (RS_TMEM) {
+        // the row sum for the output epilogue, in a TMEM column by chunk parity
+        tmem_st1(tmem + lane_base + G::T_RS + (c & 1), __float_as_uint(rowsum));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+    }
+    if (lane == 0) mbar_arrive(&bar[G::B_P_READY]);
+    return true;
+}
+
 template <int C, int D, int FORM, int MODE, typename InT, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -1073,6 +1174,11 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         } else {
             for (int c = 0; ok && c < nch; ++c) {
+                if constexpr (G::PW) {
+                    float rs;
+                    ok = p_epilogue<C, D, FORM, MODE, true>(smem, bar, Fsm, p, ab, tmem, c, q, lane, rs);
+                    if (!ok) break;
+                }
                 if constexpr (G::QS) {
                     ok = q_weight<C, D, DECAY, MODE>(smem, bar, Fsm, ab, tmem, c, tw);
                     if (!ok) break;
@@ -1152,77 +1258,19 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int c = 0; c < nch; ++c) {
             const int s = c % G::NKV;
             const long t0 = t_begin + (long)c * C;
-            if (!mbar_wait(&bar[G::B_PHI + s], (c / G::NKV) & 1, ab, 12)) break;
-            if (!mbar_wait(&bar[G::B_SC_FULL], c & 1, ab, 13)) break;
-            if (DECAY && !mbar_wait(&bar[G::B_L_READY + s], (c / G::NKV) & 1, ab, 28)) break;
-            tc_fence_after();
-            const float *L = Fsm + G::F_L + s * C;
-            const float *Lk = key_log_weights<C, D, DECAY, MODE>(Fsm, p, s);   // key side (gain folded in)
-            const float Li = (DECAY && rvalid_lane) ? L[min(i, C - 1)] : 0.f;
-            // scores -> P, one 32-column block per TMEM round trip (small code;
-            // measured faster than two).  For this warp's rows [r0, r0 + R) a
-            // block lies fully below the diagonal (no mask), fully above it
-            // (P = 0, scores not read) or on it.
-            const int r0 = q * G::ROWS_PER_WARP, r1 = r0 + G::ROWS_PER_WARP - 1;
             float rowsum = 0.f;
-#pragma unroll 1
-            for (int cb0 = 0; cb0 < C / 32; cb0 += 1) {
-                uint32_t u[1][32];
-                bool live[1];
-#pragma unroll
-                for (int h = 0; h < 1; ++h) {
-                    live[h] = (cb0 + h) * 32 <= r1;
-                    if (live[h]) tmem_ld32(tmem + lane_base + G::T_SC + (cb0 + h) * 32, u[h]);
-                }
-                tmem_ld_wait();
-#pragma unroll
-                for (int h = 0; h < 1; ++h) {
-                    const int cb = cb0 + h;
-                    uint32_t pk[16];
-                    if (!live[h]) {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) pk[k] = 0u;
-                    } else {
-                        const bool full = cb * 32 + 31 < r0;   // every j < every row of the warp
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const int j = cb * 32 + 2 * k;
-                            float v0 = __uint_as_float(u[h][2 * k]), v1 = __uint_as_float(u[h][2 * k + 1]);
-                            if constexpr (FLASH) {
-                                // exact squared-ReLU weight of the chunk form
-                                v0 = fmaxf(v0 * p.inv_s, 0.f);
-                                v1 = fmaxf(v1 * p.inv_s, 0.f);
-                                v0 *= v0;
-                                v1 *= v1;
-                            } else if constexpr (DECAY) {
-                                v0 *= ex2_approx(Li - Lk[j]);
-                                v1 *= ex2_approx(Li - Lk[j + 1]);
-                            }
-                            v0 = (full || j <= i) ? v0 : 0.f;
-                            v1 = (full || j + 1 <= i) ? v1 : 0.f;
-                            rowsum += v0 + v1;
-                            pk[k] = pack_bf16x2(v0, v1);
-                        }
-                    }
-                    if constexpr (G::PT) {
-                        tmem_st16(tmem + lane_base + G::T_SC + cb * 16, pk);
-                    } else if (rvalid_lane) {
-                        uint8_t *pr = smem + G::OFF_P;
-#pragma unroll
-                        for (int m = 0; m < 4; ++m)
-                            *reinterpret_cast<uint4 *>(pr + sw128_off(i, cb * 4 + m)) =
-                                make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
-                    }
-                }
+            if constexpr (!G::PW) {
+                if (!p_epilogue<C, D, FORM, MODE, false>(smem, bar, Fsm, p, ab, tmem, c, q, lane, rowsum)) break;
             }
-            if constexpr (G::PT) tmem_st_wait();
-            else fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[G::B_P_READY]);
 
             if (!mbar_wait(&bar[G::B_O_FULL], c & 1, ab, 14)) break;
             tc_fence_after();
+            if constexpr (G::PW) {
+                uint32_t rsb;
+                tmem_ld1(tmem + lane_base + G::T_RS + (c & 1), rsb);
+                tmem_ld_wait();
+                rowsum = __uint_as_float(rsb);
+            }
             // output: 32 columns per TMEM round trip, scaled, converted and
             // written swizzled to this warp's staging rows, then stored by TMA
             // (each warp stores its own rows; rows beyond T are clipped).  The
