@@ -37,7 +37,8 @@
 // registers at 128 per thread):
 //   warps 0-3    epilogue: scores -> P (mask, decay, row sums), output division
 //                and store.  Warp w reads TMEM lanes 32w..32w+31.  In the
-//                state-only pass: the second half of phi(K).
+//                state-only pass: the second half of phi(K).  Without decay
+//                at chunk 128 the P epilogue runs on warps 6-9 instead.
 //   warp  4      TMA producer (one elected thread).
 //   warp  5      TMEM allocator and MMA issuer (one elected thread).
 //   warps 6-9    phi(Q) (into TMEM for chunk 128) and the state epilogue
