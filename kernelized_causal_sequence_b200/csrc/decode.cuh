@@ -30,6 +30,11 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k, const I
     __shared__ float4 red[RSTEP][CG];
     __shared__ float den_part[kDecodeThreads / 32];
     const int bh = blockIdx.x, tid = threadIdx.x;
+    // launched with programmatic stream serialisation: the next kernel may be
+    // scheduled now; this one waits for the previous kernel (which may have
+    // written q, k, v or the state) before reading anything
+    pdl_trigger();
+    pdl_wait();
     const float a = decay ? decay[bh] : 1.f;
     const float b = gain ? gain[bh] : 1.f;
     if (tid < D) {

@@ -222,9 +222,24 @@ template <typename IT, typename OT, int D> struct SimtNoncausalF {
 template <typename IT, typename OT, int D> struct DecodeF {
     static la_status run(const void *q, const void *k, const void *v, const float *decay, const float *gain,
                          int mlstm, float eps, float *S, float *z, void *out, long BH, cudaStream_t st) {
-        decode_step_kernel<IT, OT, D><<<(unsigned)BH, kDecodeThreads, 0, st>>>(
-            (const IT *)q, (const IT *)k, (const IT *)v, decay, gain, mlstm, eps, S, z, (OT *)out);
+        // programmatic dependent launch: the step may be scheduled while the
+        // previous kernel in the stream drains; it waits for that kernel's
+        // completion (griddepcontrol.wait) before its first global access
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.gridDim = dim3((unsigned)BH);
+        cfg.blockDim = dim3(kDecodeThreads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t err = cudaLaunchKernelEx(&cfg, decode_step_kernel<IT, OT, D>, (const IT *)q,
+                                                   (const IT *)k, (const IT *)v, decay, gain, mlstm, eps, S, z,
+                                                   (OT *)out);
         count_launches(1);
+        if (err != cudaSuccess) return cuda_fail("decode_step launch", err);
         return cuda_check("decode_step launch", cudaGetLastError());
     }
 };
