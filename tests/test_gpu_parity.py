@@ -510,6 +510,41 @@ def test_mlstm_prefill_small(la, orc, dtype, d, T, chunk, gates, B, H):
         assert row_rel_err(z.cpu().numpy(), rz) < tol
 
 
+@pytest.mark.parametrize("form,d,chunk", [("rfa", 128, 64), ("gain", 64, 128), ("mlstm", 128, 128),
+                                          ("mlstm", 64, 64)])
+def test_gated_and_mlstm_state_split(la, orc, form, d, chunk):
+    """The gated and mLSTM prefills in two calls, the state carried in place
+    (INOUT) and the first piece ragged (not a whole number of chunks): equal to
+    the oracle over the whole sequence, outputs and final state."""
+    B, H, T1, T2 = 2, 2, 333, 470
+    T = T1 + T2
+    if form == "mlstm":
+        q, k, v, a, b = _mlstm_inputs(torch.bfloat16, d, T, True, B, H, seed=61)
+        ro, rS, rz = orc.causal(q, k, v, a, gain=b, mlstm=True)
+    else:
+        q, k, v, a, b = _gated_inputs(torch.bfloat16, d, T, form, B, H, seed=62)
+        ro, rS, rz = orc.causal(q, k, v, a, 1e-6, gain=b)
+    dev = lambda x, lo, hi: None if x is None else x[:, :, lo:hi].contiguous().to(DEV)
+    S = torch.zeros((B, H, d, d), device=DEV)
+    z = torch.zeros((B, H, d), device=DEV)
+    outs = []
+    for lo, hi in ((0, T1), (T1, T)):
+        if form == "mlstm":
+            o = la.la_prefill_causal_mlstm(dev(q, lo, hi), dev(k, lo, hi), dev(v, lo, hi), forget=dev(a, lo, hi),
+                                           input_gate=dev(b, lo, hi), chunk=chunk, state_S=S, state_z=z,
+                                           mode=la.LA_STATE_INOUT, out_dtype=torch.float32)
+        else:
+            o = la.la_prefill_causal(dev(q, lo, hi), dev(k, lo, hi), dev(v, lo, hi), decay=dev(a, lo, hi),
+                                     gain=dev(b, lo, hi), chunk=chunk, state_S=S, state_z=z,
+                                     mode=la.LA_STATE_INOUT, out_dtype=torch.float32)
+        outs.append(o)
+    torch.cuda.synchronize()
+    o = torch.cat(outs, dim=2).cpu().numpy()
+    assert row_rel_err(o, ro) < 2e-2, f"output rel err {row_rel_err(o, ro)}"
+    assert row_rel_err(S.cpu().numpy().reshape(B, H, -1), rS.reshape(B, H, -1)) < 2e-2
+    assert row_rel_err(z.cpu().numpy(), rz) < 2e-2
+
+
 def test_workload_mlstm(la, orc):
     w = W["mlstm_bf16_b2h16_t8192_d128"]
     q, k, v, f = inputs.qkv(w)
@@ -697,7 +732,8 @@ def test_prefill_from_host(la, orc, dtype, d, chunk, decay, gain):
     oracle over the whole sequence, with a state in and out, the last piece
     ragged."""
     from kernelized_causal_sequence_b200 import hostio
-    B, H, T = 2, 3, 1000
+    B, H = 2, 3
+    T = 1000 if chunk == 128 else 1024   # pieces of 256 with a ragged last one / whole pieces only
     q, k, v, a = _small_inputs(dtype, d, T, decay, B, H, seed=91)
     rng = np.random.default_rng(92)
     b = torch.from_numpy(rng.uniform(0.2, 1.5, (B, H, T)).astype(np.float32)) if gain else None
@@ -714,6 +750,20 @@ def test_prefill_from_host(la, orc, dtype, d, chunk, decay, gain):
     assert row_rel_err(out.numpy(), ro) < tol
     assert row_rel_err(S.cpu().numpy().reshape(B, H, -1), rS.reshape(B, H, -1)) < tol
     assert row_rel_err(z.cpu().numpy(), rz) < tol
+
+
+def test_prefill_from_host_one_short_piece(la, orc):
+    """The host-input prefill when the whole sequence is shorter than one
+    chunk (a single ragged piece), no state given."""
+    from kernelized_causal_sequence_b200 import hostio
+    q, k, v, a = _small_inputs(torch.bfloat16, 128, 100, True, 1, 2, seed=93)
+    pin = lambda x: x.contiguous().pin_memory()
+    out, S, z = hostio.prefill_causal_from_host(pin(q), pin(k), pin(v), decay=pin(a), chunk=128,
+                                                out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ro, rS, rz = orc.causal(q, k, v, a)
+    assert row_rel_err(out.numpy(), ro) < 2e-2
+    assert row_rel_err(S.cpu().numpy().reshape(1, 2, -1), rS.reshape(1, 2, -1)) < 2e-2
 
 
 @pytest.mark.parametrize("B,H,Lq,Lk", [(16, 16, 500, 2000), (16, 64, 129, 65), (2, 3, 1, 5000)])
