@@ -22,11 +22,11 @@ import kernelized_causal_sequence_b200 as _la
 _STREAMS = {}
 
 
-def _streams(device):
-    key = torch.device(device).index
-    if key not in _STREAMS:
-        _STREAMS[key] = (torch.cuda.Stream(device=device), torch.cuda.Stream(device=device))
-    return _STREAMS[key]
+def _streams(dev):
+    # the copy streams of device `dev` (an explicit index), made once
+    if dev.index not in _STREAMS:
+        _STREAMS[dev.index] = (torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev))
+    return _STREAMS[dev.index]
 
 
 def _copy2d(dst_ptr, dpitch, src_ptr, spitch, width, height, stream):
@@ -53,12 +53,16 @@ def prefill_causal_from_host(q, k, v, decay=None, gain=None, eps=1e-6, chunk=64,
     dv = v.shape[-1]
     BH = B * H
     dev = torch.device(device)
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
     out_dtype = q.dtype if out_dtype is None else out_dtype
     for x in (q, k, v) + tuple(y for y in (decay, gain) if y is not None):
         if x.is_cuda or not x.is_contiguous() or not x.is_pinned():
             raise ValueError("inputs: contiguous pinned host tensors")
     if out is None:
         out = torch.empty((B, H, T, dv), dtype=out_dtype).pin_memory()
+    elif out.is_cuda or not out.is_contiguous() or not out.is_pinned() or tuple(out.shape) != (B, H, T, dv):
+        raise ValueError("out: a contiguous pinned host tensor [B, H, T, d_v]")
     if state_S is None:
         state_S = torch.zeros((B, H, dk, dv), dtype=torch.float32, device=dev)
         state_z = torch.zeros((B, H, dk), dtype=torch.float32, device=dev)
