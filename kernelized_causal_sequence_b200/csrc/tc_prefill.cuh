@@ -79,6 +79,14 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     // rescaled in place once MMA1 has read them, so one accumulator holds
     // inter + intra; likewise phi(K) becomes w o phi(K) in place for MMA3.
     static constexpr bool QS = OUT && DECAY;
+    // Decay forms at chunk 64: the inter term and its normaliser are formed
+    // from the plain phi(Q) in an accumulator of their own, and the output
+    // epilogue applies 2^(L_i) in fp32 (inter * 2^(L_i) + intra), instead of
+    // rescaling the phi(Q) tile in place after MMA1: the query warps are spared
+    // that pass and MMA2 need not wait for it.  (Chunk 128 has no TMEM left for
+    // the second accumulator and rescales phi(Q) in place.)
+    static constexpr bool QSEP = QS && C == 64;
+    static constexpr bool QW = QS && !QSEP;       // phi(Q) rescaled in place after MMA1
     // Output pass, no decay, chunk 128: the P epilogue (scores -> P, row sums)
     // runs on the state-epilogue warps, whose other work is light here, so the
     // output warps only read out O and the intra-chunk product of chunk c does
@@ -133,7 +141,8 @@ template <int C_, int D_, bool DECAY_, int MODE_> struct Cfg {
     // ---- TMEM columns
     static constexpr int T_SC = 0;
     static constexpr int T_O = OUT ? C : 0;
-    static constexpr int T_S = T_O + (OUT ? D : 0);
+    static constexpr int T_OI = T_O + D;                      // QSEP: the inter term (D columns)
+    static constexpr int T_S = T_O + (OUT ? D : 0) + (QSEP ? D : 0);
     static constexpr int T_Z = T_S + D;                       // z (column 0; MMAz accumulator)
     static constexpr int T_DEN = T_Z + 16;                    // phi(Q) z of the carried state
     static constexpr int T_Q = T_DEN + (OUT ? 16 : 0);
@@ -661,7 +670,7 @@ __device__ __forceinline__ bool phi_keys_second_half(uint8_t *smem, uint64_t *ba
 template <int C, int D, int FORM, int MODE, bool RS_TMEM>
 __device__ __forceinline__ bool p_epilogue(uint8_t *smem, uint64_t *bar, float *Fsm, const TcParams &p,
                                            const AbortCtx ab, uint32_t tmem, int c, int q, int lane,
-                                           float &rowsum) {
+                                           float &rowsum, float &li_out) {
     constexpr bool DECAY = FORM != 0;
     constexpr bool FLASH = FORM == 2;
     using G = Cfg<C, D, DECAY, MODE>;
@@ -677,6 +686,7 @@ __device__ __forceinline__ bool p_epilogue(uint8_t *smem, uint64_t *bar, float *
     const float *L = Fsm + G::F_L + s * C;
     const float *Lk = key_log_weights<C, D, DECAY, MODE>(Fsm, p, s);   // key side (gain folded in)
     const float Li = (DECAY && rvalid_lane) ? L[min(i, C - 1)] : 0.f;
+    li_out = Li;
     // scores -> P, one 32-column block per TMEM round trip (small code;
     // measured faster than two).  For this warp's rows [r0, r0 + R) a
     // block lies fully below the diagonal (no mask), fully above it
@@ -995,7 +1005,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     // (with decay: from the 2^(L_i)-scaled phi(Q))
                     if (!mbar_wait(&bar[G::B_S_READY], c & 1, ab, 5)) break;
                     if (c > 0 && !mbar_wait(&bar[G::B_O_EMPTY], (c - 1) & 1, ab, 6)) break;
-                    if (G::QS && !mbar_wait(&bar[G::B_QS_READY], c & 1, ab, 24)) break;
+                    if (G::QW && !mbar_wait(&bar[G::B_QS_READY], c & 1, ab, 24)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
@@ -1006,7 +1016,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             mma_ts(tmem + G::T_DEN, tmem + G::T_Q + kk * 8, bZ, ID_DEN, kk > 0);
                         } else {
                             const uint64_t aQ = dQk + (uint64_t)(((kk >> 2) * G::BOXB + (kk & 3) * 32) >> 4);
-                            mma_ss(tmem + G::T_O, aQ, bS, ID_INT, kk > 0);
+                            mma_ss(tmem + (G::QSEP ? G::T_OI : G::T_O), aQ, bS, ID_INT, kk > 0);
                             mma_ss(tmem + G::T_DEN, aQ, bZ, ID_DEN, kk > 0);
                         }
                     }
@@ -1034,12 +1044,12 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     // MMA4: exact intra-chunk product with the masked, decayed scores
                     if (!mbar_wait(&bar[G::B_P_READY], c & 1, ab, 7)) break;
                     tc_fence_after();
-                    // O (+)= P V
+                    // O (+)= P V  (QSEP: O = P V, the inter term has its own accumulator)
                     const uint32_t dst = tmem + G::T_O;
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk) {
                         const uint64_t bV = dVm + (uint64_t)((kk * 2048) >> 4);
-                        const uint32_t acc = 1;
+                        const uint32_t acc = (G::QSEP && kk == 0) ? 0u : 1u;
                         if constexpr (G::PT)
                             mma_ts(dst, tmem + G::T_SC + kk * 8, bV, ID_PV, acc);
                         else
@@ -1177,10 +1187,11 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int c = 0; ok && c < nch; ++c) {
                 if constexpr (G::PW) {
                     float rs;
-                    ok = p_epilogue<C, D, FORM, MODE, true>(smem, bar, Fsm, p, ab, tmem, c, q, lane, rs);
+                    float li_unused;
+                    ok = p_epilogue<C, D, FORM, MODE, true>(smem, bar, Fsm, p, ab, tmem, c, q, lane, rs, li_unused);
                     if (!ok) break;
                 }
-                if constexpr (G::QS) {
+                if constexpr (G::QW) {
                     ok = q_weight<C, D, DECAY, MODE>(smem, bar, Fsm, ab, tmem, c, tw);
                     if (!ok) break;
                 }
@@ -1259,10 +1270,12 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int c = 0; c < nch; ++c) {
             const int s = c % G::NKV;
             const long t0 = t_begin + (long)c * C;
-            float rowsum = 0.f;
+            float rowsum = 0.f, Li = 0.f;
             if constexpr (!G::PW) {
-                if (!p_epilogue<C, D, FORM, MODE, false>(smem, bar, Fsm, p, ab, tmem, c, q, lane, rowsum)) break;
+                if (!p_epilogue<C, D, FORM, MODE, false>(smem, bar, Fsm, p, ab, tmem, c, q, lane, rowsum, Li)) break;
             }
+            // QSEP: the decay of the carried state at this row, applied to the inter term here
+            const float wq = G::QSEP ? ex2_approx(Li) : 1.f;
 
             if (!mbar_wait(&bar[G::B_O_FULL], c & 1, ab, 14)) break;
             tc_fence_after();
@@ -1293,7 +1306,15 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         tmem_ld1(tmem + lane_base + G::T_DEN + 1, ud_lo);   // phi(q).z_lo
                     }
                     tmem_ld32(tmem + lane_base + G::T_O + g * 32, u);
+                    uint32_t ui[32];
+                    if constexpr (G::QSEP) tmem_ld32(tmem + lane_base + G::T_OI + g * 32, ui);
                     tmem_ld_wait();
+                    if constexpr (G::QSEP) {
+                        // O = 2^(L_i) inter + intra
+#pragma unroll
+                        for (int k = 0; k < 32; ++k)
+                            u[k] = __float_as_uint(fmaf(wq, __uint_as_float(ui[k]), __uint_as_float(u[k])));
+                    }
                     if (g == D / 32 - 1) {
                         // every TMEM read of O is complete: the next chunk's MMA2 may overwrite it
                         tc_fence_before();
@@ -1305,7 +1326,8 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         if constexpr (FLASH) {
                             inv = 1.f;   // no normaliser
                         } else if constexpr (DECAY) {
-                            const float den = (__uint_as_float(ud) + __uint_as_float(ud_lo)) + rowsum;
+                            // (QSEP: the carried-state part from the plain phi(Q), scaled here)
+                            const float den = wq * (__uint_as_float(ud) + __uint_as_float(ud_lo)) + rowsum;
                             // mLSTM read-out: divide by max(|den|, 1)
                             inv = p.mlstm ? 1.f / fmaxf(fabsf(den), 1.f) : 1.f / (den + p.eps);
                         } else {
