@@ -19,9 +19,11 @@
 // 2^(L_i - L_j) for j <= i (L = chunk-local inclusive cumsum of log2 a), the
 // inter term of row i is scaled by 2^(L_i), and the state is rescaled by the
 // chunk's total decay before each update.  MMA1 reads the plain phi(Q) and
-// phi(K); once it has, the two tiles are rescaled in place (rows of phi(Q) by
-// 2^(L_i) for MMA2/MMAd, rows of phi(K) by w_j for MMA3/MMAz), so a single
-// accumulator holds the inter and intra terms and no second K tile is needed.
+// phi(K); once it has, the rows of phi(K) are rescaled in place by w_j for
+// MMA3/MMAz, so no second K tile is needed.  At chunk 128 the rows of phi(Q)
+// are likewise rescaled by 2^(L_i) for MMA2/MMAd and one accumulator holds
+// the inter and intra terms; at chunk 64 the inter term has an accumulator of
+// its own and the output epilogue applies 2^(L_i) to it.
 //
 // The decay instantiations also serve two forms of the concept card:
 // - a per-token gain b_j on the new term (the RFA gate's 1 - g): it folds
@@ -41,8 +43,9 @@
 //                at chunk 128 the P epilogue runs on warps 6-9 instead.
 //   warp  4      TMA producer (one elected thread).
 //   warp  5      TMEM allocator and MMA issuer (one elected thread).
-//   warps 6-9    phi(Q) (into TMEM for chunk 128) and the state epilogue
-//                (TMEM S -> bf16 operand, decay rescale).
+//   warps 6-9    phi(Q) (into TMEM for chunk 128; with decay at chunk 128
+//                then rescaled by 2^(L_i)) and the state epilogue (TMEM S ->
+//                bf16 operand, decay rescale).
 //   warps 10-13  decay cumsum and phi(K) (then w o phi(K) in place).
 //
 // Every wait is bounded (see tc_ptx.cuh); on expiry the CTA raises its abort
