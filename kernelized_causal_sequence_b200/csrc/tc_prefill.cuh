@@ -35,18 +35,21 @@
 // q.z keeps about 16 mantissa bits.  The state-only pass covers every segment
 // but a head's last; the output pass of that segment writes the final state.
 //
-// Warp roles (448 threads; at most four warps share a scheduler, which caps
+// Warp roles (480 threads; at most four warps share a scheduler, which caps
 // registers at 128 per thread):
 //   warps 0-3    epilogue: scores -> P (mask, decay, row sums), output division
-//                and store.  Warp w reads TMEM lanes 32w..32w+31.  In the
-//                state-only pass: the second half of phi(K).  Without decay
-//                at chunk 128 the P epilogue runs on warps 6-9 instead.
+//                and store.  Warp w reads TMEM lanes 32w..32w+31; at chunk 64
+//                (M = 64 products, rows in lanes 0-15 of each quarter) threads
+//                0-15 and 16-31 take the two column halves of the same 16 rows.
+//                In the state-only pass: the second half of phi(K).  Without
+//                decay at chunk 128 the P epilogue runs on warps 6-9 instead.
 //   warp  4      TMA producer (one elected thread).
 //   warp  5      TMEM allocator and MMA issuer (one elected thread).
 //   warps 6-9    phi(Q) (into TMEM for chunk 128; with decay at chunk 128
 //                then rescaled by 2^(L_i)) and the state epilogue (TMEM S ->
 //                bf16 operand, decay rescale).
 //   warps 10-13  decay cumsum and phi(K) (then w o phi(K) in place).
+//   warp  14     TMA producer of the query tiles (output mode).
 //
 // Every wait is bounded (see tc_ptx.cuh); on expiry the CTA raises its abort
 // flag and the call's status word (LA_ERR_TIMEOUT and the id of the wait),
@@ -678,8 +681,12 @@ __device__ __forceinline__ bool p_epilogue(uint8_t *smem, uint64_t *bar, float *
     constexpr bool FLASH = FORM == 2;
     using G = Cfg<C, D, DECAY, MODE>;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    const bool rvalid_lane = lane < G::ROWS_PER_WARP;
-    const int i = q * G::ROWS_PER_WARP + lane;   // row of the chunk held by this thread
+    // HS (chunk 64): threads 0-15 and 16-31 hold the low and high 16 columns
+    // of each 32-column block of the same row
+    constexpr bool HS = G::ROWS_PER_WARP == 16;
+    constexpr int NV = HS ? 16 : 32;                          // values per thread per block
+    const int hc = HS ? (lane >> 4) * 16 : 0;                 // this thread's column offset in a block
+    const int i = q * G::ROWS_PER_WARP + (HS ? (lane & 15) : lane);   // row of the chunk held by this thread
     const int s = c % G::NKV;
     rowsum = 0.f;
     if (!mbar_wait(&bar[G::B_PHI + s], (c / G::NKV) & 1, ab, 12)) return false;
@@ -688,7 +695,7 @@ __device__ __forceinline__ bool p_epilogue(uint8_t *smem, uint64_t *bar, float *
     tc_fence_after();
     const float *L = Fsm + G::F_L + s * C;
     const float *Lk = key_log_weights<C, D, DECAY, MODE>(Fsm, p, s);   // key side (gain folded in)
-    const float Li = (DECAY && rvalid_lane) ? L[min(i, C - 1)] : 0.f;
+    const float Li = DECAY ? L[i] : 0.f;
     li_out = Li;
     // scores -> P, one 32-column block per TMEM round trip (small code;
     // measured faster than two).  For this warp's rows [r0, r0 + R) a
@@ -697,26 +704,29 @@ __device__ __forceinline__ bool p_epilogue(uint8_t *smem, uint64_t *bar, float *
     const int r0 = q * G::ROWS_PER_WARP, r1 = r0 + G::ROWS_PER_WARP - 1;
 #pragma unroll 1
     for (int cb0 = 0; cb0 < C / 32; cb0 += 1) {
-        uint32_t u[1][32];
+        uint32_t u[1][NV];
         bool live[1];
 #pragma unroll
         for (int h = 0; h < 1; ++h) {
             live[h] = (cb0 + h) * 32 <= r1;
-            if (live[h]) tmem_ld32(tmem + lane_base + G::T_SC + (cb0 + h) * 32, u[h]);
+            if (live[h]) {
+                if constexpr (HS) tmem_ld16x2<16>(tmem + lane_base + G::T_SC + (cb0 + h) * 32, u[h]);
+                else tmem_ld32(tmem + lane_base + G::T_SC + (cb0 + h) * 32, u[h]);
+            }
         }
         tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < 1; ++h) {
             const int cb = cb0 + h;
-            uint32_t pk[16];
+            uint32_t pk[NV / 2];
             if (!live[h]) {
 #pragma unroll
-                for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                for (int k = 0; k < NV / 2; ++k) pk[k] = 0u;
             } else {
                 const bool full = cb * 32 + 31 < r0;   // every j < every row of the warp
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int j = cb * 32 + 2 * k;
+                for (int k = 0; k < NV / 2; ++k) {
+                    const int j = cb * 32 + hc + 2 * k;
                     float v0 = __uint_as_float(u[h][2 * k]), v1 = __uint_as_float(u[h][2 * k + 1]);
                     if constexpr (FLASH) {
                         // exact squared-ReLU weight of the chunk form
@@ -736,15 +746,16 @@ __device__ __forceinline__ bool p_epilogue(uint8_t *smem, uint64_t *bar, float *
             }
             if constexpr (G::PT) {
                 tmem_st16(tmem + lane_base + G::T_SC + cb * 16, pk);
-            } else if (rvalid_lane) {
+            } else {
                 uint8_t *pr = smem + G::OFF_P;
 #pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    *reinterpret_cast<uint4 *>(pr + sw128_off(i, cb * 4 + m)) =
+                for (int m = 0; m < NV / 8; ++m)
+                    *reinterpret_cast<uint4 *>(pr + sw128_off(i, cb * 4 + hc / 8 + m)) =
                         make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
             }
         }
     }
+    if constexpr (HS) rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);   // both column halves
     if constexpr (G::PT) tmem_st_wait();
     else fence_proxy_async_smem();
     tc_fence_before();
@@ -1268,8 +1279,13 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // ================= epilogue (warps 0-3): scores -> P, output division and store
         const int q = warp;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const bool rvalid_lane = lane < G::ROWS_PER_WARP;
-        const int i = q * G::ROWS_PER_WARP + lane;   // row of the chunk held by this thread
+        // HS (chunk 64, rows in lanes 0-15 of the warp's quarter): thread t
+        // holds row t & 15 and the columns [16 (t >> 4), + 16) of each
+        // 32-column group; otherwise thread t holds row t and all 32 columns
+        constexpr bool HS = G::ROWS_PER_WARP == 16;
+        constexpr int NV = HS ? 16 : 32;
+        const int r = HS ? (lane & 15) : lane;    // this thread's row in the warp's rows
+        const int hm = HS ? (lane >> 4) : 0;      // its column half (16-byte chunks 2hm.. / 4hm..)
         for (int c = 0; c < nch; ++c) {
             const int s = c % G::NKV;
             const long t0 = t_begin + (long)c * C;
@@ -1301,21 +1317,33 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             float inv = 0.f;
 #pragma unroll 1
             for (int g = 0; g < D / 32; ++g) {
-                float o[32];
+                float o[NV];
                 {
-                    uint32_t u[32], ud = 0u, ud_lo = 0u;
+                    uint32_t u[NV], ud = 0u, ud_lo = 0u;
                     if (g == 0) {
                         tmem_ld1(tmem + lane_base + G::T_DEN, ud);
                         tmem_ld1(tmem + lane_base + G::T_DEN + 1, ud_lo);   // phi(q).z_lo
                     }
-                    tmem_ld32(tmem + lane_base + G::T_O + g * 32, u);
-                    uint32_t ui[32];
-                    if constexpr (G::QSEP) tmem_ld32(tmem + lane_base + G::T_OI + g * 32, ui);
+                    uint32_t ui[NV];
+                    if constexpr (HS) {
+                        tmem_ld16x2<16>(tmem + lane_base + G::T_O + g * 32, u);
+                        if constexpr (G::QSEP) tmem_ld16x2<16>(tmem + lane_base + G::T_OI + g * 32, ui);
+                    } else {
+                        tmem_ld32(tmem + lane_base + G::T_O + g * 32, u);
+                        if constexpr (G::QSEP) tmem_ld32(tmem + lane_base + G::T_OI + g * 32, ui);
+                    }
                     tmem_ld_wait();
+                    if constexpr (HS) {
+                        // the denominator terms sit in lane r's row (read by threads 0-15)
+                        if (g == 0) {
+                            ud = __shfl_sync(0xffffffffu, ud, r);
+                            ud_lo = __shfl_sync(0xffffffffu, ud_lo, r);
+                        }
+                    }
                     if constexpr (G::QSEP) {
                         // O = 2^(L_i) inter + intra
 #pragma unroll
-                        for (int k = 0; k < 32; ++k)
+                        for (int k = 0; k < NV; ++k)
                             u[k] = __float_as_uint(fmaf(wq, __uint_as_float(ui[k]), __uint_as_float(u[k])));
                     }
                     if (g == D / 32 - 1) {
@@ -1338,7 +1366,7 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         }
                     }
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) o[k] = __uint_as_float(u[k]) * inv;
+                    for (int k = 0; k < NV; ++k) o[k] = __uint_as_float(u[k]) * inv;
                 }
                 if constexpr (NARROW) {
                     // buffer (c * D/32 + g) & 1 of this warp: [R][64 B], 64-byte swizzle
@@ -1346,19 +1374,18 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     uint8_t *stg = stg_w + (nb & 1) * (G::ROWS_PER_WARP * 64);
                     if (lane == 0) bulk_wait_read1();   // the store that last used this buffer has read it
                     __syncwarp();
-                    if (rvalid_lane) {
 #pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            float x[8];
+                    for (int mm = 0; mm < NV / 8; ++mm) {
+                        const int m = (NV / 8) * hm + mm;   // 16-byte chunk of the 64-byte row
+                        float x[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] = o[8 * m + e];
-                            uint4 w;
-                            if constexpr (std::is_same<OutT, bf16>::value) w = pack8_bf16(x);
-                            else
-                                w = make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]),
-                                               pack_f16x2(x[4], x[5]), pack_f16x2(x[6], x[7]));
-                            *reinterpret_cast<uint4 *>(stg + lane * 64 + ((m ^ ((lane >> 1) & 3)) << 4)) = w;
-                        }
+                        for (int e = 0; e < 8; ++e) x[e] = o[8 * mm + e];
+                        uint4 w;
+                        if constexpr (std::is_same<OutT, bf16>::value) w = pack8_bf16(x);
+                        else
+                            w = make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]),
+                                           pack_f16x2(x[4], x[5]), pack_f16x2(x[6], x[7]));
+                        *reinterpret_cast<uint4 *>(stg + r * 64 + ((m ^ ((r >> 1) & 3)) << 4)) = w;
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -1370,12 +1397,10 @@ tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     // this warp's previous store must have read its staging rows
                     if (lane == 0) bulk_wait_read0();
                     __syncwarp();
-                    if (rvalid_lane) {
 #pragma unroll
-                        for (int m = 0; m < 8; ++m)
-                            *reinterpret_cast<float4 *>(stg_w + sw128_off(lane, m)) =
-                                make_float4(o[4 * m], o[4 * m + 1], o[4 * m + 2], o[4 * m + 3]);
-                    }
+                    for (int mm = 0; mm < NV / 4; ++mm)
+                        *reinterpret_cast<float4 *>(stg_w + sw128_off(r, (NV / 4) * hm + mm)) =
+                            make_float4(o[4 * mm], o[4 * mm + 1], o[4 * mm + 2], o[4 * mm + 3]);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
