@@ -40,8 +40,8 @@ METRIC = "causal linear-attn prefill tokens/s on 1 B200 and % of roofline; decod
 # x4, the scan's segment states x1; profiles/dram_traffic_prefill_b1h16_t32768_d128.md):
 # K3 alone, and the whole call (K1 + scan + K3).  Valid only for that workload
 # and the kernel source they were captured from.
-K3_TRAFFIC_LONG_CONTEXT = 4 * (412234240 + 105414912)
-CALL_TRAFFIC_LONG_CONTEXT = K3_TRAFFIC_LONG_CONTEXT + 4 * (243306752 + 3481856) + 8465152
+K3_TRAFFIC_LONG_CONTEXT = 4 * (412253184 + 105545984)
+CALL_TRAFFIC_LONG_CONTEXT = K3_TRAFFIC_LONG_CONTEXT + 4 * (243309056 + 3817728) + 8465408
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
