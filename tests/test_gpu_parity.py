@@ -60,6 +60,10 @@ SMALL = [
     (torch.bfloat16, 128, 3000, 128, False, 1, 2),
     (torch.float16, 32, 300, 128, False, 2, 2),
     (torch.float16, 128, 513, 64, True, 1, 2),
+    # chunk 64 without decay at d 128 (bf16 out) and d 64 (fp16 out): the
+    # output epilogues' half-warp column split, ragged tails
+    (torch.bfloat16, 128, 700, 64, False, 1, 2),
+    (torch.float16, 64, 450, 64, False, 2, 1),
     # chunk 128 with decay on the tensor cores (in-place decay weights)
     (torch.bfloat16, 128, 1000, 128, True, 1, 2),
     (torch.bfloat16, 64, 777, 128, True, 2, 1),
