@@ -18,8 +18,11 @@ namespace la {
 
 constexpr int kDecodeThreads = 256;
 
+// 8 CTAs per SM (at most 32 registers a thread): a decode step of 1024 heads
+// (B64 H16) is then one wave on 148 SMs; at 40 registers only 6 fit and the
+// last 136 heads ran as a second, mostly idle wave
 template <typename InT, typename OutT, int D>
-__global__ void __launch_bounds__(kDecodeThreads)
+__global__ void __launch_bounds__(kDecodeThreads, 8)
 decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k, const InT *__restrict__ v,
                    const float *__restrict__ decay, const float *__restrict__ gain, int mlstm,
                    float eps, float *__restrict__ S,
@@ -62,7 +65,7 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k, const I
     // state rows: S[r] <- a S[r] + phi(k)_r v ; num += phi(q)_r S[r]
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
     float4 *Sp = reinterpret_cast<float4 *>(S + (size_t)bh * D * D) + cg;
-#pragma unroll 4
+#pragma unroll 2   // (4 spills under the 32-register bound and measured slower)
     for (int r = r0; r < D; r += RSTEP) {
         float4 s = Sp[(size_t)r * CG];
         const float f = fk[r], g = fq[r];
