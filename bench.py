@@ -342,23 +342,38 @@ def measure_workloads(dev, peaks, iters=10, only=None):
     return res
 
 
-def measure_l2_copy_gbs(dev, mib=32, reps=200):
-    """Device copy rate with source and destination resident in L2 (bytes read
-    + written per second): the denominator of an L2-resident kernel."""
+def measure_l2_gbs(dev, reps=200):
+    """The best of two L2-resident streaming rates (bytes read + written per
+    second), the denominator of an L2-resident kernel: a device copy between
+    two 32 MiB buffers, and an in-place update of one 64 MiB fp32 buffer (the
+    decode state's access: every element read once and written back).
+    Returns (rate, which)."""
     import torch
-    n = (mib << 20) // 4
+    st = torch.cuda.current_stream(dev)
+
+    def timed(fn, nbytes):
+        for _ in range(10):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(reps):
+            fn()
+        e1.record(st)
+        e1.synchronize()
+        return nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9
+
+    n = (32 << 20) // 4
     a = torch.ones(n, dtype=torch.float32, device=dev)
     b = torch.empty_like(a)
-    for _ in range(10):
-        b.copy_(a)
-    st = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(reps):
-        b.copy_(a)
-    e1.record(st)
-    e1.synchronize()
-    return 2 * n * 4 * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    copy = timed(lambda: b.copy_(a), 2 * n * 4)
+    del a, b
+    m = (64 << 20) // 4
+    x = torch.ones(m, dtype=torch.float32, device=dev)
+    rmw = timed(lambda: x.mul_(1.0), 2 * m * 4)
+    del x
+    if rmw > copy:
+        return rmw, "L2-resident in-place update of a 64 MiB fp32 buffer (best of it and a 2 x 32 MiB copy)"
+    return copy, "L2-resident device copy, 2 x 32 MiB (best of it and a 64 MiB in-place update)"
 
 
 def decode_cold_step_ms(la, dec, steps, n_sets=4, reps=3):
@@ -618,19 +633,19 @@ def run_ours(args, w):
     if dec:
         dbytes = decode_bytes_per_step(dec["w"])
         per_step_ms = dec_avg / args.decode_steps
-        l2_gbs = measure_l2_copy_gbs(dev)
+        l2_gbs, l2_src = measure_l2_gbs(dev)
         cold_ms = decode_cold_step_ms(la, dec, args.decode_steps)
         line["decode"] = {
             "value": job_rate(world, 1, per_step_ms), "unit": "steps/s", "steps_per_bench_step": args.decode_steps,
             "B": dec["w"].B, "H": dec["w"].H, "d": dec["w"].d, "us_per_step": per_step_ms * 1e3,
             "bytes_per_step": dbytes,
             # the 67.6 MB fp32 state stays in the 126 MB L2 across the loop, as in a
-            # real decode loop: its bound is the L2, measured here as a copy whose
-            # source and destination fit in L2
+            # real decode loop: its bound is the L2, measured here as the best of two
+            # L2-resident streaming kernels
             "roofline": {"bound": "l2", "achieved": dbytes / (per_step_ms * 1e-3) / 1e9,
                          "peak": l2_gbs, "unit": "GB/s",
                          "frac": dbytes / (per_step_ms * 1e-3) / 1e9 / l2_gbs,
-                         "peak_source": "measured in this run: L2-resident device copy (2 x 32 MiB)",
+                         "peak_source": "measured in this run: " + l2_src,
                          "note": "fp32 state (67.6 MB) stays L2-resident across the loop"},
             # the same steps rotating over four state sets (270 MB > L2), so every
             # step reads and writes its state in HBM
